@@ -1,0 +1,199 @@
+"""PyTorch-facing API of the B200 BitLinear: pack_weights, quant_act, forward.
+
+PyTorch supplies device memory and streams; the arithmetic is in
+libbitlinear (C ABI, include/bitlinear.h). Shapes follow torch.nn.Linear:
+W [N, K] (out_features x in_features), x [M, K], y [M, N]. The per-row scale D
+is a [N, 1] tensor, as the ternary kernel of "Core AI model zoo - BitVLA"
+section 2 requires ([1, N] is rejected: that layout made the Metal kernel of
+the page read out of bounds).
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+
+__all__ = [
+    "pack_weights",
+    "quant_act",
+    "forward",
+    "forward_acc",
+    "forward_host",
+    "prepare_act",
+    "forward_prepared",
+    "workspace_size",
+    "workspace_error",
+    "BitLinear",
+]
+
+
+def _stream_handle(device: torch.device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _need_cuda(t: torch.Tensor, name: str, dtype: torch.dtype) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _check_D(D: torch.Tensor, N: int) -> None:
+    if tuple(D.shape) != (N, 1):
+        raise ValueError(f"D must have shape [N, 1] = [{N}, 1], got {list(D.shape)}")
+    _need_cuda(D, "D", torch.float32)
+
+
+def _alloc_ws(nbytes: int, device: torch.device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks.
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def workspace_size(M: int, N: int, K: int) -> int:
+    return int(_lib.lib().bitlinear_workspace_size(M, N, K))
+
+
+def pack_weights(W: torch.Tensor, ws: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """WeightQuant + pack: fp32 W [N, K] -> (packed int32 [N, K/16], D fp32 [N, 1])."""
+    _need_cuda(W, "W", torch.float32)
+    N, K = W.shape
+    packed = torch.empty((N, K // 16), dtype=torch.int32, device=W.device)
+    D = torch.empty((N, 1), dtype=torch.float32, device=W.device)
+    L = _lib.lib()
+    if ws is None:
+        ws = _alloc_ws(L.bitlinear_pack_workspace_size(N, K), W.device)
+    _lib.call("bitlinear_pack_weights", W.data_ptr(), N, K, packed.data_ptr(), D.data_ptr(),
+              ws.data_ptr(), ws.numel(), _stream_handle(W.device))
+    return packed, D
+
+
+def quant_act(x: torch.Tensor):
+    """ActQuant: fp32 x [M, K] -> (q int8 [M, K], s_x fp32 [M], rowsum int32 [M])."""
+    _need_cuda(x, "x", torch.float32)
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s_x = torch.empty((M,), dtype=torch.float32, device=x.device)
+    rs = torch.empty((M,), dtype=torch.int32, device=x.device)
+    _lib.call("bitlinear_quant_act", x.data_ptr(), M, K, q.data_ptr(), s_x.data_ptr(), rs.data_ptr(),
+              _stream_handle(x.device))
+    return q, s_x, rs
+
+
+def _fwd_args(x, packed, K):
+    _need_cuda(x, "x", torch.float32)
+    _need_cuda(packed, "packed", torch.int32)
+    if x.dim() != 2 or packed.dim() != 2:
+        raise ValueError("x must be [M, K] and packed [N, K/16]")
+    M, Kx = x.shape
+    if Kx != K or packed.shape[1] * 16 != K:
+        raise ValueError(f"K mismatch: x has {Kx}, packed has {packed.shape[1] * 16}")
+    return M, packed.shape[0]
+
+
+def forward(x: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,
+            out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = F.linear(ActQuant(x), WeightQuant(W)) from packed weights."""
+    K = x.shape[-1]
+    M, N = _fwd_args(x, packed, K)
+    _check_D(D, N)
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _need_cuda(y, "out", torch.float32)
+    need = workspace_size(M, N, K)
+    if ws is None:
+        ws = _alloc_ws(need, x.device)
+    _lib.call("bitlinear_forward", x.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(), y.data_ptr(),
+              ws.data_ptr(), ws.numel(), _stream_handle(x.device))
+    return y
+
+
+def forward_acc(x: torch.Tensor, packed: torch.Tensor, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Exact int32 accumulators acc[m, n] = sum_k q[m, k] * code[n, k]."""
+    K = x.shape[-1]
+    M, N = _fwd_args(x, packed, K)
+    acc = torch.empty((M, N), dtype=torch.int32, device=x.device)
+    if ws is None:
+        ws = _alloc_ws(workspace_size(M, N, K), x.device)
+    _lib.call("bitlinear_forward_acc", x.data_ptr(), M, N, K, packed.data_ptr(), acc.data_ptr(),
+              ws.data_ptr(), ws.numel(), _stream_handle(x.device))
+    return acc
+
+
+def prepare_act(x: torch.Tensor, ws: torch.Tensor) -> torch.Tensor:
+    """Quantise x [M, K] once into `ws` for several forward_prepared calls."""
+    _need_cuda(x, "x", torch.float32)
+    M, K = x.shape
+    _lib.call("bitlinear_prepare_act", x.data_ptr(), M, K, ws.data_ptr(), ws.numel(), _stream_handle(x.device))
+    return ws
+
+
+def forward_prepared(M: int, K: int, packed: torch.Tensor, D: torch.Tensor, ws: torch.Tensor,
+                     out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Contraction + rescale from a workspace filled by prepare_act (tensor-core path)."""
+    _need_cuda(packed, "packed", torch.int32)
+    N = packed.shape[0]
+    if packed.shape[1] * 16 != K:
+        raise ValueError("K mismatch with packed")
+    _check_D(D, N)
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=packed.device)
+    _need_cuda(y, "out", torch.float32)
+    _lib.call("bitlinear_forward_prepared", M, N, K, packed.data_ptr(), D.data_ptr(), y.data_ptr(),
+              ws.data_ptr(), ws.numel(), _stream_handle(packed.device))
+    return y
+
+
+def forward_host(x_host: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,
+                 y_host: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """End-to-end call with host x / y (pinned recommended); synchronous."""
+    if x_host.is_cuda or x_host.dtype != torch.float32 or not x_host.is_contiguous():
+        raise ValueError("x_host must be a contiguous fp32 CPU tensor")
+    M, K = x_host.shape
+    _need_cuda(packed, "packed", torch.int32)
+    N = packed.shape[0]
+    _check_D(D, N)
+    if y_host is None:
+        y_host = torch.empty((M, N), dtype=torch.float32, pin_memory=True)
+    L = _lib.lib()
+    if ws is None:
+        ws = _alloc_ws(L.bitlinear_host_workspace_size(M, N, K), packed.device)
+    _lib.call("bitlinear_forward_host", x_host.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(),
+              y_host.data_ptr(), ws.data_ptr(), ws.numel(), _stream_handle(packed.device))
+    return y_host
+
+
+def workspace_error(ws: torch.Tensor) -> int:
+    """Synchronise and read/clear the device error word of a forward workspace."""
+    return int(_lib.lib().bitlinear_workspace_error(ws.data_ptr(), ws.numel(), _stream_handle(ws.device)))
+
+
+class BitLinear:
+    """A packed BitNet b1.58 linear layer: holds packed codes and D [N, 1]."""
+
+    def __init__(self, packed: torch.Tensor, D: torch.Tensor):
+        _need_cuda(packed, "packed", torch.int32)
+        _check_D(D, packed.shape[0])
+        self.packed = packed
+        self.D = D
+        self.out_features = packed.shape[0]
+        self.in_features = packed.shape[1] * 16
+        self._ws = None
+
+    @classmethod
+    def from_float(cls, W: torch.Tensor) -> "BitLinear":
+        packed, D = pack_weights(W.contiguous().float())
+        return cls(packed, D)
+
+    def workspace(self, M: int) -> torch.Tensor:
+        need = workspace_size(M, self.out_features, self.in_features)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = _alloc_ws(need, self.packed.device)
+        return self._ws
+
+    def __call__(self, x: torch.Tensor) -> torch.Tensor:
+        lead = x.shape[:-1]
+        x2 = x.reshape(-1, self.in_features).contiguous().float()
+        y = forward(x2, self.packed, self.D, ws=self.workspace(x2.shape[0]))
+        return y.reshape(*lead, self.out_features)

@@ -1,0 +1,234 @@
+// bl_api.cu - the extern "C" entry points of libbitlinear (see include/bitlinear.h).
+// Host-side validation and dispatch only; all arithmetic of the path runs in
+// the kernels of bl_quant.cu, bl_gemv.cu and bl_gemm.cu.
+#include "bitlinear.h"
+#include "bl_internal.h"
+
+#include <mutex>
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+// Number of SMs of the current device (cached per device id).
+int num_sms_current(int* out_dev = nullptr) {
+  static int cache[64];
+  static std::once_flag once;
+  std::call_once(once, [] {
+    for (int i = 0; i < 64; ++i) cache[i] = 0;
+  });
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  if (out_dev) *out_dev = dev;
+  if (cache[dev] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+int check_k(int64_t K) {
+  if (K <= 0 || K > bl::kMaxK || (K % 16) != 0) return BL_ERR_SHAPE;
+  return BL_OK;
+}
+
+int check_mn(int64_t M, int64_t N) {
+  if (M < 0 || N < 0 || M > 0x7FFFFFFF || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  return BL_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? BL_OK : BL_ERR_CUDA; }
+
+int forward_impl(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D,
+                 float* y, int32_t* acc, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  st = check_mn(M, N);
+  if (st != BL_OK) return st;
+  if (M == 0 || N == 0) return BL_OK;
+  if (x == nullptr || packed == nullptr || ws == nullptr || (y == nullptr && acc == nullptr) ||
+      (y != nullptr && D == nullptr))
+    return BL_ERR_NULL;
+  if (!aligned16(x) || !aligned16(packed) || (y && !aligned16(y)) || (acc && !aligned16(acc)) ||
+      (D && !aligned16(D)) || !aligned256(ws))
+    return BL_ERR_ALIGN;
+  if (ws_bytes < bitlinear_workspace_size(M, N, K)) return BL_ERR_WORKSPACE;
+  const int sms = num_sms_current();
+  if (sms <= 0) return BL_ERR_CUDA;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* err = reinterpret_cast<uint32_t*>(base);
+  if (bl::gemv_eligible(M, K))
+    return cuda_status(bl::launch_gemv(x, M, N, K, packed, D, y, acc, err, stream, sms));
+  cudaError_t e = bl::launch_act_quant(x, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
+                                       reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
+                                       reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), true, stream, err);
+  if (e != cudaSuccess) return BL_ERR_CUDA;
+  return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, acc, ws, stream, sms));
+}
+
+}  // namespace
+
+extern "C" {
+
+int bitlinear_abi_version(void) { return kAbiVersion; }
+
+const char* bitlinear_status_string(int status) {
+  switch (status) {
+    case BL_OK: return "ok";
+    case BL_ERR_NULL: return "null pointer";
+    case BL_ERR_SHAPE: return "bad shape (need 0 < K <= 131072, K % 16 == 0, 0 <= M, N < 2^31)";
+    case BL_ERR_ALIGN: return "misaligned pointer (device buffers 16 B, workspace 256 B)";
+    case BL_ERR_WORKSPACE: return "workspace too small";
+    case BL_ERR_NONFINITE: return "weights hold Inf or NaN";
+    case BL_ERR_DEVICE: return "device-side failure recorded (bounded wait expired)";
+    case BL_ERR_CUDA: return "CUDA runtime error";
+    case BL_ERR_UNSUPPORTED: return "device is not sm_100 (B200 class)";
+    default: return "unknown status";
+  }
+}
+
+int bitlinear_device_check(void) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BL_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return BL_ERR_CUDA;
+  return (major == 10 && minor == 0) ? BL_OK : BL_ERR_UNSUPPORTED;
+}
+
+size_t bitlinear_pack_workspace_size(int64_t N, int64_t K) {
+  (void)N;
+  (void)K;
+  return bl::kPackWsBytes;
+}
+
+int bitlinear_pack_weights(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
+                           size_t ws_bytes, bl_stream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  if (N <= 0 || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  if (W == nullptr || packed == nullptr || D == nullptr || ws == nullptr) return BL_ERR_NULL;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(D) || !aligned256(ws)) return BL_ERR_ALIGN;
+  if (ws_bytes < bl::kPackWsBytes) return BL_ERR_WORKSPACE;
+  const int sms = num_sms_current();
+  if (sms <= 0) return BL_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (bl::launch_pack(W, N, K, packed, D, ws, s, sms) != cudaSuccess) return BL_ERR_CUDA;
+  uint32_t status = 0;
+  if (cudaMemcpyAsync(&status, ws, sizeof(status), cudaMemcpyDeviceToHost, s) != cudaSuccess) return BL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
+  return status == 0u ? BL_OK : BL_ERR_NONFINITE;
+}
+
+int bitlinear_quant_act(const float* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
+                        bl_stream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  if (M < 0 || M > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  if (M == 0) return BL_OK;
+  if (x == nullptr || q == nullptr || s_x == nullptr) return BL_ERR_NULL;
+  if (!aligned16(x) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s_x) & 3u) ||
+      (rowsum && (reinterpret_cast<uintptr_t>(rowsum) & 3u)))
+    return BL_ERR_ALIGN;
+  return cuda_status(
+      bl::launch_act_quant(x, M, K, q, s_x, rowsum, false, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
+size_t bitlinear_workspace_size(int64_t M, int64_t N, int64_t K) {
+  (void)N;
+  if (M < 0 || K < 0) return 0;
+  return bl::ws_forward_bytes(M, K);
+}
+
+int bitlinear_forward(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D,
+                      float* y, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  if (y == nullptr && M > 0 && N > 0) return BL_ERR_NULL;
+  return forward_impl(x, M, N, K, packed, D, y, nullptr, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_forward_acc(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed, int32_t* acc,
+                          void* ws, size_t ws_bytes, bl_stream_t stream) {
+  if (acc == nullptr && M > 0 && N > 0) return BL_ERR_NULL;
+  return forward_impl(x, M, N, K, packed, nullptr, nullptr, acc, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_prepare_act(const float* x, int64_t M, int64_t K, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  if (M < 0 || M > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  if (M == 0) return BL_OK;
+  if (x == nullptr || ws == nullptr) return BL_ERR_NULL;
+  if (!aligned16(x) || !aligned256(ws)) return BL_ERR_ALIGN;
+  if (ws_bytes < bl::ws_forward_bytes(M, K)) return BL_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  return cuda_status(bl::launch_act_quant(x, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
+                                          reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
+                                          reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), true,
+                                          reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<uint32_t*>(base)));
+}
+
+int bitlinear_forward_prepared(int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D, float* y,
+                               void* ws, size_t ws_bytes, bl_stream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  st = check_mn(M, N);
+  if (st != BL_OK) return st;
+  if (M == 0 || N == 0) return BL_OK;
+  if (packed == nullptr || D == nullptr || y == nullptr || ws == nullptr) return BL_ERR_NULL;
+  if (!aligned16(packed) || !aligned16(D) || !aligned16(y) || !aligned256(ws)) return BL_ERR_ALIGN;
+  if (ws_bytes < bl::ws_forward_bytes(M, K)) return BL_ERR_WORKSPACE;
+  const int sms = num_sms_current();
+  if (sms <= 0) return BL_ERR_CUDA;
+  return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, nullptr, ws, reinterpret_cast<cudaStream_t>(stream), sms));
+}
+
+size_t bitlinear_host_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return 0;
+  return bl::ws_forward_bytes(M, K) + bl::align256(4 * (size_t)M * (size_t)K) +
+         bl::align256(4 * (size_t)M * (size_t)N);
+}
+
+int bitlinear_forward_host(const float* x_host, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                           const float* D, float* y_host, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  st = check_mn(M, N);
+  if (st != BL_OK) return st;
+  if (M == 0 || N == 0) return BL_OK;
+  if (x_host == nullptr || y_host == nullptr || ws == nullptr) return BL_ERR_NULL;
+  if (!aligned256(ws)) return BL_ERR_ALIGN;
+  if (ws_bytes < bitlinear_host_workspace_size(M, N, K)) return BL_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const size_t fw = bl::ws_forward_bytes(M, K);
+  float* xd = reinterpret_cast<float*>(base + fw);
+  float* yd = reinterpret_cast<float*>(base + fw + bl::align256(4 * (size_t)M * (size_t)K));
+  if (cudaMemcpyAsync(xd, x_host, 4 * (size_t)M * (size_t)K, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return BL_ERR_CUDA;
+  st = forward_impl(xd, M, N, K, packed, D, yd, nullptr, ws, fw, s);
+  if (st != BL_OK) return st;
+  if (cudaMemcpyAsync(y_host, yd, 4 * (size_t)M * (size_t)N, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return BL_ERR_CUDA;
+  return cudaStreamSynchronize(s) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+int bitlinear_workspace_error(void* ws, size_t ws_bytes, bl_stream_t stream) {
+  if (ws == nullptr) return BL_ERR_NULL;
+  if (ws_bytes < bl::kHeaderBytes) return BL_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t word = 0;
+  if (cudaMemcpyAsync(&word, ws, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess) return BL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
+  if (word == 0u) return BL_OK;
+  if (cudaMemsetAsync(ws, 0, sizeof(word), s) != cudaSuccess) return BL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
+  return BL_ERR_DEVICE;
+}
+
+}  // extern "C"

@@ -1,0 +1,288 @@
+// bl_quant.cu - WeightQuant + 2-bit pack and per-token ActQuant kernels.
+//
+// WeightQuant ("Core AI model zoo - BitVLA", section 1; "BitNet-Embeddings
+// I2_S guide", section 3.3): s = 1/mean(|W|), code = round(W*s).clamp(-1,1),
+// stored as code+1, 16 codes per 32-bit word (BitVLA page, section 2).
+// ActQuant (BitVLA page, section 1): per token, round(x*127/max|x|)
+// clamped to int8.
+//
+// The mean of |W| must be identical however the reduction is ordered, so it is
+// an exact integer sum: every |w| = m * 2^(max(e,1)-150), and the 24-bit
+// significands m are summed per biased exponent e in 64-bit integers (exact
+// and order independent). A single thread then forms the exact total and
+// divides it by N*K with one correct rounding to fp32.
+#include "bl_internal.h"
+
+namespace bl {
+
+// ------------------------------------------------------------------ pack --
+constexpr int kBinThreads = 256;
+constexpr int kBinWarps = kBinThreads / 32;
+
+__global__ void __launch_bounds__(kBinThreads) absum_bins_kernel(const float4* __restrict__ W, int64_t n4,
+                                                                  unsigned long long* __restrict__ bins) {
+  __shared__ unsigned long long sbins[kBinWarps][256];
+  const int warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kBinWarps * 256; i += blockDim.x) (&sbins[0][0])[i] = 0ull;
+  __syncthreads();
+  unsigned long long* my = sbins[warp];
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = __ldg(W + i);
+    const float vals[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t b = __float_as_uint(vals[j]) & 0x7FFFFFFFu;
+      const uint32_t e = b >> 23;
+      uint32_t m = b & 0x7FFFFFu;
+      if (e != 0) m |= 0x800000u;
+      if (m != 0 || e == 255) atomicAdd(&my[e], (unsigned long long)(m | (e == 255 ? 1u : 0u)));
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+    unsigned long long s = 0;
+#pragma unroll
+    for (int w = 0; w < kBinWarps; ++w) s += sbins[w][e];
+    if (s) atomicAdd(&bins[e], s);
+  }
+}
+
+// Correctly rounded fp32 of S * 2^-149 / n, where S = sum_e bins[e] * 2^(max(e,1)-1).
+// Results below the normal range are returned as 0 (they lie far below the
+// 1e-5 floor that is applied afterwards). One thread.
+__global__ void absmean_finalize_kernel(const unsigned long long* __restrict__ bins, uint64_t n,
+                                        float* __restrict__ scal, uint32_t* __restrict__ status) {
+  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  if (bins[255] != 0ull) {
+    *status = 1u;  // non-finite input
+    scal[0] = __int_as_float(0x7FC00000);
+    scal[1] = __int_as_float(0x7FC00000);
+    return;
+  }
+  // S as 11 little-endian 32-bit limbs (bins < 2^50, shifts < 254: < 2^304).
+  constexpr int L = 11;
+  uint32_t S[L];
+#pragma unroll
+  for (int i = 0; i < L; ++i) S[i] = 0u;
+  for (int e = 0; e < 255; ++e) {
+    const unsigned long long v = bins[e];
+    if (v == 0ull) continue;
+    const int sh = (e > 1 ? e : 1) - 1;
+    const int limb = sh >> 5, bit = sh & 31;
+    // v << bit spans up to three limbs.
+    const uint32_t p0 = (uint32_t)(v << bit);
+    const uint32_t p1 = (uint32_t)((v >> (32 - bit)) >> 0);
+    uint32_t parts[3];
+    parts[0] = p0;
+    if (bit == 0) {
+      parts[1] = (uint32_t)(v >> 32);
+      parts[2] = 0u;
+    } else {
+      parts[1] = (uint32_t)(v >> (32 - bit));
+      parts[2] = (uint32_t)((v >> 32) >> (32 - bit));
+    }
+    (void)p1;
+    unsigned long long carry = 0ull;
+    for (int i = limb; i < L; ++i) {
+      const unsigned long long add = (i - limb < 3 ? parts[i - limb] : 0u);
+      const unsigned long long t = (unsigned long long)S[i] + add + carry;
+      S[i] = (uint32_t)t;
+      carry = t >> 32;
+      if (i - limb >= 2 && carry == 0ull) break;
+    }
+  }
+  // Long division of S * 2^F by n, one quotient bit at a time (MSB first).
+  constexpr int F = 32;
+  const int nbits = 32 * L + F;
+  unsigned long long rem = 0ull;
+  int lead = -1;        // bit index of the leading 1 of the quotient
+  uint32_t sig = 0u;    // leading 24 bits of the quotient
+  int taken = 0;        // bits collected into sig
+  uint32_t round_bit = 0u, sticky = 0u;
+  for (int i = nbits - 1; i >= 0; --i) {
+    uint32_t bit = 0u;
+    if (i >= F) {
+      const int j = i - F;
+      bit = (S[j >> 5] >> (j & 31)) & 1u;
+    }
+    rem = (rem << 1) | bit;
+    uint32_t qb = 0u;
+    if (rem >= n) {
+      rem -= n;
+      qb = 1u;
+    }
+    if (lead < 0) {
+      if (qb) {
+        lead = i;
+        sig = 1u;
+        taken = 1;
+      }
+    } else if (taken < 24) {
+      sig = (sig << 1) | qb;
+      ++taken;
+    } else if (taken == 24) {
+      round_bit = qb;
+      ++taken;
+    } else {
+      sticky |= qb;
+    }
+  }
+  sticky |= (rem != 0ull) ? 1u : 0u;
+  float mean = 0.0f;
+  if (lead >= 0 && taken >= 25) {
+    int E = lead - 149 - F;  // value = 1.xxx * 2^E
+    if (round_bit && (sticky || (sig & 1u))) {
+      ++sig;
+      if (sig == (1u << 24)) {
+        sig >>= 1;
+        ++E;
+      }
+    }
+    if (E >= -126 && E <= 127) mean = __uint_as_float(((uint32_t)(E + 127) << 23) | (sig & 0x7FFFFFu));
+  }
+  const float mean_c = fmaxf(mean, kFloor);
+  scal[0] = mean_c;
+  scal[1] = __fdiv_rn(1.0f, mean_c);
+  *status = 0u;
+}
+
+// Each thread ternarises one float4 (4 codes = one byte of a packed word);
+// lanes 4j..4j+3 of a warp hold the four bytes of one word and combine them
+// with shuffles. Also writes D[n] = mean_c.
+__global__ void __launch_bounds__(256) ternarize_pack_kernel(const float4* __restrict__ W, int64_t n4,
+                                                             const float* __restrict__ scal,
+                                                             const uint32_t* __restrict__ status,
+                                                             uint32_t* __restrict__ packed, float* __restrict__ D,
+                                                             int64_t N) {
+  if (*status != 0u) return;
+  const float mean_c = scal[0];
+  const float s = scal[1];
+  const int lane = threadIdx.x & 31;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  // Loop bound is warp-uniform so every lane reaches the shuffles.
+  const int64_t warp_base0 = (blockIdx.x * (int64_t)blockDim.x + (threadIdx.x & ~31));
+  for (int64_t base = warp_base0; base < n4; base += stride) {
+    const int64_t i = base + lane;
+    uint32_t byte = 0u;
+    if (i < n4) {
+      const float4 v = __ldg(W + i);
+      byte = code_plus_one(v.x, s) | (code_plus_one(v.y, s) << 2) | (code_plus_one(v.z, s) << 4) |
+             (code_plus_one(v.w, s) << 6);
+    }
+    uint32_t word = byte << (8 * (lane & 3));
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+    if ((lane & 3) == 0 && i < n4) packed[i >> 2] = word;
+  }
+  for (int64_t n = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; n < N; n += stride) D[n] = mean_c;
+}
+
+// -------------------------------------------------------------- ActQuant --
+// One CTA per token row. Pass 1: max|x| (exact). Pass 2: quantise 16 columns
+// per thread-iteration and store them as one 16-byte vector, in natural
+// column order or in the kernel-private order perm16 (see bl_device.cuh).
+template <bool kPerm>
+__global__ void __launch_bounds__(256) act_quant_kernel(const float* __restrict__ x, int64_t K,
+                                                        int8_t* __restrict__ q, float* __restrict__ s_out,
+                                                        int32_t* __restrict__ rowsum_out,
+                                                        uint32_t* __restrict__ err_reset) {
+  if (err_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err_reset = 0u;
+  __shared__ float red_f[8];
+  __shared__ int red_i[8];
+  const int64_t m = blockIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(x + m * K);
+  const int ngroups = (int)(K >> 4);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+
+  float amax = 0.0f;
+  for (int g = threadIdx.x; g < ngroups; g += blockDim.x) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 v = __ldg(xr + 4 * g + j);
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if (lane == 0) red_f[warp] = amax;
+  __syncthreads();
+  amax = 0.0f;
+  for (int w = 0; w < nwarps; ++w) amax = fmaxf(amax, red_f[w]);
+  const float sx = __fdiv_rn(kQmax, fmaxf(amax, kFloor));
+
+  int rsum = 0;
+  int8_t* qr = q + m * K;
+  for (int g = threadIdx.x; g < ngroups; g += blockDim.x) {
+    int v[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 f = __ldg(xr + 4 * g + j);
+      v[4 * j + 0] = quant_i8(f.x, sx);
+      v[4 * j + 1] = quant_i8(f.y, sx);
+      v[4 * j + 2] = quant_i8(f.z, sx);
+      v[4 * j + 3] = quant_i8(f.w, sx);
+    }
+    uint32_t w4[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      uint32_t word = 0u;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int p = 4 * r + b;
+        const int src = kPerm ? perm16(p) : p;
+        word |= (uint32_t)(v[src] & 0xFF) << (8 * b);
+      }
+      w4[r] = word;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) rsum += v[j];
+    *reinterpret_cast<uint4*>(qr + 16 * (int64_t)g) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) rsum += __shfl_xor_sync(0xFFFFFFFFu, rsum, o);
+  if (lane == 0) red_i[warp] = rsum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int w = 0; w < nwarps; ++w) t += red_i[w];
+    s_out[m] = sx;
+    if (rowsum_out != nullptr) rowsum_out[m] = t;
+  }
+}
+
+// ------------------------------------------------------------ launchers --
+cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
+                        cudaStream_t stream, int num_sms) {
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  float* scal = reinterpret_cast<float*>(base + 16);
+  unsigned long long* bins = reinterpret_cast<unsigned long long*>(base + kHeaderBytes);
+  cudaError_t err = cudaMemsetAsync(base, 0, kPackWsBytes, stream);
+  if (err != cudaSuccess) return err;
+  const int64_t n4 = N * K / 4;
+  const int64_t want = (n4 + kBinThreads * 8 - 1) / (kBinThreads * 8);
+  const int grid1 = (int)(want < 4 * num_sms ? (want < 1 ? 1 : want) : 4 * num_sms);
+  absum_bins_kernel<<<grid1, kBinThreads, 0, stream>>>(reinterpret_cast<const float4*>(W), n4, bins);
+  absmean_finalize_kernel<<<1, 32, 0, stream>>>(bins, (uint64_t)(N * K), scal, status);
+  const int64_t want2 = (n4 + 255) / 256;
+  const int grid2 = (int)(want2 < 16 * num_sms ? (want2 < 1 ? 1 : want2) : 16 * num_sms);
+  ternarize_pack_kernel<<<grid2, 256, 0, stream>>>(reinterpret_cast<const float4*>(W), n4, scal, status, packed,
+                                                    D, N);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_act_quant(const float* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
+                             bool permuted, cudaStream_t stream, uint32_t* err_reset) {
+  const int64_t ngroups = K / 16;
+  int threads = (int)(ngroups < 256 ? ((ngroups + 31) / 32) * 32 : 256);
+  if (threads < 32) threads = 32;
+  // One CTA per token; grids beyond 2^31-1 are rejected by validation.
+  if (permuted)
+    act_quant_kernel<true><<<(unsigned)M, threads, 0, stream>>>(x, K, q, s_x, rowsum, err_reset);
+  else
+    act_quant_kernel<false><<<(unsigned)M, threads, 0, stream>>>(x, K, q, s_x, rowsum, err_reset);
+  return cudaGetLastError();
+}
+
+}  // namespace bl

@@ -1,0 +1,180 @@
+/*
+ * bitlinear.h - C ABI of libbitlinear, the B200 (sm_100a) BitNet b1.58
+ * BitLinear (W1.58-A8) hot path:  y = F.linear(ActQuant(x), WeightQuant(W)).
+ *
+ * Definitions followed (page title, section):
+ *   WeightQuant  "Core AI model zoo - BitVLA", section 1: per-tensor absmean,
+ *                s = 1/mean(|W|), code = round(W*s).clamp(-1, 1); also
+ *                "BitNet-Embeddings I2_S guide", section 3.3 (I2_S packing).
+ *   ActQuant     BitVLA page, section 1: per-token int8 absmax,
+ *                q = round(x*127/max|x|).clamp(-128, 127).
+ *   Storage      BitVLA page, section 2: codes stored as code+1, 16 codes per
+ *                32-bit word, K only needs K % 16 == 0, N need not be a
+ *                multiple of 32, and the scale D is one fp32 per output row,
+ *                laid out [N, 1].
+ *   Product      BitVLA page, section 2: the wrapper applies ActQuant before
+ *                the kernel, so the result equals
+ *                F.linear(ActQuant(x), WeightQuant(W)).
+ *
+ * Numerics (identical to the CPU oracle, bit for bit):
+ *   mean  = mean(|W|) over the whole tensor, exact sum, correctly rounded
+ *           to fp32; mean_c = max(mean, 1e-5);  s = RN(1 / mean_c)
+ *   code  = clamp(rint(RN(W * s)), -1, 1)      (rint: half to even)
+ *   packed word n*(K/16) + k/16, bits [2*(k%16), 2*(k%16)+2) = code + 1
+ *   D[n]  = mean_c for every row n
+ *   s_x   = RN(127 / max(max_k |x[m,k]|, 1e-5))
+ *   q     = clamp(rint(RN(x * s_x)), -128, 127)
+ *   acc   = sum_k q[m,k] * code[n,k]          (exact int32)
+ *   y     = RN( RN(float(acc) / s_x[m]) * D[n] )
+ *
+ * Conventions for every entry point:
+ *   - All pointers named "device" are device pointers on the current CUDA
+ *     device; the caller owns every buffer (this library allocates nothing and
+ *     keeps no state beyond cached device attributes).
+ *   - Matrices are dense row-major with no padding: x [M,K] fp32, W [N,K] fp32,
+ *     packed [N, K/16] uint32, D [N] fp32 (a torch [N,1] tensor), y [M,N] fp32.
+ *   - Device buffers must be 16-byte aligned, the workspace 256-byte aligned.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream). Entry points marked "synchronous" synchronise that stream.
+ *   - No exception crosses this boundary and no kernel traps; every error is a
+ *     returned bl_status. Kernels that wait on barriers give up after a bounded
+ *     time and record the failure in the workspace (see
+ *     bitlinear_workspace_error).
+ *   - Limits: 0 < K <= 131072 and K % 16 == 0 (so |acc| < 2^24 and fp32
+ *     holds it exactly); 0 <= M, N <= 2^31 - 1. M == 0 or N == 0 is a no-op.
+ */
+#ifndef BITLINEAR_H_
+#define BITLINEAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BL_API __attribute__((visibility("default")))
+#else
+#define BL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared here so the header needs no CUDA headers. */
+typedef struct CUstream_st* bl_stream_t;
+
+typedef enum {
+  BL_OK = 0,
+  BL_ERR_NULL = 1,        /* a required pointer is NULL */
+  BL_ERR_SHAPE = 2,       /* K % 16 != 0, K <= 0, K > 131072, or M/N out of range */
+  BL_ERR_ALIGN = 3,       /* a device pointer is not 16-byte aligned (workspace: 256) */
+  BL_ERR_WORKSPACE = 4,   /* ws_bytes smaller than the *_workspace_size query */
+  BL_ERR_NONFINITE = 5,   /* pack: W holds Inf or NaN, so mean(|W|) is not finite */
+  BL_ERR_DEVICE = 6,      /* a kernel recorded a device-side failure (bounded wait expired) */
+  BL_ERR_CUDA = 7,        /* a CUDA runtime call failed (launch, copy, attribute) */
+  BL_ERR_UNSUPPORTED = 8  /* the current device is not sm_100 (B200 class) */
+} bl_status;
+
+/* Version of this ABI (incremented on any incompatible change). */
+BL_API int bitlinear_abi_version(void);
+
+/* Static string for a status code; never NULL. */
+BL_API const char* bitlinear_status_string(int status);
+
+/* BL_OK if the current device can run the kernels (compute capability 10.0). */
+BL_API int bitlinear_device_check(void);
+
+/* ---------------------------------------------------------------- pack --- */
+
+/* Bytes of scratch that bitlinear_pack_weights needs (a few KB). */
+BL_API size_t bitlinear_pack_workspace_size(int64_t N, int64_t K);
+
+/* WeightQuant + 2-bit pack (BitVLA page sections 1 and 2; I2_S guide 3.3).
+ *   W       device fp32 [N, K], read only.
+ *   packed  device uint32 [N, K/16], fully overwritten.
+ *   D       device fp32 [N] (the [N,1] scale), every entry set to mean_c.
+ *   ws      device scratch of ws_bytes >= bitlinear_pack_workspace_size().
+ * Synchronous: it waits on `stream` so that it can report BL_ERR_NONFINITE
+ * (packed and D are left unwritten in that case). N >= 1 is required. */
+BL_API int bitlinear_pack_weights(const float* W, int64_t N, int64_t K,
+                           uint32_t* packed, float* D,
+                           void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* ------------------------------------------------------------ ActQuant --- */
+
+/* Per-token int8 absmax quantisation (BitVLA page section 1).
+ *   x       device fp32 [M, K].
+ *   q       device int8 [M, K], natural column order.
+ *   s_x     device fp32 [M]: the scale 127/max|x| (not its reciprocal).
+ *   rowsum  device int32 [M] or NULL: sum_k q[m,k] (exact).
+ * Asynchronous. */
+BL_API int bitlinear_quant_act(const float* x, int64_t M, int64_t K,
+                        int8_t* q, float* s_x, int32_t* rowsum,
+                        bl_stream_t stream);
+
+/* ------------------------------------------------------------- forward --- */
+
+/* Bytes of scratch that bitlinear_forward / bitlinear_forward_acc need:
+ * the quantised activations (M*K bytes, in a kernel-private column order),
+ * s_x and row sums (4*M bytes each) and a 256-byte header holding the
+ * device error word. */
+BL_API size_t bitlinear_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* y = F.linear(ActQuant(x), WeightQuant(W)) from packed weights (BitVLA page
+ * section 2: the wrapper applies ActQuant, then the ternary kernel).
+ *   x       device fp32 [M, K].
+ *   packed  device uint32 [N, K/16] from bitlinear_pack_weights.
+ *   D       device fp32 [N] per-row scale.
+ *   y       device fp32 [M, N], fully overwritten; nothing outside it is written.
+ *   ws      device scratch, ws_bytes >= bitlinear_workspace_size(M, N, K).
+ * M <= 16 runs a fused quantise + GEMV kernel that streams the packed weights
+ * once; larger M quantises into ws and runs the tcgen05 tensor-core GEMM.
+ * Asynchronous. */
+BL_API int bitlinear_forward(const float* x, int64_t M, int64_t N, int64_t K,
+                      const uint32_t* packed, const float* D, float* y,
+                      void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* As bitlinear_forward, but writes the exact int32 accumulators
+ * acc[m,n] = sum_k q[m,k] * code[n,k] to device int32 [M, N] instead of y. */
+BL_API int bitlinear_forward_acc(const float* x, int64_t M, int64_t N, int64_t K,
+                          const uint32_t* packed, int32_t* acc,
+                          void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* Two-phase form of bitlinear_forward for projections that share one input
+ * (q/k/v, or gate/up): quantise x once, then contract with several weights.
+ * bitlinear_prepare_act writes the int8 codes (kernel-private column order),
+ * s_x and row sums of x [M,K] into ws (ws_bytes >=
+ * bitlinear_workspace_size(M, N, K) for any N). Asynchronous. */
+BL_API int bitlinear_prepare_act(const float* x, int64_t M, int64_t K,
+                                 void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* Contraction + rescale from a workspace filled by bitlinear_prepare_act with
+ * the same M and K: y [M,N] = RN(RN(acc/s_x) * D). Runs the tcgen05
+ * tensor-core kernel for every M (the fused GEMV of bitlinear_forward
+ * quantises x itself). The workspace is only read (and its error word reset),
+ * so several calls may follow one prepare. Asynchronous. */
+BL_API int bitlinear_forward_prepared(int64_t M, int64_t N, int64_t K,
+                                      const uint32_t* packed, const float* D, float* y,
+                                      void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* Scratch for bitlinear_forward_host: the forward workspace plus room for x
+ * and y on the device. */
+BL_API size_t bitlinear_host_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* End-to-end call with HOST activations: copies x_host (fp32 [M,K], pinned
+ * memory recommended) to the device, runs bitlinear_forward, copies y back to
+ * y_host (fp32 [M,N]) and synchronises `stream`. packed and D are device
+ * buffers (the weights stay resident). Synchronous. */
+BL_API int bitlinear_forward_host(const float* x_host, int64_t M, int64_t N, int64_t K,
+                           const uint32_t* packed, const float* D, float* y_host,
+                           void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word in a
+ * forward workspace. BL_OK if no kernel recorded a failure, else
+ * BL_ERR_DEVICE. */
+BL_API int bitlinear_workspace_error(void* ws, size_t ws_bytes, bl_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H_ */

@@ -1,0 +1,96 @@
+"""CPU-side checks of the C ABI: the library builds/loads, exports every symbol
+include/bitlinear.h declares, and host-side validation rejects bad arguments
+before any CUDA work (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_ternary_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build_library()
+    return _lib.lib()
+
+
+def declared_symbols():
+    with open(os.path.join(ROOT, "include", "bitlinear.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"BL_API\s+[\w\s\*]*?\b(bitlinear_\w+)\s*\(", text)))
+
+
+def test_header_declares_entry_points():
+    names = declared_symbols()
+    for must in ("bitlinear_pack_weights", "bitlinear_quant_act", "bitlinear_forward"):
+        assert must in names
+    assert set(names) == set(_lib.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.bitlinear_abi_version() == 1
+    for st in range(0, 9):
+        s = L.bitlinear_status_string(st)
+        assert s and isinstance(s, bytes)
+    assert L.bitlinear_status_string(99) == b"unknown status"
+
+
+def test_workspace_queries(L):
+    assert L.bitlinear_pack_workspace_size(10, 32) >= 256 + 2048
+    ws = L.bitlinear_workspace_size(4096, 13824, 2560)
+    assert ws >= 4096 * 2560 + 8 * 4096
+    assert ws % 256 == 0
+    assert L.bitlinear_host_workspace_size(4096, 13824, 2560) >= ws + 4 * 4096 * (2560 + 13824)
+    assert L.bitlinear_workspace_size(0, 5, 16) == 256
+
+
+FAKE = 0x10000  # never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("K", [0, -16, 8, 24, 131072 + 16])
+def test_bad_k_rejected_before_cuda(L, K):
+    assert L.bitlinear_forward(FAKE, 1, 1, K, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 2
+    assert L.bitlinear_quant_act(FAKE, 1, K, FAKE, FAKE, None, None) == 2
+    assert L.bitlinear_pack_weights(FAKE, 1, K, FAKE, FAKE, FAKE, 4096, None) == 2
+
+
+def test_empty_is_noop(L):
+    assert L.bitlinear_forward(None, 0, 5, 16, None, None, None, None, 0, None) == 0
+    assert L.bitlinear_forward(None, 3, 0, 16, None, None, None, None, 0, None) == 0
+    assert L.bitlinear_quant_act(None, 0, 16, None, None, None, None) == 0
+
+
+def test_null_and_alignment_rejected(L):
+    assert L.bitlinear_forward(None, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.bitlinear_forward(FAKE + 4, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 3
+    assert L.bitlinear_forward(FAKE, 1, 1, 16, FAKE, FAKE, FAKE, FAKE + 16, 1 << 20, None) == 3
+    assert L.bitlinear_forward(FAKE, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, 10, None) == 4
+    assert L.bitlinear_pack_weights(FAKE, 0, 16, FAKE, FAKE, FAKE, 4096, None) == 2
+    assert L.bitlinear_pack_weights(FAKE, 4, 16, FAKE, FAKE, FAKE, 16, None) == 4
+    assert L.bitlinear_forward_acc(FAKE, 1, 1, 16, FAKE, None, FAKE, 1 << 20, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(_lib, "_lib", None)
+    monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        _lib.lib()
+
+
+def test_product_path_does_not_import_oracle():
+    pkg = os.path.join(ROOT, "bit_ternary_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for fn in files:
+            if fn.endswith((".py", ".cu", ".cuh", ".h")):
+                with open(os.path.join(dirpath, fn)) as f:
+                    src = f.read()
+                assert "import oracle" not in src and "from oracle" not in src, fn

@@ -1,0 +1,290 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Bar (numerics of the BitVLA page, sections 1-2, with the readings in the
+oracle's header): packed codes, D, int8 activation codes, s_x, row sums and
+int32 accumulators are bit-exact; fp32 outputs are within 1e-6 relative of the
+oracle (the kernels use the same two correctly rounded steps, so they are
+expected to match bit for bit, and that is asserted too where noted).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle as O
+from bit_ternary_b200 import workloads as WL
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 1e-6
+
+
+@pytest.fixture(scope="module")
+def B():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_ternary_b200 import build, bitlinear, _lib
+
+    build.build_library()
+    assert _lib.lib().bitlinear_device_check() == 0, "device is not sm_100"
+    return bitlinear
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def assert_y_close(y_gpu, y_ref, bitexact=True):
+    y_gpu = np.asarray(y_gpu, np.float32)
+    assert y_gpu.shape == y_ref.shape
+    assert np.all(np.isfinite(y_gpu))
+    den = np.maximum(np.abs(y_ref), np.float32(np.finfo(np.float32).tiny))
+    rel = np.abs(y_gpu.astype(np.float64) - y_ref.astype(np.float64)) / den
+    assert rel.max(initial=0.0) <= REL_TOL
+    if bitexact:
+        assert np.array_equal(y_gpu.view(np.uint32), y_ref.view(np.uint32))
+
+
+# ------------------------------------------------------------ golden example
+def test_golden_hand_example_gpu(B, golden_dir):
+    with open(os.path.join(golden_dir, "hand_4x16.json")) as f:
+        g = json.load(f)
+    W = np.array(g["W"], np.float32)
+    x = np.array(g["x"], np.float32)
+    packed, D = B.pack_weights(dev(W))
+    assert [hex(int(v) & 0xFFFFFFFF) for v in packed.cpu().numpy()[:, 0]] == g["packed_hex"]
+    assert np.all(D.cpu().numpy() == np.float32(g["mean"]))
+    q, s_x, rs = B.quant_act(dev(x))
+    assert np.array_equal(q.cpu().numpy(), np.array(g["q"], np.int8))
+    assert np.array_equal(s_x.cpu().numpy(), np.array(g["s_x"], np.float32))
+    acc = B.forward_acc(dev(x), packed).cpu().numpy()
+    assert np.array_equal(acc, np.array(g["acc"]))
+    y = B.forward(dev(x), packed, D).cpu().numpy()
+    assert [[hex(int(v)) for v in row] for row in y.view(np.uint32)] == g["y_hex"]
+
+
+# ------------------------------------------------------------------- pack
+PACK_SHAPES = [(1, 16), (3, 48), (17, 496), (31, 528), (33, 1152), (64, 4304), (257, 6912), (2560, 2560)]
+
+
+@pytest.mark.parametrize("N,K", PACK_SHAPES)
+@pytest.mark.parametrize("dist", ["normal", "laplace"])
+def test_pack_bitexact(B, N, K, dist):
+    W = WL.weight(N, K, dist, 7000 + N + K)
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)
+    assert np.array_equal(D.cpu().numpy(), D_ref)
+
+
+def test_pack_full_gate_up_shape(B):
+    """Largest weight of the decode layer set (13824 x 2560 = 35.4M weights)."""
+    W = WL.weight(13824, 2560, "normal", 1001, layer=2)
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)
+    assert np.array_equal(D.cpu().numpy(), D_ref)
+
+
+def test_pack_special_values(B):
+    W = WL.weight(8, 64, "normal", 3)
+    W[0, :5] = [0.0, -0.0, 1e-45, -1e-42, 3.4e38]  # zeros, subnormals, huge
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)
+    assert np.array_equal(D.cpu().numpy(), D_ref)
+
+
+def test_pack_all_zero_uses_floor(B):
+    W = np.zeros((4, 32), np.float32)
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)
+    assert np.all(D.cpu().numpy() == np.float32(1e-5))
+
+
+def test_pack_nonfinite_rejected(B):
+    from bit_ternary_b200._lib import BitLinearError
+
+    W = np.ones((4, 32), np.float32)
+    W[2, 7] = np.nan
+    with pytest.raises(BitLinearError, match="NONFINITE"):
+        B.pack_weights(dev(W))
+
+
+# --------------------------------------------------------------- ActQuant
+@pytest.mark.parametrize("M,K", [(1, 16), (3, 2560), (17, 1152), (64, 6912), (5, 4304)])
+def test_quant_act_bitexact(B, M, K):
+    x = WL.activations(M, K, "student_t", 77 + K, meta={"df": 3.0})
+    if M > 1:
+        x[-1] = 0.0  # all-zero token: floor path
+    q, s_x, rs = B.quant_act(dev(x))
+    q_ref, s_ref = O.act_quant(x)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s_x.cpu().numpy(), s_ref)
+    assert np.array_equal(rs.cpu().numpy(), q_ref.astype(np.int64).sum(axis=1))
+
+
+# ---------------------------------------------------------------- forward
+def run_case(B, M, N, K, wdist="normal", xdist="normal", seed=0):
+    W = WL.weight(N, K, wdist, seed)
+    x = WL.activations(M, K, xdist, seed, meta={"df": 3.0, "frac": 0.02, "scale": 20.0})
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    y_ref, parts = O.bitlinear_forward(x, p_ref, D_ref, K, return_parts=True)
+    xd = dev(x)
+    acc = B.forward_acc(xd, packed).cpu().numpy()
+    assert np.array_equal(acc, parts["acc"])
+    y = B.forward(xd, packed, D).cpu().numpy()
+    assert_y_close(y, y_ref)
+
+
+GEMV_CASES = [
+    (1, 1, 16), (1, 17, 48), (1, 31, 496), (1, 33, 528), (2, 64, 1152), (1, 2560, 2560),
+    (4, 100, 4304), (8, 4304, 1152), (9, 257, 6912), (16, 300, 2560), (1, 3840, 2560), (13, 65, 80),
+]
+
+
+@pytest.mark.parametrize("M,N,K", GEMV_CASES)
+def test_forward_gemv(B, M, N, K):
+    run_case(B, M, N, K, xdist="student_t", seed=M * 1000 + N + K)
+
+
+GEMM_CASES = [
+    (17, 16, 16), (17, 128, 128), (100, 129, 256), (256, 4304, 1152), (256, 1152, 4304),
+    (300, 700, 2560), (129, 33, 6912), (512, 384, 528), (1000, 257, 48), (640, 640, 640),
+]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_CASES)
+def test_forward_gemm(B, M, N, K):
+    run_case(B, M, N, K, wdist="laplace", xdist="outlier_channels", seed=M + N * 7 + K)
+
+
+def test_gemm_edge_zero_tokens_and_rows(B):
+    """All-zero token (floor path) and rows whose weights ternarise to 0."""
+    M, N, K = 40, 200, 512
+    W = WL.weight(N, K, "normal", 5)
+    W[3] = 1e-9  # ternarises to all zeros
+    x = WL.activations(M, K, "normal", 5)
+    x[7] = 0.0
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    y_ref = O.bitlinear_forward(x, p_ref, D_ref, K)
+    y = B.forward(dev(x), packed, D).cpu().numpy()
+    assert_y_close(y, y_ref)
+    assert np.all(y[7] == 0.0)
+
+
+def test_output_written_exactly(B):
+    """Every element of y is written, nothing past it (poisoned guard)."""
+    for (M, N, K) in [(1, 33, 64), (37, 131, 272)]:
+        W = WL.weight(N, K, "normal", 1)
+        x = WL.activations(M, K, "normal", 1)
+        packed, D = B.pack_weights(dev(W))
+        buf = torch.full((M * N + 4096,), float("nan"), device="cuda")
+        y = buf[: M * N].view(M, N)
+        B.forward(dev(x), packed, D, out=y)
+        torch.cuda.synchronize()
+        assert torch.isfinite(y).all()
+        assert torch.isnan(buf[M * N:]).all()
+
+
+def test_D_row_layout_enforced(B):
+    W = WL.weight(8, 32, "normal", 2)
+    packed, D = B.pack_weights(dev(W))
+    with pytest.raises(ValueError, match=r"\[N, 1\]"):
+        B.forward(dev(np.ones((1, 32), np.float32)), packed, D.reshape(1, -1))
+
+
+def test_forward_host_matches_device(B):
+    M, N, K = 3, 500, 1024
+    W = WL.weight(N, K, "normal", 9)
+    x = WL.activations(M, K, "normal", 9)
+    packed, D = B.pack_weights(dev(W))
+    y_dev = B.forward(dev(x), packed, D).cpu().numpy()
+    xh = torch.from_numpy(x).pin_memory()
+    y_host = B.forward_host(xh, packed, D).numpy()
+    assert np.array_equal(y_dev.view(np.uint32), y_host.view(np.uint32))
+    # and the tensor-core path
+    M = 300
+    x = WL.activations(M, K, "normal", 10)
+    y_dev = B.forward(dev(x), packed, D).cpu().numpy()
+    y_host = B.forward_host(torch.from_numpy(x).pin_memory(), packed, D).numpy()
+    assert np.array_equal(y_dev.view(np.uint32), y_host.view(np.uint32))
+
+
+def test_workspace_error_word_clear_after_gemm(B):
+    M, N, K = 200, 256, 512
+    W = WL.weight(N, K, "normal", 4)
+    x = WL.activations(M, K, "normal", 4)
+    packed, D = B.pack_weights(dev(W))
+    ws = torch.full((B.workspace_size(M, N, K),), 0x5A, dtype=torch.uint8, device="cuda")
+    B.forward(dev(x), packed, D, ws=ws)
+    assert B.workspace_error(ws) == 0
+
+
+def test_misaligned_and_small_workspace_rejected(B):
+    from bit_ternary_b200._lib import BitLinearError
+
+    M, N, K = 2, 64, 64
+    W = WL.weight(N, K, "normal", 4)
+    packed, D = B.pack_weights(dev(W))
+    x = torch.zeros(M * K + 1, device="cuda")[1:].view(M, K)  # 4-byte offset
+    with pytest.raises(BitLinearError, match="ALIGN"):
+        B.forward(x, packed, D)
+    small = torch.empty(64, dtype=torch.uint8, device="cuda")
+    with pytest.raises(BitLinearError, match="WORKSPACE"):
+        B.forward(torch.zeros(M, K, device="cuda"), packed, D, ws=small)
+
+
+# ------------------------------------------------ workload shapes (full size)
+def _layer_case(B, key, li, M, rows=None):
+    wl = WL.WORKLOADS[key]
+    layer = wl.layers[li]
+    W = WL.weight(layer.N, layer.K, wl.w_dist, wl.seed, layer=li)
+    x = WL.activations(M, layer.K, wl.x_dist, wl.seed, layer=li, meta=wl.meta)
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)
+    y = B.forward(dev(x), packed, D).cpu().numpy()
+    if rows is None:
+        y_ref = O.bitlinear_forward(x, p_ref, D_ref, layer.K)
+        assert_y_close(y, y_ref)
+    else:
+        y_ref = O.bitlinear_forward_rows(x, p_ref, D_ref, layer.K, rows)
+        assert_y_close(y[rows], y_ref)
+
+
+@pytest.mark.parametrize("li", range(4))
+def test_decode_layer_set_full(B, li):
+    _layer_case(B, "decode_layer_set", li, 1)
+
+
+def test_decode_2560_full(B):
+    _layer_case(B, "decode_2560", 0, 1)
+
+
+@pytest.mark.parametrize("li", range(2))
+def test_siglip_full(B, li):
+    _layer_case(B, "siglip_m256", li, 256)
+
+
+def _sample_rows(M, extra=()):
+    rows = set(range(0, M, 64)) | {0, M - 1} | set(int(r) for r in extra)
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("li", range(3))
+@pytest.mark.parametrize("M", [512, 4096])
+def test_prefill_sweep_sampled(B, li, M):
+    _layer_case(B, "prefill_sweep", li, M, rows=_sample_rows(M))
+
+
+@pytest.mark.parametrize("li", [0, 2, 3, 5])
+def test_embed_batch_sampled(B, li):
+    M = 32768
+    seed = WL.WORKLOADS["embed_batch"].seed
+    _layer_case(B, "embed_batch", li, M, rows=_sample_rows(M, WL.outlier_rows(M, seed)))
