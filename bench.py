@@ -59,7 +59,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ncu-small", action="store_true",
-                    help="tiny run for profiler launch lists (no extras, few steps)")
+                    help="small decode-only run for profiler captures (4 weight copies, no extras)")
+    ap.add_argument("--ncu-prefill", action="store_true",
+                    help="small prefill-only run for profiler captures (gate_up layer, M=4096)")
     a = ap.parse_args(argv)
     a.warmup = max(3, a.warmup)
     a.steps = max(1, a.steps)
@@ -80,6 +82,23 @@ def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return rank, world, local
+
+
+def max_over_ranks(v, device=None):
+    """Max of a per-rank float over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(v)
+    t = torch.tensor([float(v)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_gbs(world, bytes_per_step, steps, ms_max):
+    """Whole-job GB/s: every rank moved bytes_per_step per step; time is the slowest rank's."""
+    return world * bytes_per_step * steps / (ms_max * 1e-3) / 1e9
 
 
 def decode_bytes(layers, M):
@@ -234,6 +253,8 @@ def run_ours(a):
     dev = torch.device("cuda", local)
     if _lib.lib().bitlinear_device_check() != 0:
         raise SystemExit("device is not sm_100 (B200)")
+    if a.ncu_prefill:
+        return run_prefill_small(a, B, torch, dev)
     if world > 1:
         import datetime
 
@@ -243,12 +264,8 @@ def run_ours(a):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v):
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def max_ranks(v):
+        return max_over_ranks(v, dev)
 
     peaks, peak_src = load_peaks()
     hbm_peak = float(peaks["hbm_gbs"])
@@ -295,9 +312,10 @@ def run_ours(a):
         torch.cuda.synchronize(dev)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        g.replay()
-        e1.record(stream)
+        with torch.cuda.stream(stream):  # replay() launches on the current stream
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
         return e0.elapsed_time(e1)
@@ -318,12 +336,13 @@ def run_ours(a):
     # soak: keep the GPU under this load ~1 s before the timed replay (clock samples)
     t_soak = time.perf_counter()
     while time.perf_counter() - t_soak < 1.0:
-        g_dec.replay()
-    torch.cuda.synchronize(dev)
-    ms = max_over_ranks(time_graph(g_dec))
+        with torch.cuda.stream(stream):
+            g_dec.replay()
+        torch.cuda.synchronize(dev)
+    ms = max_ranks(time_graph(g_dec))
     clk = clocks.stop()
     ms_step = ms / a.steps
-    value = world * step_bytes * a.steps / (ms * 1e-3) / 1e9
+    value = weak_scaling_gbs(world, step_bytes, a.steps, ms)
     launches_per_step = len(layers)
     achieved = step_bytes / (ms_step * 1e-3) / 1e9
 
@@ -337,8 +356,9 @@ def run_ours(a):
                 p, D = packs[r][li]
                 B.forward(xs[r][li], p, D, out=ys[r][li], ws=wss[li])
             g = capture(one, nl)
-            g.replay()
-            t = max_over_ranks(time_graph(g)) / nl
+            with torch.cuda.stream(stream):
+                g.replay()
+            t = max_ranks(time_graph(g)) / nl
             b = decode_bytes([l], M)
             per_layer.append({"layer": l.name, "K": l.K, "N": l.N, "us": round(t * 1e3, 3),
                               "GB/s": round(b / (t * 1e-3) / 1e9, 1),
@@ -374,8 +394,8 @@ def run_ours(a):
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1)) / n_e2e
-    e2e_val = world * step_bytes / (ms_e2e * 1e-3) / 1e9
+    ms_e2e = max_ranks(e0.elapsed_time(e1)) / n_e2e
+    e2e_val = weak_scaling_gbs(world, step_bytes, 1, ms_e2e)
 
     # free decode buffers before prefill
     del g_dec
@@ -386,7 +406,7 @@ def run_ours(a):
     # ------------------------------------------------------------------ prefill
     prefill = None
     if not a.no_prefill and not a.ncu_small:
-        prefill = bench_prefill(a, B, torch, dev, stream, capture, time_graph, max_over_ranks, hbm_peak,
+        prefill = bench_prefill(a, B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak,
                                 i8_burst, i8_sust, rank)
 
     # --------------------------------------------------------------------- pack
@@ -451,7 +471,7 @@ def load_traffic(kernel):
         return None
 
 
-def bench_prefill(a, B, torch, dev, stream, capture, time_graph, max_over_ranks, hbm_peak, i8_burst, i8_sust, rank):
+def bench_prefill(a, B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, i8_burst, i8_sust, rank):
     wl = WL.WORKLOADS[PREFILL]
     M = PREFILL_M
     layers = list(wl.layers)
@@ -478,8 +498,9 @@ def bench_prefill(a, B, torch, dev, stream, capture, time_graph, max_over_ranks,
             whole(i)
     torch.cuda.synchronize(dev)
     g = capture(whole, n)
-    g.replay()
-    ms_step = max_over_ranks(time_graph(g)) / n
+    with torch.cuda.stream(stream):
+        g.replay()
+    ms_step = max_ranks(time_graph(g)) / n
     ops = sum(2 * M * l.N * l.K for l in layers)
     res = {"workload": f"{PREFILL}: M={M}, qkv 2560->3840, gate_up 2560->13824, down 6912->2560, "
                        "Laplace(0,0.02) weights", "ms_per_step": round(ms_step, 4),
@@ -497,11 +518,13 @@ def bench_prefill(a, B, torch, dev, stream, capture, time_graph, max_over_ranks,
             B.prepare_act(xs[li], wss[li])
 
         gg = capture(gemm, n)
-        gg.replay()
-        tg = max_over_ranks(time_graph(gg)) / n
+        with torch.cuda.stream(stream):
+            gg.replay()
+        tg = max_ranks(time_graph(gg)) / n
         gq = capture(quant, n)
-        gq.replay()
-        tq = max_over_ranks(time_graph(gq)) / n
+        with torch.cuda.stream(stream):
+            gq.replay()
+        tq = max_ranks(time_graph(gq)) / n
         o = 2 * M * l.N * l.K
         y_bytes = 4 * M * l.N
         x_bytes = M * l.K + 8 * M  # int8 codes + s_x + row sums read
@@ -548,6 +571,25 @@ def bench_pack(B, torch, dev, stream, hbm_peak):
     return {"layer": f"gate_up {l.K}->{l.N}", "ms": round(t, 4), "GB/s_algorithmic": round(alg / (t * 1e-3) / 1e9, 1),
             "frac_hbm": round(alg / (t * 1e-3) / 1e9 / hbm_peak, 4),
             "note": "two passes over W (exact integer mean, then ternarise+pack); synchronous call"}
+
+
+def run_prefill_small(a, B, torch, dev):
+    """Bounded prefill case for profiler captures: gate_up (2560->13824) at M=4096."""
+    wl = WL.WORKLOADS[PREFILL]
+    l = wl.layers[1]
+    M = PREFILL_M
+    W = torch.from_numpy(WL.weight(l.N, l.K, wl.w_dist, wl.seed, layer=1)).to(dev)
+    p, D = B.pack_weights(W)
+    del W
+    x = torch.from_numpy(WL.activations(M, l.K, wl.x_dist, wl.seed, layer=1)).to(dev)
+    y = torch.empty((M, l.N), dtype=torch.float32, device=dev)
+    ws = torch.zeros(B.workspace_size(M, l.N, l.K), dtype=torch.uint8, device=dev)
+    for _ in range(a.warmup + a.steps):
+        B.forward(x, p, D, out=y, ws=ws)
+    torch.cuda.synchronize(dev)
+    assert B.workspace_error(ws) == 0
+    print(json.dumps({"prefill_small": "ok", "M": M, "K": l.K, "N": l.N, "calls": a.warmup + a.steps}))
+    return 0
 
 
 def main(argv=None):

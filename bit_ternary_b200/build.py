@@ -47,6 +47,18 @@ def _inputs():
     ]
 
 
+def sources_sha() -> str:
+    """Hash of the kernel sources and header (identifies the measured kernels)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in _inputs():
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def up_to_date() -> bool:
     if not os.path.exists(LIB_PATH):
         return False

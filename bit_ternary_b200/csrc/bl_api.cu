@@ -231,4 +231,13 @@ int bitlinear_workspace_error(void* ws, size_t ws_bytes, bl_stream_t stream) {
   return BL_ERR_DEVICE;
 }
 
+int bitlinear_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns, bl_stream_t stream) {
+  if (ws == nullptr) return BL_ERR_NULL;
+  if (!aligned256(ws)) return BL_ERR_ALIGN;
+  if (ws_bytes < bl::kHeaderBytes) return BL_ERR_WORKSPACE;
+  const uint64_t cap = 100000000ull;
+  return cuda_status(bl::launch_selftest_wait(static_cast<uint32_t*>(ws), limit_ns < cap ? limit_ns : cap,
+                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -35,6 +35,7 @@ enum DevErr : uint32_t {
   kDevTimeoutUnpack = 0x103,
   kDevTimeoutEpilogue = 0x104,
   kDevTimeoutDrain = 0x105,
+  kDevTimeoutSelftest = 0x1FF,
 };
 
 // ------------------------------------------------------------- general ---
@@ -205,6 +206,25 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 // y = RN(RN(float(acc) / s_x) * d), the two-step rescale of the definition.
 __device__ __forceinline__ float rescale(int32_t acc, float s_x, float d) {
   return __fmul_rn(__fdiv_rn(__int2float_rn(acc), s_x), d);
+}
+
+// Exact int32 -> double without the conversion unit: the bit pattern
+// 0x43300000:(a ^ 0x80000000) is 2^52 + 2^31 + a, so one fp64 subtraction
+// recovers a exactly.
+__device__ __forceinline__ double int_to_double_exact(int32_t a) {
+  return __hiloint2double(0x43300000, a ^ (int32_t)0x80000000) - 4503601774854144.0;
+}
+
+// RN(float(a) / s_x) computed as RN_f32(RN_f64(a * inv)), with inv = RN_f64(1/s_x)
+// precomputed per token (__drcp_rn). This equals the correctly rounded fp32
+// quotient for every |a| < 2^24 and normal s_x. The fp64 value carries a
+// relative error below 2^-51.9. A quotient of a 24-bit integer by a 24-bit
+// significand is either an fp32 midpoint's distant neighbour or lies more than
+// 2^-49 (relative) away from every fp32 rounding midpoint, so the final
+// rounding to fp32 cannot differ (the same argument as S. A. Figueroa, "When
+// is double rounding innocuous?", SIGNUM Newsletter 30(3), 1995, for 53 >= 2*24+2).
+__device__ __forceinline__ float div_by_scale(int32_t a, double inv) {
+  return __double2float_rn(int_to_double_exact(a) * inv);
 }
 
 // Ternary code of one weight: clamp(rint(RN(w*s)), -1, 1) + 1, in {0, 1, 2}.

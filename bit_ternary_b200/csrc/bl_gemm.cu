@@ -35,7 +35,8 @@ constexpr int kBN = 128;  // tokens per tile (MMA N)
 constexpr int kBK = 128;  // codes per stage (4 MMAs of K=32)
 constexpr int kAStages = 8;
 constexpr int kBStages = 6;
-constexpr int kGemmThreads = 384;  // 12 warps
+constexpr int kGemmThreads = 512;  // 16 warps
+constexpr int kEpiWarps = 8;       // warps 8..15: two per TMEM lane quarter, 64 tokens each
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAccCol = 0;    // accumulator buffer b at column 128*b
 constexpr int kACol = 256;    // A stage s at column 256 + 32*s
@@ -52,6 +53,10 @@ struct GemmSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
+  // Per-token epilogue constants, one private slice per epilogue warp:
+  // 1/s_x in fp64 and sum_k q for the warp's 64 tokens.
+  double tok_inv[kEpiWarps][64];
+  int32_t tok_rs[kEpiWarps][64];
 };
 
 struct GemmParams {
@@ -73,7 +78,7 @@ struct GemmParams {
 
 // Smem: [B stages, 1024-aligned][GemmSmem]; padded so only one CTA fits per SM
 // (each CTA allocates all 512 TMEM columns).
-constexpr size_t kGemmSmemBytes = 1024 /*align slack*/ + (size_t)kBStages * kBStageBytes + 1024;
+constexpr size_t kGemmSmemBytes = 1024 /*align slack*/ + (size_t)kBStages * kBStageBytes + sizeof(GemmSmem);
 constexpr size_t kGemmSmemLaunch = kGemmSmemBytes > 120 * 1024 ? kGemmSmemBytes : 120 * 1024;
 
 // Warp-uniform bounded wait: lane 0 polls, the whole warp gets its verdict, so
@@ -133,7 +138,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&S.acc_full[b], 1);
-      mbar_init(&S.acc_empty[b], 4);
+      mbar_init(&S.acc_empty[b], kEpiWarps);
     }
     mbar_init(&S.drain, 1);
     S.abort_flag = 0;
@@ -244,37 +249,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp >= 8) {
     // ------------------------------------------------ epilogue: one weight row per thread
+    // Warp 8+e reads TMEM lane quarter e%4 and the 64 token columns of half e/4.
+    const int ew = warp - 8;
     const int quarter = warp & 3;
+    const int half = ew >> 2;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    double* s_inv = S.tok_inv[ew];
+    int32_t* s_rs = S.tok_rs[ew];
     for (int lt = 0; lt < my_tiles; ++lt) {
       const int b = lt & 1;
       const int tile = blockIdx.x + lt * gridDim.x;
-      const int m0 = (tile / p.tiles_n) * kBN;
+      const int m0 = (tile / p.tiles_n) * kBN + 64 * half;
       const int64_t n = (int64_t)(tile % p.tiles_n) * kBM + quarter * 32 + lane;
       const bool nvalid = n < p.N;
       const float dn = nvalid ? __ldg(p.D + n) : 0.0f;
+      // Per-token constants of this warp's 64 tokens (two per lane).
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int mm = m0 + 32 * h + lane;
+        const bool ok = mm < p.M;
+        s_inv[32 * h + lane] = ok ? __drcp_rn((double)__ldg(p.s_x + mm)) : 0.0;
+        s_rs[32 * h + lane] = ok ? __ldg(p.rowsum + mm) : 0;
+      }
+      __syncwarp();
       if (!warp_wait(&S.acc_full[b], (lt >> 1) & 1, abort_flag, p.err, kDevTimeoutEpilogue)) break;
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_base + kAccCol + 128 * b + 32 * c, v);
-        // Per-token values for these 32 tokens, one per lane, broadcast by shuffle.
-        const int mm = m0 + 32 * c + lane;
-        const float my_sx = mm < p.M ? __ldg(p.s_x + mm) : 1.0f;
-        const int my_rs = mm < p.M ? __ldg(p.rowsum + mm) : 0;
+        tmem_ld_32x32b_x32(lane_base + kAccCol + 128 * b + 64 * half + 32 * c, v);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float sx = __shfl_sync(0xFFFFFFFFu, my_sx, j);
-          const int rs = __shfl_sync(0xFFFFFFFFu, my_rs, j);
-          const int m = m0 + 32 * c + j;
+          const int t = 32 * c + j;
+          const int m = m0 + t;
+          const int a = (int)v[j] - s_rs[t];
           if (m < p.M && nvalid) {
-            const int a = (int)v[j] - rs;
             if (kAccOut)
               p.acc_out[(int64_t)m * p.N + n] = a;
             else
-              __stcs(p.y + (int64_t)m * p.N + n, rescale(a, sx, dn));
+              __stcs(p.y + (int64_t)m * p.N + n, __fmul_rn(div_by_scale(a, s_inv[t]), dn));
           }
         }
       }

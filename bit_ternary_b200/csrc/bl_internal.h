@@ -35,4 +35,6 @@ cudaError_t launch_gemv(const float* x, int64_t M, int64_t N, int64_t K, const u
 cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D, float* y,
                         int32_t* acc_out, void* ws, cudaStream_t stream, int num_sms);
 
+cudaError_t launch_selftest_wait(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);
+
 }  // namespace bl

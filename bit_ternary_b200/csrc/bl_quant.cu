@@ -251,6 +251,24 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const float* __restrict_
   }
 }
 
+// ------------------------------------------------------ wait self-test --
+// One thread waits on a barrier that is never completed; the bounded wait must
+// give up after limit_ns and record kDevTimeoutSelftest in the error word.
+__global__ void selftest_wait_kernel(uint32_t* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x != 0) return;
+  abort_flag = 0;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  mbar_wait(&bar, 0, &abort_flag, err, kDevTimeoutSelftest, limit_ns);
+}
+
+cudaError_t launch_selftest_wait(uint32_t* err, uint64_t limit_ns, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------ launchers --
 cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
                         cudaStream_t stream, int num_sms) {

@@ -173,6 +173,16 @@ BL_API int bitlinear_forward_host(const float* x_host, int64_t M, int64_t N, int
  * BL_ERR_DEVICE. */
 BL_API int bitlinear_workspace_error(void* ws, size_t ws_bytes, bl_stream_t stream);
 
+/* Diagnostic for the failure-detection path. Launches one thread that waits
+ * on a shared-memory barrier that nothing ever completes, using the same
+ * time-bounded wait as the tensor-core kernel, with a limit of limit_ns
+ * (capped at 100 ms). The wait gives up, records its code in the workspace
+ * error word and the kernel returns normally, so
+ * bitlinear_workspace_error() then reports BL_ERR_DEVICE. No fault, trap or
+ * hang is involved. Asynchronous. */
+BL_API int bitlinear_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns,
+                                           bl_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

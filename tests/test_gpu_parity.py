@@ -288,3 +288,22 @@ def test_embed_batch_sampled(B, li):
     M = 32768
     seed = WL.WORKLOADS["embed_batch"].seed
     _layer_case(B, "embed_batch", li, M, rows=_sample_rows(M, WL.outlier_rows(M, seed)))
+
+
+def test_bounded_wait_reports_device_error(B):
+    """A barrier wait that can never complete gives up within its limit and the
+    host sees BL_ERR_DEVICE; the context stays usable afterwards."""
+    import time
+
+    from bit_ternary_b200 import _lib
+
+    L = _lib.lib()
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    t0 = time.perf_counter()
+    assert L.bitlinear_selftest_wait_timeout(ws.data_ptr(), ws.numel(), 20_000_000, stream) == 0
+    assert L.bitlinear_workspace_error(ws.data_ptr(), ws.numel(), stream) == 6  # BL_ERR_DEVICE
+    assert time.perf_counter() - t0 < 5.0
+    assert int(ws[:4].view(torch.int32).item()) == 0  # cleared by the read
+    assert L.bitlinear_workspace_error(ws.data_ptr(), ws.numel(), stream) == 0
+    run_case(B, 2, 40, 64, seed=3)  # the context still works
