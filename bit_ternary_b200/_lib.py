@@ -46,6 +46,7 @@ SIGNATURES = {
     "bitlinear_forward_host": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "bitlinear_workspace_error": (ctypes.c_int, [_VP, _SZ, _VP]),
     "bitlinear_selftest_wait_timeout": (ctypes.c_int, [_VP, _SZ, ctypes.c_uint64, _VP]),
+    "bitlinear_forward_noalloc": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP]),
 }
 
 _lock = threading.Lock()

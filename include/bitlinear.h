@@ -173,6 +173,32 @@ BL_API int bitlinear_forward_host(const float* x_host, int64_t M, int64_t N, int
  * BL_ERR_DEVICE. */
 BL_API int bitlinear_workspace_error(void* ws, size_t ws_bytes, bl_stream_t stream);
 
+/* Size of the fixed device scratch used by bitlinear_forward_noalloc:
+ * 16 MiB per GPU that loads this library, held until the process exits. */
+#define BITLINEAR_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+
+/* bitlinear_forward for callers that cannot allocate device memory: a plugin
+ * whose host framework owns all device memory through its own allocator, a C
+ * program with no device allocator of its own, or a latency-critical loop that
+ * cannot afford cudaMalloc's possible device synchronisation. The pages have no
+ * counterpart; this is an interface convenience, not part of the method.
+ *   x, packed, D, y   as for bitlinear_forward (the caller still owns them).
+ * Scratch: instead of a caller workspace, the call uses a 16 MiB array in the
+ * library's device image (BITLINEAR_NOALLOC_SCRATCH_BYTES). It returns
+ * BL_ERR_WORKSPACE, without touching the GPU, when
+ * bitlinear_workspace_size(M, N, K) exceeds that size (e.g. M*K above about
+ * 16.7 million). It calls no cudaMalloc, cudaFree or other allocating routine.
+ * The first call on a device looks up the array's device address there (once
+ * per device, with that device current); make that first call before any
+ * stream capture. Every call shares the one array per device, and the array
+ * keeps the last call's contents. Calls that can overlap on the same GPU
+ * (other streams, other host threads) race on it and must be serialised by the
+ * caller. The device error word of these calls lives in that array and is not
+ * readable through bitlinear_workspace_error. Asynchronous. */
+BL_API int bitlinear_forward_noalloc(const float* x, int64_t M, int64_t N, int64_t K,
+                                     const uint32_t* packed, const float* D, float* y,
+                                     bl_stream_t stream);
+
 /* Diagnostic for the failure-detection path. Launches one thread that waits
  * on a shared-memory barrier that nothing ever completes, using the same
  * time-bounded wait as the tensor-core kernel, with a limit of limit_ns
