@@ -6,57 +6,75 @@
 // M=1 decode kernel; a prefill of many tokens is a dense int8 contraction, so
 // it runs on tcgen05.mma kind::i8 with int32 accumulators in tensor memory.
 //
+// Tile: 128 weight rows (MMA M) x 128 tokens (MMA N); 256 codes per pipeline
+// stage (8 MMAs of K=32 per barrier round trip, so the single issuing thread
+// keeps the tensor pipe fed), 4 stages.
+//
 // Operand placement (chosen for shared-memory bandwidth):
-//   A = unpacked ternary weights, 128 rows x 128 codes per stage, written by
-//       four "unpack" warps straight from registers into TMEM (tcgen05.st).
-//       The packed words are read from global memory; `(w >> 2c) & 0x03030303`
-//       yields code+1 for columns {c, 4+c, 8+c, 12+c} of a word, so TMEM holds
-//       the columns of every 16-column group in the order 4c+b <- 4b+c.
+//   A = unpacked ternary weights, written by four unpack warps straight from
+//       registers into TMEM (tcgen05.st). `(w >> 2c) & 0x03030303` yields
+//       code+1 for columns {c, 4+c, 8+c, 12+c} of a packed word, so TMEM
+//       holds each 16-column group in the order 4c+b <- 4b+c.
 //   B = int8 activations in the same order (written so by the ActQuant
 //       kernel), loaded by TMA as 128 tokens x 128 bytes with 128-byte swizzle.
-//   D = int32 accumulators in TMEM, two buffers of 128 columns so the epilogue
-//       of one tile overlaps the MMAs of the next.
-// The MMA thread issues tcgen05.mma (M=128 weight rows, N=128 tokens, K=32)
-// and signals stage reuse with tcgen05.commit. The epilogue warps read the
-// accumulators with tcgen05.ld, subtract sum_k q (the +1 of the stored codes)
-// and write y = RN(RN(acc/s_x)*D) with coalesced stores.
+//   D = int32 accumulators in TMEM, two buffers of 128 columns.
+// Warp roles: 0 TMA producer, 1 MMA issuer (TMEM owner), 2 per-token
+// constants (1/s_x in fp64 and sum_k q) into a shared ring, 4..7 unpack,
+// 8..15 epilogue. An epilogue warp reads its 32 rows x 64 tokens of the
+// accumulator, releases the TMEM buffer at once, rescales
+// y = RN(RN(acc/s_x)*D), stages the block in shared memory and writes it with
+// one TMA bulk store (or plain stores when N % 4 != 0).
 // Every barrier wait is bounded in time; a timeout sets a shared abort flag
 // and the error word in the workspace, and all roles drain and exit.
 #include "bl_internal.h"
 
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 namespace bl {
 
-constexpr int kBM = 128;  // weight rows per tile (MMA M)
-constexpr int kBN = 128;  // tokens per tile (MMA N)
-constexpr int kBK = 128;  // codes per stage (4 MMAs of K=32)
-constexpr int kAStages = 8;
-constexpr int kBStages = 6;
-constexpr int kGemmThreads = 512;  // 16 warps
-constexpr int kEpiWarps = 8;       // warps 8..15: two per TMEM lane quarter, 64 tokens each
+constexpr int kBM = 128;   // weight rows per tile (MMA M)
+constexpr int kBN = 128;   // tokens per tile (MMA N)
+constexpr int kBK = 256;   // codes per stage
+constexpr int kStages = 4;
+constexpr int kStageWords = kBK / 16;          // packed words per row per stage
+constexpr int kACols = kBK / 4;                // TMEM columns of one A stage
+constexpr uint32_t kBHalfBytes = kBN * 128;    // one TMA box: 128 tokens x 128 codes
+constexpr uint32_t kBStageBytes = 2 * kBHalfBytes;
 constexpr uint32_t kTmemCols = 512;
-constexpr int kAccCol = 0;    // accumulator buffer b at column 128*b
-constexpr int kACol = 256;    // A stage s at column 256 + 32*s
-constexpr int kUnpackPrefetch = 4;
-constexpr uint32_t kBStageBytes = kBN * kBK;  // 16 KB
+constexpr int kAccCol = 0;                     // accumulator b at column 128*b
+constexpr int kACol = 256;                     // A stage s at column 256 + 64*s
+static_assert(kACol + kStages * kACols <= (int)kTmemCols, "TMEM budget");
+
+constexpr int kWarpConst = 2;
+constexpr int kUnpackWarp0 = 4;                // 4..7: one per TMEM lane quarter
+constexpr int kEpiWarp0 = 8;                   // 8..15: two per lane quarter
+constexpr int kEpiWarps = 8;
+constexpr int kEpiTokens = kBN / 2;            // tokens per epilogue warp
+constexpr int kGemmThreads = 32 * (kEpiWarp0 + kEpiWarps);  // 512
+constexpr int kUnpackPrefetch = 2;             // stages of packed words in flight
+constexpr int kConstRing = 4;                  // tiles of per-token constants in flight
+constexpr uint32_t kYSliceBytes = kEpiTokens * 32 * 4;  // one epilogue warp's output block
+
+struct TokConst {
+  double inv;  // RN_f64(1 / s_x)
+  int32_t rs;  // sum_k q[m, k]
+  int32_t pad;
+};
 
 struct GemmSmem {
-  uint64_t b_full[kBStages];
-  uint64_t b_empty[kBStages];
-  uint64_t a_full[kAStages];
-  uint64_t a_empty[kAStages];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
+  uint64_t cst_full[kConstRing];
+  uint64_t cst_empty[kConstRing];
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  // Per-token epilogue constants, one private slice per epilogue warp:
-  // 1/s_x in fp64 and sum_k q for the warp's 64 tokens.
-  double tok_inv[kEpiWarps][64];
-  int32_t tok_rs[kEpiWarps][64];
+  TokConst cst[kConstRing][kBN];
 };
 
 struct GemmParams {
@@ -76,10 +94,11 @@ struct GemmParams {
   int num_tiles;
 };
 
-// Smem: [B stages, 1024-aligned][GemmSmem]; padded so only one CTA fits per SM
-// (each CTA allocates all 512 TMEM columns).
-constexpr size_t kGemmSmemBytes = 1024 /*align slack*/ + (size_t)kBStages * kBStageBytes + sizeof(GemmSmem);
-constexpr size_t kGemmSmemLaunch = kGemmSmemBytes > 120 * 1024 ? kGemmSmemBytes : 120 * 1024;
+// Smem: [B stages | Y slices | GemmSmem], 1024-aligned; one CTA per SM (each
+// CTA owns all 512 TMEM columns).
+constexpr size_t kSmemB = (size_t)kStages * kBStageBytes;
+constexpr size_t kSmemY = (size_t)kEpiWarps * kYSliceBytes;
+constexpr size_t kGemmSmemBytes = 1024 + kSmemB + kSmemY + ((sizeof(GemmSmem) + 127) & ~size_t(127));
 
 // Warp-uniform bounded wait: lane 0 polls, the whole warp gets its verdict, so
 // the warp stays converged for the .sync.aligned tcgen05 instructions.
@@ -91,59 +110,80 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return ok != 0;
 }
 
+// Position in this CTA's job sequence (tile-major, k-block-minor), advanced
+// without integer divisions.
+struct JobCursor {
+  int tile_local;
+  int kb;
+  __device__ __forceinline__ void next(int kblocks) {
+    if (++kb == kblocks) {
+      kb = 0;
+      ++tile_local;
+    }
+  }
+};
+
 template <bool kAligned>
-__device__ __forceinline__ void unpack_load(const GemmParams& p, int job, int row_in_tile, uint32_t (&w)[8]) {
-  const int tile_local = job / p.kblocks;
-  const int kb = job - tile_local * p.kblocks;
-  const int tile = blockIdx.x + tile_local * gridDim.x;
-  const int tn = tile % p.tiles_n;
-  const int64_t n = (int64_t)tn * kBM + row_in_tile;
-  const int w0 = kb * (kBK / 16);
+__device__ __forceinline__ void unpack_load(const GemmParams& p, const JobCursor& jc, int row_in_tile,
+                                            uint32_t (&w)[kStageWords]) {
+  const int tile = blockIdx.x + jc.tile_local * gridDim.x;
+  const int64_t n = (int64_t)(tile % p.tiles_n) * kBM + row_in_tile;
+  const int w0 = jc.kb * kStageWords;
   if (n < p.N) {
     const uint32_t* rp = p.packed + n * (int64_t)p.wpr + w0;
-    if (kAligned && w0 + 8 <= p.wpr) {
-      const uint4 v0 = __ldg(reinterpret_cast<const uint4*>(rp));
-      const uint4 v1 = __ldg(reinterpret_cast<const uint4*>(rp + 4));
-      w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-      w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+    if (kAligned) {
+      // wpr % 4 == 0 and w0 % 4 == 0: each group of four words is all in or all out.
+#pragma unroll
+      for (int q = 0; q < kStageWords / 4; ++q) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (w0 + 4 * q < p.wpr) v = __ldg(reinterpret_cast<const uint4*>(rp) + q);
+        w[4 * q] = v.x;
+        w[4 * q + 1] = v.y;
+        w[4 * q + 2] = v.z;
+        w[4 * q + 3] = v.w;
+      }
     } else {
 #pragma unroll
-      for (int j = 0; j < 8; ++j) w[j] = (w0 + j < p.wpr) ? __ldg(rp + j) : 0u;
+      for (int j = 0; j < kStageWords; ++j) w[j] = (w0 + j < p.wpr) ? __ldg(rp + j) : 0u;
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) w[j] = 0u;
+    for (int j = 0; j < kStageWords; ++j) w[j] = 0u;
   }
 }
 
-template <bool kAligned, bool kAccOut>
+template <bool kAligned, bool kAccOut, bool kTmaStore>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const GemmParams p) {
+    gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_out,
+                const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sB = smem;
-  GemmSmem& S = *reinterpret_cast<GemmSmem*>(smem + (size_t)kBStages * kBStageBytes);
+  uint8_t* sY = smem + kSmemB;
+  GemmSmem& S = *reinterpret_cast<GemmSmem*>(smem + kSmemB + kSmemY);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int my_tiles = p.num_tiles > (int)blockIdx.x ? (p.num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int jobs = my_tiles * p.kblocks;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kBStages; ++s) {
-      mbar_init(&S.b_full[s], 1);
-      mbar_init(&S.b_empty[s], 1);
-    }
-    for (int s = 0; s < kAStages; ++s) {
-      mbar_init(&S.a_full[s], 4);
-      mbar_init(&S.a_empty[s], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&S.full[s], 1 + 4);  // TMA producer + one unpack warp per lane quarter
+      mbar_init(&S.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&S.acc_full[b], 1);
       mbar_init(&S.acc_empty[b], kEpiWarps);
     }
+    for (int r = 0; r < kConstRing; ++r) {
+      mbar_init(&S.cst_full[r], 1);
+      mbar_init(&S.cst_empty[r], kEpiWarps);
+    }
     mbar_init(&S.drain, 1);
     S.abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tmap_q);
+    if (kTmaStore) tma_prefetch_desc(&tmap_out);
   }
   if (warp == 1) {
     tmem_alloc(&S.tmem_base, kTmemCols);
@@ -158,53 +198,69 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------ TMA producer (x)
     if (lane == 0) {
-      int it = 0;
-      bool ok = true;
-      for (int lt = 0; lt < my_tiles && ok; ++lt) {
-        const int tile = blockIdx.x + lt * gridDim.x;
+      int s = 0;
+      uint32_t ph = 0;
+      JobCursor c{0, 0};
+      int issued = 0;
+      for (int j = 0; j < jobs; ++j) {
+        if (!mbar_wait(&S.empty[s], ph ^ 1, abort_flag, p.err, kDevTimeoutProducer)) break;
+        const int tile = blockIdx.x + c.tile_local * gridDim.x;
         const int m0 = (tile / p.tiles_n) * kBN;
-        for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-          const int s = it % kBStages;
-          const uint32_t ph = (it / kBStages) & 1;
-          if (!mbar_wait(&S.b_empty[s], ph ^ 1, abort_flag, p.err, kDevTimeoutProducer)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&S.b_full[s], kBStageBytes);
-          tma_load_2d(sB + (size_t)s * kBStageBytes, &tmap_q, kb * kBK, m0, &S.b_full[s]);
+        const int k0 = c.kb * kBK;
+        // A box lying wholly past K is not loaded: its A codes are zero, so
+        // whatever the stage buffer holds there contributes nothing.
+        const bool second = k0 + 128 < p.K;
+        mbar_arrive_expect_tx(&S.full[s], second ? kBStageBytes : kBHalfBytes);
+        tma_load_2d(sB + (size_t)s * kBStageBytes, &tmap_q, k0, m0, &S.full[s]);
+        if (second) tma_load_2d(sB + (size_t)s * kBStageBytes + kBHalfBytes, &tmap_q, k0 + 128, m0, &S.full[s]);
+        ++issued;
+        c.next(p.kblocks);
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1;
         }
       }
       // Let every issued copy land before the CTA can exit.
-      const int first = it > kBStages ? it - kBStages : 0;
-      for (int j = first; j < it; ++j)
-        mbar_wait(&S.b_full[j % kBStages], (j / kBStages) & 1, nullptr, p.err, kDevTimeoutDrain, 100000000ull);
+      const int first = issued > kStages ? issued - kStages : 0;
+      for (int j = first; j < issued; ++j)
+        mbar_wait(&S.full[j % kStages], (j / kStages) & 1, nullptr, p.err, kDevTimeoutDrain, 100000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_i8(kBM, kBN);
-      int it = 0;
+      const uint64_t bdesc0 = umma_sdesc_sw128(sB);
+      int s = 0;
+      uint32_t ph = 0;
       bool ok = true;
       for (int lt = 0; lt < my_tiles && ok; ++lt) {
         const int b = lt & 1;
         if (!mbar_wait(&S.acc_empty[b], ((lt >> 1) & 1) ^ 1, abort_flag, p.err, kDevTimeoutMma)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + kAccCol + 128 * b;
-        for (int kb = 0; kb < p.kblocks; ++kb, ++it) {
-          const int sa = it % kAStages, sb = it % kBStages;
-          if (!mbar_wait(&S.a_full[sa], (it / kAStages) & 1, abort_flag, p.err, kDevTimeoutMma) ||
-              !mbar_wait(&S.b_full[sb], (it / kBStages) & 1, abort_flag, p.err, kDevTimeoutMma)) {
+        for (int kb = 0; kb < p.kblocks; ++kb) {
+          if (!mbar_wait(&S.full[s], ph, abort_flag, p.err, kDevTimeoutMma)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint64_t bdesc = umma_sdesc_sw128(sB + (size_t)sb * kBStageBytes);
-          const uint32_t a_tmem = tmem + kACol + 32 * sa;
+          const uint32_t a_tmem = tmem + kACol + kACols * s;
+          // K=32 steps of this stage that hold real codes (the rest are zero).
+          const int rem = p.K - kb * kBK;
+          const int steps = rem >= kBK ? kBK / 32 : (rem + 31) / 32;
 #pragma unroll
-          for (int k4 = 0; k4 < kBK / 32; ++k4)
-            umma_i8_ts(d_tmem, a_tmem + 8 * k4, bdesc + 2 * k4, idesc, (kb | k4) != 0 ? 1u : 0u);
-          tc_commit(&S.b_empty[sb]);
-          tc_commit(&S.a_empty[sa]);
+          for (int k8 = 0; k8 < kBK / 32; ++k8) {
+            if (k8 < steps) {
+              const uint64_t bdesc = bdesc0 + (uint64_t)((s * kBStageBytes + (k8 >> 2) * kBHalfBytes) >> 4) +
+                                     2 * (k8 & 3);
+              umma_i8_ts(d_tmem, a_tmem + 8 * k8, bdesc, idesc, (kb | k8) != 0 ? 1u : 0u);
+            }
+          }
+          tc_commit(&S.empty[s]);
+          if (++s == kStages) {
+            s = 0;
+            ph ^= 1;
+          }
         }
         if (ok) tc_commit(&S.acc_full[b]);
       }
@@ -212,89 +268,150 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_commit(&S.drain);
       mbar_wait(&S.drain, 0, nullptr, p.err, kDevTimeoutDrain, 100000000ull);
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp == kWarpConst) {
+    // ------------------------------------------------ per-token constants, ahead of the epilogue
+    int r = 0;
+    uint32_t ph = 0;
+    for (int lt = 0; lt < my_tiles; ++lt) {
+      const int tile = blockIdx.x + lt * gridDim.x;
+      const int m0 = (tile / p.tiles_n) * kBN;
+      double inv[kBN / 32];
+      int32_t rs[kBN / 32];
+#pragma unroll
+      for (int h = 0; h < kBN / 32; ++h) {
+        const int m = m0 + 32 * h + lane;
+        const bool ok = m < p.M;
+        inv[h] = ok ? __drcp_rn((double)__ldg(p.s_x + m)) : 0.0;
+        rs[h] = ok ? __ldg(p.rowsum + m) : 0;
+      }
+      if (!warp_wait(&S.cst_empty[r], ph ^ 1, abort_flag, p.err, kDevTimeoutEpilogue)) break;
+#pragma unroll
+      for (int h = 0; h < kBN / 32; ++h) {
+        S.cst[r][32 * h + lane].inv = inv[h];
+        S.cst[r][32 * h + lane].rs = rs[h];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.cst_full[r]);
+      if (++r == kConstRing) {
+        r = 0;
+        ph ^= 1;
+      }
+    }
+  } else if (warp >= kUnpackWarp0 && warp < kUnpackWarp0 + 4) {
     // ------------------------------------------------ A unpackers: one weight row per thread
-    const int quarter = warp & 3;
+    const int quarter = warp & 3;  // TMEM lane quarter (hardware rule: warp id % 4)
     const int row_in_tile = quarter * 32 + lane;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int jobs = my_tiles * p.kblocks;
-    uint32_t buf[kUnpackPrefetch][8];
+    JobCursor lc{0, 0};
+    uint32_t buf[kUnpackPrefetch][kStageWords];
 #pragma unroll
-    for (int j = 0; j < kUnpackPrefetch; ++j)
-      if (j < jobs) unpack_load<kAligned>(p, j, row_in_tile, buf[j]);
+    for (int q = 0; q < kUnpackPrefetch; ++q) {
+      if (q < jobs) unpack_load<kAligned>(p, lc, row_in_tile, buf[q]);
+      lc.next(p.kblocks);
+    }
+    int s = 0;
+    uint32_t ph = 0;
     bool ok = true;
     for (int j0 = 0; j0 < jobs && ok; j0 += kUnpackPrefetch) {
 #pragma unroll
-      for (int jj = 0; jj < kUnpackPrefetch; ++jj) {
-        const int j = j0 + jj;
+      for (int q = 0; q < kUnpackPrefetch; ++q) {
+        const int j = j0 + q;
         if (j >= jobs) break;
-        const int s = j % kAStages;
-        uint32_t v[32];
-#pragma unroll
-        for (int w = 0; w < 8; ++w)
-#pragma unroll
-          for (int c = 0; c < 4; ++c) v[4 * w + c] = (buf[jj][w] >> (2 * c)) & 0x03030303u;
-        if (j + kUnpackPrefetch < jobs) unpack_load<kAligned>(p, j + kUnpackPrefetch, row_in_tile, buf[jj]);
-        if (!warp_wait(&S.a_empty[s], ((j / kAStages) & 1) ^ 1, abort_flag, p.err, kDevTimeoutUnpack)) {
+        if (!warp_wait(&S.empty[s], ph ^ 1, abort_flag, p.err, kDevTimeoutUnpack)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        tmem_st_32x32b_x32(lane_base + kACol + 32 * s, v);
+#pragma unroll
+        for (int h = 0; h < kStageWords / 8; ++h) {
+          uint32_t v[32];
+#pragma unroll
+          for (int w = 0; w < 8; ++w)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) v[4 * w + c] = (buf[q][8 * h + w] >> (2 * c)) & 0x03030303u;
+          tmem_st_32x32b_x32(lane_base + kACol + kACols * s + 32 * h, v);
+        }
+        if (j + kUnpackPrefetch < jobs) unpack_load<kAligned>(p, lc, row_in_tile, buf[q]);
+        lc.next(p.kblocks);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.a_full[s]);
+        if (lane == 0) mbar_arrive(&S.full[s]);
+        if (++s == kStages) {
+          s = 0;
+          ph ^= 1;
+        }
       }
     }
-  } else if (warp >= 8) {
-    // ------------------------------------------------ epilogue: one weight row per thread
-    // Warp 8+e reads TMEM lane quarter e%4 and the 64 token columns of half e/4.
-    const int ew = warp - 8;
+  } else if (warp >= kEpiWarp0) {
+    // ------------------------------------------------ epilogue: 32 weight rows x 64 tokens per warp
+    const int ew = warp - kEpiWarp0;
     const int quarter = warp & 3;
     const int half = ew >> 2;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    double* s_inv = S.tok_inv[ew];
-    int32_t* s_rs = S.tok_rs[ew];
+    uint32_t* sy = reinterpret_cast<uint32_t*>(sY + (size_t)ew * kYSliceBytes);
+    int r = 0;
+    uint32_t rph = 0;
     for (int lt = 0; lt < my_tiles; ++lt) {
       const int b = lt & 1;
       const int tile = blockIdx.x + lt * gridDim.x;
-      const int m0 = (tile / p.tiles_n) * kBN + 64 * half;
-      const int64_t n = (int64_t)(tile % p.tiles_n) * kBM + quarter * 32 + lane;
+      const int m0 = (tile / p.tiles_n) * kBN + kEpiTokens * half;
+      const int n0 = (tile % p.tiles_n) * kBM + quarter * 32;
+      const int64_t n = (int64_t)n0 + lane;
       const bool nvalid = n < p.N;
-      const float dn = nvalid ? __ldg(p.D + n) : 0.0f;
-      // Per-token constants of this warp's 64 tokens (two per lane).
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int mm = m0 + 32 * h + lane;
-        const bool ok = mm < p.M;
-        s_inv[32 * h + lane] = ok ? __drcp_rn((double)__ldg(p.s_x + mm)) : 0.0;
-        s_rs[32 * h + lane] = ok ? __ldg(p.rowsum + mm) : 0;
-      }
-      __syncwarp();
+      const float dn = (!kAccOut && nvalid) ? __ldg(p.D + n) : 0.0f;
       if (!warp_wait(&S.acc_full[b], (lt >> 1) & 1, abort_flag, p.err, kDevTimeoutEpilogue)) break;
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_base + kAccCol + 128 * b + 64 * half + 32 * c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int t = 32 * c + j;
-          const int m = m0 + t;
-          const int a = (int)v[j] - s_rs[t];
-          if (m < p.M && nvalid) {
-            if (kAccOut)
-              p.acc_out[(int64_t)m * p.N + n] = a;
-            else
-              __stcs(p.y + (int64_t)m * p.N + n, __fmul_rn(div_by_scale(a, s_inv[t]), dn));
-          }
-        }
-      }
+      uint32_t v0[32], v1[32];
+      tmem_ld_32x32b_x32(lane_base + kAccCol + 128 * b + kEpiTokens * half, v0);
+      tmem_ld_32x32b_x32(lane_base + kAccCol + 128 * b + kEpiTokens * half + 32, v1);
+      tmem_wait_ld();
+      // The accumulator is in registers: hand the TMEM buffer back to the MMA.
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.acc_empty[b]);
+      if (!warp_wait(&S.cst_full[r], rph, abort_flag, p.err, kDevTimeoutEpilogue)) break;
+      const TokConst* cst = &S.cst[r][kEpiTokens * half];
+      if (kTmaStore) {
+        // The previous block's bulk store must have read this slice.
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+      }
+#pragma unroll
+      for (int t = 0; t < kEpiTokens; ++t) {
+        const TokConst kc = cst[t];
+        const int a = (int)(t < 32 ? v0[t] : v1[t - 32]) - kc.rs;
+        const uint32_t out = kAccOut ? (uint32_t)a : __float_as_uint(__fmul_rn(div_by_scale(a, kc.inv), dn));
+        if (kTmaStore) {
+          sy[t * 32 + lane] = out;
+        } else {
+          const int m = m0 + t;
+          if (m < p.M && nvalid) {
+            if (kAccOut)
+              p.acc_out[(int64_t)m * p.N + n] = (int32_t)out;
+            else
+              __stcs(p.y + (int64_t)m * p.N + n, __uint_as_float(out));
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.cst_empty[r]);
+      if (++r == kConstRing) {
+        r = 0;
+        rph ^= 1;
+      }
+      if (kTmaStore) {
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tmap_out, n0, m0, sy);
+          bulk_commit_group();
+        }
+      }
+    }
+    if (kTmaStore) {
+      if (lane == 0) bulk_wait_group0();
+      __syncwarp();
     }
   }
 
@@ -320,12 +437,13 @@ static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-template <bool kAligned, bool kAccOut>
-static cudaError_t launch_gemm_t(const CUtensorMap& tmap, const GemmParams& p, int grid, cudaStream_t stream) {
-  auto kern = gemm_kernel<kAligned, kAccOut>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemLaunch);
+template <bool kAligned, bool kAccOut, bool kTmaStore>
+static cudaError_t launch_gemm_t(const CUtensorMap& tq, const CUtensorMap& to, const GemmParams& p, int grid,
+                                 cudaStream_t stream) {
+  auto kern = gemm_kernel<kAligned, kAccOut, kTmaStore>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kGemmThreads, kGemmSmemLaunch, stream>>>(tmap, p);
+  kern<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tq, to, p);
   return cudaGetLastError();
 }
 
@@ -335,15 +453,31 @@ cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed,
   int8_t* q = reinterpret_cast<int8_t*>(base + ws_q_off(M));
   PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
   if (encode == nullptr) return cudaErrorNotSupported;
-  CUtensorMap tmap;
-  const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
-  const cuuint64_t gstride[1] = {(cuuint64_t)K};
-  const cuuint32_t box[2] = {(cuuint32_t)kBK, (cuuint32_t)kBN};
-  const cuuint32_t estride[2] = {1, 1};
-  CUresult r = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, gdim, gstride, box, estride,
-                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  CUtensorMap tmap_q, tmap_out;
+  {
+    const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+    const cuuint64_t gstride[1] = {(cuuint64_t)K};
+    const cuuint32_t box[2] = {128u, (cuuint32_t)kBN};
+    const cuuint32_t estride[2] = {1, 1};
+    if (encode(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, gdim, gstride, box, estride,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  // Output via TMA bulk stores when every output row starts on a 16-byte boundary.
+  void* out = acc_out != nullptr ? static_cast<void*>(acc_out) : static_cast<void*>(y);
+  const bool tma_store = (N % 4) == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0;
+  std::memset(&tmap_out, 0, sizeof(tmap_out));
+  if (tma_store) {
+    const cuuint64_t gdim[2] = {(cuuint64_t)N, (cuuint64_t)M};
+    const cuuint64_t gstride[1] = {(cuuint64_t)N * 4};
+    const cuuint32_t box[2] = {32u, (cuuint32_t)kEpiTokens};
+    const cuuint32_t estride[2] = {1, 1};
+    if (encode(&tmap_out, acc_out != nullptr ? CU_TENSOR_MAP_DATA_TYPE_INT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+               out, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
 
   GemmParams p;
   p.packed = packed;
@@ -365,9 +499,19 @@ cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed,
   p.num_tiles = (int)nt;
   const int grid = (int)(nt < num_sms ? nt : num_sms);
   const bool aligned = (p.wpr % 4) == 0;
-  if (acc_out != nullptr)
-    return aligned ? launch_gemm_t<true, true>(tmap, p, grid, stream) : launch_gemm_t<false, true>(tmap, p, grid, stream);
-  return aligned ? launch_gemm_t<true, false>(tmap, p, grid, stream) : launch_gemm_t<false, false>(tmap, p, grid, stream);
+  const bool accout = acc_out != nullptr;
+#define BL_GEMM_CASE(AL, AO, TS) \
+  if (aligned == AL && accout == AO && tma_store == TS) return launch_gemm_t<AL, AO, TS>(tmap_q, tmap_out, p, grid, stream);
+  BL_GEMM_CASE(true, false, true)
+  BL_GEMM_CASE(true, false, false)
+  BL_GEMM_CASE(false, false, true)
+  BL_GEMM_CASE(false, false, false)
+  BL_GEMM_CASE(true, true, true)
+  BL_GEMM_CASE(true, true, false)
+  BL_GEMM_CASE(false, true, true)
+  BL_GEMM_CASE(false, true, false)
+#undef BL_GEMM_CASE
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace bl

@@ -23,6 +23,7 @@ namespace bl {
 
 constexpr int kGemvThreads = 256;
 constexpr int kGemvWarps = 8;
+constexpr int kRing = 4;  // 256-code units of packed weights in flight per warp
 
 struct GemvParams {
   const float* x;
@@ -85,11 +86,15 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvParams p) 
   const uint32_t* rowpA = p.packed + (validA ? rowA : 0) * (int64_t)p.wpr;
   const uint32_t* rowpB = p.packed + (validB ? rowB : 0) * (int64_t)p.wpr;
 
-  // Issue the first unit's weight loads before quantising, to overlap latency.
-  uint32_t wa[4], wb[4];
-  int u = ks;
-  load_unit<kAligned>(rowpA, validA, u * 16 + 4 * t, p.wpr, wa);
-  load_unit<kAligned>(rowpB, validB, u * 16 + 4 * t, p.wpr, wb);
+  // Issue the weight loads of this warp's first kRing units (units ks, ks+nks, ...)
+  // before quantising, so their DRAM latency overlaps the ActQuant phase.
+  uint32_t wa[kRing][4], wb[kRing][4];
+#pragma unroll
+  for (int i = 0; i < kRing; ++i) {
+    const int u = ks + i * nks;
+    load_unit<kAligned>(rowpA, validA && u < p.n_units, u * 16 + 4 * t, p.wpr, wa[i]);
+    load_unit<kAligned>(rowpB, validB && u < p.n_units, u * 16 + 4 * t, p.wpr, wb[i]);
+  }
 
   if (p.err_reset != nullptr && blockIdx.x == 0 && tid == 0) *p.err_reset = 0u;
   if (tid < 16) {
@@ -153,46 +158,45 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvParams p) 
 #pragma unroll
       for (int i = 0; i < 4; ++i) acc[c][mt][i] = 0;
 
-  for (; u < p.n_units; u += nks) {
-    uint32_t na[4], nb[4];
-    const int un = u + nks;
-    load_unit<kAligned>(rowpA, validA && un < p.n_units, un * 16 + 4 * t, p.wpr, na);
-    load_unit<kAligned>(rowpB, validB && un < p.n_units, un * 16 + 4 * t, p.wpr, nb);
-
-    uint4 Q[MT][4];
+  for (int base = 0; ks + base * nks < p.n_units; base += kRing) {
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      const int tok = g + 8 * mt;
-      if (tok < p.M) {
-        const uint8_t* qp = sq + (int64_t)tok * p.q_stride + 16 * (u * 16 + 4 * t);
+    for (int i = 0; i < kRing; ++i) {
+      const int u = ks + (base + i) * nks;
+      if (u >= p.n_units) break;
+      uint4 Q[MT][4];
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) Q[mt][i4] = *reinterpret_cast<const uint4*>(qp + 16 * i4);
-      } else {
+      for (int mt = 0; mt < MT; ++mt) {
+        const int tok = g + 8 * mt;
+        if (tok < p.M) {
+          const uint8_t* qp = sq + (int64_t)tok * p.q_stride + 16 * (u * 16 + 4 * t);
 #pragma unroll
-        for (int i4 = 0; i4 < 4; ++i4) Q[mt][i4] = make_uint4(0u, 0u, 0u, 0u);
-      }
-    }
+          for (int i4 = 0; i4 < 4; ++i4) Q[mt][i4] = *reinterpret_cast<const uint4*>(qp + 16 * i4);
+        } else {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint32_t mask = 0x03030303u << (2 * c);
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const uint32_t a0 = wa[2 * h] & mask, a2 = wa[2 * h + 1] & mask;
-        const uint32_t a1 = wb[2 * h] & mask, a3 = wb[2 * h + 1] & mask;
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const uint4& q0 = Q[mt][2 * h];
-          const uint4& q1 = Q[mt][2 * h + 1];
-          const uint32_t b0 = c == 0 ? q0.x : (c == 1 ? q0.y : (c == 2 ? q0.z : q0.w));
-          const uint32_t b1 = c == 0 ? q1.x : (c == 1 ? q1.y : (c == 2 ? q1.z : q1.w));
-          mma_u8s8(acc[c][mt], a0, a1, a2, a3, b0, b1);
+          for (int i4 = 0; i4 < 4; ++i4) Q[mt][i4] = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-    }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      wa[j] = na[j];
-      wb[j] = nb[j];
+      for (int c = 0; c < 4; ++c) {
+        const uint32_t mask = 0x03030303u << (2 * c);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t a0 = wa[i][2 * h] & mask, a2 = wa[i][2 * h + 1] & mask;
+          const uint32_t a1 = wb[i][2 * h] & mask, a3 = wb[i][2 * h + 1] & mask;
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            const uint4& q0 = Q[mt][2 * h];
+            const uint4& q1 = Q[mt][2 * h + 1];
+            const uint32_t b0 = c == 0 ? q0.x : (c == 1 ? q0.y : (c == 2 ? q0.z : q0.w));
+            const uint32_t b1 = c == 0 ? q1.x : (c == 1 ? q1.y : (c == 2 ? q1.z : q1.w));
+            mma_u8s8(acc[c][mt], a0, a1, a2, a3, b0, b1);
+          }
+        }
+      }
+      // Refill this ring slot with the unit kRing positions further on.
+      const int un = u + kRing * nks;
+      load_unit<kAligned>(rowpA, validA && un < p.n_units, un * 16 + 4 * t, p.wpr, wa[i]);
+      load_unit<kAligned>(rowpB, validB && un < p.n_units, un * 16 + 4 * t, p.wpr, wb[i]);
     }
   }
 
@@ -255,8 +259,18 @@ cudaError_t launch_gemv(const float* x, int64_t M, int64_t N, int64_t K, const u
   p.wpr = (int)(K / 16);
   p.n_units = (p.wpr + 15) / 16;
   p.q_stride = (int)gemv_q_stride(K);
+  // Rows per CTA: as many 16-row tiles as keep every warp within kRing units
+  // (so all of its loads are in flight at once) while the grid still covers
+  // every SM; more rows per CTA amortise the per-CTA quantisation of x.
   const int64_t tiles = (N + 15) / 16;
-  p.R = tiles >= 4 * (int64_t)num_sms ? 4 : (tiles >= 2 * (int64_t)num_sms ? 2 : 1);
+  p.R = 1;
+  for (int r : {4, 2}) {
+    const int units_per_warp = (p.n_units * r + kGemvWarps - 1) / kGemvWarps;
+    if (units_per_warp <= kRing && (tiles + r - 1) / r >= num_sms) {
+      p.R = r;
+      break;
+    }
+  }
   const int64_t grid = (tiles + p.R - 1) / p.R;
   const int MT = M <= 8 ? 1 : 2;
   const size_t smem = (size_t)M * p.q_stride + 3 * 16 * 4 + (size_t)kGemvWarps * 32 * 4 * MT * 4;

@@ -179,8 +179,11 @@ def test_gemm_edge_zero_tokens_and_rows(B):
 
 
 def test_output_written_exactly(B):
-    """Every element of y is written, nothing past it (poisoned guard)."""
-    for (M, N, K) in [(1, 33, 64), (37, 131, 272)]:
+    """Every element of y is written, nothing past it (poisoned guard), and the
+    values match the oracle."""
+    # (37, 131): plain-store epilogue (N % 4 != 0); (37, 132) and (300, 260):
+    # TMA bulk-store epilogue, which must clip the M and N tails.
+    for (M, N, K) in [(1, 33, 64), (37, 131, 272), (37, 132, 272), (300, 260, 528)]:
         W = WL.weight(N, K, "normal", 1)
         x = WL.activations(M, K, "normal", 1)
         packed, D = B.pack_weights(dev(W))
@@ -190,6 +193,8 @@ def test_output_written_exactly(B):
         torch.cuda.synchronize()
         assert torch.isfinite(y).all()
         assert torch.isnan(buf[M * N:]).all()
+        p_ref, D_ref = O.pack_weights(W)
+        assert_y_close(y.cpu().numpy(), O.bitlinear_forward(x, p_ref, D_ref, K))
 
 
 def test_D_row_layout_enforced(B):
