@@ -42,6 +42,8 @@ SIGNATURES = {
     "bitlinear_forward_acc": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
     "bitlinear_prepare_act": (ctypes.c_int, [_VP, _I64, _I64, _VP, _SZ, _VP]),
     "bitlinear_forward_prepared": (ctypes.c_int, [_I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "bitlinear_batch_workspace_size": (_SZ, [_VP, ctypes.c_int]),
+    "bitlinear_forward_batch": (ctypes.c_int, [_VP, ctypes.c_int, ctypes.c_uint32, _VP, _SZ, _VP]),
     "bitlinear_host_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "bitlinear_forward_host": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "bitlinear_workspace_error": (ctypes.c_int, [_VP, _SZ, _VP]),
@@ -51,6 +53,23 @@ SIGNATURES = {
 
 _lock = threading.Lock()
 _lib = None
+
+
+class LinearCall(ctypes.Structure):
+    """Mirror of bl_linear_call (include/bitlinear.h)."""
+
+    _fields_ = [
+        ("x", ctypes.c_void_p),
+        ("M", ctypes.c_int64),
+        ("N", ctypes.c_int64),
+        ("K", ctypes.c_int64),
+        ("packed", ctypes.c_void_p),
+        ("D", ctypes.c_void_p),
+        ("y", ctypes.c_void_p),
+    ]
+
+
+BL_FLAG_STREAM_WEIGHTS_EARLY = 1
 
 
 class BitLinearError(RuntimeError):

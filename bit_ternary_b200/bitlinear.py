@@ -21,6 +21,7 @@ __all__ = [
     "forward",
     "forward_acc",
     "forward_host",
+    "forward_batch",
     "prepare_act",
     "forward_prepared",
     "workspace_size",
@@ -143,6 +144,36 @@ def forward_prepared(M: int, K: int, packed: torch.Tensor, D: torch.Tensor, ws: 
     _lib.call("bitlinear_forward_prepared", M, N, K, packed.data_ptr(), D.data_ptr(), y.data_ptr(),
               ws.data_ptr(), ws.numel(), _stream_handle(packed.device))
     return y
+
+
+def forward_batch(calls, flags: int = 0, ws: Optional[torch.Tensor] = None):
+    """Run independent BitLinears [(x, packed, D, out), ...] in one C call.
+
+    Decode-sized calls (M <= 16) are fused into grouped launches; `flags` may
+    hold BL_FLAG_STREAM_WEIGHTS_EARLY (weights are static, so the decode
+    kernels may stream them while the previous work on the stream finishes).
+    Returns the list of outputs.
+    """
+    n = len(calls)
+    arr = (_lib.LinearCall * max(n, 1))()
+    outs = []
+    device = None
+    for i, (x, packed, D, out) in enumerate(calls):
+        K = x.shape[-1]
+        M, N = _fwd_args(x, packed, K)
+        _check_D(D, N)
+        y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x.device)
+        _need_cuda(y, "out", torch.float32)
+        arr[i] = _lib.LinearCall(x.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(), y.data_ptr())
+        outs.append(y)
+        device = x.device
+    if n == 0:
+        return outs
+    L = _lib.lib()
+    if ws is None:
+        ws = _alloc_ws(L.bitlinear_batch_workspace_size(arr, n), device)
+    _lib.call("bitlinear_forward_batch", arr, n, flags, ws.data_ptr(), ws.numel(), _stream_handle(device))
+    return outs
 
 
 def forward_host(x_host: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,

@@ -61,8 +61,10 @@ int forward_impl(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t
   if (sms <= 0) return BL_ERR_CUDA;
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint32_t* err = reinterpret_cast<uint32_t*>(base);
-  if (bl::gemv_eligible(M, K))
-    return cuda_status(bl::launch_gemv(x, M, N, K, packed, D, y, acc, err, stream, sms));
+  if (bl::gemv_group_fits(M, K)) {
+    const bl::GemvCall call{x, packed, D, y, acc, M, N, K};
+    return cuda_status(bl::launch_gemv_group(&call, 1, err, false, stream, sms));
+  }
   cudaError_t e = bl::launch_act_quant(x, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
                                        reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
                                        reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), true, stream, err);
@@ -186,6 +188,74 @@ int bitlinear_forward_prepared(int64_t M, int64_t N, int64_t K, const uint32_t* 
   const int sms = num_sms_current();
   if (sms <= 0) return BL_ERR_CUDA;
   return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, nullptr, ws, reinterpret_cast<cudaStream_t>(stream), sms));
+}
+
+size_t bitlinear_batch_workspace_size(const bl_linear_call* calls, int count) {
+  size_t need = bl::kHeaderBytes;
+  if (calls == nullptr || count < 0) return 0;
+  for (int i = 0; i < count; ++i) {
+    const size_t w = bitlinear_workspace_size(calls[i].M, calls[i].N, calls[i].K);
+    need = w > need ? w : need;
+  }
+  return need;
+}
+
+int bitlinear_forward_batch(const bl_linear_call* calls, int count, uint32_t flags, void* ws, size_t ws_bytes,
+                            bl_stream_t stream) {
+  if (count < 0) return BL_ERR_SHAPE;
+  if (count == 0) return BL_OK;
+  if (calls == nullptr || ws == nullptr) return BL_ERR_NULL;
+  if (!aligned256(ws)) return BL_ERR_ALIGN;
+  if (flags & ~(uint32_t)BL_FLAG_STREAM_WEIGHTS_EARLY) return BL_ERR_SHAPE;
+  // Validate every call before launching anything.
+  for (int i = 0; i < count; ++i) {
+    const bl_linear_call& c = calls[i];
+    int st = check_k(c.K);
+    if (st != BL_OK) return st;
+    st = check_mn(c.M, c.N);
+    if (st != BL_OK) return st;
+    if (c.M == 0 || c.N == 0) continue;
+    if (c.x == nullptr || c.packed == nullptr || c.D == nullptr || c.y == nullptr) return BL_ERR_NULL;
+    if (!aligned16(c.x) || !aligned16(c.packed) || !aligned16(c.D) || !aligned16(c.y)) return BL_ERR_ALIGN;
+  }
+  if (ws_bytes < bitlinear_batch_workspace_size(calls, count)) return BL_ERR_WORKSPACE;
+  const int sms = num_sms_current();
+  if (sms <= 0) return BL_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* err = static_cast<uint32_t*>(ws);
+  const bool early = (flags & BL_FLAG_STREAM_WEIGHTS_EARLY) != 0;
+  // Decode-sized calls are grouped, in order, into launches of up to
+  // kGemvMaxGroup; every other call runs on its own.
+  bl::GemvCall group[bl::kGemvMaxGroup];
+  int ng = 0;
+  int64_t gM = 0, gK = 0;
+  auto flush = [&]() -> int {
+    if (ng == 0) return BL_OK;
+    const cudaError_t e = bl::launch_gemv_group(group, ng, err, early, s, sms);
+    ng = 0;
+    gM = gK = 0;
+    return cuda_status(e);
+  };
+  for (int i = 0; i < count; ++i) {
+    const bl_linear_call& c = calls[i];
+    if (c.M == 0 || c.N == 0) continue;
+    const int64_t nM = c.M > gM ? c.M : gM, nK = c.K > gK ? c.K : gK;
+    if (bl::gemv_group_fits(c.M, c.K)) {
+      if (ng == bl::kGemvMaxGroup || !bl::gemv_group_fits(nM, nK)) {
+        const int st = flush();
+        if (st != BL_OK) return st;
+      }
+      group[ng++] = bl::GemvCall{c.x, c.packed, c.D, c.y, nullptr, c.M, c.N, c.K};
+      gM = c.M > gM ? c.M : gM;
+      gK = c.K > gK ? c.K : gK;
+      continue;
+    }
+    int st = flush();
+    if (st != BL_OK) return st;
+    st = forward_impl(c.x, c.M, c.N, c.K, c.packed, c.D, c.y, nullptr, ws, ws_bytes, s);
+    if (st != BL_OK) return st;
+  }
+  return flush();
 }
 
 size_t bitlinear_host_workspace_size(int64_t M, int64_t N, int64_t K) {

@@ -1,44 +1,66 @@
-// bl_gemv.cu - decode GEMV (M <= 16 tokens) with ActQuant fused in.
+// bl_gemv.cu - decode GEMV (M <= 16 tokens) with ActQuant fused in, for one
+// or several independent BitLinears per launch.
 //
 // The operation is the BitLinear product of "Core AI model zoo - BitVLA",
 // section 2 (M=1 decode, arbitrary K with K % 16 == 0, any N, per-row scale
 // D [N,1]), with the wrapper's ActQuant (section 1) done inside the kernel.
 //
-// Design (B200): the packed weights are the only large stream (2 bits per
-// weight), read once with 128-bit coalesced loads. A warp works on a 16-row
-// tile; lane (g, t) = (lane/4, lane%4) loads words 4t..4t+3 of a 16-word
-// (256-code) unit for rows g and g+8, so the four lanes of a row read 64
-// contiguous bytes. Unpacking is one AND per 4 codes: for class c in 0..3,
+// Design (B200). The packed weights are the only large stream (2 bits per
+// weight). The grid is persistent: CTA c owns a contiguous, balanced range of
+// 16-row tiles over all problems of the launch. One thread issues
+// cp.async.bulk copies of whole tiles (16 rows x K/4 bytes, contiguous in
+// memory) into a ring of shared-memory stages the moment the CTA starts, so
+// every byte the CTA needs is in flight before x is even read. With
+// programmatic dependent launch the weight copies of this kernel may overlap
+// the kernel before it; the activations are read only after
+// griddepcontrol.wait.
+//
+// Math. A warp computes a 16-row tile on a K-slice; lane (g, t) =
+// (lane/4, lane%4) takes words 4t..4t+3 of each 256-code unit for rows g and
+// g+8. Unpacking is one AND per 4 codes: for class c in 0..3,
 // word & (0x03030303 << 2c) leaves, in byte b, (code[4b+c]+1) << 2c. Those
-// bytes feed mma.sync.m16n8k32 (u8 weights x s8 activations) directly, with
-// one accumulator set per class; the classes are recombined exactly as
-// acc0 + acc1/4 + acc2/16 + acc3/64 (each accumulator is an exact multiple).
-// The activations are quantised per CTA into shared memory in the matching
-// order (inside every 16 columns, position 4c+b holds column 4b+c), so the
-// B fragments are plain 32-bit shared loads. sum q*(code+1) - sum q gives the
-// signed result.
+// bytes feed mma.sync.m16n8k32 (u8 weights x s8 activations) with one
+// accumulator set per class, recombined exactly as acc0 + acc1/4 + acc2/16 +
+// acc3/64. The activations are quantised per CTA into shared memory in the
+// matching order (inside every 16 columns, position 4c+b holds column 4b+c).
+// sum q*(code+1) - sum q gives the signed result.
 #include "bl_internal.h"
+
+#include <cstring>
 
 namespace bl {
 
-constexpr int kGemvThreads = 256;
-constexpr int kGemvWarps = 8;
-constexpr int kRing = 4;  // 256-code units of packed weights in flight per warp
+constexpr int kGemvWarps = 16;  // warps per CTA: enough independent work to hide latency
+constexpr int kGemvThreads = 32 * kGemvWarps;
+constexpr int kGemvMaxGrid = 256;
 
-struct GemvParams {
+struct GemvProblem {
   const float* x;
   const uint32_t* packed;
   const float* D;
   float* y;
-  int32_t* acc_out;
-  uint32_t* err_reset;
+  int32_t* acc;
   int M;
-  int64_t N;
+  int N;
   int K;
   int wpr;       // packed words per row = K/16
   int n_units;   // ceil(wpr / 16)
-  int R;         // 16-row tiles per CTA (1, 2 or 4)
-  int q_stride;  // shared bytes per token row
+  int tiles;     // ceil(N / 16)
+  int tile0;     // index of this problem's first tile in the launch
+  int q_stride;  // shared bytes per token row of quantised activations
+};
+
+struct GemvLaunch {
+  GemvProblem pr[kGemvMaxGroup];
+  int nprob;
+  int total_tiles;
+  int stage_bytes;  // bytes of one tile slot of the double-buffered mode (widest problem)
+  int round_tiles;  // tile slots per round buffer
+  int nbuf;         // 1: all of a CTA's tiles in flight, packed by size; 2: double-buffered rounds
+  int buf_bytes;    // capacity of one round buffer
+  int q_bytes;
+  uint32_t* err;
+  int cta_start[kGemvMaxGrid + 1];  // CTA c owns launch tiles [cta_start[c], cta_start[c+1])
 };
 
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -49,80 +71,76 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, 
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <bool kAligned>
-__device__ __forceinline__ void load_unit(const uint32_t* __restrict__ rowp, bool valid, int w0, int wpr,
-                                          uint32_t (&w)[4]) {
-  if (kAligned) {
-    // wpr % 4 == 0 and w0 % 4 == 0: the four words are all in or all out.
-    if (valid && w0 < wpr) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(rowp + w0));
-      w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
-    } else {
-      w[0] = w[1] = w[2] = w[3] = 0u;
-    }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) w[j] = (valid && w0 + j < wpr) ? __ldg(rowp + w0 + j) : 0u;
-  }
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
-template <int MT, bool kAligned, bool kAccOut>
-__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvParams p) {
-  extern __shared__ __align__(16) uint8_t smem[];
-  uint8_t* sq = smem;                                            // [M][q_stride] permuted int8
-  float* s_sx = reinterpret_cast<float*>(smem + p.M * p.q_stride);  // [16]
-  int32_t* s_rsum = reinterpret_cast<int32_t*>(s_sx + 16);          // [16]
-  uint32_t* s_amax = reinterpret_cast<uint32_t*>(s_rsum + 16);      // [16]
-  int32_t* s_red = reinterpret_cast<int32_t*>(s_amax + 16);         // [8][32][4*MT]
+__device__ __forceinline__ int problem_of(const GemvLaunch& L, int gt) {
+  int p = 0;
+#pragma unroll 1
+  while (p + 1 < L.nprob && gt >= L.pr[p + 1].tile0) ++p;
+  return p;
+}
 
+// Bytes of launch tile `gt` in shared memory (rows x K/4, rounded up to 128).
+__device__ __forceinline__ uint32_t tile_slot_bytes(const GemvLaunch& L, int gt) {
+  const GemvProblem& P = L.pr[problem_of(L, gt)];
+  const int row0 = (gt - P.tile0) * 16;
+  const int rows = P.N - row0 < 16 ? P.N - row0 : 16;
+  return ((uint32_t)rows * (uint32_t)P.wpr * 4u + 127u) & ~127u;
+}
+
+// Start the copy of launch tile `gt` into shared memory (one thread). A tile
+// is rows_valid x K/4 contiguous bytes. Whole 16-byte chunks go by bulk copy;
+// a remainder of 4..12 bytes (only possible on a problem's last tile) is
+// copied with plain loads before the barrier's arrival, which orders it for
+// the readers.
+__device__ __forceinline__ void issue_tile(const GemvLaunch& L, int gt, uint8_t* dst, uint64_t* bar) {
+  const GemvProblem& P = L.pr[problem_of(L, gt)];
+  const int lt = gt - P.tile0;
+  const int row0 = lt * 16;
+  const int rows = P.N - row0 < 16 ? P.N - row0 : 16;
+  const uint32_t bytes = (uint32_t)rows * (uint32_t)P.wpr * 4u;
+  const uint32_t bulk = bytes & ~15u;
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(P.packed + (int64_t)row0 * P.wpr);
+  for (uint32_t o = bulk; o < bytes; o += 4)
+    *reinterpret_cast<uint32_t*>(dst + o) = __ldg(reinterpret_cast<const uint32_t*>(src + o));
+  mbar_arrive_expect_tx(bar, bulk);
+  if (bulk) bulk_g2s(dst, src, bulk, bar);
+}
+
+// Quantise problem P's activations into shared memory (kernel-private column
+// order), with per-token scale and sum of codes. Block-wide.
+__device__ __forceinline__ void quantise_x(const GemvProblem& P, uint8_t* sq, float* s_sx, int32_t* s_rs,
+                                           uint32_t* s_amax) {
   const int tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int R = p.R;
-  const int rt = warp % R, ks = warp / R, nks = kGemvWarps / R;
-  const int64_t row0 = ((int64_t)blockIdx.x * R + rt) * 16;
-  const int64_t rowA = row0 + g, rowB = row0 + g + 8;
-  const bool validA = rowA < p.N, validB = rowB < p.N;
-  const uint32_t* rowpA = p.packed + (validA ? rowA : 0) * (int64_t)p.wpr;
-  const uint32_t* rowpB = p.packed + (validB ? rowB : 0) * (int64_t)p.wpr;
-
-  // Issue the weight loads of this warp's first kRing units (units ks, ks+nks, ...)
-  // before quantising, so their DRAM latency overlaps the ActQuant phase.
-  uint32_t wa[kRing][4], wb[kRing][4];
-#pragma unroll
-  for (int i = 0; i < kRing; ++i) {
-    const int u = ks + i * nks;
-    load_unit<kAligned>(rowpA, validA && u < p.n_units, u * 16 + 4 * t, p.wpr, wa[i]);
-    load_unit<kAligned>(rowpB, validB && u < p.n_units, u * 16 + 4 * t, p.wpr, wb[i]);
-  }
-
-  if (p.err_reset != nullptr && blockIdx.x == 0 && tid == 0) *p.err_reset = 0u;
   if (tid < 16) {
     s_amax[tid] = 0u;
-    s_rsum[tid] = 0;
+    s_rs[tid] = 0;
   }
   __syncthreads();
-
-  // ---- fused ActQuant: pass 1, max|x| per token (non-negative floats order as uints)
-  const int G = p.K >> 4;
-  const int total = p.M * G;
+  const int G = P.K >> 4;
+  const int total = P.M * G;
   for (int idx = tid; idx < total; idx += kGemvThreads) {
     const int m = idx / G, grp = idx - m * G;
-    const float4* xr = reinterpret_cast<const float4*>(p.x + (int64_t)m * p.K) + 4 * grp;
+    const float4* xr = reinterpret_cast<const float4*>(P.x + (int64_t)m * P.K) + 4 * grp;
     float a = 0.0f;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float4 v = __ldg(xr + j);
       a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
     }
-    atomicMax(&s_amax[m], __float_as_uint(a));
+    atomicMax(&s_amax[m], __float_as_uint(a));  // non-negative floats order as their bit patterns
   }
   __syncthreads();
-  // ---- pass 2: quantise into shared memory in the permuted order, row sums
   for (int idx = tid; idx < total; idx += kGemvThreads) {
     const int m = idx / G, grp = idx - m * G;
     const float sx = __fdiv_rn(kQmax, fmaxf(__uint_as_float(s_amax[m]), kFloor));
-    const float4* xr = reinterpret_cast<const float4*>(p.x + (int64_t)m * p.K) + 4 * grp;
+    const float4* xr = reinterpret_cast<const float4*>(P.x + (int64_t)m * P.K) + 4 * grp;
     int v[16];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
@@ -143,151 +161,362 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const GemvParams p) 
     }
 #pragma unroll
     for (int j = 0; j < 16; ++j) rs += v[j];
-    *reinterpret_cast<uint4*>(sq + (int64_t)m * p.q_stride + 16 * grp) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-    atomicAdd(&s_rsum[m], rs);
+    *reinterpret_cast<uint4*>(sq + (int64_t)m * P.q_stride + 16 * grp) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    atomicAdd(&s_rs[m], rs);
     if (grp == 0) s_sx[m] = sx;
   }
   __syncthreads();
+}
 
-  // ---- main loop over 256-code units
-  int acc[4][MT][4];
-#pragma unroll
-  for (int c = 0; c < 4; ++c)
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) acc[c][mt][i] = 0;
-
-  for (int base = 0; ks + base * nks < p.n_units; base += kRing) {
-#pragma unroll
-    for (int i = 0; i < kRing; ++i) {
-      const int u = ks + (base + i) * nks;
-      if (u >= p.n_units) break;
-      uint4 Q[MT][4];
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        const int tok = g + 8 * mt;
-        if (tok < p.M) {
-          const uint8_t* qp = sq + (int64_t)tok * p.q_stride + 16 * (u * 16 + 4 * t);
-#pragma unroll
-          for (int i4 = 0; i4 < 4; ++i4) Q[mt][i4] = *reinterpret_cast<const uint4*>(qp + 16 * i4);
-        } else {
-#pragma unroll
-          for (int i4 = 0; i4 < 4; ++i4) Q[mt][i4] = make_uint4(0u, 0u, 0u, 0u);
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint32_t mask = 0x03030303u << (2 * c);
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const uint32_t a0 = wa[i][2 * h] & mask, a2 = wa[i][2 * h + 1] & mask;
-          const uint32_t a1 = wb[i][2 * h] & mask, a3 = wb[i][2 * h + 1] & mask;
-#pragma unroll
-          for (int mt = 0; mt < MT; ++mt) {
-            const uint4& q0 = Q[mt][2 * h];
-            const uint4& q1 = Q[mt][2 * h + 1];
-            const uint32_t b0 = c == 0 ? q0.x : (c == 1 ? q0.y : (c == 2 ? q0.z : q0.w));
-            const uint32_t b1 = c == 0 ? q1.x : (c == 1 ? q1.y : (c == 2 ? q1.z : q1.w));
-            mma_u8s8(acc[c][mt], a0, a1, a2, a3, b0, b1);
-          }
-        }
-      }
-      // Refill this ring slot with the unit kRing positions further on.
-      const int un = u + kRing * nks;
-      load_unit<kAligned>(rowpA, validA && un < p.n_units, un * 16 + 4 * t, p.wpr, wa[i]);
-      load_unit<kAligned>(rowpB, validB && un < p.n_units, un * 16 + 4 * t, p.wpr, wb[i]);
-    }
-  }
-
-  // ---- recombine the four classes (exact) and reduce over the K-split warps
+// Add a warp's partial sums for one 16-row tile into the tile's shared block.
+// The four classes are recombined exactly: class c holds 4^c * sum q*(code+1).
+template <int MT, int DA>
+__device__ __forceinline__ void flush_tile(const int (&acc)[4][DA][MT][4], int* dst, int g, int t) {
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = acc[0][mt][i] + (acc[1][mt][i] >> 2) + (acc[2][mt][i] >> 4) + (acc[3][mt][i] >> 6);
-      s_red[(warp * 32 + lane) * (4 * MT) + mt * 4 + i] = r;
+    for (int q = 0; q < 4; ++q) {
+      int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+#pragma unroll
+      for (int d = 0; d < DA; ++d) {
+        c0 += acc[0][d][mt][q];
+        c1 += acc[1][d][mt][q];
+        c2 += acc[2][d][mt][q];
+        c3 += acc[3][d][mt][q];
+      }
+      const int v = c0 + (c1 >> 2) + (c2 >> 4) + (c3 >> 6);
+      const int row = g + 8 * (q >> 1), tok = 8 * mt + 2 * t + (q & 1);
+      atomicAdd(dst + row * 8 * MT + tok, v);
     }
-  __syncthreads();
+}
 
-  const int rows_cta = 16 * R;
-  const int outs = rows_cta * p.M;
-  for (int idx = tid; idx < outs; idx += kGemvThreads) {
-    const int tok = idx / rows_cta;
-    const int rr = idx - tok * rows_cta;
-    const int rt2 = rr >> 4, r16 = rr & 15;
-    const int64_t row = ((int64_t)blockIdx.x * R + rt2) * 16 + r16;
-    if (row >= p.N) continue;
-    const int gg = r16 & 7, half = r16 >> 3;
-    const int mt = tok >> 3, col = tok & 7;
-    const int ln = gg * 4 + (col >> 1);
-    const int reg = mt * 4 + half * 2 + (col & 1);
-    int sum = 0;
-    for (int k2 = 0; k2 < nks; ++k2) sum += s_red[((rt2 + R * k2) * 32 + ln) * (4 * MT) + reg];
-    const int a = sum - s_rsum[tok];
-    if (kAccOut)
-      p.acc_out[(int64_t)tok * p.N + row] = a;
-    else
-      p.y[(int64_t)tok * p.N + row] = rescale(a, s_sx[tok], __ldg(p.D + row));
+template <int MT, bool kAccOut>
+__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constant__ GemvLaunch L) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int RT = L.round_tiles;                                           // tiles per round buffer
+  uint8_t* bufs = smem;                                                   // [nbuf][buf_bytes]
+  uint8_t* sq = smem + (size_t)L.nbuf * L.buf_bytes;
+  float* s_sx = reinterpret_cast<float*>(sq + L.q_bytes);                 // [16]
+  int32_t* s_rs = reinterpret_cast<int32_t*>(s_sx + 16);                  // [16]
+  uint32_t* s_amax = reinterpret_cast<uint32_t*>(s_rs + 16);              // [16]
+  int32_t* s_acc = reinterpret_cast<int32_t*>(s_amax + 16);               // [RT][16 rows][8*MT tokens]
+  uint64_t* full = reinterpret_cast<uint64_t*>(s_acc + (size_t)RT * 16 * 8 * MT);  // [nbuf][RT]
+  uint32_t* s_off = reinterpret_cast<uint32_t*>(full + (size_t)L.nbuf * RT);       // [nbuf][RT] tile offsets
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(s_off + (size_t)L.nbuf * RT);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int c = blockIdx.x;
+  const int t0 = L.cta_start[c];
+  const int nt = L.cta_start[c + 1] - t0;
+  const int nrounds = (nt + RT - 1) / RT;
+
+  if (tid == 0) {
+    for (int s = 0; s < L.nbuf * RT; ++s) mbar_init(&full[s], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  // Issue every copy of round r into buffer r % nbuf (one thread). Tiles are
+  // packed by size; the offset table is written before each tile's barrier
+  // arrival, so a reader that has waited on the barrier sees it.
+  auto issue_round = [&](int r) {
+    const int b = r % L.nbuf;
+    const int a = r * RT, e = (a + RT < nt) ? a + RT : nt;
+    uint32_t off = 0;
+    for (int i = a; i < e; ++i) {
+      s_off[b * RT + (i - a)] = off;
+      issue_tile(L, t0 + i, bufs + (size_t)b * L.buf_bytes + off, &full[b * RT + (i - a)]);
+      off += tile_slot_bytes(L, t0 + i);
+    }
+  };
+  int issued = 0;  // rounds issued (thread 0)
+  if (tid == 0) {
+    // Dependents may be scheduled as soon as every CTA of this grid is running.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    for (int r = 0; r < L.nbuf && r < nrounds; ++r) {
+      issue_round(r);
+      issued = r + 1;
+    }
+  }
+  // Everything below reads activations or writes outputs: wait for the grid
+  // this launch depends on (returns at once without programmatic dependence).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  if (tid == 0 && c == 0 && L.err != nullptr) *L.err = 0u;
+
+  int cur = -1;
+  for (int r = 0; r < nrounds; ++r) {
+    const int b = r % L.nbuf;
+    const uint32_t ph = (uint32_t)(r / L.nbuf) & 1u;
+    const int ra = r * RT, re = (ra + RT < nt) ? ra + RT : nt;
+    // One segment per problem met in this round.
+    for (int sa = ra; sa < re;) {
+      __syncthreads();  // the previous segment's output loop is done with s_rs / s_sx / sq
+      const int p = problem_of(L, t0 + sa);
+      const GemvProblem& P = L.pr[p];
+      int se = P.tile0 + P.tiles - t0;
+      se = se < re ? se : re;
+      if (p != cur) {
+        quantise_x(P, sq, s_sx, s_rs, s_amax);  // block-wide, ends with a barrier
+        cur = p;
+      }
+      for (int i = tid; i < (se - sa) * 16 * 8 * MT; i += kGemvThreads) s_acc[(sa - ra) * 16 * 8 * MT + i] = 0;
+      __syncthreads();
+      // Flat (tile, unit) tasks of this segment; warp w takes tasks w, w+8, ...
+      const int ntask = (se - sa) * P.n_units;
+      const bool al = (P.wpr & 3) == 0;
+      int ti = 0, u = warp;  // tile index within the segment, unit
+      while (u >= P.n_units) {
+        u -= P.n_units;
+        ++ti;
+      }
+      // Separate accumulators per (class, half) give 4*DA independent MMA chains.
+      constexpr int DA = MT == 1 ? 2 : 1;
+      int acc[4][DA][MT][4];
+      int acc_tile = -1;
+      for (int task = warp; task < ntask; task += kGemvWarps) {
+        const int li = sa - ra + ti;  // tile slot in the round buffer
+        if (acc_tile != ti) {
+          if (acc_tile >= 0) flush_tile<MT, DA>(acc, s_acc + (size_t)(sa - ra + acc_tile) * 16 * 8 * MT, g, t);
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int d = 0; d < DA; ++d)
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) acc[cc][d][mt][q] = 0;
+          acc_tile = ti;
+          int ok = 1;
+          if (lane == 0) ok = mbar_wait(&full[b * RT + li], ph, abort_flag, L.err, kDevTimeoutProducer) ? 1 : 0;
+          ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+          if (!ok) break;
+        }
+        const uint32_t* tile = reinterpret_cast<const uint32_t*>(bufs + (size_t)b * L.buf_bytes + s_off[b * RT + li]);
+        const int w0 = u * 16 + 4 * t;
+        uint32_t wa[4], wb[4];
+        if (al && w0 + 4 <= P.wpr) {
+          const uint4 va = *reinterpret_cast<const uint4*>(tile + g * P.wpr + w0);
+          const uint4 vb = *reinterpret_cast<const uint4*>(tile + (g + 8) * P.wpr + w0);
+          wa[0] = va.x; wa[1] = va.y; wa[2] = va.z; wa[3] = va.w;
+          wb[0] = vb.x; wb[1] = vb.y; wb[2] = vb.z; wb[3] = vb.w;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const bool in = w0 + j < P.wpr;  // words past the row belong to the next row: zero them
+            wa[j] = in ? tile[g * P.wpr + w0 + j] : 0u;
+            wb[j] = in ? tile[(g + 8) * P.wpr + w0 + j] : 0u;
+          }
+        }
+        uint4 Q[MT][4];
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const int tok = g + 8 * mt;
+          if (tok < P.M) {
+            const uint8_t* qp = sq + (int64_t)tok * P.q_stride + 16 * w0;
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) Q[mt][i4] = *reinterpret_cast<const uint4*>(qp + 16 * i4);
+          } else {
+#pragma unroll
+            for (int i4 = 0; i4 < 4; ++i4) Q[mt][i4] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const uint32_t mask = 0x03030303u << (2 * cc);
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t a0 = wa[2 * h] & mask, a2 = wa[2 * h + 1] & mask;
+            const uint32_t a1 = wb[2 * h] & mask, a3 = wb[2 * h + 1] & mask;
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              const uint4& q0 = Q[mt][2 * h];
+              const uint4& q1 = Q[mt][2 * h + 1];
+              const uint32_t b0 = cc == 0 ? q0.x : (cc == 1 ? q0.y : (cc == 2 ? q0.z : q0.w));
+              const uint32_t b1 = cc == 0 ? q1.x : (cc == 1 ? q1.y : (cc == 2 ? q1.z : q1.w));
+              mma_u8s8(acc[cc][h % DA][mt], a0, a1, a2, a3, b0, b1);
+            }
+          }
+        }
+        u += kGemvWarps;
+        while (u >= P.n_units) {
+          u -= P.n_units;
+          ++ti;
+        }
+      }
+      if (acc_tile >= 0) flush_tile<MT, DA>(acc, s_acc + (size_t)(sa - ra + acc_tile) * 16 * 8 * MT, g, t);
+      __syncthreads();
+      if (*abort_flag) {
+        // Block-uniform after the barrier. Let the copies already issued land
+        // before the CTA exits.
+        if (tid == 0) {
+          for (int rr = r; rr < issued; ++rr) {
+            const int bb = rr % L.nbuf, na = (rr * RT + RT < nt ? RT : nt - rr * RT);
+            for (int li = 0; li < na; ++li)
+              mbar_wait(&full[bb * RT + li], (uint32_t)(rr / L.nbuf) & 1u, nullptr, L.err, kDevTimeoutDrain,
+                        100000000ull);
+          }
+        }
+        return;
+      }
+      // Outputs of this segment: rows x tokens, coalesced along the rows.
+      const int nout = (se - sa) * 16 * P.M;
+      for (int idx = tid; idx < nout; idx += kGemvThreads) {
+        const int tok = idx / ((se - sa) * 16);
+        const int rr = idx - tok * (se - sa) * 16;
+        const int ti2 = rr >> 4, r16 = rr & 15;
+        const int64_t row = (int64_t)(t0 + sa + ti2 - P.tile0) * 16 + r16;
+        if (row >= P.N) continue;
+        const int a = s_acc[((size_t)(sa - ra + ti2) * 16 + r16) * 8 * MT + tok] - s_rs[tok];
+        if (kAccOut)
+          P.acc[(int64_t)tok * P.N + row] = a;
+        else
+          P.y[(int64_t)tok * P.N + row] = rescale(a, s_sx[tok], __ldg(P.D + row));
+      }
+      sa = se;
+    }
+    __syncthreads();
+    // This round's buffer is consumed: start the round that reuses it.
+    if (tid == 0 && r + L.nbuf < nrounds) {
+      issue_round(r + L.nbuf);
+      issued = r + L.nbuf + 1;
+    }
   }
 }
 
-template <int MT, bool kAligned, bool kAccOut>
-static cudaError_t launch_gemv_t(const GemvParams& p, int grid, size_t smem, cudaStream_t stream) {
-  auto kern = gemv_kernel<MT, kAligned, kAccOut>;
+template <int MT, bool kAccOut>
+static cudaError_t launch_gemv_t(const GemvLaunch& L, int grid, size_t smem, bool pdl, cudaStream_t stream) {
+  auto kern = gemv_kernel<MT, kAccOut>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  kern<<<grid, kGemvThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemvThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, L);
 }
 
-cudaError_t launch_gemv(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
-                        const float* D, float* y, int32_t* acc_out, uint32_t* err_reset, cudaStream_t stream,
-                        int num_sms) {
-  GemvParams p;
-  p.err_reset = err_reset;
-  p.x = x;
-  p.packed = packed;
-  p.D = D;
-  p.y = y;
-  p.acc_out = acc_out;
-  p.M = (int)M;
-  p.N = N;
-  p.K = (int)K;
-  p.wpr = (int)(K / 16);
-  p.n_units = (p.wpr + 15) / 16;
-  p.q_stride = (int)gemv_q_stride(K);
-  // Rows per CTA: as many 16-row tiles as keep every warp within kRing units
-  // (so all of its loads are in flight at once) while the grid still covers
-  // every SM; more rows per CTA amortise the per-CTA quantisation of x.
-  const int64_t tiles = (N + 15) / 16;
-  p.R = 1;
-  for (int r : {4, 2}) {
-    const int units_per_warp = (p.n_units * r + kGemvWarps - 1) / kGemvWarps;
-    if (units_per_warp <= kRing && (tiles + r - 1) / r >= num_sms) {
-      p.R = r;
-      break;
+static size_t gemv_smem_bytes(const GemvLaunch& L, int MT) {
+  return (size_t)L.nbuf * L.buf_bytes + L.q_bytes + 3 * 16 * 4 + (size_t)L.round_tiles * 16 * 8 * MT * 4 +
+         (size_t)L.nbuf * L.round_tiles * (8 + 4) + 16;
+}
+
+// Shared-memory bytes of launch tile gt (rows x K/4 rounded up to 128 B).
+static int64_t host_tile_bytes(const GemvLaunch& L, int gt) {
+  int p = 0;
+  while (p + 1 < L.nprob && gt >= L.pr[p + 1].tile0) ++p;
+  const GemvProblem& P = L.pr[p];
+  const int64_t row0 = (int64_t)(gt - P.tile0) * 16;
+  const int64_t rows = P.N - row0 < 16 ? P.N - row0 : 16;
+  return (rows * P.wpr * 4 + 127) / 128 * 128;
+}
+
+// Split the launch's tiles into `grid` contiguous ranges of about equal bytes
+// (problems of different K have tiles of different size). Returns the largest
+// range in bytes and the largest range in tiles.
+static void partition_by_bytes(GemvLaunch& L, int grid, int64_t* max_bytes, int* max_tiles) {
+  int64_t total = 0;
+  for (int gt = 0; gt < L.total_tiles; ++gt) total += host_tile_bytes(L, gt);
+  int64_t acc = 0, best_b = 0, cur_b = 0;
+  int c = 0, best_t = 0, start = 0;
+  L.cta_start[0] = 0;
+  for (int gt = 0; gt < L.total_tiles; ++gt) {
+    const int64_t tb = host_tile_bytes(L, gt);
+    // Close CTA c once it holds its share, keeping at least one tile for each later CTA.
+    const int64_t target = total * (c + 1) / grid;
+    if (c + 1 < grid && gt > start && acc + tb / 2 > target && L.total_tiles - gt >= grid - c - 1) {
+      best_b = cur_b > best_b ? cur_b : best_b;
+      best_t = gt - start > best_t ? gt - start : best_t;
+      L.cta_start[++c] = gt;
+      start = gt;
+      cur_b = 0;
     }
+    acc += tb;
+    cur_b += tb;
   }
-  const int64_t grid = (tiles + p.R - 1) / p.R;
-  const int MT = M <= 8 ? 1 : 2;
-  const size_t smem = (size_t)M * p.q_stride + 3 * 16 * 4 + (size_t)kGemvWarps * 32 * 4 * MT * 4;
-  const bool aligned = (p.wpr % 4) == 0;
-  const bool accout = acc_out != nullptr;
-#define BL_GEMV_CASE(MT_, AL_, AO_) \
-  if (MT == MT_ && aligned == AL_ && accout == AO_) return launch_gemv_t<MT_, AL_, AO_>(p, (int)grid, smem, stream);
-  BL_GEMV_CASE(1, true, false)
-  BL_GEMV_CASE(1, false, false)
-  BL_GEMV_CASE(2, true, false)
-  BL_GEMV_CASE(2, false, false)
-  BL_GEMV_CASE(1, true, true)
-  BL_GEMV_CASE(1, false, true)
-  BL_GEMV_CASE(2, true, true)
-  BL_GEMV_CASE(2, false, true)
-#undef BL_GEMV_CASE
-  return cudaErrorInvalidValue;
+  best_b = cur_b > best_b ? cur_b : best_b;
+  best_t = L.total_tiles - start > best_t ? L.total_tiles - start : best_t;
+  // Any CTA left without tiles gets an empty range.
+  for (int k = c + 1; k <= grid; ++k) L.cta_start[k] = L.total_tiles;
+  *max_bytes = best_b;
+  *max_tiles = best_t;
+}
+
+int64_t gemv_stage_bytes(int64_t K) { return ((16 * (K / 4)) + 127) / 128 * 128; }
+
+bool gemv_group_fits(int64_t maxM, int64_t maxK) {
+  if (maxM > kGemvMaxM) return false;
+  const int64_t q = (maxM * gemv_q_stride(maxK) + 127) / 128 * 128;
+  return q + 2 * gemv_stage_bytes(maxK) + 16 * 1024 <= kGemvMaxSmem;
+}
+
+cudaError_t launch_gemv_group(const GemvCall* calls, int n, uint32_t* err, bool pdl, cudaStream_t stream,
+                              int num_sms) {
+  if (n < 1 || n > kGemvMaxGroup) return cudaErrorInvalidValue;
+  GemvLaunch L;
+  std::memset(&L, 0, sizeof(L));
+  int64_t maxM = 0, maxK = 0;
+  int tiles = 0;
+  for (int i = 0; i < n; ++i) {
+    GemvProblem& P = L.pr[i];
+    P.x = calls[i].x;
+    P.packed = calls[i].packed;
+    P.D = calls[i].D;
+    P.y = calls[i].y;
+    P.acc = calls[i].acc;
+    P.M = (int)calls[i].M;
+    P.N = (int)calls[i].N;
+    P.K = (int)calls[i].K;
+    P.wpr = P.K / 16;
+    P.n_units = (P.wpr + 15) / 16;
+    P.tiles = (P.N + 15) / 16;
+    P.tile0 = tiles;
+    P.q_stride = (int)gemv_q_stride(P.K);
+    tiles += P.tiles;
+    maxM = calls[i].M > maxM ? calls[i].M : maxM;
+    maxK = calls[i].K > maxK ? calls[i].K : maxK;
+  }
+  L.nprob = n;
+  L.total_tiles = tiles;
+  L.err = err;
+  L.stage_bytes = (int)gemv_stage_bytes(maxK);
+  L.q_bytes = (int)((maxM * gemv_q_stride(maxK) + 127) / 128 * 128);
+  const int MT = maxM <= 8 ? 1 : 2;
+  int grid0 = tiles < num_sms ? tiles : num_sms;
+  if (grid0 > kGemvMaxGrid) grid0 = kGemvMaxGrid;
+  int64_t cta_bytes = 0;
+  int per_cta = 0;
+  partition_by_bytes(L, grid0, &cta_bytes, &per_cta);
+  // Per tile slot: its partial-sum block, barrier and offset entry.
+  const int64_t slot_extra = 16 * 8 * MT * 4 + 8 + 4;
+  const int64_t fixed = L.q_bytes + 3 * 16 * 4 + 16;
+  if (fixed + cta_bytes + per_cta * slot_extra <= kGemvMaxSmem) {
+    L.nbuf = 1;  // every tile of a CTA in flight at once
+    L.round_tiles = per_cta;
+    L.buf_bytes = (int)cta_bytes;
+  } else {
+    L.nbuf = 2;
+    int64_t rt = (kGemvSmemTarget - fixed) / (2 * (L.stage_bytes + slot_extra));
+    if (rt < 1) rt = 1;
+    L.round_tiles = (int)rt;
+    L.buf_bytes = (int)(rt * L.stage_bytes);
+  }
+  const size_t smem = gemv_smem_bytes(L, MT);
+  if ((int64_t)smem > kGemvMaxSmem) return cudaErrorInvalidValue;
+  const int grid = grid0;
+  const bool accout = calls[0].acc != nullptr;
+  if (MT == 1) return accout ? launch_gemv_t<1, true>(L, grid, smem, pdl, stream)
+                             : launch_gemv_t<1, false>(L, grid, smem, pdl, stream);
+  return accout ? launch_gemv_t<2, true>(L, grid, smem, pdl, stream) : launch_gemv_t<2, false>(L, grid, smem, pdl, stream);
 }
 
 }  // namespace bl

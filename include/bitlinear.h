@@ -156,6 +156,41 @@ BL_API int bitlinear_forward_prepared(int64_t M, int64_t N, int64_t K,
                                       const uint32_t* packed, const float* D, float* y,
                                       void* ws, size_t ws_bytes, bl_stream_t stream);
 
+/* ---------------------------------------------------------------- batch --- */
+
+/* One BitLinear of a batch: y [M,N] = F.linear(ActQuant(x [M,K]), W) from
+ * packed [N, K/16] and D [N] (same meaning and layout as bitlinear_forward). */
+typedef struct {
+  const float* x;
+  int64_t M;
+  int64_t N;
+  int64_t K;
+  const uint32_t* packed;
+  const float* D;
+  float* y;
+} bl_linear_call;
+
+/* Flag for bitlinear_forward_batch: the packed weights and D of the calls are
+ * not written by the work enqueued on `stream` just before the batch (as in a
+ * decode loop, where weights are static). The decode kernels may then start
+ * streaming them while that work still runs (programmatic dependent launch);
+ * activations are still read only after it has finished. */
+#define BL_FLAG_STREAM_WEIGHTS_EARLY 1u
+
+/* Bytes of scratch for bitlinear_forward_batch: the largest
+ * bitlinear_workspace_size of its calls. */
+BL_API size_t bitlinear_batch_workspace_size(const bl_linear_call* calls, int count);
+
+/* Runs `count` independent BitLinears, in order, on `stream`. Consecutive
+ * decode-sized calls (M <= 16) are fused into one launch of up to 8 calls
+ * (one persistent kernel streams all of their packed weights); other calls
+ * run through the tensor-core path one at a time. No output may overlap any
+ * input or another output of the same batch. A one-call batch without flags
+ * is the same as bitlinear_forward. Errors of any call are reported before
+ * anything is launched. Asynchronous. */
+BL_API int bitlinear_forward_batch(const bl_linear_call* calls, int count, uint32_t flags,
+                                   void* ws, size_t ws_bytes, bl_stream_t stream);
+
 /* Scratch for bitlinear_forward_host: the forward workspace plus room for x
  * and y on the device. */
 BL_API size_t bitlinear_host_workspace_size(int64_t M, int64_t N, int64_t K);

@@ -94,3 +94,16 @@ def test_product_path_does_not_import_oracle():
                 with open(os.path.join(dirpath, fn)) as f:
                     src = f.read()
                 assert "import oracle" not in src and "from oracle" not in src, fn
+
+
+def test_batch_validation_before_cuda(L):
+    calls = (_lib.LinearCall * 2)()
+    calls[0] = _lib.LinearCall(FAKE, 1, 8, 64, FAKE, FAKE, FAKE)
+    calls[1] = _lib.LinearCall(FAKE, 1, 8, 24, FAKE, FAKE, FAKE)  # K % 16 != 0
+    assert L.bitlinear_forward_batch(calls, 2, 0, FAKE, 1 << 20, None) == 2
+    calls[1] = _lib.LinearCall(None, 1, 8, 64, FAKE, FAKE, FAKE)
+    assert L.bitlinear_forward_batch(calls, 2, 0, FAKE, 1 << 20, None) == 1
+    calls[1] = _lib.LinearCall(FAKE, 1, 8, 64, FAKE, FAKE, FAKE)
+    assert L.bitlinear_forward_batch(calls, 2, 0x80, FAKE, 1 << 20, None) == 2  # unknown flag
+    assert L.bitlinear_forward_batch(calls, 0, 0, None, 0, None) == 0
+    assert L.bitlinear_batch_workspace_size(calls, 2) == 256 + 256 + 256 + 256  # header, s_x, sums, q

@@ -312,3 +312,59 @@ def test_bounded_wait_reports_device_error(B):
     assert int(ws[:4].view(torch.int32).item()) == 0  # cleared by the read
     assert L.bitlinear_workspace_error(ws.data_ptr(), ws.numel(), stream) == 0
     run_case(B, 2, 40, 64, seed=3)  # the context still works
+
+
+# ------------------------------------------------------------ batched calls
+def _oracle_y(W, x):
+    p_ref, D_ref = O.pack_weights(W)
+    return O.bitlinear_forward(x, p_ref, D_ref, W.shape[1])
+
+
+@pytest.mark.parametrize("flags", [0, 1])
+def test_forward_batch_grouped_matches_oracle(B, flags):
+    """Decode-sized calls of different shapes fused into grouped launches, with
+    a tensor-core call in the middle and a group split by the 8-call limit."""
+    shapes = [(1, 3840, 2560), (1, 2560, 2560), (2, 100, 528), (1, 13824 // 8, 2560), (3, 257, 6912),
+              (40, 300, 512),  # tensor-core path in the middle
+              (1, 33, 48), (16, 64, 1152), (1, 17, 16), (1, 500, 1024), (1, 64, 64), (5, 31, 4304),
+              (1, 48, 256), (2, 129, 2560)]
+    calls, refs = [], []
+    for i, (M, N, K) in enumerate(shapes):
+        W = WL.weight(N, K, "normal", 500 + i)
+        x = WL.activations(M, K, "student_t", 600 + i, meta={"df": 3.0})
+        packed, D = B.pack_weights(dev(W))
+        calls.append((dev(x), packed, D, None))
+        refs.append(_oracle_y(W, x))
+    outs = B.forward_batch(calls, flags=flags)
+    torch.cuda.synchronize()
+    for y, ref in zip(outs, refs):
+        assert_y_close(y.cpu().numpy(), ref)
+
+
+def test_forward_batch_chain_with_early_weights(B):
+    """A dependent chain (each call's x is the previous call's y) with the
+    early-weights flag: activations must still be read only after the
+    previous kernel finished."""
+    K = 2560
+    Ws = [WL.weight(K, K, "normal", 700 + i) for i in range(4)]
+    packs = [B.pack_weights(dev(W)) for W in Ws]
+    x0 = WL.activations(1, K, "normal", 7)
+    xd = dev(x0)
+    for (packed, D) in packs:
+        (xd,) = B.forward_batch([(xd, packed, D, None)], flags=1)
+    torch.cuda.synchronize()
+    ref = x0
+    for W in Ws:
+        ref = _oracle_y(W, ref)
+    assert_y_close(xd.cpu().numpy(), ref)
+
+
+def test_forward_batch_rejects_before_launch(B):
+    from bit_ternary_b200._lib import BitLinearError
+
+    W = WL.weight(64, 64, "normal", 1)
+    packed, D = B.pack_weights(dev(W))
+    good = (dev(np.ones((1, 64), np.float32)), packed, D, None)
+    bad_y = torch.zeros(1 * 64 + 1, device="cuda")[1:].view(1, 64)
+    with pytest.raises(BitLinearError, match="ALIGN"):
+        B.forward_batch([good, (good[0], packed, D, bad_y)])
