@@ -269,6 +269,81 @@ cudaError_t launch_selftest_wait(uint32_t* err, uint64_t limit_ns, cudaStream_t 
   return cudaGetLastError();
 }
 
+// Register-resident variant for rows of up to 256 * 16 * kG columns: each
+// thread loads its kG groups of 16 values once, the block reduces max|x|, and
+// the same registers are quantised and stored (one read of x, one write of q).
+template <bool kPerm, int kG>
+__global__ void __launch_bounds__(256) act_quant_reg_kernel(const float* __restrict__ x, int64_t K,
+                                                            int8_t* __restrict__ q, float* __restrict__ s_out,
+                                                            int32_t* __restrict__ rowsum_out,
+                                                            uint32_t* __restrict__ err_reset) {
+  __shared__ float red_f[8];
+  __shared__ int red_i[8];
+  if (err_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err_reset = 0u;
+  const int64_t m = blockIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(x + m * K);
+  const int ngroups = (int)(K >> 4);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  float4 f[kG][4];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kG; ++i) {
+    const int g = threadIdx.x + i * blockDim.x;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) f[i][j] = g < ngroups ? __ldg(xr + 4 * g + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f[i][j].x), fabsf(f[i][j].y)), fmaxf(fabsf(f[i][j].z), fabsf(f[i][j].w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if (lane == 0) red_f[warp] = amax;
+  __syncthreads();
+  amax = 0.0f;
+  for (int w = 0; w < nwarps; ++w) amax = fmaxf(amax, red_f[w]);
+  const float sx = __fdiv_rn(kQmax, fmaxf(amax, kFloor));
+  int rsum = 0;
+  int8_t* qr = q + m * K;
+#pragma unroll
+  for (int i = 0; i < kG; ++i) {
+    const int g = threadIdx.x + i * blockDim.x;
+    if (g >= ngroups) continue;
+    int v[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[4 * j + 0] = quant_i8(f[i][j].x, sx);
+      v[4 * j + 1] = quant_i8(f[i][j].y, sx);
+      v[4 * j + 2] = quant_i8(f[i][j].z, sx);
+      v[4 * j + 3] = quant_i8(f[i][j].w, sx);
+    }
+    uint32_t w4[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      uint32_t word = 0u;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int p = 4 * r + b;
+        word |= (uint32_t)(v[kPerm ? perm16(p) : p] & 0xFF) << (8 * b);
+      }
+      w4[r] = word;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) rsum += v[j];
+    *reinterpret_cast<uint4*>(qr + 16 * (int64_t)g) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) rsum += __shfl_xor_sync(0xFFFFFFFFu, rsum, o);
+  if (lane == 0) red_i[warp] = rsum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int w = 0; w < nwarps; ++w) tot += red_i[w];
+    s_out[m] = sx;
+    if (rowsum_out != nullptr) rowsum_out[m] = tot;
+  }
+}
+
 // ------------------------------------------------------------ launchers --
 cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
                         cudaStream_t stream, int num_sms) {
@@ -293,8 +368,22 @@ cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* packed, 
 cudaError_t launch_act_quant(const float* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
                              bool permuted, cudaStream_t stream, uint32_t* err_reset) {
   const int64_t ngroups = K / 16;
-  int threads = (int)(ngroups < 256 ? ((ngroups + 31) / 32) * 32 : 256);
-  if (threads < 32) threads = 32;
+  // Rows of up to 256 threads x 4 groups x 16 values stay in registers.
+  int kg = (int)((ngroups + 255) / 256);
+  if (kg <= 4) {
+    kg = kg <= 1 ? 1 : (kg <= 2 ? 2 : 4);
+    int threads = (int)(((ngroups + kg - 1) / kg + 31) / 32 * 32);
+    if (threads < 32) threads = 32;
+#define BL_AQ(P, G) act_quant_reg_kernel<P, G><<<(unsigned)M, threads, 0, stream>>>(x, K, q, s_x, rowsum, err_reset)
+    if (permuted) {
+      if (kg == 1) BL_AQ(true, 1); else if (kg == 2) BL_AQ(true, 2); else BL_AQ(true, 4);
+    } else {
+      if (kg == 1) BL_AQ(false, 1); else if (kg == 2) BL_AQ(false, 2); else BL_AQ(false, 4);
+    }
+#undef BL_AQ
+    return cudaGetLastError();
+  }
+  const int threads = 256;
   // One CTA per token; grids beyond 2^31-1 are rejected by validation.
   if (permuted)
     act_quant_kernel<true><<<(unsigned)M, threads, 0, stream>>>(x, K, q, s_x, rowsum, err_reset);
