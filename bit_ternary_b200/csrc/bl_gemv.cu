@@ -6,24 +6,32 @@
 // D [N,1]), with the wrapper's ActQuant (section 1) done inside the kernel.
 //
 // Design (B200). The packed weights are the only large stream (2 bits per
-// weight). The grid is persistent: CTA c owns a contiguous, balanced range of
-// 16-row tiles over all problems of the launch. One thread issues
+// weight). The grid is persistent: CTA c owns a contiguous, byte-balanced
+// range of 16-row tiles over all problems of the launch. One thread issues
 // cp.async.bulk copies of whole tiles (16 rows x K/4 bytes, contiguous in
-// memory) into a ring of shared-memory stages the moment the CTA starts, so
-// every byte the CTA needs is in flight before x is even read. With
-// programmatic dependent launch the weight copies of this kernel may overlap
-// the kernel before it; the activations are read only after
-// griddepcontrol.wait.
+// memory) into shared memory the moment the CTA starts, and the row scales D
+// follow by cp.async, so every byte of weights the CTA needs is in flight
+// before x is read. A CTA needs at most ~100 KB of shared memory and 64
+// registers per thread for M <= 8, so two CTAs fit on an SM: under
+// programmatic dependent launch the next launch's CTAs become resident while
+// this one runs and stream their weights in the meantime; activations are read
+// only after griddepcontrol.wait.
 //
-// Math. A warp computes a 16-row tile on a K-slice; lane (g, t) =
-// (lane/4, lane%4) takes words 4t..4t+3 of each 256-code unit for rows g and
-// g+8. Unpacking is one AND per 4 codes: for class c in 0..3,
+// Quantise. Every CTA quantises x itself (x is small and L2-resident): a
+// thread takes one 16-column group, the per-token absmax is a warp reduction
+// plus one shared atomic per warp, and the codes are written as one 16-byte
+// store in the kernel-private column order (inside every 16 columns, position
+// 4c+b holds column 4b+c). Wider activations stride over float4s instead.
+//
+// Math. Lane (g, t) = (lane/4, lane%4) of a warp takes words 4t..4t+3 of each
+// 256-code unit for rows g and g+8 of a tile; warp w takes a contiguous range
+// of (tile, unit) tasks, so it flushes its sums to the tile's shared block once
+// per tile. Unpacking is one AND per 4 codes: for class c in 0..3,
 // word & (0x03030303 << 2c) leaves, in byte b, (code[4b+c]+1) << 2c. Those
 // bytes feed mma.sync.m16n8k32 (u8 weights x s8 activations) with one
 // accumulator set per class, recombined exactly as acc0 + acc1/4 + acc2/16 +
-// acc3/64. The activations are quantised per CTA into shared memory in the
-// matching order (inside every 16 columns, position 4c+b holds column 4b+c).
-// sum q*(code+1) - sum q gives the signed result.
+// acc3/64; only lanes of existing tokens load activations (the other MMA
+// columns are never read). sum q*(code+1) - sum q gives the signed result.
 #include "bl_internal.h"
 
 #include <cstring>
@@ -59,6 +67,7 @@ struct GemvLaunch {
   int nbuf;         // 1: all of a CTA's tiles in flight, packed by size; 2: double-buffered rounds
   int buf_bytes;    // capacity of one round buffer
   int q_bytes;
+  int xs_bytes;     // staging of fp32 activations between the absmax and the quantise
   uint32_t* err;
   int cta_start[kGemvMaxGrid + 1];  // CTA c owns launch tiles [cta_start[c], cta_start[c+1])
 };
@@ -104,69 +113,95 @@ __device__ __forceinline__ void issue_tile(const GemvLaunch& L, int gt, uint8_t*
   const int lt = gt - P.tile0;
   const int row0 = lt * 16;
   const int rows = P.N - row0 < 16 ? P.N - row0 : 16;
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(P.packed + (int64_t)row0 * P.wpr);
   const uint32_t bytes = (uint32_t)rows * (uint32_t)P.wpr * 4u;
   const uint32_t bulk = bytes & ~15u;
-  const uint8_t* src = reinterpret_cast<const uint8_t*>(P.packed + (int64_t)row0 * P.wpr);
   for (uint32_t o = bulk; o < bytes; o += 4)
     *reinterpret_cast<uint32_t*>(dst + o) = __ldg(reinterpret_cast<const uint32_t*>(src + o));
   mbar_arrive_expect_tx(bar, bulk);
   if (bulk) bulk_g2s(dst, src, bulk, bar);
 }
 
-// Quantise problem P's activations into shared memory (kernel-private column
-// order), with per-token scale and sum of codes. Block-wide.
-__device__ __forceinline__ void quantise_x(const GemvProblem& P, uint8_t* sq, float* s_sx, int32_t* s_rs,
-                                           uint32_t* s_amax) {
-  const int tid = threadIdx.x;
-  if (tid < 16) {
-    s_amax[tid] = 0u;
-    s_rs[tid] = 0;
-  }
-  __syncthreads();
-  const int G = P.K >> 4;
-  const int total = P.M * G;
-  for (int idx = tid; idx < total; idx += kGemvThreads) {
-    const int m = idx / G, grp = idx - m * G;
-    const float4* xr = reinterpret_cast<const float4*>(P.x + (int64_t)m * P.K) + 4 * grp;
-    float a = 0.0f;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float4 v = __ldg(xr + j);
-      a = fmaxf(a, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-    }
-    atomicMax(&s_amax[m], __float_as_uint(a));  // non-negative floats order as their bit patterns
-  }
-  __syncthreads();
-  for (int idx = tid; idx < total; idx += kGemvThreads) {
-    const int m = idx / G, grp = idx - m * G;
-    const float sx = __fdiv_rn(kQmax, fmaxf(__uint_as_float(s_amax[m]), kFloor));
-    const float4* xr = reinterpret_cast<const float4*>(P.x + (int64_t)m * P.K) + 4 * grp;
-    int v[16];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float4 f = __ldg(xr + j);
-      v[4 * j + 0] = quant_i8(f.x, sx);
-      v[4 * j + 1] = quant_i8(f.y, sx);
-      v[4 * j + 2] = quant_i8(f.z, sx);
-      v[4 * j + 3] = quant_i8(f.w, sx);
-    }
-    uint32_t w4[4];
-    int rs = 0;
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      uint32_t word = 0u;
-#pragma unroll
-      for (int b = 0; b < 4; ++b) word |= (uint32_t)(v[perm16(4 * r + b)] & 0xFF) << (8 * b);
-      w4[r] = word;
-    }
-#pragma unroll
-    for (int j = 0; j < 16; ++j) rs += v[j];
-    *reinterpret_cast<uint4*>(sq + (int64_t)m * P.q_stride + 16 * grp) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
-    atomicAdd(&s_rs[m], rs);
-    if (grp == 0) s_sx[m] = sx;
-  }
-  __syncthreads();
+// Activations of one problem are quantised per CTA into shared memory, in the
+// kernel-private column order, with per-token scale s_x and sum of codes.
+// Threads stride over the float4s of the row-major [M, K] block twice
+// (absmax, then quantise; the second pass hits L1), kXBatch float4 loads in
+// flight per thread. Element 4j+e of a
+// 16-column group (float4 j, lane e) goes to byte 4e+j of the group: the
+// order perm16 describes.
+
+constexpr int kXBatch = 4;
+
+__device__ __forceinline__ float absmax4(const float4 v) {
+  return fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
 }
+
+// Warp-aggregated shared atomics. The lanes of a warp usually hold one token,
+// and then one lane updates for all of them. tok < 0 marks an idle lane; idle
+// lanes are always the last ones of the warp. Called by all 32 lanes.
+__device__ __forceinline__ void warp_amax(uint32_t* s_amax, int tok, float a) {
+  const int t0 = __shfl_sync(0xFFFFFFFFu, tok, 0);
+  if (__all_sync(0xFFFFFFFFu, tok == t0 || tok < 0)) {
+    // non-negative floats order as their bit patterns
+    const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(a));
+    if ((threadIdx.x & 31) == 0 && t0 >= 0) atomicMax(&s_amax[t0], m);
+  } else if (tok >= 0) {
+    atomicMax(&s_amax[tok], __float_as_uint(a));
+  }
+}
+
+__device__ __forceinline__ void warp_rowsum(int32_t* s_rs, int tok, int s) {
+  const int t0 = __shfl_sync(0xFFFFFFFFu, tok, 0);
+  if (__all_sync(0xFFFFFFFFu, tok == t0 || tok < 0)) {
+    const int sum = __reduce_add_sync(0xFFFFFFFFu, s);
+    if ((threadIdx.x & 31) == 0 && t0 >= 0) atomicAdd(&s_rs[t0], sum);
+  } else if (tok >= 0) {
+    atomicAdd(&s_rs[tok], s);
+  }
+}
+
+// int8 code clamp(rint(RN(x*s_x)), -128, 127), rounding by the addition of
+// 1.5*2^23: for |v| < 2^22 the fp32 sum v + 1.5*2^23 lies in [2^23, 2^24),
+// where the spacing is 1, so the addition itself rounds v to the nearest
+// integer, ties to even, exactly as rint does; the integer is the difference
+// of the bit patterns. Larger or non-finite products take the conversion
+// instruction, so every input gives the same code as quant_i8.
+__device__ __forceinline__ int quant_i8_fast(float x, float s_x) {
+  const float v = __fmul_rn(x, s_x);
+  int q;
+  if (fabsf(v) < 4194304.0f)
+    q = __float_as_int(__fadd_rn(v, 12582912.0f)) - 0x4B400000;
+  else
+    q = __float2int_rn(v);
+  return q < -128 ? -128 : (q > 127 ? 127 : q);
+}
+
+// Quantise one float4 (token m, float4 column c4) into shared memory; returns
+// the sum of its four codes.
+__device__ __forceinline__ int quant_store4(uint8_t* sq, int q_stride, int m, int c4, const float4 f, float sx) {
+  const int q0 = quant_i8_fast(f.x, sx), q1 = quant_i8_fast(f.y, sx), q2 = quant_i8_fast(f.z, sx),
+            q3 = quant_i8_fast(f.w, sx);
+  uint8_t* dst = sq + (int64_t)m * q_stride + 16 * (c4 >> 2) + (c4 & 3);
+  dst[0] = (uint8_t)q0;
+  dst[4] = (uint8_t)q1;
+  dst[8] = (uint8_t)q2;
+  dst[12] = (uint8_t)q3;
+  return q0 + q1 + q2 + q3;
+}
+
+__device__ __forceinline__ float token_scale(const uint32_t* s_amax, int m) {
+  return __fdiv_rn(kQmax, fmaxf(__uint_as_float(s_amax[m]), kFloor));
+}
+
+// 4-byte asynchronous copy global -> shared (row scales), waited for with
+// cp.async.wait_all before the outputs are written.
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)),
+               "l"(__cvta_generic_to_global(src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Add a warp's partial sums for one 16-row tile into the tile's shared block.
 // The four classes are recombined exactly: class c holds 4^c * sum q*(code+1).
@@ -191,15 +226,18 @@ __device__ __forceinline__ void flush_tile(const int (&acc)[4][DA][MT][4], int* 
 }
 
 template <int MT, bool kAccOut>
-__global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constant__ GemvLaunch L) {
+__global__ void __launch_bounds__(kGemvThreads, MT == 1 ? 2 : 1) gemv_kernel(const __grid_constant__ GemvLaunch L) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int RT = L.round_tiles;                                           // tiles per round buffer
   uint8_t* bufs = smem;                                                   // [nbuf][buf_bytes]
   uint8_t* sq = smem + (size_t)L.nbuf * L.buf_bytes;
-  float* s_sx = reinterpret_cast<float*>(sq + L.q_bytes);                 // [16]
-  int32_t* s_rs = reinterpret_cast<int32_t*>(s_sx + 16);                  // [16]
-  uint32_t* s_amax = reinterpret_cast<uint32_t*>(s_rs + 16);              // [16]
-  int32_t* s_acc = reinterpret_cast<int32_t*>(s_amax + 16);               // [RT][16 rows][8*MT tokens]
+  float4* s_xs = reinterpret_cast<float4*>(sq + L.q_bytes);              // [xs_bytes / 16]
+  // Per-token state in two sets: consecutive problems of a CTA alternate.
+  float* s_sx = reinterpret_cast<float*>(sq + L.q_bytes + L.xs_bytes);    // [2][16]
+  int32_t* s_rs = reinterpret_cast<int32_t*>(s_sx + 32);                  // [2][16]
+  uint32_t* s_amax = reinterpret_cast<uint32_t*>(s_rs + 32);              // [2][16]
+  float* s_D = reinterpret_cast<float*>(s_amax + 32);                     // [RT * 16] row scales of the round
+  int32_t* s_acc = reinterpret_cast<int32_t*>(s_D + (size_t)RT * 16);     // [RT][16 rows][8*MT tokens]
   uint64_t* full = reinterpret_cast<uint64_t*>(s_acc + (size_t)RT * 16 * 8 * MT);  // [nbuf][RT]
   uint32_t* s_off = reinterpret_cast<uint32_t*>(full + (size_t)L.nbuf * RT);       // [nbuf][RT] tile offsets
   volatile int* abort_flag = reinterpret_cast<volatile int*>(s_off + (size_t)L.nbuf * RT);
@@ -217,6 +255,10 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
     *abort_flag = 0;
     fence_barrier_init();
   }
+  if (tid < 32) {
+    s_amax[tid] = 0u;
+    s_rs[tid] = 0;
+  }
   __syncthreads();
   // Issue every copy of round r into buffer r % nbuf (one thread). Tiles are
   // packed by size; the offset table is written before each tile's barrier
@@ -231,6 +273,19 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
       off += tile_slot_bytes(L, t0 + i);
     }
   };
+  // Row scales D of round r's tiles into s_D (all threads). The int32
+  // accumulator output has no D.
+  auto load_D = [&](int r) {
+    if (kAccOut) return;
+    const int a = r * RT, e = (a + RT < nt) ? a + RT : nt;
+    for (int i = tid; i < (e - a) * 16; i += kGemvThreads) {
+      const int gt = t0 + a + (i >> 4);
+      const GemvProblem& P = L.pr[problem_of(L, gt)];
+      const int row = (gt - P.tile0) * 16 + (i & 15);
+      if (row < P.N && P.D != nullptr) cp_async4(s_D + i, P.D + row);
+    }
+    cp_async_commit();
+  };
   int issued = 0;  // rounds issued (thread 0)
   if (tid == 0) {
     // Dependents may be scheduled as soon as every CTA of this grid is running.
@@ -240,112 +295,234 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
       issued = r + 1;
     }
   }
+  if (nrounds > 0) load_D(0);
   // Everything below reads activations or writes outputs: wait for the grid
   // this launch depends on (returns at once without programmatic dependence).
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0 && c == 0 && L.err != nullptr) *L.err = 0u;
 
-  int cur = -1;
+  int cur = -1, qs = 1;  // current problem and its per-token set
   for (int r = 0; r < nrounds; ++r) {
     const int b = r % L.nbuf;
     const uint32_t ph = (uint32_t)(r / L.nbuf) & 1u;
     const int ra = r * RT, re = (ra + RT < nt) ? ra + RT : nt;
+    if (r > 0) {
+      __syncthreads();  // the previous round's outputs are done with s_D, sq and s_acc
+      load_D(r);
+    }
     // One segment per problem met in this round.
     for (int sa = ra; sa < re;) {
-      __syncthreads();  // the previous segment's output loop is done with s_rs / s_sx / sq
+      if (sa != ra) __syncthreads();  // the previous segment's outputs are done with sq and s_acc
       const int p = problem_of(L, t0 + sa);
       const GemvProblem& P = L.pr[p];
       int se = P.tile0 + P.tiles - t0;
       se = se < re ? se : re;
-      if (p != cur) {
-        quantise_x(P, sq, s_sx, s_rs, s_amax);  // block-wide, ends with a barrier
-        cur = p;
-      }
-      for (int i = tid; i < (se - sa) * 16 * 8 * MT; i += kGemvThreads) s_acc[(sa - ra) * 16 * 8 * MT + i] = 0;
-      __syncthreads();
-      // Flat (tile, unit) tasks of this segment; warp w takes tasks w, w+8, ...
-      const int ntask = (se - sa) * P.n_units;
-      const bool al = (P.wpr & 3) == 0;
-      int ti = 0, u = warp;  // tile index within the segment, unit
-      while (u >= P.n_units) {
-        u -= P.n_units;
-        ++ti;
-      }
-      // Separate accumulators per (class, half) give 4*DA independent MMA chains.
-      constexpr int DA = MT == 1 ? 2 : 1;
-      int acc[4][DA][MT][4];
-      int acc_tile = -1;
-      for (int task = warp; task < ntask; task += kGemvWarps) {
-        const int li = sa - ra + ti;  // tile slot in the round buffer
-        if (acc_tile != ti) {
-          if (acc_tile >= 0) flush_tile<MT, DA>(acc, s_acc + (size_t)(sa - ra + acc_tile) * 16 * 8 * MT, g, t);
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-            for (int d = 0; d < DA; ++d)
-#pragma unroll
-              for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int q = 0; q < 4; ++q) acc[cc][d][mt][q] = 0;
-          acc_tile = ti;
-          int ok = 1;
-          if (lane == 0) ok = mbar_wait(&full[b * RT + li], ph, abort_flag, L.err, kDevTimeoutProducer) ? 1 : 0;
-          ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-          if (!ok) break;
+      const bool newp = p != cur;
+      const int K4 = P.K >> 2, total4 = P.M * K4;
+      const int G = P.K >> 4, ngroups = P.M * G;
+      // One 16-column group per thread, one read of x (staged in shared memory).
+      const bool greg = ngroups <= kGemvThreads && ngroups * 64 <= L.xs_bytes;
+      if (newp) {
+        // Per-token absmax. The other set is cleared for the problem after this one.
+        qs ^= 1;
+        if (tid < 16) {
+          s_amax[(qs ^ 1) * 16 + tid] = 0u;
+          s_rs[(qs ^ 1) * 16 + tid] = 0;
         }
-        const uint32_t* tile = reinterpret_cast<const uint32_t*>(bufs + (size_t)b * L.buf_bytes + s_off[b * RT + li]);
-        const int w0 = u * 16 + 4 * t;
-        uint32_t wa[4], wb[4];
-        if (al && w0 + 4 <= P.wpr) {
-          const uint4 va = *reinterpret_cast<const uint4*>(tile + g * P.wpr + w0);
-          const uint4 vb = *reinterpret_cast<const uint4*>(tile + (g + 8) * P.wpr + w0);
-          wa[0] = va.x; wa[1] = va.y; wa[2] = va.z; wa[3] = va.w;
-          wb[0] = vb.x; wb[1] = vb.y; wb[2] = vb.z; wb[3] = vb.w;
+        const float4* x4 = reinterpret_cast<const float4*>(P.x);
+        if (greg) {
+          // One 16-column group per thread (groups never straddle tokens).
+          int m = -1;
+          float a = 0.0f;
+          if (tid < ngroups) {
+            m = tid / G;
+            float4 xg[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) xg[j] = __ldg(x4 + 4 * tid + j);
+            a = fmaxf(fmaxf(absmax4(xg[0]), absmax4(xg[1])), fmaxf(absmax4(xg[2]), absmax4(xg[3])));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) s_xs[4 * tid + j] = xg[j];  // read back after the barrier
+          }
+          warp_amax(s_amax + qs * 16, m, a);
         } else {
+          for (int base = 0; base < total4; base += kXBatch * kGemvThreads) {
+            float a[kXBatch];  // all loads of the batch in flight before any reduction
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const bool in = w0 + j < P.wpr;  // words past the row belong to the next row: zero them
-            wa[j] = in ? tile[g * P.wpr + w0 + j] : 0u;
-            wb[j] = in ? tile[(g + 8) * P.wpr + w0 + j] : 0u;
-          }
-        }
-        uint4 Q[MT][4];
+            for (int j = 0; j < kXBatch; ++j) {
+              const int i4 = base + j * kGemvThreads + tid;
+              a[j] = 0.0f;
+              if (i4 < total4) a[j] = absmax4(__ldg(x4 + i4));
+            }
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          const int tok = g + 8 * mt;
-          if (tok < P.M) {
-            const uint8_t* qp = sq + (int64_t)tok * P.q_stride + 16 * w0;
-#pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4) Q[mt][i4] = *reinterpret_cast<const uint4*>(qp + 16 * i4);
-          } else {
-#pragma unroll
-            for (int i4 = 0; i4 < 4; ++i4) Q[mt][i4] = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const uint32_t mask = 0x03030303u << (2 * cc);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const uint32_t a0 = wa[2 * h] & mask, a2 = wa[2 * h + 1] & mask;
-            const uint32_t a1 = wb[2 * h] & mask, a3 = wb[2 * h + 1] & mask;
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-              const uint4& q0 = Q[mt][2 * h];
-              const uint4& q1 = Q[mt][2 * h + 1];
-              const uint32_t b0 = cc == 0 ? q0.x : (cc == 1 ? q0.y : (cc == 2 ? q0.z : q0.w));
-              const uint32_t b1 = cc == 0 ? q1.x : (cc == 1 ? q1.y : (cc == 2 ? q1.z : q1.w));
-              mma_u8s8(acc[cc][h % DA][mt], a0, a1, a2, a3, b0, b1);
+            for (int j = 0; j < kXBatch; ++j) {
+              const int i4 = base + j * kGemvThreads + tid;
+              warp_amax(s_amax + qs * 16, i4 < total4 ? i4 / K4 : -1, a[j]);
             }
           }
         }
-        u += kGemvWarps;
-        while (u >= P.n_units) {
-          u -= P.n_units;
-          ++ti;
-        }
       }
-      if (acc_tile >= 0) flush_tile<MT, DA>(acc, s_acc + (size_t)(sa - ra + acc_tile) * 16 * 8 * MT, g, t);
+      for (int i = tid; i < (se - sa) * 16 * 8 * MT; i += kGemvThreads) s_acc[(sa - ra) * 16 * 8 * MT + i] = 0;
+      if (newp) {
+        __syncthreads();  // absmax complete
+        const float4* x4 = reinterpret_cast<const float4*>(P.x);
+        if (greg) {
+          int m = -1, sum = 0;
+          if (tid < ngroups) {
+            m = tid / G;
+            const int grp = tid - m * G;
+            const float sx = token_scale(s_amax + qs * 16, m);
+            // Byte b of word r is column 4b + r of the group: component r of float4 b.
+            int q[4][4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float4 xv = s_xs[4 * tid + j];
+              q[j][0] = quant_i8_fast(xv.x, sx);
+              q[j][1] = quant_i8_fast(xv.y, sx);
+              q[j][2] = quant_i8_fast(xv.z, sx);
+              q[j][3] = quant_i8_fast(xv.w, sx);
+              sum += q[j][0] + q[j][1] + q[j][2] + q[j][3];
+            }
+            uint32_t w[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r)
+              w[r] = (uint32_t)(q[0][r] & 0xFF) | ((uint32_t)(q[1][r] & 0xFF) << 8) |
+                     ((uint32_t)(q[2][r] & 0xFF) << 16) | ((uint32_t)(q[3][r] & 0xFF) << 24);
+            *reinterpret_cast<uint4*>(sq + (int64_t)m * P.q_stride + 16 * grp) = make_uint4(w[0], w[1], w[2], w[3]);
+            if (grp == 0) s_sx[qs * 16 + m] = sx;
+          }
+          warp_rowsum(s_rs + qs * 16, m, sum);
+        } else {
+          int mprev = -1;
+          float sx = 0.0f;
+          for (int base = 0; base < total4; base += kXBatch * kGemvThreads) {
+            float4 v[kXBatch];
+#pragma unroll
+            for (int j = 0; j < kXBatch; ++j) {
+              const int i4 = base + j * kGemvThreads + tid;
+              v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (i4 < total4) v[j] = __ldg(x4 + i4);
+            }
+#pragma unroll
+            for (int j = 0; j < kXBatch; ++j) {
+              const int i4 = base + j * kGemvThreads + tid;
+              int m = -1, sum = 0;
+              if (i4 < total4) {
+                m = i4 / K4;
+                const int c4 = i4 - m * K4;
+                if (m != mprev) {
+                  sx = token_scale(s_amax + qs * 16, m);
+                  mprev = m;
+                }
+                sum = quant_store4(sq, P.q_stride, m, c4, v[j], sx);
+                if (c4 == 0) s_sx[qs * 16 + m] = sx;
+              }
+              warp_rowsum(s_rs + qs * 16, m, sum);
+            }
+          }
+        }
+        cur = p;
+      }
+      __syncthreads();  // codes, scales, row sums and zeroed partial sums visible
+      // Tasks of this segment are (tile, 256-code unit) pairs in tile-major
+      // order; warp w takes the contiguous range [ntask*w/W, ntask*(w+1)/W), so
+      // a warp meets one or two tiles and flushes its sums once per tile.
+      const int ntask = (se - sa) * P.n_units;
+      const int wpr = P.wpr, nu = P.n_units;
+      const bool al = (wpr & 3) == 0;
+      // Lane (g, t) reads words 4t..4t+3 of each unit for rows g and g+8, and
+      // the activation codes of token g + 8*mt. Lanes past the last token load
+      // nothing (their MMA columns are never used), which keeps the shared
+      // traffic of the activations to the tokens that exist.
+      const uint8_t* qrow[MT];
+      bool qon[MT];
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        qon[mt] = g + 8 * mt < P.M;
+        qrow[mt] = sq + (int64_t)(qon[mt] ? g + 8 * mt : 0) * P.q_stride + 64 * t;
+      }
+      // One accumulator set per class: four independent MMA chains per unit.
+      constexpr int DA = 1;
+      int acc[4][DA][MT][4];
+      const int tb = (int)(((int64_t)ntask * (warp + 1)) / kGemvWarps);
+      int task = (int)(((int64_t)ntask * warp) / kGemvWarps);
+      while (task < tb) {
+        const int ti = task / nu;
+        const int u0 = task - ti * nu;
+        const int u1 = (nu < u0 + (tb - task)) ? nu : u0 + (tb - task);
+        const int li = sa - ra + ti;  // tile slot in the round buffer
+        int okw = 1;
+        if (lane == 0) okw = mbar_wait(&full[b * RT + li], ph, abort_flag, L.err, kDevTimeoutProducer) ? 1 : 0;
+        okw = __shfl_sync(0xFFFFFFFFu, okw, 0);
+        if (!okw) break;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) acc[cc][0][mt][q] = 0;
+        const uint32_t* tile = reinterpret_cast<const uint32_t*>(bufs + (size_t)b * L.buf_bytes + s_off[b * RT + li]);
+        // Rows past N are not in the tile's slot: lanes on them read nothing.
+        const int rv = P.N - (t0 + sa + ti - P.tile0) * 16;
+        const bool aon = g < rv, bon = g + 8 < rv;
+        const uint32_t* rowa = tile + (aon ? g : 0) * wpr + 4 * t;
+        const uint32_t* rowb = tile + (bon ? g + 8 : 0) * wpr + 4 * t;
+        for (int u = u0; u < u1; ++u) {
+          uint32_t wa[4], wb[4];
+          const int w0 = u * 16 + 4 * t;
+          if (al && w0 + 4 <= wpr) {
+            uint4 va = make_uint4(0u, 0u, 0u, 0u), vb = make_uint4(0u, 0u, 0u, 0u);
+            if (aon) va = *reinterpret_cast<const uint4*>(rowa + 16 * u);
+            if (bon) vb = *reinterpret_cast<const uint4*>(rowb + 16 * u);
+            wa[0] = va.x;
+            wa[1] = va.y;
+            wa[2] = va.z;
+            wa[3] = va.w;
+            wb[0] = vb.x;
+            wb[1] = vb.y;
+            wb[2] = vb.z;
+            wb[3] = vb.w;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const bool in = w0 + j < wpr;  // words past the row belong to the next row: zero them
+              wa[j] = in && aon ? rowa[16 * u + j] : 0u;
+              wb[j] = in && bon ? rowb[16 * u + j] : 0u;
+            }
+          }
+          // Half h covers words 2h, 2h+1 of the lane (codes 32h .. 32h+31 of its 64).
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint4 Q[MT][2];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              const uint8_t* qp = qrow[mt] + 256 * u + 32 * h;
+              Q[mt][0] = make_uint4(0u, 0u, 0u, 0u);
+              Q[mt][1] = make_uint4(0u, 0u, 0u, 0u);
+              if (qon[mt]) {
+                Q[mt][0] = *reinterpret_cast<const uint4*>(qp);
+                Q[mt][1] = *reinterpret_cast<const uint4*>(qp + 16);
+              }
+            }
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+              const uint32_t mask = 0x03030303u << (2 * cc);
+              const uint32_t a0 = wa[2 * h] & mask, a2 = wa[2 * h + 1] & mask;
+              const uint32_t a1 = wb[2 * h] & mask, a3 = wb[2 * h + 1] & mask;
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                const uint4& q0 = Q[mt][0];
+                const uint4& q1 = Q[mt][1];
+                const uint32_t b0 = cc == 0 ? q0.x : (cc == 1 ? q0.y : (cc == 2 ? q0.z : q0.w));
+                const uint32_t b1 = cc == 0 ? q1.x : (cc == 1 ? q1.y : (cc == 2 ? q1.z : q1.w));
+                mma_u8s8(acc[cc][0][mt], a0, a1, a2, a3, b0, b1);
+              }
+            }
+          }
+        }
+        flush_tile<MT, DA>(acc, s_acc + (size_t)li * 16 * 8 * MT, g, t);
+        task += u1 - u0;
+      }
+      cp_async_wait_all();  // this thread's row-scale copies
       __syncthreads();
       if (*abort_flag) {
         // Block-uniform after the barrier. Let the copies already issued land
@@ -360,6 +537,12 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
         }
         return;
       }
+      // This round's buffer is consumed once its last segment is: start the
+      // round that reuses it while the outputs are written.
+      if (se == re && tid == 0 && r + L.nbuf < nrounds) {
+        issue_round(r + L.nbuf);
+        issued = r + L.nbuf + 1;
+      }
       // Outputs of this segment: rows x tokens, coalesced along the rows.
       const int nout = (se - sa) * 16 * P.M;
       for (int idx = tid; idx < nout; idx += kGemvThreads) {
@@ -368,19 +551,13 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
         const int ti2 = rr >> 4, r16 = rr & 15;
         const int64_t row = (int64_t)(t0 + sa + ti2 - P.tile0) * 16 + r16;
         if (row >= P.N) continue;
-        const int a = s_acc[((size_t)(sa - ra + ti2) * 16 + r16) * 8 * MT + tok] - s_rs[tok];
+        const int a = s_acc[((size_t)(sa - ra + ti2) * 16 + r16) * 8 * MT + tok] - s_rs[qs * 16 + tok];
         if (kAccOut)
           P.acc[(int64_t)tok * P.N + row] = a;
         else
-          P.y[(int64_t)tok * P.N + row] = rescale(a, s_sx[tok], __ldg(P.D + row));
+          P.y[(int64_t)tok * P.N + row] = rescale(a, s_sx[qs * 16 + tok], s_D[(sa - ra + ti2) * 16 + r16]);
       }
       sa = se;
-    }
-    __syncthreads();
-    // This round's buffer is consumed: start the round that reuses it.
-    if (tid == 0 && r + L.nbuf < nrounds) {
-      issue_round(r + L.nbuf);
-      issued = r + L.nbuf + 1;
     }
   }
 }
@@ -406,8 +583,8 @@ static cudaError_t launch_gemv_t(const GemvLaunch& L, int grid, size_t smem, boo
 }
 
 static size_t gemv_smem_bytes(const GemvLaunch& L, int MT) {
-  return (size_t)L.nbuf * L.buf_bytes + L.q_bytes + 3 * 16 * 4 + (size_t)L.round_tiles * 16 * 8 * MT * 4 +
-         (size_t)L.nbuf * L.round_tiles * (8 + 4) + 16;
+  return (size_t)L.nbuf * L.buf_bytes + L.q_bytes + L.xs_bytes + 3 * 32 * 4 + (size_t)L.round_tiles * 16 * 4 +
+         (size_t)L.round_tiles * 16 * 8 * MT * 4 + (size_t)L.nbuf * L.round_tiles * (8 + 4) + 16;
 }
 
 // Shared-memory bytes of launch tile gt (rows x K/4 rounded up to 128 B).
@@ -456,7 +633,8 @@ int64_t gemv_stage_bytes(int64_t K) { return ((16 * (K / 4)) + 127) / 128 * 128;
 bool gemv_group_fits(int64_t maxM, int64_t maxK) {
   if (maxM > kGemvMaxM) return false;
   const int64_t q = (maxM * gemv_q_stride(maxK) + 127) / 128 * 128;
-  return q + 2 * gemv_stage_bytes(maxK) + 16 * 1024 <= kGemvMaxSmem;
+  const int64_t xs = maxM * maxK <= 16 * kGemvThreads ? maxM * maxK * 4 : 0;
+  return q + xs + 2 * gemv_stage_bytes(maxK) + 16 * 1024 <= kGemvMaxSmem;
 }
 
 cudaError_t launch_gemv_group(const GemvCall* calls, int n, uint32_t* err, bool pdl, cudaStream_t stream,
@@ -490,15 +668,22 @@ cudaError_t launch_gemv_group(const GemvCall* calls, int n, uint32_t* err, bool 
   L.err = err;
   L.stage_bytes = (int)gemv_stage_bytes(maxK);
   L.q_bytes = (int)((maxM * gemv_q_stride(maxK) + 127) / 128 * 128);
+  // Problems with at most one 16-column group per thread stage x in shared memory.
+  int64_t xs = 0;
+  for (int i = 0; i < n; ++i) {
+    const int64_t mk = calls[i].M * calls[i].K;
+    if (mk / 16 <= kGemvThreads && mk * 4 > xs) xs = mk * 4;
+  }
+  L.xs_bytes = (int)xs;
   const int MT = maxM <= 8 ? 1 : 2;
   int grid0 = tiles < num_sms ? tiles : num_sms;
   if (grid0 > kGemvMaxGrid) grid0 = kGemvMaxGrid;
   int64_t cta_bytes = 0;
   int per_cta = 0;
   partition_by_bytes(L, grid0, &cta_bytes, &per_cta);
-  // Per tile slot: its partial-sum block, barrier and offset entry.
-  const int64_t slot_extra = 16 * 8 * MT * 4 + 8 + 4;
-  const int64_t fixed = L.q_bytes + 3 * 16 * 4 + 16;
+  // Per tile slot: its partial-sum block, row scales, barrier and offset entry.
+  const int64_t slot_extra = 16 * 8 * MT * 4 + 16 * 4 + 8 + 4;
+  const int64_t fixed = L.q_bytes + L.xs_bytes + 3 * 32 * 4 + 16;
   if (fixed + cta_bytes + per_cta * slot_extra <= kGemvMaxSmem) {
     L.nbuf = 1;  // every tile of a CTA in flight at once
     L.round_tiles = per_cta;

@@ -152,6 +152,62 @@ def test_forward_gemv(B, M, N, K):
     run_case(B, M, N, K, xdist="student_t", seed=M * 1000 + N + K)
 
 
+@pytest.mark.parametrize("M,N,K", [(1, 2560, 2560), (3, 300, 528), (16, 257, 6912), (1, 33, 48), (200, 129, 1152)])
+def test_forward_per_row_scale(B, M, N, K):
+    """D is a per-row [N,1] scale: distinct values per row must land on their
+    own rows (decode and tensor-core paths)."""
+    rng = np.random.default_rng(N * 7 + K)
+    W = WL.weight(N, K, "normal", 31)
+    x = WL.activations(M, K, "student_t", 32, meta={"df": 3.0})
+    packed, _ = B.pack_weights(dev(W))
+    p_ref, _ = O.pack_weights(W)
+    D_rows = rng.uniform(1e-3, 2.0, size=(N, 1)).astype(np.float32)
+    y = B.forward(dev(x), packed, dev(D_rows)).cpu().numpy()
+    assert_y_close(y, O.bitlinear_forward(x, p_ref, D_rows, K))
+
+
+@pytest.mark.parametrize("M", [1, 3, 100])
+def test_quant_ties_round_to_even(B, M):
+    """Products x*s_x that land exactly on .5 round to even (rint), in the
+    decode kernel's own quantiser (M <= 16) and in the ActQuant kernel (M > 16).
+    amax = 127 gives s_x = 1, so the codes are rint(x)."""
+    K = 64
+    halves = np.array([0.5, 1.5, 2.5, -0.5, -1.5, -2.5, 126.5, -126.5, 3.5, 4.5], np.float32)
+    x = np.zeros((M, K), np.float32)
+    for m in range(M):
+        row = np.resize(np.roll(halves, m), K)
+        row[10 + (7 * m) % (K - 10)] = 127.0 if m % 2 == 0 else -127.0
+        x[m] = row
+    W = WL.weight(48, K, "normal", 77)
+    packed, _ = B.pack_weights(dev(W))
+    p_ref, _ = O.pack_weights(W)
+    q_ref, s_ref = O.act_quant(x)
+    assert np.all(s_ref == 1.0)
+    assert q_ref[0, 0] == 0 and q_ref[0, 1] == 2 and q_ref[0, 2] == 2 and q_ref[0, 6] == 126
+    _, parts = O.bitlinear_forward(x, p_ref, np.ones((48, 1), np.float32), K, return_parts=True)
+    acc = B.forward_acc(dev(x), packed).cpu().numpy()
+    assert np.array_equal(acc, parts["acc"])
+
+
+def test_gemv_streamed_rounds(B):
+    """A decode layer too large for one shot of shared memory per CTA
+    (~38 MB of packed weights): the kernel streams double-buffered rounds.
+    Codes are drawn directly (uniform over {-1,0,1}), D per row; sampled
+    rows are checked against the oracle on those rows' weights."""
+    M, N, K = 1, 9477, 16384
+    rng = np.random.default_rng(99)
+    packed = np.empty((N, K // 16), dtype=np.uint32)
+    for r0 in range(0, N, 512):
+        r1 = min(N, r0 + 512)
+        packed[r0:r1] = O.pack_codes(rng.integers(-1, 2, size=(r1 - r0, K), dtype=np.int8))
+    D_rows = rng.uniform(1e-3, 2.0, size=(N, 1)).astype(np.float32)
+    x = WL.activations(M, K, "student_t", 98, meta={"df": 3.0})
+    y = B.forward(dev(x), dev(packed.view(np.int32)), dev(D_rows)).cpu().numpy()
+    rows = np.array(sorted(set(range(0, N, 5)) | set(range(N - 40, N))))
+    y_ref = O.bitlinear_forward(x, packed[rows], D_rows[rows], K)
+    assert_y_close(y[:, rows], y_ref)
+
+
 GEMM_CASES = [
     (17, 16, 16), (17, 128, 128), (100, 129, 256), (256, 4304, 1152), (256, 1152, 4304),
     (300, 700, 2560), (129, 33, 6912), (512, 384, 528), (1000, 257, 48), (640, 640, 640),
