@@ -499,7 +499,8 @@ def load_traffic(kernel):
 
         if d.get("sources_sha") != build.sources_sha():
             return None
-        return d.get("kernels", {}).get(kernel)
+        v = d.get("kernels", {}).get(kernel)
+        return v.get("bytes_per_launch") if isinstance(v, dict) else v
     except Exception:
         return None
 
