@@ -46,6 +46,8 @@ SIGNATURES = {
     "bitlinear_forward_batch": (ctypes.c_int, [_VP, ctypes.c_int, ctypes.c_uint32, _VP, _SZ, _VP]),
     "bitlinear_host_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "bitlinear_forward_host": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "bitlinear_forward_host_async": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "bitlinear_forward_q": (ctypes.c_int, [_VP, _VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "bitlinear_workspace_error": (ctypes.c_int, [_VP, _SZ, _VP]),
     "bitlinear_selftest_wait_timeout": (ctypes.c_int, [_VP, _SZ, ctypes.c_uint64, _VP]),
     "bitlinear_forward_noalloc": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP]),

@@ -146,6 +146,31 @@ def forward_prepared(M: int, K: int, packed: torch.Tensor, D: torch.Tensor, ws: 
     return y
 
 
+def forward_q(q: torch.Tensor, s_x: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,
+              out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y from pre-quantised activations: q int8 [M,K] (natural order) and s_x fp32 [M]
+    as quant_act returns them."""
+    _need_cuda(q, "q", torch.int8)
+    _need_cuda(s_x, "s_x", torch.float32)
+    if q.dim() != 2 or not q.is_contiguous() or not s_x.is_contiguous():
+        raise ValueError("q must be a contiguous [M, K] tensor and s_x contiguous")
+    M, K = q.shape
+    if s_x.numel() != M:
+        raise ValueError("s_x must hold one scale per token")
+    _need_cuda(packed, "packed", torch.int32)
+    N = packed.shape[0]
+    if packed.shape[1] * 16 != K:
+        raise ValueError("K mismatch with packed")
+    _check_D(D, N)
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=q.device)
+    _need_cuda(y, "out", torch.float32)
+    if ws is None:
+        ws = _alloc_ws(_lib.lib().bitlinear_workspace_size(M, N, K), q.device)
+    _lib.call("bitlinear_forward_q", q.data_ptr(), s_x.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(),
+              y.data_ptr(), ws.data_ptr(), ws.numel(), _stream_handle(q.device))
+    return y
+
+
 def forward_batch(calls, flags: int = 0, ws: Optional[torch.Tensor] = None):
     """Run independent BitLinears [(x, packed, D, out), ...] in one C call.
 
@@ -177,8 +202,11 @@ def forward_batch(calls, flags: int = 0, ws: Optional[torch.Tensor] = None):
 
 
 def forward_host(x_host: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,
-                 y_host: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """End-to-end call with host x / y (pinned recommended); synchronous."""
+                 y_host: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                 sync: bool = True) -> torch.Tensor:
+    """End-to-end call with host x / y. sync=True: synchronous (pinned memory
+    recommended). sync=False: enqueued on the current stream; x_host and y_host
+    must be pinned, and y_host is valid after the stream is synchronised."""
     if x_host.is_cuda or x_host.dtype != torch.float32 or not x_host.is_contiguous():
         raise ValueError("x_host must be a contiguous fp32 CPU tensor")
     M, K = x_host.shape
@@ -187,10 +215,13 @@ def forward_host(x_host: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,
     _check_D(D, N)
     if y_host is None:
         y_host = torch.empty((M, N), dtype=torch.float32, pin_memory=True)
+    if not sync and not (x_host.is_pinned() and y_host.is_pinned()):
+        raise ValueError("the asynchronous host call needs pinned x_host and y_host")
     L = _lib.lib()
     if ws is None:
         ws = _alloc_ws(L.bitlinear_host_workspace_size(M, N, K), packed.device)
-    _lib.call("bitlinear_forward_host", x_host.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(),
+    fn = "bitlinear_forward_host" if sync else "bitlinear_forward_host_async"
+    _lib.call(fn, x_host.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(),
               y_host.data_ptr(), ws.data_ptr(), ws.numel(), _stream_handle(packed.device))
     return y_host
 

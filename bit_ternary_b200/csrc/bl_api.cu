@@ -190,6 +190,29 @@ int bitlinear_forward_prepared(int64_t M, int64_t N, int64_t K, const uint32_t* 
   return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, nullptr, ws, reinterpret_cast<cudaStream_t>(stream), sms));
 }
 
+int bitlinear_forward_q(const int8_t* q, const float* s_x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                        const float* D, float* y, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  st = check_mn(M, N);
+  if (st != BL_OK) return st;
+  if (M == 0 || N == 0) return BL_OK;
+  if (q == nullptr || s_x == nullptr || packed == nullptr || D == nullptr || y == nullptr || ws == nullptr)
+    return BL_ERR_NULL;
+  if (!aligned16(q) || !aligned16(packed) || !aligned16(D) || !aligned16(y) || !aligned256(ws)) return BL_ERR_ALIGN;
+  if (ws_bytes < bitlinear_workspace_size(M, N, K)) return BL_ERR_WORKSPACE;
+  const int sms = num_sms_current();
+  if (sms <= 0) return BL_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  st = cuda_status(bl::launch_q_prepare(q, s_x, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
+                                        reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
+                                        reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), s,
+                                        reinterpret_cast<uint32_t*>(base)));
+  if (st != BL_OK) return st;
+  return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, nullptr, ws, s, sms));
+}
+
 size_t bitlinear_batch_workspace_size(const bl_linear_call* calls, int count) {
   size_t need = bl::kHeaderBytes;
   if (calls == nullptr || count < 0) return 0;
@@ -264,8 +287,9 @@ size_t bitlinear_host_workspace_size(int64_t M, int64_t N, int64_t K) {
          bl::align256(4 * (size_t)M * (size_t)N);
 }
 
-int bitlinear_forward_host(const float* x_host, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
-                           const float* D, float* y_host, void* ws, size_t ws_bytes, bl_stream_t stream) {
+static int forward_host_impl(const float* x_host, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                             const float* D, float* y_host, void* ws, size_t ws_bytes, bl_stream_t stream,
+                             bool sync) {
   int st = check_k(K);
   if (st != BL_OK) return st;
   st = check_mn(M, N);
@@ -285,7 +309,18 @@ int bitlinear_forward_host(const float* x_host, int64_t M, int64_t N, int64_t K,
   if (st != BL_OK) return st;
   if (cudaMemcpyAsync(y_host, yd, 4 * (size_t)M * (size_t)N, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return BL_ERR_CUDA;
+  if (!sync) return BL_OK;
   return cudaStreamSynchronize(s) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+int bitlinear_forward_host(const float* x_host, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                           const float* D, float* y_host, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  return forward_host_impl(x_host, M, N, K, packed, D, y_host, ws, ws_bytes, stream, true);
+}
+
+int bitlinear_forward_host_async(const float* x_host, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                                 const float* D, float* y_host, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  return forward_host_impl(x_host, M, N, K, packed, D, y_host, ws, ws_bytes, stream, false);
 }
 
 int bitlinear_workspace_error(void* ws, size_t ws_bytes, bl_stream_t stream) {

@@ -43,6 +43,10 @@ cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* packed, 
 // err_reset (nullable): the workspace error word, cleared by the kernel.
 cudaError_t launch_act_quant(const float* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
                              bool permuted, cudaStream_t stream, uint32_t* err_reset);
+// Natural-order int8 codes and scales (bitlinear_quant_act's output) into the
+// forward workspace layout (private order, row sums); err_reset as above.
+cudaError_t launch_q_prepare(const int8_t* q, const float* s_x, int64_t M, int64_t K, int8_t* wq, float* wsx,
+                             int32_t* wrs, cudaStream_t stream, uint32_t* err_reset);
 // Expects the permuted activations, s_x and row sums already in the forward
 // workspace (launch_act_quant with permuted = true).
 cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D, float* y,

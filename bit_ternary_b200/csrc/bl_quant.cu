@@ -365,6 +365,51 @@ cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* packed, 
   return cudaGetLastError();
 }
 
+// Pre-quantised input: natural-order int8 codes q [M,K] and scales s_x [M]
+// (as bitlinear_quant_act writes them) into the forward workspace, in the
+// kernel-private column order, with the row sums. One CTA per token; each
+// thread moves 16-column groups: byte j of output word r is byte r of input
+// word j (the 4x4 byte transpose perm16 describes).
+__global__ void __launch_bounds__(256) q_prepare_kernel(const int8_t* __restrict__ q, const float* __restrict__ s_x,
+                                                        int64_t K, int8_t* __restrict__ wq, float* __restrict__ wsx,
+                                                        int32_t* __restrict__ wrs, uint32_t* __restrict__ err_reset) {
+  if (err_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err_reset = 0u;
+  __shared__ int red[8];
+  const int64_t m = blockIdx.x;
+  const uint4* src = reinterpret_cast<const uint4*>(q + m * K);
+  uint4* dst = reinterpret_cast<uint4*>(wq + m * K);
+  const int ngroups = (int)(K >> 4);
+  int sum = 0;
+  for (int g = threadIdx.x; g < ngroups; g += blockDim.x) {
+    const uint4 v = __ldg(src + g);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+      o[r] = ((w[0] >> (8 * r)) & 0xFFu) | (((w[1] >> (8 * r)) & 0xFFu) << 8) | (((w[2] >> (8 * r)) & 0xFFu) << 16) |
+             (((w[3] >> (8 * r)) & 0xFFu) << 24);
+    dst[g] = make_uint4(o[0], o[1], o[2], o[3]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) sum = __dp4a((int)w[j], 0x01010101, sum);  // sum of the four signed bytes
+  }
+  sum = __reduce_add_sync(0xFFFFFFFFu, sum);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) red[warp] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int t = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) t += red[i];
+    wrs[m] = t;
+    wsx[m] = s_x[m];
+  }
+}
+
+cudaError_t launch_q_prepare(const int8_t* q, const float* s_x, int64_t M, int64_t K, int8_t* wq, float* wsx,
+                             int32_t* wrs, cudaStream_t stream, uint32_t* err_reset) {
+  q_prepare_kernel<<<(unsigned)M, 256, 0, stream>>>(q, s_x, K, wq, wsx, wrs, err_reset);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_act_quant(const float* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
                              bool permuted, cudaStream_t stream, uint32_t* err_reset) {
   const int64_t ngroups = K / 16;

@@ -156,6 +156,17 @@ BL_API int bitlinear_forward_prepared(int64_t M, int64_t N, int64_t K,
                                       const uint32_t* packed, const float* D, float* y,
                                       void* ws, size_t ws_bytes, bl_stream_t stream);
 
+/* Forward from pre-quantised activations: q device int8 [M, K] in natural
+ * column order and s_x device fp32 [M] (the scale 127/max|x| per token), as
+ * bitlinear_quant_act writes them. y [M,N] = RN(RN(acc/s_x) * D) with
+ * acc = sum_k q*code exactly. Any int8 codes are accepted (-128 included).
+ * q, packed, D and y must be 16-byte aligned, ws 256-byte aligned with
+ * ws_bytes >= bitlinear_workspace_size(M, N, K). Reorders q into ws, then runs
+ * the tensor-core kernel (every M). Asynchronous. */
+BL_API int bitlinear_forward_q(const int8_t* q, const float* s_x, int64_t M, int64_t N, int64_t K,
+                               const uint32_t* packed, const float* D, float* y,
+                               void* ws, size_t ws_bytes, bl_stream_t stream);
+
 /* ---------------------------------------------------------------- batch --- */
 
 /* One BitLinear of a batch: y [M,N] = F.linear(ActQuant(x [M,K]), W) from
@@ -202,6 +213,15 @@ BL_API size_t bitlinear_host_workspace_size(int64_t M, int64_t N, int64_t K);
 BL_API int bitlinear_forward_host(const float* x_host, int64_t M, int64_t N, int64_t K,
                            const uint32_t* packed, const float* D, float* y_host,
                            void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* The same three steps as bitlinear_forward_host, enqueued on `stream`
+ * without synchronising: y_host holds the result once the stream has been
+ * synchronised. x_host and y_host must be pinned (page-locked) for the copies
+ * to overlap the host; they must stay valid and untouched until then. Calls on
+ * one stream may share a workspace (stream order serialises them). */
+BL_API int bitlinear_forward_host_async(const float* x_host, int64_t M, int64_t N, int64_t K,
+                                 const uint32_t* packed, const float* D, float* y_host,
+                                 void* ws, size_t ws_bytes, bl_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device error word in a
  * forward workspace. BL_OK if no kernel recorded a failure, else

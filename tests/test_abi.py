@@ -107,3 +107,18 @@ def test_batch_validation_before_cuda(L):
     assert L.bitlinear_forward_batch(calls, 2, 0x80, FAKE, 1 << 20, None) == 2  # unknown flag
     assert L.bitlinear_forward_batch(calls, 0, 0, None, 0, None) == 0
     assert L.bitlinear_batch_workspace_size(calls, 2) == 256 + 256 + 256 + 256  # header, s_x, sums, q
+
+
+def test_forward_q_and_async_host_validation_before_cuda(L):
+    # bitlinear_forward_q(q, s_x, M, N, K, packed, D, y, ws, ws_bytes, stream)
+    assert L.bitlinear_forward_q(FAKE, FAKE, 1, 1, 24, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 2
+    assert L.bitlinear_forward_q(None, FAKE, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.bitlinear_forward_q(FAKE, None, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.bitlinear_forward_q(FAKE + 8, FAKE, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 3
+    assert L.bitlinear_forward_q(FAKE, FAKE, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, 16, None) == 4
+    assert L.bitlinear_forward_q(None, None, 0, 4, 16, None, None, None, None, 0, None) == 0
+    # bitlinear_forward_host_async(x_host, M, N, K, packed, D, y_host, ws, ws_bytes, stream)
+    assert L.bitlinear_forward_host_async(None, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.bitlinear_forward_host_async(FAKE, 1, 1, 40, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 2
+    assert L.bitlinear_forward_host_async(FAKE, 1, 1, 16, FAKE, FAKE, FAKE, FAKE + 16, 1 << 20, None) == 3
+    assert L.bitlinear_forward_host_async(FAKE, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, 8, None) == 4

@@ -277,6 +277,51 @@ def test_forward_host_matches_device(B):
     assert np.array_equal(y_dev.view(np.uint32), y_host.view(np.uint32))
 
 
+def test_forward_host_async_shared_workspace(B):
+    """Several asynchronous host calls on one stream share a workspace; after
+    one synchronise every y_host holds its own result (decode and GEMM paths)."""
+    shapes = [(1, 3840, 2560), (1, 2560, 2560), (5, 700, 1152), (40, 300, 512)]
+    calls, refs = [], []
+    for i, (M, N, K) in enumerate(shapes):
+        W = WL.weight(N, K, "normal", 900 + i)
+        x = WL.activations(M, K, "student_t", 910 + i, meta={"df": 3.0})
+        packed, D = B.pack_weights(dev(W))
+        calls.append((torch.from_numpy(x).pin_memory(), packed, D,
+                      torch.empty((M, N), dtype=torch.float32).pin_memory()))
+        refs.append(_oracle_y(W, x))
+    L = __import__("bit_ternary_b200._lib", fromlist=["lib"]).lib()
+    ws_bytes = max(L.bitlinear_host_workspace_size(M, N, K) for (M, N, K) in shapes)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
+    for xh, packed, D, yh in calls:
+        B.forward_host(xh, packed, D, y_host=yh, ws=ws, sync=False)
+    torch.cuda.current_stream().synchronize()
+    for (_, _, _, yh), ref in zip(calls, refs):
+        assert_y_close(yh.numpy(), ref)
+    with pytest.raises(ValueError):
+        B.forward_host(torch.zeros(1, 16), calls[0][1][:, :1].contiguous(), calls[0][2], sync=False)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 300, 2560), (37, 257, 528), (300, 700, 1152)])
+def test_forward_q_from_quant_act(B, M, N, K):
+    """forward_q on quant_act's natural-order codes equals the oracle's
+    contraction and rescale of the same codes; arbitrary codes (-128 included)
+    and scales too."""
+    W = WL.weight(N, K, "normal", 60 + K)
+    x = WL.activations(M, K, "student_t", 61 + M, meta={"df": 3.0})
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    q, s_x, _ = B.quant_act(dev(x))
+    y = B.forward_q(q, s_x, packed, D).cpu().numpy()
+    assert_y_close(y, O.bitlinear_forward(x, p_ref, D_ref, K))
+    rng = np.random.default_rng(M + N + K)
+    q2 = rng.integers(-128, 128, size=(M, K), dtype=np.int8)
+    s2 = rng.uniform(0.5, 300.0, size=M).astype(np.float32)
+    codes = O.unpack_codes(p_ref, K)
+    y_ref = O.rescale(O.int_matmul(q2, codes), s2, D_ref)
+    y2 = B.forward_q(dev(q2), dev(s2), packed, D).cpu().numpy()
+    assert_y_close(y2, y_ref)
+
+
 def test_workspace_error_word_clear_after_gemm(B):
     M, N, K = 200, 256, 512
     W = WL.weight(N, K, "normal", 4)
