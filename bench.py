@@ -62,6 +62,8 @@ def parse_args(argv=None):
                     help="small decode-only run for profiler captures (4 weight copies, no extras)")
     ap.add_argument("--ncu-prefill", action="store_true",
                     help="small prefill-only run for profiler captures (gate_up layer, M=4096)")
+    ap.add_argument("--ncu-layer", default=None, metavar="WORKLOAD:LAYER:M",
+                    help="one layer of a workload, M tokens, for profiler captures (e.g. embed_batch:0:32768)")
     a = ap.parse_args(argv)
     a.warmup = max(3, a.warmup)
     a.steps = max(1, a.steps)
@@ -253,7 +255,7 @@ def run_ours(a):
     dev = torch.device("cuda", local)
     if _lib.lib().bitlinear_device_check() != 0:
         raise SystemExit("device is not sm_100 (B200)")
-    if a.ncu_prefill:
+    if a.ncu_prefill or a.ncu_layer:
         return run_prefill_small(a, B, torch, dev)
     if world > 1:
         import datetime
@@ -669,14 +671,18 @@ def bench_pack(B, torch, dev, stream, hbm_peak):
 
 
 def run_prefill_small(a, B, torch, dev):
-    """Bounded prefill case for profiler captures: gate_up (2560->13824) at M=4096."""
-    wl = WL.WORKLOADS[PREFILL]
-    l = wl.layers[1]
-    M = PREFILL_M
-    W = torch.from_numpy(WL.weight(l.N, l.K, wl.w_dist, wl.seed, layer=1)).to(dev)
+    """Bounded case for profiler captures: one layer of one workload (default: the prefill
+    gate_up layer, 2560->13824, at M=4096)."""
+    key, li, M = PREFILL, 1, PREFILL_M
+    if a.ncu_layer:
+        k, i, m = a.ncu_layer.split(":")
+        key, li, M = k, int(i), int(m)
+    wl = WL.WORKLOADS[key]
+    l = wl.layers[li]
+    W = torch.from_numpy(WL.weight(l.N, l.K, wl.w_dist, wl.seed, layer=li)).to(dev)
     p, D = B.pack_weights(W)
     del W
-    x = torch.from_numpy(WL.activations(M, l.K, wl.x_dist, wl.seed, layer=1)).to(dev)
+    x = torch.from_numpy(WL.activations(M, l.K, wl.x_dist, wl.seed, layer=li, meta=wl.meta)).to(dev)
     y = torch.empty((M, l.N), dtype=torch.float32, device=dev)
     ws = torch.zeros(B.workspace_size(M, l.N, l.K), dtype=torch.uint8, device=dev)
     for _ in range(a.warmup + a.steps):

@@ -9,8 +9,12 @@
 
 namespace bl {
 
-// Pack workspace: header (status word at 0, mean_c and s at 16/20) + 256 bins.
-constexpr size_t kPackWsBytes = kHeaderBytes + 256 * sizeof(unsigned long long);
+// Pack workspace: header (status word at 0, mean_c and s at 16/20) + bins:
+// kPackBins sums of significands by weight (bin b weighs 2^(max(b,1)-1) units
+// of 2^-149) and, at kPackNonFiniteBin, a count of non-finite weights.
+constexpr int kPackBins = 320;
+constexpr int kPackNonFiniteBin = kPackBins - 1;
+constexpr size_t kPackWsBytes = kHeaderBytes + kPackBins * sizeof(unsigned long long);
 
 // Decode path (fused quantise + GEMV): at most 16 tokens, and the quantised
 // activations plus two ring stages of packed weights must fit in shared memory.

@@ -8,9 +8,9 @@
 //
 // The mean of |W| must be identical however the reduction is ordered, so it is
 // an exact integer sum: every |w| = m * 2^(max(e,1)-150), and the 24-bit
-// significands m are summed per biased exponent e in 64-bit integers (exact
-// and order independent). A single thread then forms the exact total and
-// divides it by N*K with one correct rounding to fp32.
+// significands m are summed, in integers, into bins by weight (exact and order
+// independent). A single thread then forms the exact total and divides it by
+// N*K with one correct rounding to fp32.
 #include "bl_internal.h"
 
 namespace bl {
@@ -18,28 +18,74 @@ namespace bl {
 // ------------------------------------------------------------------ pack --
 constexpr int kBinThreads = 256;
 constexpr int kBinWarps = kBinThreads / 32;
+constexpr int kWindow = 38;  // binades below a batch's largest exponent summed in one 64-bit word
 
+// Exact per-weight sums of the significands of |W|. |w| = m * 2^(ee-1) units
+// of 2^-149, with m < 2^24 and ee = max(biased exponent, 1). A warp takes 128
+// weights at a time (one float4 per lane) and the batch's largest ee, E; each
+// lane adds m << (ee - base) for base = max(E - kWindow, 1) into a 64-bit word
+// (4 terms below 2^62 each), the warp sums that word in three 21-bit chunks
+// (each chunk sum < 2^27) and lane 0 adds them to the bins base, base+21 and
+// base+42 of a per-warp shared copy. Weights below the window go to their own
+// bin. Every step is integer arithmetic, so the result does not depend on the
+// order of the reduction.
 __global__ void __launch_bounds__(kBinThreads) absum_bins_kernel(const float4* __restrict__ W, int64_t n4,
                                                                   unsigned long long* __restrict__ bins) {
-  __shared__ unsigned long long sbins[kBinWarps][256];
-  const int warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < kBinWarps * 256; i += blockDim.x) (&sbins[0][0])[i] = 0ull;
+  __shared__ unsigned long long sbins[kBinWarps][kPackBins];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kBinWarps * kPackBins; i += blockDim.x) (&sbins[0][0])[i] = 0ull;
   __syncthreads();
   unsigned long long* my = sbins[warp];
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
-    const float4 v = __ldg(W + i);
-    const float vals[4] = {v.x, v.y, v.z, v.w};
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  // Warp-uniform loop bound: every lane reaches the warp reductions.
+  const int64_t base0 = blockIdx.x * (int64_t)blockDim.x + (threadIdx.x & ~31);
+  for (int64_t wb = base0; wb < n4; wb += stride) {
+    const int64_t i = wb + lane;
+    uint32_t m[4], ee[4];
+    uint32_t emax = 0u, nonfinite = 0u;
+    if (i < n4) {
+      const float4 v = __ldg(W + i);
+      const float vals[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t b = __float_as_uint(vals[j]) & 0x7FFFFFFFu;
+        const uint32_t e = b >> 23;
+        m[j] = (b & 0x7FFFFFu) | (e != 0 ? 0x800000u : 0u);
+        ee[j] = e > 1 ? e : 1;
+        if (e == 255) {
+          nonfinite = 1u;
+          m[j] = 0u;
+        }
+        if (m[j] != 0u && ee[j] > emax) emax = ee[j];
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) m[j] = 0u, ee[j] = 1u;
+    }
+    const uint32_t E = __reduce_max_sync(0xFFFFFFFFu, emax);
+    const uint32_t base = E > (uint32_t)kWindow + 1u ? E - (uint32_t)kWindow : 1u;
+    unsigned long long acc = 0ull;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const uint32_t b = __float_as_uint(vals[j]) & 0x7FFFFFFFu;
-      const uint32_t e = b >> 23;
-      uint32_t m = b & 0x7FFFFFu;
-      if (e != 0) m |= 0x800000u;
-      if (m != 0 || e == 255) atomicAdd(&my[e], (unsigned long long)(m | (e == 255 ? 1u : 0u)));
+      if (m[j] == 0u) continue;
+      if (ee[j] >= base)
+        acc += (unsigned long long)m[j] << (ee[j] - base);
+      else
+        atomicAdd(&my[ee[j]], (unsigned long long)m[j]);  // more than kWindow binades below the batch maximum
+    }
+    const uint32_t c0 = __reduce_add_sync(0xFFFFFFFFu, (uint32_t)(acc & 0x1FFFFFull));
+    const uint32_t c1 = __reduce_add_sync(0xFFFFFFFFu, (uint32_t)((acc >> 21) & 0x1FFFFFull));
+    const uint32_t c2 = __reduce_add_sync(0xFFFFFFFFu, (uint32_t)(acc >> 42));
+    const uint32_t nf = __reduce_add_sync(0xFFFFFFFFu, nonfinite);
+    if (lane == 0) {
+      if (c0) atomicAdd(&my[base], (unsigned long long)c0);
+      if (c1) atomicAdd(&my[base + 21], (unsigned long long)c1);
+      if (c2) atomicAdd(&my[base + 42], (unsigned long long)c2);
+      if (nf) atomicAdd(&my[kPackNonFiniteBin], (unsigned long long)nf);
     }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < 256; e += blockDim.x) {
+  for (int e = threadIdx.x; e < kPackBins; e += blockDim.x) {
     unsigned long long s = 0;
 #pragma unroll
     for (int w = 0; w < kBinWarps; ++w) s += sbins[w][e];
@@ -49,22 +95,25 @@ __global__ void __launch_bounds__(kBinThreads) absum_bins_kernel(const float4* _
 
 // Correctly rounded fp32 of S * 2^-149 / n, where S = sum_e bins[e] * 2^(max(e,1)-1).
 // Results below the normal range are returned as 0 (they lie far below the
-// 1e-5 floor that is applied afterwards). One thread.
+// 1e-5 floor that is applied afterwards). One thread. n = N*K < 2^48 (N < 2^31,
+// K <= 2^17), and a tensor that fits in device memory has n < 2^36, so every
+// bin is below 2^60 and S below 2^313.
 __global__ void absmean_finalize_kernel(const unsigned long long* __restrict__ bins, uint64_t n,
                                         float* __restrict__ scal, uint32_t* __restrict__ status) {
   if (threadIdx.x != 0 || blockIdx.x != 0) return;
-  if (bins[255] != 0ull) {
+  if (bins[kPackNonFiniteBin] != 0ull) {
     *status = 1u;  // non-finite input
     scal[0] = __int_as_float(0x7FC00000);
     scal[1] = __int_as_float(0x7FC00000);
     return;
   }
-  // S as 11 little-endian 32-bit limbs (bins < 2^50, shifts < 254: < 2^304).
+  // S as 11 little-endian 32-bit limbs (used bins < 2^60 at indices <= 258:
+  // S < 2^318).
   constexpr int L = 11;
   uint32_t S[L];
 #pragma unroll
   for (int i = 0; i < L; ++i) S[i] = 0u;
-  for (int e = 0; e < 255; ++e) {
+  for (int e = 0; e < kPackNonFiniteBin; ++e) {
     const unsigned long long v = bins[e];
     if (v == 0ull) continue;
     const int sh = (e > 1 ? e : 1) - 1;
@@ -91,45 +140,39 @@ __global__ void absmean_finalize_kernel(const unsigned long long* __restrict__ b
       if (i - limb >= 2 && carry == 0ull) break;
     }
   }
-  // Long division of S * 2^F by n, one quotient bit at a time (MSB first).
+  // Long division of S * 2^F by n (n < 2^48), 16-bit digits MSB first: the
+  // remainder stays below n, so remainder * 2^16 + digit fits in 64 bits.
   constexpr int F = 32;
-  const int nbits = 32 * L + F;
+  constexpr int kDigits = (32 * L + F) / 16;  // 24
+  uint16_t qd[kDigits];
   unsigned long long rem = 0ull;
-  int lead = -1;        // bit index of the leading 1 of the quotient
-  uint32_t sig = 0u;    // leading 24 bits of the quotient
-  int taken = 0;        // bits collected into sig
-  uint32_t round_bit = 0u, sticky = 0u;
-  for (int i = nbits - 1; i >= 0; --i) {
-    uint32_t bit = 0u;
-    if (i >= F) {
-      const int j = i - F;
-      bit = (S[j >> 5] >> (j & 31)) & 1u;
+  for (int d = 0; d < kDigits; ++d) {
+    const int bit = 32 * L + F - 16 * (d + 1);  // weight of this digit's lowest bit in S * 2^F
+    uint32_t digit = 0u;
+    if (bit >= F) {
+      const int j = bit - F;
+      digit = (S[j >> 5] >> (j & 31)) & 0xFFFFu;
     }
-    rem = (rem << 1) | bit;
-    uint32_t qb = 0u;
-    if (rem >= n) {
-      rem -= n;
-      qb = 1u;
-    }
-    if (lead < 0) {
-      if (qb) {
-        lead = i;
-        sig = 1u;
-        taken = 1;
-      }
-    } else if (taken < 24) {
-      sig = (sig << 1) | qb;
-      ++taken;
-    } else if (taken == 24) {
-      round_bit = qb;
-      ++taken;
-    } else {
-      sticky |= qb;
-    }
+    const unsigned long long cur = (rem << 16) | digit;
+    qd[d] = (uint16_t)(cur / n);
+    rem = cur % n;
   }
-  sticky |= (rem != 0ull) ? 1u : 0u;
+  // Leading 24 bits of the quotient, the next (round) bit, and a sticky bit
+  // for every lower bit and the final remainder.
   float mean = 0.0f;
-  if (lead >= 0 && taken >= 25) {
+  int lead = -1;  // bit index (from the quotient's LSB) of its leading 1
+  for (int d = 0; d < kDigits && lead < 0; ++d)
+    if (qd[d] != 0) lead = 16 * (kDigits - 1 - d) + (31 - __clz((uint32_t)qd[d]));
+  if (lead >= 24) {
+    auto qbit = [&](int i) -> uint32_t {  // bit i of the quotient
+      const int d = kDigits - 1 - (i >> 4);
+      return ((uint32_t)qd[d] >> (i & 15)) & 1u;
+    };
+    uint32_t sig = 0u;
+    for (int i = lead; i > lead - 24; --i) sig = (sig << 1) | qbit(i);
+    const uint32_t round_bit = qbit(lead - 24);
+    uint32_t sticky = rem != 0ull ? 1u : 0u;
+    for (int i = lead - 25; i >= 0 && !sticky; --i) sticky |= qbit(i);
     int E = lead - 149 - F;  // value = 1.xxx * 2^E
     if (round_bit && (sticky || (sig & 1u))) {
       ++sig;
