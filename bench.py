@@ -510,10 +510,10 @@ def load_traffic(kernel):
             d = json.load(f)
         from bit_ternary_b200 import build
 
-        if d.get("sources_sha") != build.sources_sha():
-            return None
         v = d.get("kernels", {}).get(kernel)
-        return v.get("bytes_per_launch") if isinstance(v, dict) else v
+        if not isinstance(v, dict) or v.get("sha") != build.kernel_sha(kernel):
+            return None
+        return v.get("bytes_per_launch")
     except Exception:
         return None
 

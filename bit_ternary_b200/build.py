@@ -59,6 +59,25 @@ def sources_sha() -> str:
     return h.hexdigest()[:16]
 
 
+KERNEL_SOURCES = {
+    "gemv_kernel": ["bl_gemv.cu", "bl_device.cuh"],
+    "gemm_kernel": ["bl_gemm.cu", "bl_device.cuh"],
+}
+
+
+def kernel_sha(kernel: str) -> str:
+    """Hash of the source file that defines `kernel` and the device helpers it
+    uses: profiler counters taken for a kernel stay valid while this holds."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kernel]:
+        h.update(name.encode())
+        with open(os.path.join(CSRC, name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def up_to_date() -> bool:
     if not os.path.exists(LIB_PATH):
         return False
