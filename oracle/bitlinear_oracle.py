@@ -30,6 +30,9 @@ Readings where the pages are silent (each is listed in the design doc):
   * Bit order: code+1 for column k sits in bits [2*(k%16), 2*(k%16)+2) of word
     k/16 (LSB first); the row stride is exactly K/16 words.
   * y[m,n] = RN( RN(float(acc[m,n]) / s_x[m]) * D[n] ).
+  * bf16 inputs (the BitVLA checkpoint is a bf16 latent master, §1; the codes
+    are built from it, §2) are widened to fp32 exactly (a bf16 is the upper
+    half of an fp32) and then follow the fp32 definition above.
 
 Every step is fp32 with IEEE round-to-nearest-even (numpy float32 arithmetic);
 integer steps are exact (Python ints / int64).
@@ -57,6 +60,10 @@ __all__ = [
     "bitlinear_forward_rows",
     "fake_quant_linear",
     "round_fraction_to_f32",
+    "bf16_to_f32",
+    "pack_weights_bf16",
+    "act_quant_bf16",
+    "bitlinear_forward_bf16",
 ]
 
 
@@ -263,3 +270,33 @@ def fake_quant_linear(x: np.ndarray, W: np.ndarray) -> np.ndarray:
     xq = q.astype(np.float64) / s_x.astype(np.float64)[:, None]
     wq = codes.astype(np.float64) / np.float64(s)
     return xq @ wq.T
+
+
+# --------------------------------------------------------------------------
+# bf16 inputs
+# --------------------------------------------------------------------------
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    """bf16 values given as their 16-bit patterns (uint16) -> fp32, exactly.
+
+    BitVLA page §1: the checkpoint is a bf16 latent master, quantised on the
+    fly; §2 builds the codes from it. A bf16 is the upper 16 bits of the fp32
+    with the same value, so the widening is a shift of the bit pattern.
+    """
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def pack_weights_bf16(W_bits: np.ndarray):
+    """WeightQuant + pack of a bf16 master weight [N, K] (uint16 bit patterns)."""
+    return pack_weights(bf16_to_f32(W_bits))
+
+
+def act_quant_bf16(x_bits: np.ndarray):
+    """ActQuant of bf16 activations [M, K] (uint16 bit patterns)."""
+    return act_quant(bf16_to_f32(x_bits))
+
+
+def bitlinear_forward_bf16(x_bits: np.ndarray, packed: np.ndarray, D: np.ndarray, K: int,
+                           return_parts: bool = False):
+    """The forward from bf16 activations (uint16 bit patterns) [M, K]."""
+    return bitlinear_forward(bf16_to_f32(x_bits), packed, D, K, return_parts=return_parts)

@@ -384,3 +384,42 @@ def test_planted_mistake_is_caught(plant, monkeypatch, golden_dir):
     PLANTS[plant](monkeypatch)
     with pytest.raises(AssertionError):
         test_golden_hand_example_oracle(golden_dir)
+
+
+# ------------------------------------------------------------- bf16 inputs
+BF16_KNOWN = {  # bit pattern -> value (bf16 = sign, 8 exponent bits, 7 fraction bits)
+    0x3F80: 1.0, 0xC000: -2.0, 0x3E80: 0.25, 0x4049: 3.140625, 0x0001: 2.0 ** -133,
+    0x0080: 2.0 ** -126, 0x7F7F: (2.0 - 2.0 ** -7) * 2.0 ** 127, 0x8000: -0.0,
+    0x7F80: float("inf"), 0xFF80: float("-inf"),
+}
+
+
+def test_bf16_widening_known_values():
+    bits = np.array(sorted(BF16_KNOWN), dtype=np.uint16)
+    got = O.bf16_to_f32(bits)
+    want = np.array([BF16_KNOWN[int(b)] for b in bits], dtype=np.float64)
+    assert got.dtype == np.float32
+    assert np.array_equal(got.astype(np.float64), want)
+    assert np.signbit(got[bits.tolist().index(0x8000)])
+
+
+def test_bf16_widening_matches_library_on_every_pattern():
+    torch = pytest.importorskip("torch")
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    ours = O.bf16_to_f32(bits)
+    lib = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).float().numpy()
+    nan = np.isnan(lib)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan].view(np.uint32), lib[~nan].view(np.uint32))
+
+
+def test_bf16_round_trip_of_fp32_with_empty_low_half():
+    rng = np.random.default_rng(5)
+    v = (rng.standard_normal(1000).astype(np.float32).view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32)
+    assert np.array_equal(O.bf16_to_f32((v.view(np.uint32) >> 16).astype(np.uint16)), v)
+
+
+def test_bf16_widening_planted_mistake_is_caught(monkeypatch):
+    monkeypatch.setattr(O, "bf16_to_f32", lambda b: np.asarray(b, np.uint16).view(np.float16).astype(np.float32))
+    with pytest.raises(AssertionError):
+        test_bf16_widening_known_values()
