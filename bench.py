@@ -454,6 +454,11 @@ def run_ours(a):
     if not a.ncu_small:
         pack = bench_pack(B, torch, dev, stream, hbm_peak)
 
+    # ------------------------------------------------------------- bf16 inputs
+    bf16 = None
+    if not a.no_prefill and not a.ncu_small:
+        bf16 = bench_bf16(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, rank)
+
     # --------------------------------------------------------------- cpu baseline
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline and not a.ncu_small:
@@ -494,6 +499,7 @@ def run_ours(a):
         "prefill": prefill,
         "configs": configs,
         "pack": pack,
+        "bf16_inputs": bf16,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
@@ -644,6 +650,85 @@ def bench_configs(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_pea
                         "l2": f"rotates over {rot} copies"})
             del g, items, ws
             torch.cuda.empty_cache()
+    return out
+
+
+def bench_bf16(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, rank):
+    """bf16 inputs (bf16 master weights, bf16 activations; fp32 outputs), each against the HBM
+    roofline with bf16 bytes counted at 2 per element."""
+    out = {}
+    wl = WL.WORKLOADS[HEADLINE]
+    layers = list(wl.layers)
+    rot = 16
+    with torch.cuda.stream(stream):
+        base = []
+        for li, l in enumerate(layers):
+            W = torch.from_numpy(WL.weight(l.N, l.K, wl.w_dist, wl.seed + 17 * rank, layer=li)).to(dev)
+            base.append(B.pack_weights(W.to(torch.bfloat16)))
+            del W
+        packs = [[(p.clone(), D.clone()) for (p, D) in base] for _ in range(rot)]
+        xs = [[torch.from_numpy(WL.activations(1, l.K, wl.x_dist, wl.seed + r, layer=li, meta=wl.meta)).to(dev)
+               .to(torch.bfloat16) for li, l in enumerate(layers)] for r in range(rot)]
+        ys = [torch.empty((1, l.N), dtype=torch.float32, device=dev) for l in layers]
+        wss = [torch.zeros(max(256, B.workspace_size(1, l.N, l.K)), dtype=torch.uint8, device=dev) for l in layers]
+    torch.cuda.synchronize(dev)
+
+    def step(i):
+        r = i % rot
+        for li in range(len(layers)):
+            p, D = packs[r][li]
+            B.forward(xs[r][li], p, D, out=ys[li], ws=wss[li])
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i)
+    torch.cuda.synchronize(dev)
+    n = 64
+    g = capture(step, n)
+    with torch.cuda.stream(stream):
+        g.replay()
+    t = max_ranks(time_graph(g)) / n * 1e-3
+    nbytes = sum(l.N * l.K // 4 + 4 * l.N + 2 * l.K + 4 * l.N for l in layers)
+    out["decode_layer_set"] = {"us_per_step": round(t * 1e6, 2), "GB/s": round(nbytes / t / 1e9, 1),
+                               "frac_hbm": round(nbytes / t / 1e9 / hbm_peak, 4),
+                               "note": "four dependent bitlinear_forward_bf16 launches per step, M=1, "
+                                       f"weights rotating over {rot} copies"}
+    del g, packs, xs
+    M = PREFILL_M
+    aq = []
+    for K in (2560, 6912):
+        with torch.cuda.stream(stream):
+            xb = torch.from_numpy(WL.activations(M, K, "normal", 3, layer=K)).to(dev).to(torch.bfloat16)
+        torch.cuda.synchronize(dev)
+        g = capture(lambda i, xb=xb: B.quant_act(xb), 20)
+        with torch.cuda.stream(stream):
+            g.replay()
+        t = max_ranks(time_graph(g)) / 20 * 1e-3
+        qb = 2 * M * K + M * K + 12 * M
+        aq.append({"M": M, "K": K, "us": round(t * 1e6, 2), "GB/s": round(qb / t / 1e9, 1),
+                   "frac_hbm": round(qb / t / 1e9 / hbm_peak, 4)})
+        del g, xb
+    out["actquant"] = aq
+    l = layers[2]
+    with torch.cuda.stream(stream):
+        Wb = torch.from_numpy(WL.weight(l.N, l.K, "normal", 5)).to(dev).to(torch.bfloat16)
+        ws = torch.zeros(4096, dtype=torch.uint8, device=dev)
+        B.pack_weights(Wb, ws=ws)
+        torch.cuda.synchronize(dev)
+        ts = []
+        for _ in range(5):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            B.pack_weights(Wb, ws=ws)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+    t = statistics.median(ts) * 1e-3
+    alg = 2 * l.N * l.K + l.N * l.K // 4 + 4 * l.N
+    out["pack"] = {"layer": f"gate_up {l.K}->{l.N}", "ms": round(t * 1e3, 4),
+                   "GB/s_algorithmic": round(alg / t / 1e9, 1), "frac_hbm": round(alg / t / 1e9 / hbm_peak, 4)}
+    torch.cuda.empty_cache()
     return out
 
 

@@ -58,34 +58,46 @@ def workspace_size(M: int, N: int, K: int) -> int:
     return int(_lib.lib().bitlinear_workspace_size(M, N, K))
 
 
+def _float_input(t: torch.Tensor, name: str) -> str:
+    """'' for fp32, '_bf16' for bf16 (passed to the library as its bit patterns)."""
+    if t.dtype == torch.bfloat16:
+        _need_cuda(t, name, torch.bfloat16)
+        return "_bf16"
+    _need_cuda(t, name, torch.float32)
+    return ""
+
+
 def pack_weights(W: torch.Tensor, ws: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """WeightQuant + pack: fp32 W [N, K] -> (packed int32 [N, K/16], D fp32 [N, 1])."""
-    _need_cuda(W, "W", torch.float32)
+    """WeightQuant + pack: fp32 or bf16 W [N, K] -> (packed int32 [N, K/16], D fp32 [N, 1])."""
+    sfx = _float_input(W, "W")
     N, K = W.shape
     packed = torch.empty((N, K // 16), dtype=torch.int32, device=W.device)
     D = torch.empty((N, 1), dtype=torch.float32, device=W.device)
     L = _lib.lib()
     if ws is None:
         ws = _alloc_ws(L.bitlinear_pack_workspace_size(N, K), W.device)
-    _lib.call("bitlinear_pack_weights", W.data_ptr(), N, K, packed.data_ptr(), D.data_ptr(),
+    _lib.call("bitlinear_pack_weights" + sfx, W.data_ptr(), N, K, packed.data_ptr(), D.data_ptr(),
               ws.data_ptr(), ws.numel(), _stream_handle(W.device))
     return packed, D
 
 
 def quant_act(x: torch.Tensor):
-    """ActQuant: fp32 x [M, K] -> (q int8 [M, K], s_x fp32 [M], rowsum int32 [M])."""
-    _need_cuda(x, "x", torch.float32)
+    """ActQuant: fp32 or bf16 x [M, K] -> (q int8 [M, K], s_x fp32 [M], rowsum int32 [M])."""
+    sfx = _float_input(x, "x")
     M, K = x.shape
     q = torch.empty((M, K), dtype=torch.int8, device=x.device)
     s_x = torch.empty((M,), dtype=torch.float32, device=x.device)
     rs = torch.empty((M,), dtype=torch.int32, device=x.device)
-    _lib.call("bitlinear_quant_act", x.data_ptr(), M, K, q.data_ptr(), s_x.data_ptr(), rs.data_ptr(),
+    _lib.call("bitlinear_quant_act" + sfx, x.data_ptr(), M, K, q.data_ptr(), s_x.data_ptr(), rs.data_ptr(),
               _stream_handle(x.device))
     return q, s_x, rs
 
 
-def _fwd_args(x, packed, K):
-    _need_cuda(x, "x", torch.float32)
+def _fwd_args(x, packed, K, allow_bf16=False):
+    if not (allow_bf16 and x.dtype == torch.bfloat16):
+        _need_cuda(x, "x", torch.float32)
+    else:
+        _need_cuda(x, "x", torch.bfloat16)
     _need_cuda(packed, "packed", torch.int32)
     if x.dim() != 2 or packed.dim() != 2:
         raise ValueError("x must be [M, K] and packed [N, K/16]")
@@ -97,16 +109,17 @@ def _fwd_args(x, packed, K):
 
 def forward(x: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,
             out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """y = F.linear(ActQuant(x), WeightQuant(W)) from packed weights."""
+    """y = F.linear(ActQuant(x), WeightQuant(W)) from packed weights; x fp32 or bf16, y fp32."""
     K = x.shape[-1]
-    M, N = _fwd_args(x, packed, K)
+    M, N = _fwd_args(x, packed, K, allow_bf16=True)
+    fn = "bitlinear_forward_bf16" if x.dtype == torch.bfloat16 else "bitlinear_forward"
     _check_D(D, N)
     y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x.device)
     _need_cuda(y, "out", torch.float32)
     need = workspace_size(M, N, K)
     if ws is None:
         ws = _alloc_ws(need, x.device)
-    _lib.call("bitlinear_forward", x.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(), y.data_ptr(),
+    _lib.call(fn, x.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(), y.data_ptr(),
               ws.data_ptr(), ws.numel(), _stream_handle(x.device))
     return y
 

@@ -43,7 +43,8 @@ int check_mn(int64_t M, int64_t N) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? BL_OK : BL_ERR_CUDA; }
 
-int forward_impl(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D,
+// x is fp32 [M, K], or bf16 bit patterns when bf16.
+int forward_impl(const void* x, bool bf16, int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D,
                  float* y, int32_t* acc, void* ws, size_t ws_bytes, cudaStream_t stream) {
   int st = check_k(K);
   if (st != BL_OK) return st;
@@ -62,10 +63,10 @@ int forward_impl(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint32_t* err = reinterpret_cast<uint32_t*>(base);
   if (bl::gemv_group_fits(M, K)) {
-    const bl::GemvCall call{x, packed, D, y, acc, M, N, K};
+    const bl::GemvCall call{x, packed, D, y, acc, M, N, K, bf16};
     return cuda_status(bl::launch_gemv_group(&call, 1, err, false, stream, sms));
   }
-  cudaError_t e = bl::launch_act_quant(x, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
+  cudaError_t e = bl::launch_act_quant(x, bf16, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
                                        reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
                                        reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), true, stream, err);
   if (e != cudaSuccess) return BL_ERR_CUDA;
@@ -109,8 +110,8 @@ size_t bitlinear_pack_workspace_size(int64_t N, int64_t K) {
   return bl::kPackWsBytes;
 }
 
-int bitlinear_pack_weights(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
-                           size_t ws_bytes, bl_stream_t stream) {
+static int pack_impl(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
+                     size_t ws_bytes, bl_stream_t stream) {
   int st = check_k(K);
   if (st != BL_OK) return st;
   if (N <= 0 || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
@@ -120,15 +121,15 @@ int bitlinear_pack_weights(const float* W, int64_t N, int64_t K, uint32_t* packe
   const int sms = num_sms_current();
   if (sms <= 0) return BL_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (bl::launch_pack(W, N, K, packed, D, ws, s, sms) != cudaSuccess) return BL_ERR_CUDA;
+  if (bl::launch_pack(W, bf16, N, K, packed, D, ws, s, sms) != cudaSuccess) return BL_ERR_CUDA;
   uint32_t status = 0;
   if (cudaMemcpyAsync(&status, ws, sizeof(status), cudaMemcpyDeviceToHost, s) != cudaSuccess) return BL_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
   return status == 0u ? BL_OK : BL_ERR_NONFINITE;
 }
 
-int bitlinear_quant_act(const float* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
-                        bl_stream_t stream) {
+static int quant_act_impl(const void* x, bool bf16, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
+                          bl_stream_t stream) {
   int st = check_k(K);
   if (st != BL_OK) return st;
   if (M < 0 || M > 0x7FFFFFFF) return BL_ERR_SHAPE;
@@ -138,7 +139,27 @@ int bitlinear_quant_act(const float* x, int64_t M, int64_t K, int8_t* q, float* 
       (rowsum && (reinterpret_cast<uintptr_t>(rowsum) & 3u)))
     return BL_ERR_ALIGN;
   return cuda_status(
-      bl::launch_act_quant(x, M, K, q, s_x, rowsum, false, reinterpret_cast<cudaStream_t>(stream), nullptr));
+      bl::launch_act_quant(x, bf16, M, K, q, s_x, rowsum, false, reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
+int bitlinear_pack_weights(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
+                           size_t ws_bytes, bl_stream_t stream) {
+  return pack_impl(W, false, N, K, packed, D, ws, ws_bytes, stream);
+}
+
+int bitlinear_pack_weights_bf16(const uint16_t* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
+                                size_t ws_bytes, bl_stream_t stream) {
+  return pack_impl(W, true, N, K, packed, D, ws, ws_bytes, stream);
+}
+
+int bitlinear_quant_act(const float* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
+                        bl_stream_t stream) {
+  return quant_act_impl(x, false, M, K, q, s_x, rowsum, stream);
+}
+
+int bitlinear_quant_act_bf16(const uint16_t* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
+                             bl_stream_t stream) {
+  return quant_act_impl(x, true, M, K, q, s_x, rowsum, stream);
 }
 
 size_t bitlinear_workspace_size(int64_t M, int64_t N, int64_t K) {
@@ -150,13 +171,20 @@ size_t bitlinear_workspace_size(int64_t M, int64_t N, int64_t K) {
 int bitlinear_forward(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D,
                       float* y, void* ws, size_t ws_bytes, bl_stream_t stream) {
   if (y == nullptr && M > 0 && N > 0) return BL_ERR_NULL;
-  return forward_impl(x, M, N, K, packed, D, y, nullptr, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+  return forward_impl(x, false, M, N, K, packed, D, y, nullptr, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+int bitlinear_forward_bf16(const uint16_t* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                           const float* D, float* y, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  if (y == nullptr && M > 0 && N > 0) return BL_ERR_NULL;
+  return forward_impl(x, true, M, N, K, packed, D, y, nullptr, ws, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int bitlinear_forward_acc(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed, int32_t* acc,
                           void* ws, size_t ws_bytes, bl_stream_t stream) {
   if (acc == nullptr && M > 0 && N > 0) return BL_ERR_NULL;
-  return forward_impl(x, M, N, K, packed, nullptr, nullptr, acc, ws, ws_bytes,
+  return forward_impl(x, false, M, N, K, packed, nullptr, nullptr, acc, ws, ws_bytes,
                       reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -169,7 +197,7 @@ int bitlinear_prepare_act(const float* x, int64_t M, int64_t K, void* ws, size_t
   if (!aligned16(x) || !aligned256(ws)) return BL_ERR_ALIGN;
   if (ws_bytes < bl::ws_forward_bytes(M, K)) return BL_ERR_WORKSPACE;
   uint8_t* base = static_cast<uint8_t*>(ws);
-  return cuda_status(bl::launch_act_quant(x, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
+  return cuda_status(bl::launch_act_quant(x, false, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
                                           reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
                                           reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), true,
                                           reinterpret_cast<cudaStream_t>(stream), reinterpret_cast<uint32_t*>(base)));
@@ -268,14 +296,14 @@ int bitlinear_forward_batch(const bl_linear_call* calls, int count, uint32_t fla
         const int st = flush();
         if (st != BL_OK) return st;
       }
-      group[ng++] = bl::GemvCall{c.x, c.packed, c.D, c.y, nullptr, c.M, c.N, c.K};
+      group[ng++] = bl::GemvCall{c.x, c.packed, c.D, c.y, nullptr, c.M, c.N, c.K, false};
       gM = c.M > gM ? c.M : gM;
       gK = c.K > gK ? c.K : gK;
       continue;
     }
     int st = flush();
     if (st != BL_OK) return st;
-    st = forward_impl(c.x, c.M, c.N, c.K, c.packed, c.D, c.y, nullptr, ws, ws_bytes, s);
+    st = forward_impl(c.x, false, c.M, c.N, c.K, c.packed, c.D, c.y, nullptr, ws, ws_bytes, s);
     if (st != BL_OK) return st;
   }
   return flush();
@@ -305,7 +333,7 @@ static int forward_host_impl(const float* x_host, int64_t M, int64_t N, int64_t 
   float* yd = reinterpret_cast<float*>(base + fw + bl::align256(4 * (size_t)M * (size_t)K));
   if (cudaMemcpyAsync(xd, x_host, 4 * (size_t)M * (size_t)K, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return BL_ERR_CUDA;
-  st = forward_impl(xd, M, N, K, packed, D, yd, nullptr, ws, fw, s);
+  st = forward_impl(xd, false, M, N, K, packed, D, yd, nullptr, ws, fw, s);
   if (st != BL_OK) return st;
   if (cudaMemcpyAsync(y_host, yd, 4 * (size_t)M * (size_t)N, cudaMemcpyDeviceToHost, s) != cudaSuccess)
     return BL_ERR_CUDA;

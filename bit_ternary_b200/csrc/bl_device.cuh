@@ -247,6 +247,21 @@ __device__ __forceinline__ float div_by_scale(int32_t a, double inv) {
   return __double2float_rn(int_to_double_exact(a) * inv);
 }
 
+// Inputs are fp32, or bf16 given as 16-bit patterns. A bf16 is the upper half
+// of the fp32 with the same value, so widening it is exact. load4 reads the
+// four consecutive elements 4*i4 .. 4*i4+3 (16 bytes of fp32 or 8 of bf16).
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t bits16) { return __uint_as_float(bits16 << 16); }
+
+template <bool kBf16>
+__device__ __forceinline__ float4 load4(const void* p, int64_t i4) {
+  if (kBf16) {
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(p) + i4);
+    return make_float4(bf16_bits_to_float(v.x & 0xFFFFu), bf16_bits_to_float(v.x >> 16),
+                       bf16_bits_to_float(v.y & 0xFFFFu), bf16_bits_to_float(v.y >> 16));
+  }
+  return __ldg(reinterpret_cast<const float4*>(p) + i4);
+}
+
 // Ternary code of one weight: clamp(rint(RN(w*s)), -1, 1) + 1, in {0, 1, 2}.
 __device__ __forceinline__ uint32_t code_plus_one(float w, float s) {
   int c = __float2int_rn(__fmul_rn(w, s));

@@ -43,7 +43,7 @@ constexpr int kGemvThreads = 32 * kGemvWarps;
 constexpr int kGemvMaxGrid = 256;
 
 struct GemvProblem {
-  const float* x;
+  const void* x;  // fp32, or bf16 bit patterns (kBf16)
   const uint32_t* packed;
   const float* D;
   float* y;
@@ -225,7 +225,7 @@ __device__ __forceinline__ void flush_tile(const int (&acc)[4][DA][MT][4], int* 
     }
 }
 
-template <int MT, bool kAccOut>
+template <int MT, bool kAccOut, bool kBf16>
 __global__ void __launch_bounds__(kGemvThreads, MT == 1 ? 2 : 1) gemv_kernel(const __grid_constant__ GemvLaunch L) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int RT = L.round_tiles;                                           // tiles per round buffer
@@ -329,7 +329,6 @@ __global__ void __launch_bounds__(kGemvThreads, MT == 1 ? 2 : 1) gemv_kernel(con
           s_amax[(qs ^ 1) * 16 + tid] = 0u;
           s_rs[(qs ^ 1) * 16 + tid] = 0;
         }
-        const float4* x4 = reinterpret_cast<const float4*>(P.x);
         if (greg) {
           // One 16-column group per thread (groups never straddle tokens).
           int m = -1;
@@ -338,7 +337,7 @@ __global__ void __launch_bounds__(kGemvThreads, MT == 1 ? 2 : 1) gemv_kernel(con
             m = tid / G;
             float4 xg[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) xg[j] = __ldg(x4 + 4 * tid + j);
+            for (int j = 0; j < 4; ++j) xg[j] = load4<kBf16>(P.x, 4 * tid + j);
             a = fmaxf(fmaxf(absmax4(xg[0]), absmax4(xg[1])), fmaxf(absmax4(xg[2]), absmax4(xg[3])));
 #pragma unroll
             for (int j = 0; j < 4; ++j) s_xs[4 * tid + j] = xg[j];  // read back after the barrier
@@ -351,7 +350,7 @@ __global__ void __launch_bounds__(kGemvThreads, MT == 1 ? 2 : 1) gemv_kernel(con
             for (int j = 0; j < kXBatch; ++j) {
               const int i4 = base + j * kGemvThreads + tid;
               a[j] = 0.0f;
-              if (i4 < total4) a[j] = absmax4(__ldg(x4 + i4));
+              if (i4 < total4) a[j] = absmax4(load4<kBf16>(P.x, i4));
             }
 #pragma unroll
             for (int j = 0; j < kXBatch; ++j) {
@@ -364,7 +363,6 @@ __global__ void __launch_bounds__(kGemvThreads, MT == 1 ? 2 : 1) gemv_kernel(con
       for (int i = tid; i < (se - sa) * 16 * 8 * MT; i += kGemvThreads) s_acc[(sa - ra) * 16 * 8 * MT + i] = 0;
       if (newp) {
         __syncthreads();  // absmax complete
-        const float4* x4 = reinterpret_cast<const float4*>(P.x);
         if (greg) {
           int m = -1, sum = 0;
           if (tid < ngroups) {
@@ -400,7 +398,7 @@ __global__ void __launch_bounds__(kGemvThreads, MT == 1 ? 2 : 1) gemv_kernel(con
             for (int j = 0; j < kXBatch; ++j) {
               const int i4 = base + j * kGemvThreads + tid;
               v[j] = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (i4 < total4) v[j] = __ldg(x4 + i4);
+              if (i4 < total4) v[j] = load4<kBf16>(P.x, i4);
             }
 #pragma unroll
             for (int j = 0; j < kXBatch; ++j) {
@@ -562,9 +560,9 @@ __global__ void __launch_bounds__(kGemvThreads, MT == 1 ? 2 : 1) gemv_kernel(con
   }
 }
 
-template <int MT, bool kAccOut>
+template <int MT, bool kAccOut, bool kBf16>
 static cudaError_t launch_gemv_t(const GemvLaunch& L, int grid, size_t smem, bool pdl, cudaStream_t stream) {
-  auto kern = gemv_kernel<MT, kAccOut>;
+  auto kern = gemv_kernel<MT, kAccOut, kBf16>;
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -699,9 +697,21 @@ cudaError_t launch_gemv_group(const GemvCall* calls, int n, uint32_t* err, bool 
   if ((int64_t)smem > kGemvMaxSmem) return cudaErrorInvalidValue;
   const int grid = grid0;
   const bool accout = calls[0].acc != nullptr;
-  if (MT == 1) return accout ? launch_gemv_t<1, true>(L, grid, smem, pdl, stream)
-                             : launch_gemv_t<1, false>(L, grid, smem, pdl, stream);
-  return accout ? launch_gemv_t<2, true>(L, grid, smem, pdl, stream) : launch_gemv_t<2, false>(L, grid, smem, pdl, stream);
+  const bool bf16 = calls[0].bf16;
+  for (int i = 1; i < n; ++i)
+    if (calls[i].bf16 != bf16) return cudaErrorInvalidValue;  // one input type per launch
+#define BL_GEMV(MTV, AO, BF) \
+  if (MT == MTV && accout == AO && bf16 == BF) return launch_gemv_t<MTV, AO, BF>(L, grid, smem, pdl, stream);
+  BL_GEMV(1, false, false)
+  BL_GEMV(1, true, false)
+  BL_GEMV(2, false, false)
+  BL_GEMV(2, true, false)
+  BL_GEMV(1, false, true)
+  BL_GEMV(1, true, true)
+  BL_GEMV(2, false, true)
+  BL_GEMV(2, true, true)
+#undef BL_GEMV
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace bl

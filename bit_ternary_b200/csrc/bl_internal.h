@@ -26,12 +26,13 @@ constexpr int64_t kGemvMaxSmem = 200 * 1024;
 inline int64_t gemv_q_stride(int64_t K) { return ((K + 255) / 256) * 256 + 16; }
 
 struct GemvCall {
-  const float* x;
+  const void* x;   // fp32 [M, K], or bf16 bit patterns when bf16
   const uint32_t* packed;
   const float* D;
   float* y;        // fp32 output, or
   int32_t* acc;    // int32 accumulators (when non-null)
   int64_t M, N, K;
+  bool bf16;
 };
 
 int64_t gemv_stage_bytes(int64_t K);
@@ -42,10 +43,12 @@ bool gemv_group_fits(int64_t maxM, int64_t maxK);
 cudaError_t launch_gemv_group(const GemvCall* calls, int n, uint32_t* err, bool pdl, cudaStream_t stream,
                               int num_sms);
 
-cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
+// W is fp32, or bf16 bit patterns when bf16 (widened exactly).
+cudaError_t launch_pack(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
                         cudaStream_t stream, int num_sms);
 // err_reset (nullable): the workspace error word, cleared by the kernel.
-cudaError_t launch_act_quant(const float* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
+// x is fp32, or bf16 bit patterns when bf16 (widened exactly).
+cudaError_t launch_act_quant(const void* x, bool bf16, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
                              bool permuted, cudaStream_t stream, uint32_t* err_reset);
 // Natural-order int8 codes and scales (bitlinear_quant_act's output) into the
 // forward workspace layout (private order, row sums); err_reset as above.

@@ -29,7 +29,8 @@ constexpr int kWindow = 38;  // binades below a batch's largest exponent summed 
 // base+42 of a per-warp shared copy. Weights below the window go to their own
 // bin. Every step is integer arithmetic, so the result does not depend on the
 // order of the reduction.
-__global__ void __launch_bounds__(kBinThreads) absum_bins_kernel(const float4* __restrict__ W, int64_t n4,
+template <bool kBf16>
+__global__ void __launch_bounds__(kBinThreads) absum_bins_kernel(const void* __restrict__ W, int64_t n4,
                                                                   unsigned long long* __restrict__ bins) {
   __shared__ unsigned long long sbins[kBinWarps][kPackBins];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -44,7 +45,7 @@ __global__ void __launch_bounds__(kBinThreads) absum_bins_kernel(const float4* _
     uint32_t m[4], ee[4];
     uint32_t emax = 0u, nonfinite = 0u;
     if (i < n4) {
-      const float4 v = __ldg(W + i);
+      const float4 v = load4<kBf16>(W, i);
       const float vals[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -192,7 +193,8 @@ __global__ void absmean_finalize_kernel(const unsigned long long* __restrict__ b
 // Each thread ternarises one float4 (4 codes = one byte of a packed word);
 // lanes 4j..4j+3 of a warp hold the four bytes of one word and combine them
 // with shuffles. Also writes D[n] = mean_c.
-__global__ void __launch_bounds__(256) ternarize_pack_kernel(const float4* __restrict__ W, int64_t n4,
+template <bool kBf16>
+__global__ void __launch_bounds__(256) ternarize_pack_kernel(const void* __restrict__ W, int64_t n4,
                                                              const float* __restrict__ scal,
                                                              const uint32_t* __restrict__ status,
                                                              uint32_t* __restrict__ packed, float* __restrict__ D,
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(256) ternarize_pack_kernel(const float4* __res
     const int64_t i = base + lane;
     uint32_t byte = 0u;
     if (i < n4) {
-      const float4 v = __ldg(W + i);
+      const float4 v = load4<kBf16>(W, i);
       byte = code_plus_one(v.x, s) | (code_plus_one(v.y, s) << 2) | (code_plus_one(v.z, s) << 4) |
              (code_plus_one(v.w, s) << 6);
     }
@@ -224,8 +226,8 @@ __global__ void __launch_bounds__(256) ternarize_pack_kernel(const float4* __res
 // One CTA per token row. Pass 1: max|x| (exact). Pass 2: quantise 16 columns
 // per thread-iteration and store them as one 16-byte vector, in natural
 // column order or in the kernel-private order perm16 (see bl_device.cuh).
-template <bool kPerm>
-__global__ void __launch_bounds__(256) act_quant_kernel(const float* __restrict__ x, int64_t K,
+template <bool kPerm, bool kBf16>
+__global__ void __launch_bounds__(256) act_quant_kernel(const void* __restrict__ x, int64_t K,
                                                         int8_t* __restrict__ q, float* __restrict__ s_out,
                                                         int32_t* __restrict__ rowsum_out,
                                                         uint32_t* __restrict__ err_reset) {
@@ -233,7 +235,7 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const float* __restrict_
   __shared__ float red_f[8];
   __shared__ int red_i[8];
   const int64_t m = blockIdx.x;
-  const float4* xr = reinterpret_cast<const float4*>(x + m * K);
+  const int64_t xr = m * (K >> 2);  // first float4 (group of 4 elements) of the row
   const int ngroups = (int)(K >> 4);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
@@ -242,7 +244,7 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const float* __restrict_
   for (int g = threadIdx.x; g < ngroups; g += blockDim.x) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float4 v = __ldg(xr + 4 * g + j);
+      const float4 v = load4<kBf16>(x, xr + 4 * g + j);
       amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
     }
   }
@@ -260,7 +262,7 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const float* __restrict_
     int v[16];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float4 f = __ldg(xr + 4 * g + j);
+      const float4 f = load4<kBf16>(x, xr + 4 * g + j);
       v[4 * j + 0] = quant_i8(f.x, sx);
       v[4 * j + 1] = quant_i8(f.y, sx);
       v[4 * j + 2] = quant_i8(f.z, sx);
@@ -315,8 +317,8 @@ cudaError_t launch_selftest_wait(uint32_t* err, uint64_t limit_ns, cudaStream_t 
 // Register-resident variant for rows of up to 256 * 16 * kG columns: each
 // thread loads its kG groups of 16 values once, the block reduces max|x|, and
 // the same registers are quantised and stored (one read of x, one write of q).
-template <bool kPerm, int kG>
-__global__ void __launch_bounds__(256) act_quant_reg_kernel(const float* __restrict__ x, int64_t K,
+template <bool kPerm, int kG, bool kBf16>
+__global__ void __launch_bounds__(256) act_quant_reg_kernel(const void* __restrict__ x, int64_t K,
                                                             int8_t* __restrict__ q, float* __restrict__ s_out,
                                                             int32_t* __restrict__ rowsum_out,
                                                             uint32_t* __restrict__ err_reset) {
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(256) act_quant_reg_kernel(const float* __restr
   __shared__ int red_i[8];
   if (err_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err_reset = 0u;
   const int64_t m = blockIdx.x;
-  const float4* xr = reinterpret_cast<const float4*>(x + m * K);
+  const int64_t xr = m * (K >> 2);  // first float4 (group of 4 elements) of the row
   const int ngroups = (int)(K >> 4);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
@@ -334,7 +336,10 @@ __global__ void __launch_bounds__(256) act_quant_reg_kernel(const float* __restr
   for (int i = 0; i < kG; ++i) {
     const int g = threadIdx.x + i * blockDim.x;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) f[i][j] = g < ngroups ? __ldg(xr + 4 * g + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int j = 0; j < 4; ++j) {
+      f[i][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (g < ngroups) f[i][j] = load4<kBf16>(x, xr + 4 * g + j);
+    }
 #pragma unroll
     for (int j = 0; j < 4; ++j)
       amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f[i][j].x), fabsf(f[i][j].y)), fmaxf(fabsf(f[i][j].z), fabsf(f[i][j].w))));
@@ -388,7 +393,7 @@ __global__ void __launch_bounds__(256) act_quant_reg_kernel(const float* __restr
 }
 
 // ------------------------------------------------------------ launchers --
-cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
+cudaError_t launch_pack(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
                         cudaStream_t stream, int num_sms) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint32_t* status = reinterpret_cast<uint32_t*>(base);
@@ -399,12 +404,17 @@ cudaError_t launch_pack(const float* W, int64_t N, int64_t K, uint32_t* packed, 
   const int64_t n4 = N * K / 4;
   const int64_t want = (n4 + kBinThreads * 8 - 1) / (kBinThreads * 8);
   const int grid1 = (int)(want < 4 * num_sms ? (want < 1 ? 1 : want) : 4 * num_sms);
-  absum_bins_kernel<<<grid1, kBinThreads, 0, stream>>>(reinterpret_cast<const float4*>(W), n4, bins);
+  if (bf16)
+    absum_bins_kernel<true><<<grid1, kBinThreads, 0, stream>>>(W, n4, bins);
+  else
+    absum_bins_kernel<false><<<grid1, kBinThreads, 0, stream>>>(W, n4, bins);
   absmean_finalize_kernel<<<1, 32, 0, stream>>>(bins, (uint64_t)(N * K), scal, status);
   const int64_t want2 = (n4 + 255) / 256;
   const int grid2 = (int)(want2 < 16 * num_sms ? (want2 < 1 ? 1 : want2) : 16 * num_sms);
-  ternarize_pack_kernel<<<grid2, 256, 0, stream>>>(reinterpret_cast<const float4*>(W), n4, scal, status, packed,
-                                                    D, N);
+  if (bf16)
+    ternarize_pack_kernel<true><<<grid2, 256, 0, stream>>>(W, n4, scal, status, packed, D, N);
+  else
+    ternarize_pack_kernel<false><<<grid2, 256, 0, stream>>>(W, n4, scal, status, packed, D, N);
   return cudaGetLastError();
 }
 
@@ -453,8 +463,9 @@ cudaError_t launch_q_prepare(const int8_t* q, const float* s_x, int64_t M, int64
   return cudaGetLastError();
 }
 
-cudaError_t launch_act_quant(const float* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
-                             bool permuted, cudaStream_t stream, uint32_t* err_reset) {
+template <bool kBf16>
+static cudaError_t launch_act_quant_t(const void* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
+                                      bool permuted, cudaStream_t stream, uint32_t* err_reset) {
   const int64_t ngroups = K / 16;
   // Rows of up to 256 threads x 4 groups x 16 values stay in registers.
   int kg = (int)((ngroups + 255) / 256);
@@ -462,7 +473,7 @@ cudaError_t launch_act_quant(const float* x, int64_t M, int64_t K, int8_t* q, fl
     kg = kg <= 1 ? 1 : (kg <= 2 ? 2 : 4);
     int threads = (int)(((ngroups + kg - 1) / kg + 31) / 32 * 32);
     if (threads < 32) threads = 32;
-#define BL_AQ(P, G) act_quant_reg_kernel<P, G><<<(unsigned)M, threads, 0, stream>>>(x, K, q, s_x, rowsum, err_reset)
+#define BL_AQ(P, G) act_quant_reg_kernel<P, G, kBf16><<<(unsigned)M, threads, 0, stream>>>(x, K, q, s_x, rowsum, err_reset)
     if (permuted) {
       if (kg == 1) BL_AQ(true, 1); else if (kg == 2) BL_AQ(true, 2); else BL_AQ(true, 4);
     } else {
@@ -474,10 +485,16 @@ cudaError_t launch_act_quant(const float* x, int64_t M, int64_t K, int8_t* q, fl
   const int threads = 256;
   // One CTA per token; grids beyond 2^31-1 are rejected by validation.
   if (permuted)
-    act_quant_kernel<true><<<(unsigned)M, threads, 0, stream>>>(x, K, q, s_x, rowsum, err_reset);
+    act_quant_kernel<true, kBf16><<<(unsigned)M, threads, 0, stream>>>(x, K, q, s_x, rowsum, err_reset);
   else
-    act_quant_kernel<false><<<(unsigned)M, threads, 0, stream>>>(x, K, q, s_x, rowsum, err_reset);
+    act_quant_kernel<false, kBf16><<<(unsigned)M, threads, 0, stream>>>(x, K, q, s_x, rowsum, err_reset);
   return cudaGetLastError();
+}
+
+cudaError_t launch_act_quant(const void* x, bool bf16, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
+                             bool permuted, cudaStream_t stream, uint32_t* err_reset) {
+  return bf16 ? launch_act_quant_t<true>(x, M, K, q, s_x, rowsum, permuted, stream, err_reset)
+              : launch_act_quant_t<false>(x, M, K, q, s_x, rowsum, permuted, stream, err_reset);
 }
 
 }  // namespace bl

@@ -99,6 +99,15 @@ BL_API int bitlinear_pack_weights(const float* W, int64_t N, int64_t K,
                            uint32_t* packed, float* D,
                            void* ws, size_t ws_bytes, bl_stream_t stream);
 
+/* As bitlinear_pack_weights, from a bf16 master weight: W holds the bf16 bit
+ * patterns [N, K] (uint16, 16-byte aligned). Each value is widened to fp32
+ * exactly (a bf16 is the upper half of an fp32), then quantised as above
+ * ("Core AI model zoo - BitVLA" section 1: the checkpoint is a bf16 latent
+ * master, quantised on the fly). Synchronous. */
+BL_API int bitlinear_pack_weights_bf16(const uint16_t* W, int64_t N, int64_t K,
+                                       uint32_t* packed, float* D,
+                                       void* ws, size_t ws_bytes, bl_stream_t stream);
+
 /* ------------------------------------------------------------ ActQuant --- */
 
 /* Per-token int8 absmax quantisation (BitVLA page section 1).
@@ -110,6 +119,11 @@ BL_API int bitlinear_pack_weights(const float* W, int64_t N, int64_t K,
 BL_API int bitlinear_quant_act(const float* x, int64_t M, int64_t K,
                         int8_t* q, float* s_x, int32_t* rowsum,
                         bl_stream_t stream);
+
+/* As bitlinear_quant_act, from bf16 activations (uint16 bit patterns [M, K],
+ * widened to fp32 exactly). Asynchronous. */
+BL_API int bitlinear_quant_act_bf16(const uint16_t* x, int64_t M, int64_t K,
+                                    int8_t* q, float* s_x, int32_t* rowsum, bl_stream_t stream);
 
 /* ------------------------------------------------------------- forward --- */
 
@@ -132,6 +146,13 @@ BL_API size_t bitlinear_workspace_size(int64_t M, int64_t N, int64_t K);
 BL_API int bitlinear_forward(const float* x, int64_t M, int64_t N, int64_t K,
                       const uint32_t* packed, const float* D, float* y,
                       void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* As bitlinear_forward, from bf16 activations: x holds bf16 bit patterns
+ * [M, K] (uint16, 16-byte aligned), widened to fp32 exactly inside the
+ * quantiser; y is fp32 [M, N]. Same workspace. Asynchronous. */
+BL_API int bitlinear_forward_bf16(const uint16_t* x, int64_t M, int64_t N, int64_t K,
+                                  const uint32_t* packed, const float* D, float* y,
+                                  void* ws, size_t ws_bytes, bl_stream_t stream);
 
 /* As bitlinear_forward, but writes the exact int32 accumulators
  * acc[m,n] = sum_k q[m,k] * code[n,k] to device int32 [M, N] instead of y. */

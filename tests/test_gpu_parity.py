@@ -469,3 +469,52 @@ def test_forward_batch_rejects_before_launch(B):
     bad_y = torch.zeros(1 * 64 + 1, device="cuda")[1:].view(1, 64)
     with pytest.raises(BitLinearError, match="ALIGN"):
         B.forward_batch([good, (good[0], packed, D, bad_y)])
+
+
+# ------------------------------------------------------------ bf16 inputs
+def _bf16(a):
+    """fp32 numpy array -> (bf16 CUDA tensor, its uint16 bit patterns)."""
+    t = torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16)
+    bits = t.view(torch.int16).numpy().view(np.uint16).copy()
+    return t.cuda(), bits
+
+
+@pytest.mark.parametrize("N,K,dist", [(3, 48, "normal"), (257, 6912, "laplace"), (2560, 2560, "normal"),
+                                      (33, 1152, "laplace")])
+def test_pack_bf16_bitexact(B, N, K, dist):
+    Wt, bits = _bf16(WL.weight(N, K, dist, 40 + K))
+    packed, D = B.pack_weights(Wt)
+    p_ref, D_ref = O.pack_weights_bf16(bits)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)
+    assert np.array_equal(D.cpu().numpy(), D_ref)
+
+
+def test_pack_bf16_special_values(B):
+    bits = np.array([[0x0001, 0x8001, 0x0000, 0x8000, 0x3F80, 0xBF80, 0x0080, 0x7F7F] * 2], dtype=np.uint16)
+    Wt = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).cuda()
+    packed, D = B.pack_weights(Wt)
+    p_ref, D_ref = O.pack_weights_bf16(bits)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)
+    assert np.array_equal(D.cpu().numpy(), D_ref)
+
+
+@pytest.mark.parametrize("M,K", [(1, 2560), (3, 528), (64, 6912), (17, 16400)])
+def test_quant_act_bf16_bitexact(B, M, K):
+    xt, bits = _bf16(WL.activations(M, K, "student_t", 50 + K, meta={"df": 3.0}))
+    q, s_x, rs = B.quant_act(xt)
+    q_ref, s_ref = O.act_quant_bf16(bits)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s_x.cpu().numpy(), s_ref)
+    assert np.array_equal(rs.cpu().numpy(), q_ref.astype(np.int64).sum(axis=1))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 3840, 2560), (1, 2560, 6912), (5, 257, 528), (16, 300, 2560),
+                                   (40, 700, 1152), (300, 129, 6912)])
+def test_forward_bf16(B, M, N, K):
+    """bf16 master weight and bf16 activations, decode (M <= 16) and tensor-core paths."""
+    Wt, wbits = _bf16(WL.weight(N, K, "normal", 70 + N))
+    xt, xbits = _bf16(WL.activations(M, K, "student_t", 71 + M, meta={"df": 3.0}))
+    packed, D = B.pack_weights(Wt)
+    p_ref, D_ref = O.pack_weights_bf16(wbits)
+    y = B.forward(xt, packed, D).cpu().numpy()
+    assert_y_close(y, O.bitlinear_forward_bf16(xbits, p_ref, D_ref, K))
