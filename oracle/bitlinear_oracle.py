@@ -30,6 +30,10 @@ Readings where the pages are silent (each is listed in the design doc):
   * Bit order: code+1 for column k sits in bits [2*(k%16), 2*(k%16)+2) of word
     k/16 (LSB first); the row stride is exactly K/16 words.
   * y[m,n] = RN( RN(float(acc[m,n]) / s_x[m]) * D[n] ).
+  * Per-projection RMSNorm before ActQuant ("BitNet-Embeddings I2_S guide"
+    §3.1; rms_norm_eps = 1e-6): ms = mean(x^2) over the row is the exact real
+    mean, correctly rounded to fp32 once; r = RN(1/RN(sqrt(RN(ms + eps))));
+    n = RN(RN(x*r)*g); then ActQuant of n.
   * bf16 inputs (the BitVLA checkpoint is a bf16 latent master, §1; the codes
     are built from it, §2) are widened to fp32 exactly (a bf16 is the upper
     half of an fp32) and then follow the fp32 definition above.
@@ -64,6 +68,11 @@ __all__ = [
     "pack_weights_bf16",
     "act_quant_bf16",
     "bitlinear_forward_bf16",
+    "RMS_EPS",
+    "mean_square_exact",
+    "rmsnorm",
+    "rmsnorm_act_quant",
+    "bitlinear_forward_rmsnorm",
 ]
 
 
@@ -300,3 +309,59 @@ def bitlinear_forward_bf16(x_bits: np.ndarray, packed: np.ndarray, D: np.ndarray
                            return_parts: bool = False):
     """The forward from bf16 activations (uint16 bit patterns) [M, K]."""
     return bitlinear_forward(bf16_to_f32(x_bits), packed, D, K, return_parts=return_parts)
+
+
+# --------------------------------------------------------------------------
+# Per-projection RMSNorm + ActQuant
+# --------------------------------------------------------------------------
+RMS_EPS = np.float32(1e-6)
+
+
+def mean_square_exact(row: np.ndarray) -> np.float32:
+    """mean(x^2) over one row: exact sum of squares, correctly rounded division.
+
+    x = m * 2^(ee-150) (ee = max(biased exponent, 1), m the 24-bit
+    significand), so x^2 = m^2 * 2^(2*(ee-1)) units of 2^-298: integer sums,
+    then one rounding of the exact rational to fp32.
+    """
+    a = np.ascontiguousarray(row, dtype=np.float32).reshape(-1)
+    bits = a.view(np.uint32) & np.uint32(0x7FFFFFFF)
+    exps = (bits >> np.uint32(23)).astype(np.int64)
+    if np.any(exps == 255):
+        raise FloatingPointError("non-finite activation")
+    mant = (bits & np.uint32(0x7FFFFF)).astype(np.int64)
+    mant = np.where(exps > 0, mant | (1 << 23), mant)
+    total = 0  # in units of 2^-298
+    for m, e in zip(mant.tolist(), exps.tolist()):
+        if m:
+            total += (m * m) << (2 * (max(e, 1) - 1))
+    return round_fraction_to_f32(Fraction(total, a.size) / (Fraction(2) ** 298))
+
+
+def rmsnorm(x: np.ndarray, g: np.ndarray, eps: np.float32 = RMS_EPS) -> np.ndarray:
+    """n = RMSNorm(x, g) per row, in fp32 (I2_S guide §3.1: each projection
+    normalises its input with its own norm.weight g before activation_quant).
+
+    ms = mean(x^2) exact, rounded once; r = RN(1 / RN(sqrt(RN(ms + eps))));
+    n[k] = RN(RN(x[k] * r) * g[k]).
+    """
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    g = np.ascontiguousarray(g, dtype=np.float32).reshape(1, -1)
+    out = np.empty_like(x)
+    for i in range(x.shape[0]):
+        ms = mean_square_exact(x[i])
+        v = np.float32(ms + np.float32(eps))
+        r = np.float32(np.float32(1.0) / np.sqrt(v))
+        out[i] = ((x[i] * r).astype(np.float32) * g[0]).astype(np.float32)
+    return out
+
+
+def rmsnorm_act_quant(x: np.ndarray, g: np.ndarray, eps: np.float32 = RMS_EPS):
+    """ActQuant(RMSNorm(x, g)): q int8 [M, K], s_x fp32 [M]."""
+    return act_quant(rmsnorm(x, g, eps))
+
+
+def bitlinear_forward_rmsnorm(x: np.ndarray, g: np.ndarray, packed: np.ndarray, D: np.ndarray, K: int,
+                              eps: np.float32 = RMS_EPS, return_parts: bool = False):
+    """y = F.linear(ActQuant(RMSNorm(x, g)), WeightQuant(W)) (I2_S guide §3.1 chain)."""
+    return bitlinear_forward(rmsnorm(x, g, eps), packed, D, K, return_parts=return_parts)

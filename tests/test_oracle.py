@@ -423,3 +423,67 @@ def test_bf16_widening_planted_mistake_is_caught(monkeypatch):
     monkeypatch.setattr(O, "bf16_to_f32", lambda b: np.asarray(b, np.uint16).view(np.float16).astype(np.float32))
     with pytest.raises(AssertionError):
         test_bf16_widening_known_values()
+
+
+# ------------------------------------------------------- RMSNorm + ActQuant
+def _rms_ref64(x, g, eps):
+    """fp64 RMSNorm from torch's own routine (a library reference)."""
+    torch = pytest.importorskip("torch")
+    xt = torch.from_numpy(x.astype(np.float64))
+    gt = torch.from_numpy(g.astype(np.float64))
+    return torch.nn.functional.rms_norm(xt, (x.shape[1],), gt, float(eps)).numpy()
+
+
+def test_rmsnorm_matches_library_fp64_within_rounding():
+    rng = np.random.default_rng(11)
+    x = np.concatenate([rng.standard_normal((6, 1024)), 20 * rng.standard_t(3, (2, 1024))]).astype(np.float32)
+    x[1] *= np.float32(1e-3)
+    g = rng.uniform(0.5, 2.0, 1024).astype(np.float32)
+    n = O.rmsnorm(x, g)
+    ref = _rms_ref64(x, g, O.RMS_EPS)
+    ulp = np.spacing(np.abs(n).astype(np.float32)).astype(np.float64)
+    assert np.all(np.abs(n.astype(np.float64) - ref) <= 4 * ulp)
+
+
+def test_mean_square_exact_brute_force_rational():
+    from fractions import Fraction
+    rng = np.random.default_rng(12)
+    for K in (16, 48, 96):
+        for scale in (1.0, 1e-20, 1e18, 1e-42):
+            row = (rng.standard_normal(K) * scale).astype(np.float32)
+            want = O.round_fraction_to_f32(sum(Fraction(float(v)) ** 2 for v in row) / K)
+            assert O.mean_square_exact(row) == want
+
+
+def test_mean_square_exact_tie_rounds_to_even():
+    a = np.float32(1 + 2.0 ** -12)  # a^2 = 1 + 2^-11 + 2^-24: halfway between two fp32 neighbours
+    assert O.mean_square_exact(np.full(32, a, np.float32)) == np.float32(1 + 2.0 ** -11)
+    # b^2 = 1 + 4098.5*2^-23 + 2^-34 + 2^-46: a hair above a midpoint, so it rounds up to 4099
+    b = np.float32(1 + 2.0 ** -12 + 2.0 ** -23)
+    assert O.mean_square_exact(np.full(16, b, np.float32)) == np.float32(1 + 4099 * 2.0 ** -23)
+    c = np.float32(1 + 3 * 2.0 ** -12)  # c^2 = 1 + 12292.5*2^-23 exactly: a tie, to the even 12292
+    assert O.mean_square_exact(np.full(16, c, np.float32)) == np.float32(1 + 12292 * 2.0 ** -23)
+
+
+def test_rmsnorm_act_quant_constant_row_and_g_scaling():
+    x = np.full((2, 64), 3.0, np.float32)
+    g = np.ones(64, np.float32)
+    q, s = O.rmsnorm_act_quant(x, g)
+    assert np.all(q == 127)
+    q2, s2 = O.rmsnorm_act_quant(x, 2 * g)  # n doubles exactly: same codes, half the scale
+    assert np.array_equal(q, q2) and np.array_equal(s2, s / np.float32(2))
+
+
+RMS_PLANTS = {
+    "mean_over_k_minus_1": lambda row: O.round_fraction_to_f32(
+        sum(__import__("fractions").Fraction(float(v)) ** 2 for v in row) / (row.size - 1)),
+    "no_square": lambda row: O.round_fraction_to_f32(
+        sum(abs(__import__("fractions").Fraction(float(v))) for v in row) / row.size),
+}
+
+
+@pytest.mark.parametrize("plant", sorted(RMS_PLANTS))
+def test_rmsnorm_planted_mistake_is_caught(plant, monkeypatch):
+    monkeypatch.setattr(O.bitlinear_oracle, "mean_square_exact", RMS_PLANTS[plant])
+    with pytest.raises(AssertionError):
+        test_rmsnorm_matches_library_fp64_within_rounding()
