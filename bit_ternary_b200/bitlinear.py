@@ -24,6 +24,9 @@ __all__ = [
     "forward_batch",
     "prepare_act",
     "forward_prepared",
+    "forward_q",
+    "rmsnorm_quant_act",
+    "forward_rmsnorm",
     "workspace_size",
     "workspace_error",
     "BitLinear",
@@ -181,6 +184,39 @@ def forward_q(q: torch.Tensor, s_x: torch.Tensor, packed: torch.Tensor, D: torch
         ws = _alloc_ws(_lib.lib().bitlinear_workspace_size(M, N, K), q.device)
     _lib.call("bitlinear_forward_q", q.data_ptr(), s_x.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(),
               y.data_ptr(), ws.data_ptr(), ws.numel(), _stream_handle(q.device))
+    return y
+
+
+def rmsnorm_quant_act(x: torch.Tensor, g: torch.Tensor, eps: float = 1e-6):
+    """ActQuant(RMSNorm(x, g)): fp32 x [M, K], norm weight g [K] -> (q int8 [M, K], s_x [M], rowsum [M])."""
+    _need_cuda(x, "x", torch.float32)
+    _need_cuda(g, "g", torch.float32)
+    M, K = x.shape
+    if g.numel() != K:
+        raise ValueError("g must hold K weights")
+    q = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    s_x = torch.empty((M,), dtype=torch.float32, device=x.device)
+    rs = torch.empty((M,), dtype=torch.int32, device=x.device)
+    _lib.call("bitlinear_rmsnorm_quant_act", x.data_ptr(), g.data_ptr(), float(eps), M, K, q.data_ptr(),
+              s_x.data_ptr(), rs.data_ptr(), _stream_handle(x.device))
+    return q, s_x, rs
+
+
+def forward_rmsnorm(x: torch.Tensor, g: torch.Tensor, packed: torch.Tensor, D: torch.Tensor, eps: float = 1e-6,
+                    out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = F.linear(ActQuant(RMSNorm(x, g)), WeightQuant(W)) from packed weights."""
+    K = x.shape[-1]
+    M, N = _fwd_args(x, packed, K)
+    _need_cuda(g, "g", torch.float32)
+    if g.numel() != K:
+        raise ValueError("g must hold K weights")
+    _check_D(D, N)
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _need_cuda(y, "out", torch.float32)
+    if ws is None:
+        ws = _alloc_ws(workspace_size(M, N, K), x.device)
+    _lib.call("bitlinear_forward_rmsnorm", x.data_ptr(), g.data_ptr(), float(eps), M, N, K, packed.data_ptr(),
+              D.data_ptr(), y.data_ptr(), ws.data_ptr(), ws.numel(), _stream_handle(x.device))
     return y
 
 

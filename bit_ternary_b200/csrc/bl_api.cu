@@ -241,6 +241,48 @@ int bitlinear_forward_q(const int8_t* q, const float* s_x, int64_t M, int64_t N,
   return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, nullptr, ws, s, sms));
 }
 
+int bitlinear_rmsnorm_quant_act(const float* x, const float* g, float eps, int64_t M, int64_t K, int8_t* q,
+                                float* s_x, int32_t* rowsum, bl_stream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  if (K > bl::kRmsMaxK || M < 0 || M > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  if (M == 0) return BL_OK;
+  if (x == nullptr || g == nullptr || q == nullptr || s_x == nullptr) return BL_ERR_NULL;
+  if (!aligned16(x) || !aligned16(g) || !aligned16(q) || (reinterpret_cast<uintptr_t>(s_x) & 3u) ||
+      (rowsum && (reinterpret_cast<uintptr_t>(rowsum) & 3u)))
+    return BL_ERR_ALIGN;
+  if (!(eps >= 0.0f) || eps > 1e30f) return BL_ERR_SHAPE;
+  return cuda_status(bl::launch_rms_act_quant(x, g, eps, M, K, q, s_x, rowsum, false,
+                                              reinterpret_cast<cudaStream_t>(stream), nullptr));
+}
+
+int bitlinear_forward_rmsnorm(const float* x, const float* g, float eps, int64_t M, int64_t N, int64_t K,
+                              const uint32_t* packed, const float* D, float* y, void* ws, size_t ws_bytes,
+                              bl_stream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  st = check_mn(M, N);
+  if (st != BL_OK) return st;
+  if (K > bl::kRmsMaxK) return BL_ERR_SHAPE;
+  if (M == 0 || N == 0) return BL_OK;
+  if (x == nullptr || g == nullptr || packed == nullptr || D == nullptr || y == nullptr || ws == nullptr)
+    return BL_ERR_NULL;
+  if (!aligned16(x) || !aligned16(g) || !aligned16(packed) || !aligned16(D) || !aligned16(y) || !aligned256(ws))
+    return BL_ERR_ALIGN;
+  if (!(eps >= 0.0f) || eps > 1e30f) return BL_ERR_SHAPE;
+  if (ws_bytes < bitlinear_workspace_size(M, N, K)) return BL_ERR_WORKSPACE;
+  const int sms = num_sms_current();
+  if (sms <= 0) return BL_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  st = cuda_status(bl::launch_rms_act_quant(x, g, eps, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
+                                            reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
+                                            reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), true, s,
+                                            reinterpret_cast<uint32_t*>(base)));
+  if (st != BL_OK) return st;
+  return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, nullptr, ws, s, sms));
+}
+
 size_t bitlinear_batch_workspace_size(const bl_linear_call* calls, int count) {
   size_t need = bl::kHeaderBytes;
   if (calls == nullptr || count < 0) return 0;

@@ -50,6 +50,11 @@ cudaError_t launch_pack(const void* W, bool bf16, int64_t N, int64_t K, uint32_t
 // x is fp32, or bf16 bit patterns when bf16 (widened exactly).
 cudaError_t launch_act_quant(const void* x, bool bf16, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
                              bool permuted, cudaStream_t stream, uint32_t* err_reset);
+// RMSNorm (weight g [K], eps) then ActQuant, per token; K <= kRmsMaxK.
+constexpr int64_t kRmsMaxK = 16384;
+cudaError_t launch_rms_act_quant(const float* x, const float* g, float eps, int64_t M, int64_t K, int8_t* q,
+                                 float* s_x, int32_t* rowsum, bool permuted, cudaStream_t stream,
+                                 uint32_t* err_reset);
 // Natural-order int8 codes and scales (bitlinear_quant_act's output) into the
 // forward workspace layout (private order, row sums); err_reset as above.
 cudaError_t launch_q_prepare(const int8_t* q, const float* s_x, int64_t M, int64_t K, int8_t* wq, float* wsx,

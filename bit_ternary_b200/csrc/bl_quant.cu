@@ -392,6 +392,210 @@ __global__ void __launch_bounds__(256) act_quant_reg_kernel(const void* __restri
   }
 }
 
+// ------------------------------------------------------ RMSNorm + ActQuant --
+// Per-projection RMSNorm before ActQuant ("BitNet-Embeddings I2_S guide",
+// section 3.1; rms_norm_eps 1e-6): n = RN(RN(x*r)*g) with
+// r = RN(1/RN(sqrt(RN(ms + eps)))) and ms = mean(x^2) correctly rounded once
+// from the exact sum. One CTA per token, x and g held in registers.
+//
+// ms: each x^2 is exact in fp64, so the fp64 sum S' of the K squares, in any
+// order, is within gamma_(K-1) = (K-1)u/(1-(K-1)u) of the exact S (u = 2^-53,
+// all terms >= 0), and q = RN64(S'/K) adds one more u. Thread 0 widens q by
+// (K+8)*2^-52 in both directions with directed rounding; if both ends round to
+// the same fp32, that is RN32(S/K). Otherwise (a rounding boundary inside the
+// interval: a few tokens in a million) the block sums the squares exactly in
+// integers and divides by K.
+constexpr int kRmsBins = 544;  // x^2 = m^2 * 2^(2(ee-1)) units of 2^-298; m^2 split in 24-bit halves
+
+// Correctly rounded fp32 of (sum_b bins[b] * 2^b) / K * 2^-298, by long
+// division on 32-bit limbs (one thread). bins[b] < 2^41.
+__device__ float mean_square_exact_f32(const unsigned long long* bins, uint32_t K) {
+  constexpr int L = 19;  // 608 bits: bins below 2^41 at shifts < 544
+  uint32_t S[L];
+  for (int i = 0; i < L; ++i) S[i] = 0u;
+  for (int b = 0; b < kRmsBins; ++b) {
+    const unsigned long long v = bins[b];
+    if (v == 0ull) continue;
+    const int limb = b >> 5, bit = b & 31;
+    uint32_t parts[3];
+    parts[0] = (uint32_t)(v << bit);
+    parts[1] = bit == 0 ? (uint32_t)(v >> 32) : (uint32_t)(v >> (32 - bit));
+    parts[2] = bit == 0 ? 0u : (uint32_t)((v >> 32) >> (32 - bit));
+    unsigned long long carry = 0ull;
+    for (int i = limb; i < L; ++i) {
+      const unsigned long long add = (i - limb < 3 ? parts[i - limb] : 0u);
+      const unsigned long long t = (unsigned long long)S[i] + add + carry;
+      S[i] = (uint32_t)t;
+      carry = t >> 32;
+      if (i - limb >= 2 && carry == 0ull) break;
+    }
+  }
+  // Q = floor(S / K), remainder r (K < 2^18, so r * 2^32 + limb fits 64 bits).
+  uint32_t Q[L];
+  unsigned long long r = 0ull;
+  for (int i = L - 1; i >= 0; --i) {
+    const unsigned long long cur = (r << 32) | S[i];
+    Q[i] = (uint32_t)(cur / K);
+    r = cur % K;
+  }
+  int lead = -1;
+  for (int i = L - 1; i >= 0 && lead < 0; --i)
+    if (Q[i]) lead = 32 * i + 31 - __clz(Q[i]);
+  if (lead < 0) return 0.0f;  // below 2^-298: rounds to zero
+  auto qbit = [&](int i) -> uint32_t { return (Q[i >> 5] >> (i & 31)) & 1u; };
+  const int E = lead - 298;                    // value = 1.xxx * 2^E
+  const int qe = E - 23 > -149 ? E - 23 : -149;  // exponent of the last significand bit
+  const int p = qe + 298;                      // its bit position in Q (>= 149)
+  uint32_t sig = 0u;
+  for (int i = lead; i >= p; --i) sig = (sig << 1) | qbit(i);
+  const uint32_t round_bit = qbit(p - 1);
+  uint32_t sticky = r != 0ull ? 1u : 0u;
+  for (int i = p - 2; i >= 0 && !sticky; --i) sticky |= qbit(i);
+  if (round_bit && (sticky || (sig & 1u))) ++sig;
+  // sig * 2^qe: subnormal when qe == -149 and sig < 2^23; a carry to 2^24 moves up one binade.
+  if (qe == -149 && sig < (1u << 23)) return __uint_as_float(sig);
+  int e2 = qe + 23;
+  if (sig == (1u << 24)) {
+    sig >>= 1;
+    ++e2;
+  }
+  return __uint_as_float(((uint32_t)(e2 + 127) << 23) | (sig & 0x7FFFFFu));
+}
+
+template <bool kPerm, int kG>
+__global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restrict__ x, const float* __restrict__ g,
+                                                            float eps, int64_t K, int8_t* __restrict__ q,
+                                                            float* __restrict__ s_out, int32_t* __restrict__ rowsum_out,
+                                                            uint32_t* __restrict__ err_reset) {
+  __shared__ double red_d[8];
+  __shared__ float red_f[8];
+  __shared__ int red_i[8];
+  __shared__ float s_ms;
+  __shared__ int s_exact;
+  __shared__ unsigned long long bins[kRmsBins];
+  if (err_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err_reset = 0u;
+  const int64_t m = blockIdx.x;
+  const int64_t xr = m * (K >> 2);
+  const int ngroups = (int)(K >> 4);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  float4 f[kG][4];
+  double ss = 0.0;
+#pragma unroll
+  for (int i = 0; i < kG; ++i) {
+    const int gi = threadIdx.x + i * blockDim.x;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      f[i][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (gi < ngroups) f[i][j] = __ldg(reinterpret_cast<const float4*>(x) + xr + 4 * gi + j);
+      ss += (double)f[i][j].x * f[i][j].x + (double)f[i][j].y * f[i][j].y;
+      ss += (double)f[i][j].z * f[i][j].z + (double)f[i][j].w * f[i][j].w;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+  if (lane == 0) red_d[warp] = ss;
+  for (int b = threadIdx.x; b < kRmsBins; b += blockDim.x) bins[b] = 0ull;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double S = 0.0;
+    for (int w = 0; w < nwarps; ++w) S += red_d[w];
+    const double qd = S / (double)K;
+    const double d = (double)(K + 8) * 2.220446049250313e-16;  // (K+8) * 2^-52
+    const float flo = __double2float_rn(__dmul_rd(qd, 1.0 - d));
+    const float fhi = __double2float_rn(__dmul_ru(qd, 1.0 + d));
+    s_exact = flo != fhi;
+    s_ms = flo;
+  }
+  __syncthreads();
+  if (s_exact) {  // block-uniform
+#pragma unroll
+    for (int i = 0; i < kG; ++i) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float v4[4] = {f[i][j].x, f[i][j].y, f[i][j].z, f[i][j].w};
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint32_t b = __float_as_uint(v4[c]) & 0x7FFFFFFFu;
+          const uint32_t e = b >> 23;
+          const unsigned long long mm = (b & 0x7FFFFFu) | (e != 0 ? 0x800000u : 0u);
+          if (mm == 0ull) continue;
+          const int sh = 2 * ((int)(e > 1 ? e : 1) - 1);
+          const unsigned long long sq = mm * mm;  // < 2^48
+          atomicAdd(&bins[sh], sq & 0xFFFFFFull);
+          atomicAdd(&bins[sh + 24], sq >> 24);
+        }
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) s_ms = mean_square_exact_f32(bins, (uint32_t)K);
+    __syncthreads();
+  }
+  const float ms = s_ms;
+  const float rr = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, eps)));
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kG; ++i) {
+    const int gi = threadIdx.x + i * blockDim.x;
+    if (gi >= ngroups) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 gw = __ldg(reinterpret_cast<const float4*>(g) + 4 * gi + j);
+      f[i][j].x = __fmul_rn(__fmul_rn(f[i][j].x, rr), gw.x);
+      f[i][j].y = __fmul_rn(__fmul_rn(f[i][j].y, rr), gw.y);
+      f[i][j].z = __fmul_rn(__fmul_rn(f[i][j].z, rr), gw.z);
+      f[i][j].w = __fmul_rn(__fmul_rn(f[i][j].w, rr), gw.w);
+      amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f[i][j].x), fabsf(f[i][j].y)), fmaxf(fabsf(f[i][j].z), fabsf(f[i][j].w))));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if (lane == 0) red_f[warp] = amax;
+  __syncthreads();
+  amax = 0.0f;
+  for (int w = 0; w < nwarps; ++w) amax = fmaxf(amax, red_f[w]);
+  const float sx = __fdiv_rn(kQmax, fmaxf(amax, kFloor));
+  int rsum = 0;
+  int8_t* qr = q + m * K;
+#pragma unroll
+  for (int i = 0; i < kG; ++i) {
+    const int gi = threadIdx.x + i * blockDim.x;
+    if (gi >= ngroups) continue;
+    int v[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[4 * j + 0] = quant_i8(f[i][j].x, sx);
+      v[4 * j + 1] = quant_i8(f[i][j].y, sx);
+      v[4 * j + 2] = quant_i8(f[i][j].z, sx);
+      v[4 * j + 3] = quant_i8(f[i][j].w, sx);
+    }
+    uint32_t w4[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      uint32_t word = 0u;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int p = 4 * r + b;
+        word |= (uint32_t)(v[kPerm ? perm16(p) : p] & 0xFF) << (8 * b);
+      }
+      w4[r] = word;
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) rsum += v[j];
+    *reinterpret_cast<uint4*>(qr + 16 * (int64_t)gi) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) rsum += __shfl_xor_sync(0xFFFFFFFFu, rsum, o);
+  if (lane == 0) red_i[warp] = rsum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int tot = 0;
+    for (int w = 0; w < nwarps; ++w) tot += red_i[w];
+    s_out[m] = sx;
+    if (rowsum_out != nullptr) rowsum_out[m] = tot;
+  }
+}
+
 // ------------------------------------------------------------ launchers --
 cudaError_t launch_pack(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
                         cudaStream_t stream, int num_sms) {
@@ -495,6 +699,30 @@ cudaError_t launch_act_quant(const void* x, bool bf16, int64_t M, int64_t K, int
                              bool permuted, cudaStream_t stream, uint32_t* err_reset) {
   return bf16 ? launch_act_quant_t<true>(x, M, K, q, s_x, rowsum, permuted, stream, err_reset)
               : launch_act_quant_t<false>(x, M, K, q, s_x, rowsum, permuted, stream, err_reset);
+}
+
+}  // namespace bl
+
+namespace bl {
+
+cudaError_t launch_rms_act_quant(const float* x, const float* g, float eps, int64_t M, int64_t K, int8_t* q,
+                                 float* s_x, int32_t* rowsum, bool permuted, cudaStream_t stream,
+                                 uint32_t* err_reset) {
+  const int64_t ngroups = K / 16;
+  int kg = (int)((ngroups + 255) / 256);
+  if (kg > 4) return cudaErrorInvalidValue;  // K <= 16384
+  kg = kg <= 1 ? 1 : (kg <= 2 ? 2 : 4);
+  int threads = (int)(((ngroups + kg - 1) / kg + 31) / 32 * 32);
+  if (threads < 32) threads = 32;
+#define BL_RQ(P, G) \
+  rms_act_quant_kernel<P, G><<<(unsigned)M, threads, 0, stream>>>(x, g, eps, K, q, s_x, rowsum, err_reset)
+  if (permuted) {
+    if (kg == 1) BL_RQ(true, 1); else if (kg == 2) BL_RQ(true, 2); else BL_RQ(true, 4);
+  } else {
+    if (kg == 1) BL_RQ(false, 1); else if (kg == 2) BL_RQ(false, 2); else BL_RQ(false, 4);
+  }
+#undef BL_RQ
+  return cudaGetLastError();
 }
 
 }  // namespace bl

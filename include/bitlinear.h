@@ -188,6 +188,24 @@ BL_API int bitlinear_forward_q(const int8_t* q, const float* s_x, int64_t M, int
                                const uint32_t* packed, const float* D, float* y,
                                void* ws, size_t ws_bytes, bl_stream_t stream);
 
+/* Per-projection RMSNorm then ActQuant ("BitNet-Embeddings I2_S guide"
+ * section 3.1: x -> RMSNorm(x, norm.weight) -> activation_quant -> matmul;
+ * rms_norm_eps 1e-6). Per token: ms = mean(x^2), the exact mean correctly
+ * rounded to fp32 once; r = RN(1/RN(sqrt(RN(ms + eps)))); n = RN(RN(x*r)*g);
+ * then the ActQuant of bitlinear_quant_act on n (q, s_x, rowsum as there).
+ *   x  device fp32 [M, K]; g device fp32 [K] (the projection's norm.weight);
+ *   eps >= 0 (finite). K <= 16384; x, g, q 16-byte aligned. Asynchronous. */
+BL_API int bitlinear_rmsnorm_quant_act(const float* x, const float* g, float eps, int64_t M, int64_t K,
+                                       int8_t* q, float* s_x, int32_t* rowsum, bl_stream_t stream);
+
+/* y = F.linear(ActQuant(RMSNorm(x, g)), WeightQuant(W)) from packed weights:
+ * the fused norm + quantiser writes the codes into ws, then the tensor-core
+ * kernel runs (every M). Same arguments as bitlinear_forward plus g and eps;
+ * K <= 16384. Asynchronous. */
+BL_API int bitlinear_forward_rmsnorm(const float* x, const float* g, float eps, int64_t M, int64_t N,
+                                     int64_t K, const uint32_t* packed, const float* D, float* y,
+                                     void* ws, size_t ws_bytes, bl_stream_t stream);
+
 /* ---------------------------------------------------------------- batch --- */
 
 /* One BitLinear of a batch: y [M,N] = F.linear(ActQuant(x [M,K]), W) from

@@ -122,3 +122,17 @@ def test_forward_q_and_async_host_validation_before_cuda(L):
     assert L.bitlinear_forward_host_async(FAKE, 1, 1, 40, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 2
     assert L.bitlinear_forward_host_async(FAKE, 1, 1, 16, FAKE, FAKE, FAKE, FAKE + 16, 1 << 20, None) == 3
     assert L.bitlinear_forward_host_async(FAKE, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, 8, None) == 4
+
+
+def test_rmsnorm_validation_before_cuda(L):
+    # bitlinear_rmsnorm_quant_act(x, g, eps, M, K, q, s_x, rowsum, stream)
+    assert L.bitlinear_rmsnorm_quant_act(FAKE, FAKE, 1e-6, 1, 16384 + 16, FAKE, FAKE, None, None) == 2
+    assert L.bitlinear_rmsnorm_quant_act(FAKE, None, 1e-6, 1, 64, FAKE, FAKE, None, None) == 1
+    assert L.bitlinear_rmsnorm_quant_act(FAKE, FAKE, -1.0, 1, 64, FAKE, FAKE, None, None) == 2
+    assert L.bitlinear_rmsnorm_quant_act(FAKE, FAKE + 4, 1e-6, 1, 64, FAKE, FAKE, None, None) == 3
+    assert L.bitlinear_rmsnorm_quant_act(None, None, 1e-6, 0, 64, None, None, None, None) == 0
+    # bitlinear_forward_rmsnorm(x, g, eps, M, N, K, packed, D, y, ws, ws_bytes, stream)
+    assert L.bitlinear_forward_rmsnorm(FAKE, FAKE, 1e-6, 1, 1, 20000 - 20000 % 16, FAKE, FAKE, FAKE, FAKE, 1 << 30,
+                                       None) == 2
+    assert L.bitlinear_forward_rmsnorm(FAKE, None, 1e-6, 1, 1, 64, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.bitlinear_forward_rmsnorm(FAKE, FAKE, 1e-6, 1, 1, 64, FAKE, FAKE, FAKE, FAKE, 16, None) == 4

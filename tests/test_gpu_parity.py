@@ -518,3 +518,45 @@ def test_forward_bf16(B, M, N, K):
     p_ref, D_ref = O.pack_weights_bf16(wbits)
     y = B.forward(xt, packed, D).cpu().numpy()
     assert_y_close(y, O.bitlinear_forward_bf16(xbits, p_ref, D_ref, K))
+
+
+# --------------------------------------------------- RMSNorm + ActQuant
+@pytest.mark.parametrize("M,K,xdist", [(1, 2560, "student_t"), (5, 1024, "outlier_tokens"), (64, 3072, "normal"),
+                                       (300, 640, "student_t"), (17, 16384, "normal")])
+def test_rmsnorm_quant_act_bitexact(B, M, K, xdist):
+    x = WL.activations(M, K, xdist, 80 + K, meta={"df": 3.0, "frac": 0.02, "scale": 20.0})
+    x[0, :5] = 0.0
+    g = np.random.default_rng(K).uniform(0.5, 2.0, K).astype(np.float32)
+    q, s_x, rs = B.rmsnorm_quant_act(dev(x), dev(g))
+    q_ref, s_ref = O.rmsnorm_act_quant(x, g)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s_x.cpu().numpy(), s_ref)
+    assert np.array_equal(rs.cpu().numpy(), q_ref.astype(np.int64).sum(axis=1))
+
+
+def test_rmsnorm_exact_path_on_rounding_ties_and_zero_row(B):
+    """Rows whose mean square is an exact fp32 rounding tie (or a hair above
+    one) leave the fp64 interval ambiguous, so the kernel takes the exact
+    integer path; an all-zero row gives ms = 0; a tiny row gives a subnormal ms."""
+    B2 = B
+    K = 64
+    rows = [np.full(K, 1 + 2.0 ** -12, np.float32), np.full(K, 1 + 3 * 2.0 ** -12, np.float32),
+            np.full(K, 1 + 2.0 ** -12 + 2.0 ** -23, np.float32), np.zeros(K, np.float32),
+            np.full(K, 3.0 * 2.0 ** -70, np.float32)]
+    x = np.stack(rows)
+    g = np.linspace(0.5, 1.5, K).astype(np.float32)
+    q, s_x, _ = B2.rmsnorm_quant_act(dev(x), dev(g))
+    q_ref, s_ref = O.rmsnorm_act_quant(x, g)
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s_x.cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 3840, 2560), (37, 700, 1024), (300, 1024, 3072), (16, 129, 528)])
+def test_forward_rmsnorm(B, M, N, K):
+    W = WL.weight(N, K, "normal", 90 + N)
+    x = WL.activations(M, K, "outlier_tokens", 91 + M, meta={"df": 3.0, "frac": 0.02, "scale": 20.0})
+    g = np.random.default_rng(N).uniform(0.5, 2.0, K).astype(np.float32)
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    y = B.forward_rmsnorm(dev(x), dev(g), packed, D).cpu().numpy()
+    assert_y_close(y, O.bitlinear_forward_rmsnorm(x, g, p_ref, D_ref, K))
