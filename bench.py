@@ -454,6 +454,11 @@ def run_ours(a):
     if not a.ncu_small:
         pack = bench_pack(B, torch, dev, stream, hbm_peak)
 
+    # ----------------------------------------------------- RMSNorm + ActQuant
+    rms = None
+    if not a.no_prefill and not a.ncu_small:
+        rms = bench_rmsnorm(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, i8_burst)
+
     # ------------------------------------------------------------- bf16 inputs
     bf16 = None
     if not a.no_prefill and not a.ncu_small:
@@ -500,6 +505,7 @@ def run_ours(a):
         "configs": configs,
         "pack": pack,
         "bf16_inputs": bf16,
+        "rmsnorm_actquant": rms,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
@@ -728,6 +734,51 @@ def bench_bf16(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, 
     alg = 2 * l.N * l.K + l.N * l.K // 4 + 4 * l.N
     out["pack"] = {"layer": f"gate_up {l.K}->{l.N}", "ms": round(t * 1e3, 4),
                    "GB/s_algorithmic": round(alg / t / 1e9, 1), "frac_hbm": round(alg / t / 1e9 / hbm_peak, 4)}
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_rmsnorm(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, i8_burst):
+    """Fused per-projection RMSNorm + ActQuant (the embedding models of C5 normalise the input of
+    every projection) against HBM: 4MK + 4K read, MK + 8M written. Also the forward with the
+    fused norm on the first C5 layer, against its true roofline."""
+    out = {"actquant": []}
+    for (M, K) in ((32768, 1024), (32768, 3072), (4096, 2560), (4096, 6912)):
+        with torch.cuda.stream(stream):
+            x = torch.from_numpy(WL.activations(M, K, "outlier_tokens", 7, layer=K,
+                                                meta={"frac": 0.01, "scale": 20.0, "df": 3.0})).to(dev)
+            g = torch.from_numpy(WL.weight(1, K, "normal", 8).reshape(-1) + np.float32(1.0)).to(dev)
+        torch.cuda.synchronize(dev)
+        g_ = capture(lambda i, x=x, g=g: B.rmsnorm_quant_act(x, g), 10)
+        with torch.cuda.stream(stream):
+            g_.replay()
+        t = max_ranks(time_graph(g_)) / 10 * 1e-3
+        nb = 4 * M * K + 4 * K + M * K + 12 * M
+        out["actquant"].append({"M": M, "K": K, "us": round(t * 1e6, 2), "GB/s": round(nb / t / 1e9, 1),
+                                "frac_hbm": round(nb / t / 1e9 / hbm_peak, 4)})
+        del g_, x, g
+    wl = WL.WORKLOADS["embed_batch"]
+    l = wl.layers[2]  # 3072 -> 1024, compute-bound
+    M = 32768
+    with torch.cuda.stream(stream):
+        W = torch.from_numpy(WL.weight(l.N, l.K, wl.w_dist, wl.seed, layer=2)).to(dev)
+        p, D = B.pack_weights(W)
+        del W
+        x = torch.from_numpy(WL.activations(M, l.K, wl.x_dist, wl.seed, layer=2, meta=wl.meta)).to(dev)
+        g = torch.from_numpy(WL.weight(1, l.K, "normal", 9).reshape(-1) + np.float32(1.0)).to(dev)
+        y = torch.empty((M, l.N), dtype=torch.float32, device=dev)
+        ws = torch.zeros(B.workspace_size(M, l.N, l.K), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize(dev)
+    gg = capture(lambda i: B.forward_rmsnorm(x, g, p, D, out=y, ws=ws), 10)
+    with torch.cuda.stream(stream):
+        gg.replay()
+    t = max_ranks(time_graph(gg)) / 10 * 1e-3
+    ops = 2 * M * l.N * l.K
+    nb = 4 * M * l.K + 4 * l.K + l.N * l.K // 4 + 4 * l.N + 4 * M * l.N
+    out["forward"] = {"layer": f"embed_batch {l.name} {l.K}->{l.N}, M={M}", "us": round(t * 1e6, 2),
+                      "TOPS": round(ops / t / 1e12, 1),
+                      "frac_true_roofline": round(max(nb / (hbm_peak * 1e9), ops / (i8_burst * 1e12)) / t, 4)}
+    del gg, x, y, ws
     torch.cuda.empty_cache()
     return out
 

@@ -479,7 +479,11 @@ __global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restr
   const int ngroups = (int)(K >> 4);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
+  // g is loaded with x when it fits in registers (kG == 1), so its latency
+  // overlaps the load of x instead of following the mean-square barrier.
+  constexpr bool kGEarly = kG == 1;
   float4 f[kG][4];
+  float4 gw[kGEarly ? kG : 1][4];
   double ss = 0.0;
 #pragma unroll
   for (int i = 0; i < kG; ++i) {
@@ -488,6 +492,10 @@ __global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restr
     for (int j = 0; j < 4; ++j) {
       f[i][j] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (gi < ngroups) f[i][j] = __ldg(reinterpret_cast<const float4*>(x) + xr + 4 * gi + j);
+      if (kGEarly) {
+        gw[kGEarly ? i : 0][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (gi < ngroups) gw[kGEarly ? i : 0][j] = __ldg(reinterpret_cast<const float4*>(g) + 4 * gi + j);
+      }
       ss += (double)f[i][j].x * f[i][j].x + (double)f[i][j].y * f[i][j].y;
       ss += (double)f[i][j].z * f[i][j].z + (double)f[i][j].w * f[i][j].w;
     }
@@ -495,7 +503,6 @@ __global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restr
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
   if (lane == 0) red_d[warp] = ss;
-  for (int b = threadIdx.x; b < kRmsBins; b += blockDim.x) bins[b] = 0ull;
   __syncthreads();
   if (threadIdx.x == 0) {
     double S = 0.0;
@@ -509,6 +516,8 @@ __global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restr
   }
   __syncthreads();
   if (s_exact) {  // block-uniform
+    for (int b = threadIdx.x; b < kRmsBins; b += blockDim.x) bins[b] = 0ull;
+    __syncthreads();
 #pragma unroll
     for (int i = 0; i < kG; ++i) {
 #pragma unroll
@@ -540,11 +549,11 @@ __global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restr
     if (gi >= ngroups) continue;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float4 gw = __ldg(reinterpret_cast<const float4*>(g) + 4 * gi + j);
-      f[i][j].x = __fmul_rn(__fmul_rn(f[i][j].x, rr), gw.x);
-      f[i][j].y = __fmul_rn(__fmul_rn(f[i][j].y, rr), gw.y);
-      f[i][j].z = __fmul_rn(__fmul_rn(f[i][j].z, rr), gw.z);
-      f[i][j].w = __fmul_rn(__fmul_rn(f[i][j].w, rr), gw.w);
+      const float4 gv = kGEarly ? gw[kGEarly ? i : 0][j] : __ldg(reinterpret_cast<const float4*>(g) + 4 * gi + j);
+      f[i][j].x = __fmul_rn(__fmul_rn(f[i][j].x, rr), gv.x);
+      f[i][j].y = __fmul_rn(__fmul_rn(f[i][j].y, rr), gv.y);
+      f[i][j].z = __fmul_rn(__fmul_rn(f[i][j].z, rr), gv.z);
+      f[i][j].w = __fmul_rn(__fmul_rn(f[i][j].w, rr), gv.w);
       amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f[i][j].x), fabsf(f[i][j].y)), fmaxf(fabsf(f[i][j].z), fabsf(f[i][j].w))));
     }
   }
