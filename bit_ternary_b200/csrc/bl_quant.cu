@@ -99,9 +99,15 @@ __global__ void __launch_bounds__(kBinThreads) absum_bins_kernel(const void* __r
 // 1e-5 floor that is applied afterwards). One thread. n = N*K < 2^48 (N < 2^31,
 // K <= 2^17), and a tensor that fits in device memory has n < 2^36, so every
 // bin is below 2^60 and S below 2^313.
-__global__ void absmean_finalize_kernel(const unsigned long long* __restrict__ bins, uint64_t n,
+__global__ void absmean_finalize_kernel(const unsigned long long* __restrict__ gbins, uint64_t n,
                                         float* __restrict__ scal, uint32_t* __restrict__ status) {
-  if (threadIdx.x != 0 || blockIdx.x != 0) return;
+  // The warp stages the bins in shared memory (parallel loads); one thread
+  // then does the exact arithmetic.
+  __shared__ unsigned long long bins[kPackBins];
+  if (blockIdx.x != 0) return;
+  for (int i = threadIdx.x; i < kPackBins; i += blockDim.x) bins[i] = gbins[i];
+  __syncthreads();
+  if (threadIdx.x != 0) return;
   if (bins[kPackNonFiniteBin] != 0ull) {
     *status = 1u;  // non-finite input
     scal[0] = __int_as_float(0x7FC00000);
