@@ -100,7 +100,7 @@ constexpr size_t kSmemB = (size_t)kStages * kBStageBytes;
 constexpr size_t kSmemY = (size_t)kEpiWarps * kYSliceBytes;
 constexpr size_t kGemmSmemBytes = 1024 + kSmemB + kSmemY + ((sizeof(GemmSmem) + 127) & ~size_t(127));
 
-// Warp-uniform bounded wait: lane 0 polls, the whole warp gets its verdict, so
+// Warp-uniform bounded wait: lane 0 polls, the whole warp gets the outcome, so
 // the warp stays converged for the .sync.aligned tcgen05 instructions.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, uint32_t* err,
                                           uint32_t code) {

@@ -21,7 +21,7 @@ What it computes, and where the pages define it:
                equals F.linear(ActQuant(x), WeightQuant(W)). Here that is an
                exact integer contraction acc = q . code, then the two scales.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent (the plainest reading in each case):
   * mean(|W|) is the exact real mean, correctly rounded to fp32.
   * A floor of 1e-5 guards mean(|W|) and max|x| (an all-zero tensor or token).
   * s = RN(1/mean); the code is rint(RN(W*s)) (the W*s spelling of §1).
