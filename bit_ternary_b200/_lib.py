@@ -51,6 +51,8 @@ SIGNATURES = {
     "bitlinear_pack_weights_bf16": (ctypes.c_int, [_VP, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
     "bitlinear_quant_act_bf16": (ctypes.c_int, [_VP, _I64, _I64, _VP, _VP, _VP, _VP]),
     "bitlinear_forward_bf16": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "bitlinear_batch_host_workspace_size": (ctypes.c_size_t, [_VP, ctypes.c_int]),
+    "bitlinear_forward_batch_host": (ctypes.c_int, [_VP, ctypes.c_int, ctypes.c_uint32, _VP, _SZ, _VP]),
     "bitlinear_rmsnorm_quant_act": (ctypes.c_int, [_VP, _VP, ctypes.c_float, _I64, _I64, _VP, _VP, _VP, _VP]),
     "bitlinear_forward_rmsnorm": (ctypes.c_int, [_VP, _VP, ctypes.c_float, _I64, _I64, _I64, _VP, _VP, _VP,
                                                  _VP, _SZ, _VP]),
@@ -78,6 +80,7 @@ class LinearCall(ctypes.Structure):
 
 
 BL_FLAG_STREAM_WEIGHTS_EARLY = 1
+BL_FLAG_ONE_LAUNCH_PER_CALL = 2
 
 
 class BitLinearError(RuntimeError):

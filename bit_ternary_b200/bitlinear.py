@@ -225,8 +225,9 @@ def forward_batch(calls, flags: int = 0, ws: Optional[torch.Tensor] = None):
 
     Decode-sized calls (M <= 16) are fused into grouped launches; `flags` may
     hold BL_FLAG_STREAM_WEIGHTS_EARLY (weights are static, so the decode
-    kernels may stream them while the previous work on the stream finishes).
-    Returns the list of outputs.
+    kernels may stream them while the previous work on the stream finishes)
+    and BL_FLAG_ONE_LAUNCH_PER_CALL (every call in its own launch, in order,
+    for calls that stand for dependent layers). Returns the list of outputs.
     """
     n = len(calls)
     arr = (_lib.LinearCall * max(n, 1))()
@@ -248,6 +249,51 @@ def forward_batch(calls, flags: int = 0, ws: Optional[torch.Tensor] = None):
         ws = _alloc_ws(L.bitlinear_batch_workspace_size(arr, n), device)
     _lib.call("bitlinear_forward_batch", arr, n, flags, ws.data_ptr(), ws.numel(), _stream_handle(device))
     return outs
+
+
+def forward_batch_host(calls, flags: int = 0, ws: Optional[torch.Tensor] = None):
+    """forward_batch with host activations and outputs: calls are
+    [(x_host, packed, D, y_host), ...] with x_host / y_host pinned CPU fp32
+    tensors (y_host None: allocated pinned) and packed / D on the device.
+    Enqueued on the current stream; the outputs are valid once it has been
+    synchronised. Calls whose host blocks follow one another in memory (views
+    of one pinned buffer) move in one copy each way. Returns the outputs."""
+    n = len(calls)
+    arr = (_lib.LinearCall * max(n, 1))()
+    outs = []
+    device = None
+    for i, (x, packed, D, y) in enumerate(calls):
+        if x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous() or x.dim() != 2:
+            raise ValueError("x_host must be a contiguous 2-D fp32 CPU tensor")
+        M, K = x.shape
+        _need_cuda(packed, "packed", torch.int32)
+        N = packed.shape[0]
+        _check_D(D, N)
+        if y is None:
+            y = torch.empty((M, N), dtype=torch.float32, pin_memory=True)
+        if y.is_cuda or y.dtype != torch.float32 or not y.is_contiguous() or tuple(y.shape) != (M, N):
+            raise ValueError("y_host must be a contiguous fp32 CPU tensor of shape (M, N)")
+        if M and N and not (x.is_pinned() and y.is_pinned()):
+            raise ValueError("the batched host call needs pinned x_host and y_host")
+        arr[i] = _lib.LinearCall(x.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(), y.data_ptr())
+        outs.append(y)
+        device = packed.device
+    if n == 0:
+        return outs
+    L = _lib.lib()
+    if ws is None:
+        ws = _alloc_ws(L.bitlinear_batch_host_workspace_size(arr, n), device)
+    _lib.call("bitlinear_forward_batch_host", arr, n, flags, ws.data_ptr(), ws.numel(), _stream_handle(device))
+    return outs
+
+
+def batch_host_workspace_size(calls) -> int:
+    """Workspace bytes for forward_batch_host over [(M, N, K), ...]."""
+    n = len(calls)
+    arr = (_lib.LinearCall * max(n, 1))()
+    for i, (M, N, K) in enumerate(calls):
+        arr[i] = _lib.LinearCall(0, M, N, K, 0, 0, 0)
+    return int(_lib.lib().bitlinear_batch_host_workspace_size(arr, n))
 
 
 def forward_host(x_host: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,

@@ -4,6 +4,8 @@
 #include "bitlinear.h"
 #include "bl_internal.h"
 
+#include <vector>
+
 #include <mutex>
 
 namespace {
@@ -299,7 +301,7 @@ int bitlinear_forward_batch(const bl_linear_call* calls, int count, uint32_t fla
   if (count == 0) return BL_OK;
   if (calls == nullptr || ws == nullptr) return BL_ERR_NULL;
   if (!aligned256(ws)) return BL_ERR_ALIGN;
-  if (flags & ~(uint32_t)BL_FLAG_STREAM_WEIGHTS_EARLY) return BL_ERR_SHAPE;
+  if (flags & ~(uint32_t)(BL_FLAG_STREAM_WEIGHTS_EARLY | BL_FLAG_ONE_LAUNCH_PER_CALL)) return BL_ERR_SHAPE;
   // Validate every call before launching anything.
   for (int i = 0; i < count; ++i) {
     const bl_linear_call& c = calls[i];
@@ -317,8 +319,9 @@ int bitlinear_forward_batch(const bl_linear_call* calls, int count, uint32_t fla
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(ws);
   const bool early = (flags & BL_FLAG_STREAM_WEIGHTS_EARLY) != 0;
+  const int max_group = (flags & BL_FLAG_ONE_LAUNCH_PER_CALL) ? 1 : bl::kGemvMaxGroup;
   // Decode-sized calls are grouped, in order, into launches of up to
-  // kGemvMaxGroup; every other call runs on its own.
+  // max_group; every other call runs on its own.
   bl::GemvCall group[bl::kGemvMaxGroup];
   int ng = 0;
   int64_t gM = 0, gK = 0;
@@ -334,7 +337,7 @@ int bitlinear_forward_batch(const bl_linear_call* calls, int count, uint32_t fla
     if (c.M == 0 || c.N == 0) continue;
     const int64_t nM = c.M > gM ? c.M : gM, nK = c.K > gK ? c.K : gK;
     if (bl::gemv_group_fits(c.M, c.K)) {
-      if (ng == bl::kGemvMaxGroup || !bl::gemv_group_fits(nM, nK)) {
+      if (ng == max_group || !bl::gemv_group_fits(nM, nK)) {
         const int st = flush();
         if (st != BL_OK) return st;
       }
@@ -349,6 +352,98 @@ int bitlinear_forward_batch(const bl_linear_call* calls, int count, uint32_t fla
     if (st != BL_OK) return st;
   }
   return flush();
+}
+
+// Bytes of x (in) or y (out) that a call stages; calls with no output move nothing.
+static size_t staged_bytes(const bl_linear_call& c, bool in) {
+  if (c.M <= 0 || c.N <= 0 || c.K < 0) return 0;
+  return 4 * (size_t)c.M * (size_t)(in ? c.K : c.N);
+}
+
+// Room a staged block takes: its bytes rounded up to 16, so every block starts
+// 16-byte aligned.
+static size_t staged_room(const bl_linear_call& c, bool in) { return (staged_bytes(c, in) + 15) & ~(size_t)15; }
+
+size_t bitlinear_batch_host_workspace_size(const bl_linear_call* calls, int count) {
+  if (calls == nullptr || count < 0) return 0;
+  size_t xs = 0, ys = 0;
+  for (int i = 0; i < count; ++i) {
+    if (calls[i].M < 0 || calls[i].N < 0 || calls[i].K < 0) return 0;
+    xs += staged_room(calls[i], true);
+    ys += staged_room(calls[i], false);
+  }
+  return bl::align256(bitlinear_batch_workspace_size(calls, count)) + bl::align256(xs) + bl::align256(ys);
+}
+
+int bitlinear_forward_batch_host(const bl_linear_call* calls, int count, uint32_t flags, void* ws, size_t ws_bytes,
+                                 bl_stream_t stream) {
+  if (count < 0) return BL_ERR_SHAPE;
+  if (count == 0) return BL_OK;
+  if (calls == nullptr || ws == nullptr) return BL_ERR_NULL;
+  if (!aligned256(ws)) return BL_ERR_ALIGN;
+  if (flags & ~(uint32_t)(BL_FLAG_STREAM_WEIGHTS_EARLY | BL_FLAG_ONE_LAUNCH_PER_CALL)) return BL_ERR_SHAPE;
+  for (int i = 0; i < count; ++i) {
+    const bl_linear_call& c = calls[i];
+    int st = check_k(c.K);
+    if (st != BL_OK) return st;
+    st = check_mn(c.M, c.N);
+    if (st != BL_OK) return st;
+    if (c.M == 0 || c.N == 0) continue;
+    if (c.x == nullptr || c.packed == nullptr || c.D == nullptr || c.y == nullptr) return BL_ERR_NULL;
+    if (!aligned16(c.packed) || !aligned16(c.D)) return BL_ERR_ALIGN;
+  }
+  if (ws_bytes < bitlinear_batch_host_workspace_size(calls, count)) return BL_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const size_t fw = bl::align256(bitlinear_batch_workspace_size(calls, count));
+  size_t xs = 0;
+  for (int i = 0; i < count; ++i) xs += staged_room(calls[i], true);
+  uint8_t* xdev = base + fw;                    // activations of all calls, back to back
+  uint8_t* ydev = base + fw + bl::align256(xs);  // outputs of all calls, back to back
+  // Device copies of the calls, pointing into the staging areas.
+  std::vector<bl_linear_call> dc(calls, calls + count);
+  size_t xo = 0, yo = 0;
+  for (int i = 0; i < count; ++i) {
+    dc[i].x = reinterpret_cast<const float*>(xdev + xo);
+    dc[i].y = reinterpret_cast<float*>(ydev + yo);
+    xo += staged_room(calls[i], true);
+    yo += staged_room(calls[i], false);
+  }
+  // Blocks that follow one another both in host memory and in the staging
+  // area move in one copy; calls that stage nothing are skipped.
+  auto copy_runs = [&](bool in) -> int {
+    const char* run_host = nullptr;
+    size_t run_off = 0, run_len = 0, off = 0;
+    auto flush = [&]() -> int {
+      if (run_len == 0) return BL_OK;
+      const cudaError_t e =
+          in ? cudaMemcpyAsync(xdev + run_off, run_host, run_len, cudaMemcpyHostToDevice, s)
+             : cudaMemcpyAsync(const_cast<char*>(run_host), ydev + run_off, run_len, cudaMemcpyDeviceToHost, s);
+      run_len = 0;
+      return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+    };
+    for (int i = 0; i < count; ++i) {
+      const size_t b = staged_bytes(calls[i], in);
+      if (b == 0) continue;
+      const char* h = in ? reinterpret_cast<const char*>(calls[i].x) : reinterpret_cast<const char*>(calls[i].y);
+      if (run_len != 0 && (h != run_host + run_len || off != run_off + run_len)) {
+        const int st = flush();
+        if (st != BL_OK) return st;
+      }
+      if (run_len == 0) {
+        run_host = h;
+        run_off = off;
+      }
+      run_len += b;
+      off += staged_room(calls[i], in);
+    }
+    return flush();
+  };
+  int st = copy_runs(true);
+  if (st != BL_OK) return st;
+  st = bitlinear_forward_batch(dc.data(), count, flags, ws, fw, stream);
+  if (st != BL_OK) return st;
+  return copy_runs(false);
 }
 
 size_t bitlinear_host_workspace_size(int64_t M, int64_t N, int64_t K) {

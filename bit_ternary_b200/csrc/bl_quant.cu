@@ -165,30 +165,33 @@ __global__ void absmean_finalize_kernel(const unsigned long long* __restrict__ g
     rem = cur % n;
   }
   // Leading 24 bits of the quotient, the next (round) bit, and a sticky bit
-  // for every lower bit and the final remainder.
+  // for every lower bit and the final remainder. The leading 25 bits lie in
+  // the first four nonzero-led digits, read as one 64-bit window.
   float mean = 0.0f;
-  int lead = -1;  // bit index (from the quotient's LSB) of its leading 1
-  for (int d = 0; d < kDigits && lead < 0; ++d)
-    if (qd[d] != 0) lead = 16 * (kDigits - 1 - d) + (31 - __clz((uint32_t)qd[d]));
-  if (lead >= 24) {
-    auto qbit = [&](int i) -> uint32_t {  // bit i of the quotient
-      const int d = kDigits - 1 - (i >> 4);
-      return ((uint32_t)qd[d] >> (i & 15)) & 1u;
-    };
-    uint32_t sig = 0u;
-    for (int i = lead; i > lead - 24; --i) sig = (sig << 1) | qbit(i);
-    const uint32_t round_bit = qbit(lead - 24);
-    uint32_t sticky = rem != 0ull ? 1u : 0u;
-    for (int i = lead - 25; i >= 0 && !sticky; --i) sticky |= qbit(i);
-    int E = lead - 149 - F;  // value = 1.xxx * 2^E
-    if (round_bit && (sticky || (sig & 1u))) {
-      ++sig;
-      if (sig == (1u << 24)) {
-        sig >>= 1;
-        ++E;
+  int dl = 0;
+  while (dl < kDigits && qd[dl] == 0) ++dl;
+  if (dl < kDigits) {
+    unsigned long long w = 0ull;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w = (w << 16) | (dl + k < kDigits ? qd[dl + k] : 0u);
+    const int lb = 31 - __clz((uint32_t)qd[dl]);          // leading bit inside digit dl
+    const int lead = 16 * (kDigits - 1 - dl) + lb;        // its index from the quotient's LSB
+    if (lead >= 24) {
+      const int top = 48 + lb;                            // the leading bit's index in w
+      uint32_t sig = (uint32_t)(w >> (top - 23)) & 0xFFFFFFu;
+      const uint32_t round_bit = (uint32_t)(w >> (top - 24)) & 1u;
+      uint32_t sticky = (rem != 0ull || (w & ((1ull << (top - 24)) - 1ull)) != 0ull) ? 1u : 0u;
+      for (int d = dl + 4; d < kDigits && !sticky; ++d) sticky |= qd[d] != 0 ? 1u : 0u;
+      int E = lead - 149 - F;  // value = 1.xxx * 2^E
+      if (round_bit && (sticky || (sig & 1u))) {
+        ++sig;
+        if (sig == (1u << 24)) {
+          sig >>= 1;
+          ++E;
+        }
       }
+      if (E >= -126 && E <= 127) mean = __uint_as_float(((uint32_t)(E + 127) << 23) | (sig & 0x7FFFFFu));
     }
-    if (E >= -126 && E <= 127) mean = __uint_as_float(((uint32_t)(E + 127) << 23) | (sig & 0x7FFFFFu));
   }
   const float mean_c = fmaxf(mean, kFloor);
   scal[0] = mean_c;

@@ -227,6 +227,12 @@ typedef struct {
  * activations are still read only after it has finished. */
 #define BL_FLAG_STREAM_WEIGHTS_EARLY 1u
 
+/* Flag for bitlinear_forward_batch: give every call its own launch, in order
+ * (for calls that stand for dependent layers; with the flag above, each
+ * launch may still stream its weights while the one before it runs). Without
+ * it, consecutive decode-sized calls share launches. */
+#define BL_FLAG_ONE_LAUNCH_PER_CALL 2u
+
 /* Bytes of scratch for bitlinear_forward_batch: the largest
  * bitlinear_workspace_size of its calls. */
 BL_API size_t bitlinear_batch_workspace_size(const bl_linear_call* calls, int count);
@@ -261,6 +267,20 @@ BL_API int bitlinear_forward_host(const float* x_host, int64_t M, int64_t N, int
 BL_API int bitlinear_forward_host_async(const float* x_host, int64_t M, int64_t N, int64_t K,
                                  const uint32_t* packed, const float* D, float* y_host,
                                  void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* Scratch for bitlinear_forward_batch_host: the batch workspace plus device
+ * room for every call's x and y. */
+BL_API size_t bitlinear_batch_host_workspace_size(const bl_linear_call* calls, int count);
+
+/* bitlinear_forward_batch with HOST activations and outputs: calls[i].x and
+ * calls[i].y are host pointers (pinned memory for the copies to run
+ * asynchronously), packed and D device pointers. Copies every x to the device
+ * (calls whose host blocks follow one another in host memory move in one
+ * copy), runs the batch with `flags`, and copies every y back the same way.
+ * Nothing is synchronised: the outputs are in host memory once `stream` has
+ * been synchronised. Errors of any call are reported before anything runs. */
+BL_API int bitlinear_forward_batch_host(const bl_linear_call* calls, int count, uint32_t flags,
+                                        void* ws, size_t ws_bytes, bl_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device error word in a
  * forward workspace. BL_OK if no kernel recorded a failure, else

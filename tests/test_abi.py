@@ -136,3 +136,26 @@ def test_rmsnorm_validation_before_cuda(L):
                                        None) == 2
     assert L.bitlinear_forward_rmsnorm(FAKE, None, 1e-6, 1, 1, 64, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 1
     assert L.bitlinear_forward_rmsnorm(FAKE, FAKE, 1e-6, 1, 1, 64, FAKE, FAKE, FAKE, FAKE, 16, None) == 4
+
+
+def test_batch_host_validation_before_cuda(L):
+    calls = (_lib.LinearCall * 3)()
+    calls[0] = _lib.LinearCall(FAKE, 1, 8, 64, FAKE, FAKE, FAKE)
+    calls[1] = _lib.LinearCall(FAKE, 3, 5, 32, FAKE, FAKE, FAKE)
+    calls[2] = _lib.LinearCall(None, 0, 8, 64, None, None, None)  # empty: stages nothing
+    need = L.bitlinear_batch_host_workspace_size(calls, 3)
+    # batch workspace, then x blocks (256 + 384 bytes) and y blocks (32 + 60 -> 64 bytes), 256-aligned each
+    assert need == L.bitlinear_batch_workspace_size(calls, 3) + 768 + 256
+    # bitlinear_forward_batch_host(calls, count, flags, ws, ws_bytes, stream)
+    assert L.bitlinear_forward_batch_host(calls, 3, 0, FAKE, need - 1, None) == 4
+    assert L.bitlinear_forward_batch_host(calls, 3, 0, FAKE + 16, need, None) == 3
+    assert L.bitlinear_forward_batch_host(calls, 3, 0x80, FAKE, need, None) == 2
+    assert L.bitlinear_forward_batch_host(calls, -1, 0, FAKE, need, None) == 2
+    assert L.bitlinear_forward_batch_host(calls, 0, 0, None, 0, None) == 0
+    calls[1] = _lib.LinearCall(FAKE, 3, 5, 40, FAKE, FAKE, FAKE)  # K % 16 != 0
+    assert L.bitlinear_forward_batch_host(calls, 3, 0, FAKE, 1 << 20, None) == 2
+    calls[1] = _lib.LinearCall(FAKE, 3, 5, 32, FAKE, FAKE, None)  # no y
+    assert L.bitlinear_forward_batch_host(calls, 3, 0, FAKE, 1 << 20, None) == 1
+    calls[1] = _lib.LinearCall(FAKE, 3, 5, 32, FAKE + 4, FAKE, FAKE)  # packed not 16-byte aligned
+    assert L.bitlinear_forward_batch_host(calls, 3, 0, FAKE, 1 << 20, None) == 3
+    assert L.bitlinear_batch_host_workspace_size(None, 3) == 0

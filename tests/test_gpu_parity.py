@@ -471,6 +471,88 @@ def test_forward_batch_rejects_before_launch(B):
         B.forward_batch([good, (good[0], packed, D, bad_y)])
 
 
+@pytest.mark.parametrize("flags", [2, 3])
+def test_forward_batch_one_launch_per_call(B, flags):
+    """Every call in its own launch (with and without early weights): the same
+    bits as the grouped launches, and the oracle's."""
+    shapes = [(1, 2560, 2560), (2, 100, 528), (1, 33, 48), (40, 300, 512), (16, 64, 1152), (3, 257, 6912)]
+    calls, refs = [], []
+    for i, (M, N, K) in enumerate(shapes):
+        W = WL.weight(N, K, "normal", 800 + i)
+        x = WL.activations(M, K, "normal", 900 + i)
+        packed, D = B.pack_weights(dev(W))
+        calls.append((dev(x), packed, D, None))
+        refs.append(_oracle_y(W, x))
+    outs = B.forward_batch(calls, flags=flags)
+    grouped = B.forward_batch(calls, flags=0)
+    torch.cuda.synchronize()
+    for y, g, ref in zip(outs, grouped, refs):
+        assert_y_close(y.cpu().numpy(), ref)
+        assert torch.equal(y, g)
+
+
+def _pinned(a):
+    t = torch.empty(a.shape, dtype=torch.float32, pin_memory=True)
+    t.copy_(torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)))
+    return t
+
+
+@pytest.mark.parametrize("flags", [0, 3])
+def test_forward_batch_host(B, flags):
+    """Host activations and outputs: views of one pinned buffer (merged
+    copies), a call with its own buffers, blocks whose bytes are not a
+    multiple of 16, an empty call, and a tensor-core call."""
+    shapes = [(1, 2560, 2560), (3, 33, 48), (0, 64, 64), (2, 129, 528), (40, 300, 512), (1, 17, 16)]
+    Ws = [WL.weight(N, K, "normal", 1000 + i) for i, (M, N, K) in enumerate(shapes)]
+    xs = [WL.activations(M, K, "student_t", 1100 + i, meta={"df": 3.0}) for i, (M, N, K) in enumerate(shapes)]
+    packs = [B.pack_weights(dev(W)) for W in Ws]
+    x_all = torch.empty(sum(M * K for M, N, K in shapes), dtype=torch.float32, pin_memory=True)
+    y_all = torch.full((sum(M * N for M, N, K in shapes),), float("nan"), dtype=torch.float32, pin_memory=True)
+    calls, xo, yo = [], 0, 0
+    for i, (M, N, K) in enumerate(shapes):
+        xv = x_all[xo:xo + M * K].view(M, K)
+        yv = y_all[yo:yo + M * N].view(M, N)
+        xo += M * K
+        yo += M * N
+        if i == 3:  # its own buffers: breaks both runs
+            xv = _pinned(np.zeros((M, K), np.float32))
+            yv = torch.empty((M, N), dtype=torch.float32, pin_memory=True)
+        xv.copy_(torch.from_numpy(xs[i]))
+        calls.append((xv, packs[i][0], packs[i][1], yv))
+    outs = B.forward_batch_host(calls, flags=flags)
+    torch.cuda.synchronize()
+    for i, (y, W, x) in enumerate(zip(outs, Ws, xs)):
+        assert y.data_ptr() == calls[i][3].data_ptr()
+        assert_y_close(y.numpy(), _oracle_y(W, x))
+    # every slot of the shared output buffer that a call owns was written
+    yo = 0
+    for i, (M, N, K) in enumerate(shapes):
+        if i != 3:
+            assert not torch.isnan(y_all[yo:yo + M * N]).any()
+        yo += M * N
+
+
+def test_forward_batch_host_chain_reuses_workspace(B):
+    """Repeated batched host calls on one stream and one workspace, each
+    feeding its output back as the next input."""
+    K = 1024
+    W = WL.weight(K, K, "normal", 1200)
+    packed, D = B.pack_weights(dev(W))
+    x0 = WL.activations(2, K, "normal", 1201)
+    xh = _pinned(x0)
+    yh = torch.empty((2, K), dtype=torch.float32, pin_memory=True)
+    ws = None
+    ref = x0
+    for _ in range(3):
+        if ws is None:
+            ws = torch.empty(B.batch_host_workspace_size([(2, K, K)]), dtype=torch.uint8, device="cuda")
+        B.forward_batch_host([(xh, packed, D, yh)], flags=1, ws=ws)
+        torch.cuda.synchronize()
+        ref = _oracle_y(W, ref)
+        assert_y_close(yh.numpy(), ref)
+        xh.copy_(yh)
+
+
 # ------------------------------------------------------------ bf16 inputs
 def _bf16(a):
     """fp32 numpy array -> (bf16 CUDA tensor, its uint16 bit patterns)."""
