@@ -476,9 +476,10 @@ def run_ours(a):
         configs = bench_configs(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, i8_burst, rank)
 
     # --------------------------------------------------------------------- pack
-    pack = None
+    pack = i2s = None
     if not a.ncu_small:
         pack = bench_pack(B, torch, dev, stream, hbm_peak)
+        i2s = bench_i2s(B, torch, dev, stream, hbm_peak)
 
     # ----------------------------------------------------- RMSNorm + ActQuant
     rms = None
@@ -531,6 +532,7 @@ def run_ours(a):
         "prefill": prefill,
         "configs": configs,
         "pack": pack,
+        "i2s": i2s,
         "bf16_inputs": bf16,
         "rmsnorm_actquant": rms,
         "cpu_baseline": cpu,
@@ -831,6 +833,46 @@ def bench_pack(B, torch, dev, stream, hbm_peak):
     return {"layer": f"gate_up {l.K}->{l.N}", "ms": round(t, 4), "GB/s_algorithmic": round(alg / (t * 1e-3) / 1e9, 1),
             "frac_hbm": round(alg / (t * 1e-3) / 1e9 / hbm_peak, 4),
             "note": "two passes over W (exact integer mean, then ternarise+pack); synchronous call"}
+
+
+def bench_i2s(B, torch, dev, stream, hbm_peak, copies=16, reps=5):
+    """I2_S export and import of a stack of `copies` gate_up weights (larger
+    than L2, so every call streams from HBM), both byte groupings."""
+    l = WL.WORKLOADS[HEADLINE].layers[2]
+    with torch.cuda.stream(stream):
+        W = torch.from_numpy(WL.weight(l.N, l.K, "normal", 6)).to(dev)
+        p1, D1 = B.pack_weights(W)
+        del W
+        packed = p1.repeat(copies, 1).contiguous()
+        D = D1.repeat(copies, 1).contiguous()
+        del p1, D1
+        N, K = packed.shape[0], packed.shape[1] * 16
+        buf = torch.empty(B.i2s_bytes(N, K), dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize(dev)
+        out = {"tensor": f"{copies} x gate_up stacked: [{N}, {K}]", "bytes_each_way": N * K // 4}
+        for layout in ("consecutive", "quarters"):
+            B.i2s_export(packed, D, layout, out=buf)
+            B.i2s_import(buf, N, K, layout)
+            res = {}
+            for name, fn, alg in (
+                    ("export", lambda: B.i2s_export(packed, D, layout, out=buf), N * K // 2 + 4 * N + 4),
+                    ("import", lambda: B.i2s_import(buf, N, K, layout), N * K // 2 + 4 * N + 4)):
+                ts = []
+                for _ in range(reps):
+                    e0 = torch.cuda.Event(enable_timing=True)
+                    e1 = torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    fn()
+                    e1.record(stream)
+                    torch.cuda.synchronize(dev)
+                    ts.append(e0.elapsed_time(e1))
+                t = statistics.median(ts)
+                res[name] = {"ms": round(t, 4), "GB/s_algorithmic": round(alg / (t * 1e-3) / 1e9, 1),
+                             "frac_hbm": round(alg / (t * 1e-3) / 1e9 / hbm_peak, 4)}
+            out[layout] = res
+    out["note"] = ("synchronous calls (status memset, one kernel, 4-byte status read); import includes allocating "
+                   "its packed and D outputs through torch's caching allocator")
+    return out
 
 
 def run_prefill_small(a, B, torch, dev):

@@ -24,6 +24,7 @@ STATUS_NAMES = {
     6: "BL_ERR_DEVICE",
     7: "BL_ERR_CUDA",
     8: "BL_ERR_UNSUPPORTED",
+    9: "BL_ERR_FORMAT",
 }
 
 # name -> (restype, argtypes), mirroring include/bitlinear.h
@@ -53,6 +54,12 @@ SIGNATURES = {
     "bitlinear_forward_bf16": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "bitlinear_batch_host_workspace_size": (ctypes.c_size_t, [_VP, ctypes.c_int]),
     "bitlinear_forward_batch_host": (ctypes.c_int, [_VP, ctypes.c_int, ctypes.c_uint32, _VP, _SZ, _VP]),
+    "bitlinear_i2s_bytes": (_SZ, [ctypes.c_int64, ctypes.c_int64]),
+    "bitlinear_i2s_workspace_size": (_SZ, []),
+    "bitlinear_i2s_export": (ctypes.c_int, [_VP, _VP, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, _VP, _VP, _SZ,
+                                            _VP]),
+    "bitlinear_i2s_import": (ctypes.c_int, [_VP, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, _VP, _VP, _VP, _SZ,
+                                            _VP]),
     "bitlinear_rmsnorm_quant_act": (ctypes.c_int, [_VP, _VP, ctypes.c_float, _I64, _I64, _VP, _VP, _VP, _VP]),
     "bitlinear_forward_rmsnorm": (ctypes.c_int, [_VP, _VP, ctypes.c_float, _I64, _I64, _I64, _VP, _VP, _VP,
                                                  _VP, _SZ, _VP]),
@@ -81,6 +88,8 @@ class LinearCall(ctypes.Structure):
 
 BL_FLAG_STREAM_WEIGHTS_EARLY = 1
 BL_FLAG_ONE_LAUNCH_PER_CALL = 2
+BL_I2S_CONSECUTIVE = 0
+BL_I2S_QUARTERS = 1
 
 
 class BitLinearError(RuntimeError):

@@ -321,6 +321,50 @@ def forward_host(x_host: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,
     return y_host
 
 
+_I2S_LAYOUTS = {"consecutive": _lib.BL_I2S_CONSECUTIVE, "quarters": _lib.BL_I2S_QUARTERS}
+
+
+def i2s_bytes(N: int, K: int) -> int:
+    """Size of the I2_S buffer of an [N, K] tensor (blocks plus the fp32 scale)."""
+    return int(_lib.lib().bitlinear_i2s_bytes(N, K))
+
+
+def i2s_export(packed: torch.Tensor, D: torch.Tensor, layout: str = "consecutive",
+               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """BitLinear packed weights + D -> one I2_S buffer (uint8 CUDA tensor).
+    Synchronous; raises BitLinearError (BL_ERR_FORMAT) on a field holding 3 or
+    rows of D that differ."""
+    _need_cuda(packed, "packed", torch.int32)
+    N, K = packed.shape[0], packed.shape[1] * 16
+    _check_D(D, N)
+    nbytes = i2s_bytes(N, K)
+    if out is None:
+        out = torch.empty(nbytes, dtype=torch.uint8, device=packed.device)
+    _need_cuda(out, "out", torch.uint8)
+    if out.numel() != nbytes:
+        raise ValueError(f"out must hold {nbytes} bytes")
+    ws = _alloc_ws(_lib.lib().bitlinear_i2s_workspace_size(), packed.device)
+    _lib.call("bitlinear_i2s_export", packed.data_ptr(), D.data_ptr(), N, K, _I2S_LAYOUTS[layout], out.data_ptr(),
+              ws.data_ptr(), ws.numel(), _stream_handle(packed.device))
+    return out
+
+
+def i2s_import(buf: torch.Tensor, N: int, K: int, layout: str = "consecutive") -> Tuple[torch.Tensor, torch.Tensor]:
+    """One I2_S buffer (uint8 CUDA tensor) of an [N, K] tensor -> (packed
+    int32 [N, K/16], D fp32 [N, 1]). Synchronous; raises BitLinearError
+    (BL_ERR_FORMAT) on a field holding 3 or a scale that is not finite and
+    positive."""
+    _need_cuda(buf, "buf", torch.uint8)
+    if buf.numel() != i2s_bytes(N, K):
+        raise ValueError(f"buf must hold {i2s_bytes(N, K)} bytes")
+    packed = torch.empty((N, K // 16), dtype=torch.int32, device=buf.device)
+    D = torch.empty((N, 1), dtype=torch.float32, device=buf.device)
+    ws = _alloc_ws(_lib.lib().bitlinear_i2s_workspace_size(), buf.device)
+    _lib.call("bitlinear_i2s_import", buf.data_ptr(), N, K, _I2S_LAYOUTS[layout], packed.data_ptr(), D.data_ptr(),
+              ws.data_ptr(), ws.numel(), _stream_handle(buf.device))
+    return packed, D
+
+
 def workspace_error(ws: torch.Tensor) -> int:
     """Synchronise and read/clear the device error word of a forward workspace."""
     return int(_lib.lib().bitlinear_workspace_error(ws.data_ptr(), ws.numel(), _stream_handle(ws.device)))

@@ -92,6 +92,7 @@ const char* bitlinear_status_string(int status) {
     case BL_ERR_DEVICE: return "device-side failure recorded (bounded wait expired)";
     case BL_ERR_CUDA: return "CUDA runtime error";
     case BL_ERR_UNSUPPORTED: return "device is not sm_100 (B200 class)";
+    case BL_ERR_FORMAT: return "I2_S: field holding 3, bad scale, or rows of D that differ";
     default: return "unknown status";
   }
 }
@@ -508,6 +509,50 @@ int bitlinear_selftest_wait_timeout(void* ws, size_t ws_bytes, uint64_t limit_ns
   const uint64_t cap = 100000000ull;
   return cuda_status(bl::launch_selftest_wait(static_cast<uint32_t*>(ws), limit_ns < cap ? limit_ns : cap,
                                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t bitlinear_i2s_bytes(int64_t N, int64_t K) {
+  if (N < 0 || K < 0) return 0;
+  return 32 * (((size_t)N * (size_t)K + 127) / 128) + 4;
+}
+
+size_t bitlinear_i2s_workspace_size(void) { return bl::kHeaderBytes; }
+
+// Shared checks and the synchronous status read of the two I2_S conversions.
+static int i2s_impl(bool to_i2s, const void* i2s, const uint32_t* packed, const float* D, int64_t N, int64_t K,
+                    int layout, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  if (N <= 0 || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  if (layout != BL_I2S_CONSECUTIVE && layout != BL_I2S_QUARTERS) return BL_ERR_SHAPE;
+  if (i2s == nullptr || packed == nullptr || D == nullptr || ws == nullptr) return BL_ERR_NULL;
+  if (!aligned16(i2s) || !aligned16(packed) || (reinterpret_cast<uintptr_t>(D) & 3u) || !aligned256(ws))
+    return BL_ERR_ALIGN;
+  if (ws_bytes < bl::kHeaderBytes) return BL_ERR_WORKSPACE;
+  const int sms = num_sms_current();
+  if (sms <= 0) return BL_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* err = static_cast<uint32_t*>(ws);
+  const cudaError_t e =
+      to_i2s ? bl::launch_i2s(true, layout == BL_I2S_QUARTERS, packed, const_cast<void*>(i2s), D, nullptr, N, K,
+                              err, s, sms)
+             : bl::launch_i2s(false, layout == BL_I2S_QUARTERS, i2s, const_cast<uint32_t*>(packed), nullptr,
+                              const_cast<float*>(D), N, K, err, s, sms);
+  if (e != cudaSuccess) return BL_ERR_CUDA;
+  uint32_t status = 0;
+  if (cudaMemcpyAsync(&status, err, sizeof(status), cudaMemcpyDeviceToHost, s) != cudaSuccess) return BL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
+  return status == 0u ? BL_OK : BL_ERR_FORMAT;
+}
+
+int bitlinear_i2s_export(const uint32_t* packed, const float* D, int64_t N, int64_t K, int layout, uint8_t* i2s,
+                         void* ws, size_t ws_bytes, bl_stream_t stream) {
+  return i2s_impl(true, i2s, packed, D, N, K, layout, ws, ws_bytes, stream);
+}
+
+int bitlinear_i2s_import(const uint8_t* i2s, int64_t N, int64_t K, int layout, uint32_t* packed, float* D, void* ws,
+                         size_t ws_bytes, bl_stream_t stream) {
+  return i2s_impl(false, i2s, packed, D, N, K, layout, ws, ws_bytes, stream);
 }
 
 }  // extern "C"

@@ -23,6 +23,14 @@ constexpr int kGemvMaxGroup = 8;                   // BitLinears per grouped lau
 constexpr int64_t kGemvSmemTarget = 100 * 1024;    // leaves room for a CTA of the next launch
 constexpr int64_t kGemvMaxSmem = 200 * 1024;
 
+// I2_S conversion (bl_i2s.cu): to_i2s packs `in` (BitLinear words, D_in)
+// into I2_S words at `out`; otherwise unpacks I2_S words at `in` into packed
+// words at `out` and D_out. err (a device word) gets bit 0 for a field
+// holding 3 and bit 1 for a scale that is not finite and positive (or rows of
+// D_in that differ).
+cudaError_t launch_i2s(bool to_i2s, bool quarters, const void* in, void* out, const float* D_in, float* D_out,
+                       int64_t N, int64_t K, uint32_t* err, cudaStream_t stream, int sms);
+
 inline int64_t gemv_q_stride(int64_t K) { return ((K + 255) / 256) * 256 + 16; }
 
 struct GemvCall {

@@ -71,7 +71,9 @@ typedef enum {
   BL_ERR_NONFINITE = 5,   /* pack: W holds Inf or NaN, so mean(|W|) is not finite */
   BL_ERR_DEVICE = 6,      /* a kernel recorded a device-side failure (bounded wait expired) */
   BL_ERR_CUDA = 7,        /* a CUDA runtime call failed (launch, copy, attribute) */
-  BL_ERR_UNSUPPORTED = 8  /* the current device is not sm_100 (B200 class) */
+  BL_ERR_UNSUPPORTED = 8, /* the current device is not sm_100 (B200 class) */
+  BL_ERR_FORMAT = 9       /* I2_S: a field holds 3, the scale is not finite and
+                             positive, or (export) the rows of D differ */
 } bl_status;
 
 /* Version of this ABI (incremented on any incompatible change). */
@@ -312,6 +314,49 @@ BL_API int bitlinear_workspace_error(void* ws, size_t ws_bytes, bl_stream_t stre
 BL_API int bitlinear_forward_noalloc(const float* x, int64_t M, int64_t N, int64_t K,
                                      const uint32_t* packed, const float* D, float* y,
                                      bl_stream_t stream);
+
+/* ---------------------------------------------------------------- I2_S --- */
+
+/* I2_S, the 2-bit ternary format of the "BitNet-Embeddings I2_S guide"
+ * (section "I2_S Ternary Packing"): codes stored as code + 1 (-1 -> 0,
+ * 0 -> 1, +1 -> 2), 128 values per 32-byte block with
+ * byte = c0 << 6 | c1 << 4 | c2 << 2 | c3, and the fp32 scale 1/mean(|w|)
+ * appended (little-endian) right after the last block. The blocks run over the
+ * flattened row-major [N, K] tensor; a tail shorter than 128 values is padded
+ * with the code 0. The page does not say which four values of a block share a
+ * byte; `layout` picks the reading:
+ *   BL_I2S_CONSECUTIVE  byte j holds values 4j, 4j+1, 4j+2, 4j+3 (c0..c3);
+ *   BL_I2S_QUARTERS     byte j holds values j, j+32, j+64, j+96 (c0..c3). */
+#define BL_I2S_CONSECUTIVE 0
+#define BL_I2S_QUARTERS 1
+
+/* Bytes of the I2_S buffer of an [N, K] tensor: 32 * ceil(N*K / 128) + 4
+ * (0 for negative sizes). */
+BL_API size_t bitlinear_i2s_bytes(int64_t N, int64_t K);
+
+/* Scratch for the two conversions (one device status word): 256 bytes. */
+BL_API size_t bitlinear_i2s_workspace_size(void);
+
+/* Export BitLinear packed weights to I2_S.
+ *   packed  device uint32 [N, K/16], D device fp32 [N] (every row the same
+ *           value, as bitlinear_pack_weights writes it).
+ *   i2s     device buffer of bitlinear_i2s_bytes(N, K) bytes (16-byte
+ *           aligned); gets the blocks, then the scale RN(1/D[0]), which for a
+ *           pack's D = mean_c is exactly the quantiser's s = RN(1/mean_c).
+ * 1 <= N, K as for the forward. Synchronous: returns BL_ERR_FORMAT if a
+ * packed field holds 3, the rows of D differ, or D[0] or 1/D[0] is not finite
+ * and positive (the contents of i2s are then unspecified). */
+BL_API int bitlinear_i2s_export(const uint32_t* packed, const float* D, int64_t N, int64_t K, int layout,
+                                uint8_t* i2s, void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* Import an I2_S buffer (device, bitlinear_i2s_bytes(N, K) bytes, 16-byte
+ * aligned) into BitLinear packed weights [N, K/16] and D [N] = RN(1/scale)
+ * for every row. Padding values of the tail block are ignored. Synchronous:
+ * returns BL_ERR_FORMAT if a value's field holds 3 or the scale (or its
+ * reciprocal) is not finite and positive (packed and D are then
+ * unspecified). */
+BL_API int bitlinear_i2s_import(const uint8_t* i2s, int64_t N, int64_t K, int layout,
+                                uint32_t* packed, float* D, void* ws, size_t ws_bytes, bl_stream_t stream);
 
 /* Diagnostic for the failure-detection path. Launches one thread that waits
  * on a shared-memory barrier that nothing ever completes, using the same

@@ -116,7 +116,10 @@ def i2s_export(packed: np.ndarray, D: np.ndarray, K: int, layout: str = "consecu
     if not (np.isfinite(Dv[0]) and Dv[0] > 0):
         raise ValueError("D must be finite and positive")
     codes = unpack_codes(np.asarray(packed), K)
-    scale = np.float32(np.float32(1.0) / Dv[0])
+    with np.errstate(over="ignore"):
+        scale = np.float32(np.float32(1.0) / Dv[0])
+    if not np.isfinite(scale):
+        raise ValueError("the reciprocal of D is not finite, so no I2_S scale holds it")
     return np.concatenate([i2s_encode_codes(codes, layout), np.array([scale], "<f4").view(np.uint8)])
 
 

@@ -38,7 +38,7 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_abi_version_and_status_strings(L):
     assert L.bitlinear_abi_version() == 1
-    for st in range(0, 9):
+    for st in range(0, 10):
         s = L.bitlinear_status_string(st)
         assert s and isinstance(s, bytes)
     assert L.bitlinear_status_string(99) == b"unknown status"
@@ -159,3 +159,27 @@ def test_batch_host_validation_before_cuda(L):
     calls[1] = _lib.LinearCall(FAKE, 3, 5, 32, FAKE + 4, FAKE, FAKE)  # packed not 16-byte aligned
     assert L.bitlinear_forward_batch_host(calls, 3, 0, FAKE, 1 << 20, None) == 3
     assert L.bitlinear_batch_host_workspace_size(None, 3) == 0
+
+
+def test_i2s_sizes_and_validation_before_cuda(L):
+    assert L.bitlinear_i2s_bytes(3, 48) == 68
+    assert L.bitlinear_i2s_bytes(2560, 2560) == 2560 * 2560 // 4 + 4
+    assert L.bitlinear_i2s_bytes(1, 16) == 36
+    assert L.bitlinear_i2s_bytes(-1, 16) == 0
+    assert L.bitlinear_i2s_workspace_size() == 256
+    # bitlinear_i2s_export(packed, D, N, K, layout, i2s, ws, ws_bytes, stream)
+    assert L.bitlinear_i2s_export(FAKE, FAKE, 3, 24, 0, FAKE, FAKE, 256, None) == 2
+    assert L.bitlinear_i2s_export(FAKE, FAKE, 0, 48, 0, FAKE, FAKE, 256, None) == 2
+    assert L.bitlinear_i2s_export(FAKE, FAKE, 3, 48, 2, FAKE, FAKE, 256, None) == 2
+    assert L.bitlinear_i2s_export(None, FAKE, 3, 48, 0, FAKE, FAKE, 256, None) == 1
+    assert L.bitlinear_i2s_export(FAKE, FAKE, 3, 48, 1, FAKE + 4, FAKE, 256, None) == 3
+    assert L.bitlinear_i2s_export(FAKE, FAKE + 2, 3, 48, 1, FAKE, FAKE, 256, None) == 3
+    assert L.bitlinear_i2s_export(FAKE, FAKE, 3, 48, 0, FAKE, FAKE, 128, None) == 4
+    # bitlinear_i2s_import(i2s, N, K, layout, packed, D, ws, ws_bytes, stream)
+    assert L.bitlinear_i2s_import(FAKE, 3, 40, 0, FAKE, FAKE, FAKE, 256, None) == 2
+    assert L.bitlinear_i2s_import(FAKE, 3, 48, -1, FAKE, FAKE, FAKE, 256, None) == 2
+    assert L.bitlinear_i2s_import(FAKE, 3, 48, 0, FAKE, None, FAKE, 256, None) == 1
+    assert L.bitlinear_i2s_import(FAKE, 3, 48, 0, FAKE + 8, FAKE, FAKE, 256, None) == 3
+    assert L.bitlinear_i2s_import(FAKE, 3, 48, 0, FAKE, FAKE, FAKE + 16, 256, None) == 3
+    assert L.bitlinear_i2s_import(FAKE, 3, 48, 0, FAKE, FAKE, FAKE, 8, None) == 4
+    assert L.bitlinear_status_string(9) == b"I2_S: field holding 3, bad scale, or rows of D that differ"

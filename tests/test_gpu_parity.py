@@ -642,3 +642,96 @@ def test_forward_rmsnorm(B, M, N, K):
     p_ref, D_ref = O.pack_weights(W)
     y = B.forward_rmsnorm(dev(x), dev(g), packed, D).cpu().numpy()
     assert_y_close(y, O.bitlinear_forward_rmsnorm(x, g, p_ref, D_ref, K))
+
+
+# ------------------------------------------------------------ I2_S import/export
+I2S_SHAPES = [(1, 16), (3, 48), (5, 1152), (17, 4304), (2560, 2560), (7, 6912)]
+
+
+@pytest.mark.parametrize("layout", ["consecutive", "quarters"])
+@pytest.mark.parametrize("N,K", I2S_SHAPES)
+def test_i2s_export_bitexact(B, layout, N, K):
+    W = WL.weight(N, K, "normal", 1300 + K + N)
+    p_ref, D_ref = O.pack_weights(W)
+    buf = B.i2s_export(dev(p_ref.view(np.int32)), dev(D_ref), layout)
+    assert np.array_equal(buf.cpu().numpy(), O.i2s_export(p_ref, D_ref, K, layout))
+
+
+@pytest.mark.parametrize("layout", ["consecutive", "quarters"])
+@pytest.mark.parametrize("N,K", I2S_SHAPES)
+def test_i2s_import_bitexact_arbitrary_codes(B, layout, N, K):
+    """Random valid fields (not only what a pack produces) and random bytes in
+    the tail padding, with a scale that is not a power of two."""
+    rng = np.random.default_rng(N * 131 + K)
+    codes = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+    blocks = O.i2s_encode_codes(codes, layout)
+    pad = blocks.size * 4 - N * K  # padding values at the end of the last block
+    if pad:
+        # overwrite the padding fields of the last block with random 2-bit values, 3 included
+        got = O.i2s_decode_codes(blocks, N * K, layout)
+        assert np.array_equal(got, codes.reshape(-1))
+        last = blocks[-32:].copy()
+        junk = rng.integers(0, 256, size=32).astype(np.uint8)
+        order = np.arange(128).reshape(32, 4) if layout == "consecutive" else np.arange(128).reshape(4, 32).T
+        for byte in range(32):
+            for f in range(4):
+                v = order[byte, f]  # value index within the block
+                if (blocks.size - 32) * 4 + v >= N * K:
+                    sh = 6 - 2 * f
+                    last[byte] = (int(last[byte]) & (0xFF ^ (3 << sh))) | (int(junk[byte]) & (3 << sh))
+        blocks = np.concatenate([blocks[:-32], last])
+    scale = np.float32(7.3)
+    buf = np.concatenate([blocks, np.array([scale], "<f4").view(np.uint8)])
+    packed, D = B.i2s_import(dev(buf), N, K, layout)
+    p_ref, D_ref = O.i2s_import(buf, N, K, layout)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)
+    assert np.array_equal(D.cpu().numpy(), D_ref)
+
+
+@pytest.mark.parametrize("layout", ["consecutive", "quarters"])
+def test_i2s_round_trip_and_forward(B, layout):
+    """pack -> export -> import gives the same codes; the forward from the
+    imported weights equals the oracle's forward with the imported D."""
+    N, K, M = 300, 1152, 5
+    W = WL.weight(N, K, "laplace", 1400)
+    x = WL.activations(M, K, "normal", 1401)
+    packed, D = B.pack_weights(dev(W))
+    buf = B.i2s_export(packed, D, layout)
+    assert np.array_equal(buf.cpu().numpy(), O.i2s_from_weight(W, layout))
+    p2, D2 = B.i2s_import(buf, N, K, layout)
+    assert torch.equal(p2, packed)
+    p_ref, D_ref = O.i2s_import(buf.cpu().numpy(), N, K, layout)
+    assert np.array_equal(D2.cpu().numpy(), D_ref)
+    y = B.forward(dev(x), p2, D2)
+    torch.cuda.synchronize()
+    assert_y_close(y.cpu().numpy(), O.bitlinear_forward(x, p_ref, D_ref, K))
+
+
+def test_i2s_rejects_invalid_buffers(B):
+    from bit_ternary_b200._lib import BitLinearError
+
+    N, K = 3, 48
+    W = WL.weight(N, K, "normal", 1500)
+    p_ref, D_ref = O.pack_weights(W)
+    good = O.i2s_export(p_ref, D_ref, K)
+    for layout in ("consecutive", "quarters"):
+        bad = good.copy()
+        bad[5] |= 0x0C  # a data value holds 3
+        with pytest.raises(BitLinearError, match="FORMAT"):
+            B.i2s_import(dev(bad), N, K, layout)
+    for scale in (0.0, -2.0, np.nan, np.inf, 1e-45):
+        b = good.copy()
+        b[-4:] = np.array([scale], "<f4").view(np.uint8)
+        with pytest.raises(BitLinearError, match="FORMAT"):
+            B.i2s_import(dev(b), N, K)
+    D_rows = D_ref.copy()
+    D_rows[2, 0] *= 2
+    with pytest.raises(BitLinearError, match="FORMAT"):
+        B.i2s_export(dev(p_ref.view(np.int32)), dev(D_rows))
+    p3 = p_ref.copy()
+    p3[1, 2] |= np.uint32(3 << 10)  # a packed field holds 3
+    with pytest.raises(BitLinearError, match="FORMAT"):
+        B.i2s_export(dev(p3.view(np.int32)), dev(D_ref))
+    # the context still works, and a good buffer still imports
+    packed, D = B.i2s_import(dev(good), N, K)
+    assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)

@@ -159,6 +159,9 @@ def test_export_rejects_per_row_scales():
     D2[1, 0] = 2.0
     with pytest.raises(ValueError, match="differ"):
         O.i2s_export(packed, D2, 16)
+    for d in (0.0, -1.0, np.nan, np.inf, 1e-45):  # no finite positive scale 1/d
+        with pytest.raises(ValueError):
+            O.i2s_export(packed, np.full((2, 1), d, np.float32), 16)
 
 
 # planted mistakes: each must fail the hand-worked block
