@@ -64,6 +64,10 @@ def parse_args(argv=None):
                     help="small prefill-only run for profiler captures (gate_up layer, M=4096)")
     ap.add_argument("--ncu-layer", default=None, metavar="WORKLOAD:LAYER:M",
                     help="one layer of a workload, M tokens, for profiler captures (e.g. embed_batch:0:32768)")
+    ap.add_argument("--ncu-i2s", action="store_true",
+                    help="I2_S export/import only (stacked gate_up weights), for profiler captures")
+    ap.add_argument("--i2s-layouts", default="consecutive,quarters",
+                    help="byte groupings timed by the I2_S part (comma-separated)")
     a = ap.parse_args(argv)
     a.warmup = max(3, a.warmup)
     a.steps = max(1, a.steps)
@@ -257,6 +261,12 @@ def run_ours(a):
         raise SystemExit("device is not sm_100 (B200)")
     if a.ncu_prefill or a.ncu_layer:
         return run_prefill_small(a, B, torch, dev)
+    if a.ncu_i2s:
+        peaks, _ = load_peaks()
+        stream = torch.cuda.Stream(device=dev)
+        print(json.dumps({"i2s": bench_i2s(B, torch, dev, stream, float(peaks["hbm_gbs"]), reps=2,
+                                           layouts=tuple(a.i2s_layouts.split(",")))}))
+        return 0
     if world > 1:
         import datetime
 
@@ -479,7 +489,7 @@ def run_ours(a):
     pack = i2s = None
     if not a.ncu_small:
         pack = bench_pack(B, torch, dev, stream, hbm_peak)
-        i2s = bench_i2s(B, torch, dev, stream, hbm_peak)
+        i2s = bench_i2s(B, torch, dev, stream, hbm_peak, layouts=tuple(a.i2s_layouts.split(",")))
 
     # ----------------------------------------------------- RMSNorm + ActQuant
     rms = None
@@ -835,9 +845,11 @@ def bench_pack(B, torch, dev, stream, hbm_peak):
             "note": "two passes over W (exact integer mean, then ternarise+pack); synchronous call"}
 
 
-def bench_i2s(B, torch, dev, stream, hbm_peak, copies=16, reps=5):
+def bench_i2s(B, torch, dev, stream, hbm_peak, copies=16, reps=10, layouts=("consecutive", "quarters")):
     """I2_S export and import of a stack of `copies` gate_up weights (larger
-    than L2, so every call streams from HBM), both byte groupings."""
+    than L2, so every call streams from HBM), both byte groupings: `reps`
+    asynchronous conversions back to back between two events (one status
+    check after them), and the synchronous call for comparison."""
     l = WL.WORKLOADS[HEADLINE].layers[2]
     with torch.cuda.stream(stream):
         W = torch.from_numpy(WL.weight(l.N, l.K, "normal", 6)).to(dev)
@@ -848,30 +860,49 @@ def bench_i2s(B, torch, dev, stream, hbm_peak, copies=16, reps=5):
         del p1, D1
         N, K = packed.shape[0], packed.shape[1] * 16
         buf = torch.empty(B.i2s_bytes(N, K), dtype=torch.uint8, device=dev)
+        p_in = torch.empty_like(packed)
+        D_in = torch.empty_like(D)
+        ws = B.i2s_workspace(dev)
         torch.cuda.synchronize(dev)
-        out = {"tensor": f"{copies} x gate_up stacked: [{N}, {K}]", "bytes_each_way": N * K // 4}
-        for layout in ("consecutive", "quarters"):
-            B.i2s_export(packed, D, layout, out=buf)
-            B.i2s_import(buf, N, K, layout)
+        alg = N * K // 2 + 4 * N + 4  # packed words + I2_S blocks + D + scale
+        out = {"tensor": f"{copies} x gate_up stacked: [{N}, {K}]", "bytes_each_way": N * K // 4,
+               "algorithmic_bytes_per_call": alg}
+        for layout in layouts:
+            calls = {
+                "export": lambda sync: B.i2s_export(packed, D, layout, out=buf, ws=ws, sync=sync),
+                "import": lambda sync: B.i2s_import(buf, N, K, layout, out=(p_in, D_in), ws=ws, sync=sync),
+            }
             res = {}
-            for name, fn, alg in (
-                    ("export", lambda: B.i2s_export(packed, D, layout, out=buf), N * K // 2 + 4 * N + 4),
-                    ("import", lambda: B.i2s_import(buf, N, K, layout), N * K // 2 + 4 * N + 4)):
-                ts = []
+            for name, fn in calls.items():
+                for _ in range(3):
+                    fn(False)
+                torch.cuda.synchronize(dev)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
                 for _ in range(reps):
-                    e0 = torch.cuda.Event(enable_timing=True)
-                    e1 = torch.cuda.Event(enable_timing=True)
-                    e0.record(stream)
-                    fn()
-                    e1.record(stream)
+                    fn(False)
+                e1.record(stream)
+                torch.cuda.synchronize(dev)
+                if B.i2s_status(ws) != 0:
+                    raise RuntimeError("I2_S conversion reported a format error")
+                t = e0.elapsed_time(e1) / reps
+                ts = []
+                for _ in range(3):
+                    f0 = torch.cuda.Event(enable_timing=True)
+                    f1 = torch.cuda.Event(enable_timing=True)
+                    f0.record(stream)
+                    fn(True)
+                    f1.record(stream)
                     torch.cuda.synchronize(dev)
-                    ts.append(e0.elapsed_time(e1))
-                t = statistics.median(ts)
-                res[name] = {"ms": round(t, 4), "GB/s_algorithmic": round(alg / (t * 1e-3) / 1e9, 1),
-                             "frac_hbm": round(alg / (t * 1e-3) / 1e9 / hbm_peak, 4)}
+                    ts.append(f0.elapsed_time(f1))
+                res[name] = {"us": round(t * 1e3, 2), "GB/s_algorithmic": round(alg / (t * 1e-3) / 1e9, 1),
+                             "frac_hbm": round(alg / (t * 1e-3) / 1e9 / hbm_peak, 4),
+                             "sync_call_us": round(statistics.median(ts) * 1e3, 2)}
             out[layout] = res
-    out["note"] = ("synchronous calls (status memset, one kernel, 4-byte status read); import includes allocating "
-                   "its packed and D outputs through torch's caching allocator")
+        assert torch.equal(p_in, packed)
+    out["note"] = ("us / GB/s: asynchronous calls back to back (one kernel each), one status check after them; "
+                   "sync_call_us: the synchronous call (status clear, kernel, status read, host wake-up)")
     return out
 
 

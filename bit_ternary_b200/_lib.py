@@ -60,6 +60,11 @@ SIGNATURES = {
                                             _VP]),
     "bitlinear_i2s_import": (ctypes.c_int, [_VP, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, _VP, _VP, _VP, _SZ,
                                             _VP]),
+    "bitlinear_i2s_export_async": (ctypes.c_int, [_VP, _VP, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, _VP, _VP,
+                                                  _SZ, _VP]),
+    "bitlinear_i2s_import_async": (ctypes.c_int, [_VP, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, _VP, _VP, _VP,
+                                                  _SZ, _VP]),
+    "bitlinear_i2s_status": (ctypes.c_int, [_VP, _SZ, _VP]),
     "bitlinear_rmsnorm_quant_act": (ctypes.c_int, [_VP, _VP, ctypes.c_float, _I64, _I64, _VP, _VP, _VP, _VP]),
     "bitlinear_forward_rmsnorm": (ctypes.c_int, [_VP, _VP, ctypes.c_float, _I64, _I64, _I64, _VP, _VP, _VP,
                                                  _VP, _SZ, _VP]),

@@ -329,11 +329,18 @@ def i2s_bytes(N: int, K: int) -> int:
     return int(_lib.lib().bitlinear_i2s_bytes(N, K))
 
 
+def i2s_workspace(device) -> torch.Tensor:
+    """A zeroed workspace (status word) for the I2_S conversions."""
+    return torch.zeros(max(256, int(_lib.lib().bitlinear_i2s_workspace_size())), dtype=torch.uint8, device=device)
+
+
 def i2s_export(packed: torch.Tensor, D: torch.Tensor, layout: str = "consecutive",
-               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+               out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+               sync: bool = True) -> torch.Tensor:
     """BitLinear packed weights + D -> one I2_S buffer (uint8 CUDA tensor).
-    Synchronous; raises BitLinearError (BL_ERR_FORMAT) on a field holding 3 or
-    rows of D that differ."""
+    sync=True: raises BitLinearError (BL_ERR_FORMAT) on a field holding 3 or
+    rows of D that differ. sync=False: enqueued on the current stream; errors
+    collect in ws (zeroed by i2s_workspace) until i2s_status(ws)."""
     _need_cuda(packed, "packed", torch.int32)
     N, K = packed.shape[0], packed.shape[1] * 16
     _check_D(D, N)
@@ -343,26 +350,49 @@ def i2s_export(packed: torch.Tensor, D: torch.Tensor, layout: str = "consecutive
     _need_cuda(out, "out", torch.uint8)
     if out.numel() != nbytes:
         raise ValueError(f"out must hold {nbytes} bytes")
-    ws = _alloc_ws(_lib.lib().bitlinear_i2s_workspace_size(), packed.device)
-    _lib.call("bitlinear_i2s_export", packed.data_ptr(), D.data_ptr(), N, K, _I2S_LAYOUTS[layout], out.data_ptr(),
+    if ws is None:
+        if not sync:
+            raise ValueError("the asynchronous conversion needs a workspace from i2s_workspace()")
+        ws = i2s_workspace(packed.device)
+    fn = "bitlinear_i2s_export" if sync else "bitlinear_i2s_export_async"
+    _lib.call(fn, packed.data_ptr(), D.data_ptr(), N, K, _I2S_LAYOUTS[layout], out.data_ptr(),
               ws.data_ptr(), ws.numel(), _stream_handle(packed.device))
     return out
 
 
-def i2s_import(buf: torch.Tensor, N: int, K: int, layout: str = "consecutive") -> Tuple[torch.Tensor, torch.Tensor]:
+def i2s_import(buf: torch.Tensor, N: int, K: int, layout: str = "consecutive",
+               out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None, ws: Optional[torch.Tensor] = None,
+               sync: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
     """One I2_S buffer (uint8 CUDA tensor) of an [N, K] tensor -> (packed
-    int32 [N, K/16], D fp32 [N, 1]). Synchronous; raises BitLinearError
+    int32 [N, K/16], D fp32 [N, 1]). sync=True: raises BitLinearError
     (BL_ERR_FORMAT) on a field holding 3 or a scale that is not finite and
-    positive."""
+    positive. sync=False: as for i2s_export."""
     _need_cuda(buf, "buf", torch.uint8)
     if buf.numel() != i2s_bytes(N, K):
         raise ValueError(f"buf must hold {i2s_bytes(N, K)} bytes")
-    packed = torch.empty((N, K // 16), dtype=torch.int32, device=buf.device)
-    D = torch.empty((N, 1), dtype=torch.float32, device=buf.device)
-    ws = _alloc_ws(_lib.lib().bitlinear_i2s_workspace_size(), buf.device)
-    _lib.call("bitlinear_i2s_import", buf.data_ptr(), N, K, _I2S_LAYOUTS[layout], packed.data_ptr(), D.data_ptr(),
+    if out is None:
+        packed = torch.empty((N, K // 16), dtype=torch.int32, device=buf.device)
+        D = torch.empty((N, 1), dtype=torch.float32, device=buf.device)
+    else:
+        packed, D = out
+        _need_cuda(packed, "packed", torch.int32)
+        _check_D(D, N)
+        if tuple(packed.shape) != (N, K // 16):
+            raise ValueError("packed must be [N, K/16]")
+    if ws is None:
+        if not sync:
+            raise ValueError("the asynchronous conversion needs a workspace from i2s_workspace()")
+        ws = i2s_workspace(buf.device)
+    fn = "bitlinear_i2s_import" if sync else "bitlinear_i2s_import_async"
+    _lib.call(fn, buf.data_ptr(), N, K, _I2S_LAYOUTS[layout], packed.data_ptr(), D.data_ptr(),
               ws.data_ptr(), ws.numel(), _stream_handle(buf.device))
     return packed, D
+
+
+def i2s_status(ws: torch.Tensor) -> int:
+    """Synchronise and read/clear the status word of asynchronous I2_S
+    conversions: 0 (BL_OK) or 9 (BL_ERR_FORMAT)."""
+    return int(_lib.lib().bitlinear_i2s_status(ws.data_ptr(), ws.numel(), _stream_handle(ws.device)))
 
 
 def workspace_error(ws: torch.Tensor) -> int:

@@ -518,9 +518,21 @@ size_t bitlinear_i2s_bytes(int64_t N, int64_t K) {
 
 size_t bitlinear_i2s_workspace_size(void) { return bl::kHeaderBytes; }
 
-// Shared checks and the synchronous status read of the two I2_S conversions.
+// Reads and clears the I2_S status word (after synchronising the stream).
+static int i2s_read_status(uint32_t* err, cudaStream_t s) {
+  uint32_t status = 0;
+  if (cudaMemcpyAsync(&status, err, sizeof(status), cudaMemcpyDeviceToHost, s) != cudaSuccess) return BL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
+  if (status == 0u) return BL_OK;
+  if (cudaMemsetAsync(err, 0, sizeof(status), s) != cudaSuccess) return BL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
+  return BL_ERR_FORMAT;
+}
+
+// Shared checks of the two I2_S conversions; `sync` clears the status word
+// first and reads it back at the end.
 static int i2s_impl(bool to_i2s, const void* i2s, const uint32_t* packed, const float* D, int64_t N, int64_t K,
-                    int layout, void* ws, size_t ws_bytes, bl_stream_t stream) {
+                    int layout, void* ws, size_t ws_bytes, bl_stream_t stream, bool sync) {
   int st = check_k(K);
   if (st != BL_OK) return st;
   if (N <= 0 || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
@@ -533,26 +545,41 @@ static int i2s_impl(bool to_i2s, const void* i2s, const uint32_t* packed, const 
   if (sms <= 0) return BL_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(ws);
+  if (sync && cudaMemsetAsync(err, 0, sizeof(uint32_t), s) != cudaSuccess) return BL_ERR_CUDA;
   const cudaError_t e =
       to_i2s ? bl::launch_i2s(true, layout == BL_I2S_QUARTERS, packed, const_cast<void*>(i2s), D, nullptr, N, K,
                               err, s, sms)
              : bl::launch_i2s(false, layout == BL_I2S_QUARTERS, i2s, const_cast<uint32_t*>(packed), nullptr,
                               const_cast<float*>(D), N, K, err, s, sms);
   if (e != cudaSuccess) return BL_ERR_CUDA;
-  uint32_t status = 0;
-  if (cudaMemcpyAsync(&status, err, sizeof(status), cudaMemcpyDeviceToHost, s) != cudaSuccess) return BL_ERR_CUDA;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
-  return status == 0u ? BL_OK : BL_ERR_FORMAT;
+  return sync ? i2s_read_status(err, s) : BL_OK;
 }
 
 int bitlinear_i2s_export(const uint32_t* packed, const float* D, int64_t N, int64_t K, int layout, uint8_t* i2s,
                          void* ws, size_t ws_bytes, bl_stream_t stream) {
-  return i2s_impl(true, i2s, packed, D, N, K, layout, ws, ws_bytes, stream);
+  return i2s_impl(true, i2s, packed, D, N, K, layout, ws, ws_bytes, stream, true);
+}
+
+int bitlinear_i2s_export_async(const uint32_t* packed, const float* D, int64_t N, int64_t K, int layout,
+                               uint8_t* i2s, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  return i2s_impl(true, i2s, packed, D, N, K, layout, ws, ws_bytes, stream, false);
 }
 
 int bitlinear_i2s_import(const uint8_t* i2s, int64_t N, int64_t K, int layout, uint32_t* packed, float* D, void* ws,
                          size_t ws_bytes, bl_stream_t stream) {
-  return i2s_impl(false, i2s, packed, D, N, K, layout, ws, ws_bytes, stream);
+  return i2s_impl(false, i2s, packed, D, N, K, layout, ws, ws_bytes, stream, true);
+}
+
+int bitlinear_i2s_import_async(const uint8_t* i2s, int64_t N, int64_t K, int layout, uint32_t* packed, float* D,
+                               void* ws, size_t ws_bytes, bl_stream_t stream) {
+  return i2s_impl(false, i2s, packed, D, N, K, layout, ws, ws_bytes, stream, false);
+}
+
+int bitlinear_i2s_status(void* ws, size_t ws_bytes, bl_stream_t stream) {
+  if (ws == nullptr) return BL_ERR_NULL;
+  if (!aligned256(ws)) return BL_ERR_ALIGN;
+  if (ws_bytes < bl::kHeaderBytes) return BL_ERR_WORKSPACE;
+  return i2s_read_status(static_cast<uint32_t*>(ws), reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

@@ -25,9 +25,9 @@ constexpr int64_t kGemvMaxSmem = 200 * 1024;
 
 // I2_S conversion (bl_i2s.cu): to_i2s packs `in` (BitLinear words, D_in)
 // into I2_S words at `out`; otherwise unpacks I2_S words at `in` into packed
-// words at `out` and D_out. err (a device word) gets bit 0 for a field
-// holding 3 and bit 1 for a scale that is not finite and positive (or rows of
-// D_in that differ).
+// words at `out` and D_out. err (a device word, not cleared here) gets bit 0
+// OR-ed in for a field holding 3 and bit 1 for a scale that is not finite and
+// positive (or rows of D_in that differ).
 cudaError_t launch_i2s(bool to_i2s, bool quarters, const void* in, void* out, const float* D_in, float* D_out,
                        int64_t N, int64_t K, uint32_t* err, cudaStream_t stream, int sms);
 

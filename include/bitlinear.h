@@ -358,6 +358,21 @@ BL_API int bitlinear_i2s_export(const uint32_t* packed, const float* D, int64_t 
 BL_API int bitlinear_i2s_import(const uint8_t* i2s, int64_t N, int64_t K, int layout,
                                 uint32_t* packed, float* D, void* ws, size_t ws_bytes, bl_stream_t stream);
 
+/* Asynchronous forms of the two conversions, for converting many tensors
+ * with one check at the end: same arguments and checks, but nothing is
+ * synchronised and a format error is OR-ed into the status word at the start
+ * of `ws` instead of being returned. The caller zeroes that word before the
+ * first call (a zero-filled workspace); bitlinear_i2s_status reads it. */
+BL_API int bitlinear_i2s_export_async(const uint32_t* packed, const float* D, int64_t N, int64_t K, int layout,
+                                      uint8_t* i2s, void* ws, size_t ws_bytes, bl_stream_t stream);
+BL_API int bitlinear_i2s_import_async(const uint8_t* i2s, int64_t N, int64_t K, int layout,
+                                      uint32_t* packed, float* D, void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the status word of `ws`: BL_OK if
+ * no asynchronous conversion since the last read met a format error, else
+ * BL_ERR_FORMAT. */
+BL_API int bitlinear_i2s_status(void* ws, size_t ws_bytes, bl_stream_t stream);
+
 /* Diagnostic for the failure-detection path. Launches one thread that waits
  * on a shared-memory barrier that nothing ever completes, using the same
  * time-bounded wait as the tensor-core kernel, with a limit of limit_ns

@@ -183,3 +183,13 @@ def test_i2s_sizes_and_validation_before_cuda(L):
     assert L.bitlinear_i2s_import(FAKE, 3, 48, 0, FAKE, FAKE, FAKE + 16, 256, None) == 3
     assert L.bitlinear_i2s_import(FAKE, 3, 48, 0, FAKE, FAKE, FAKE, 8, None) == 4
     assert L.bitlinear_status_string(9) == b"I2_S: field holding 3, bad scale, or rows of D that differ"
+
+
+def test_i2s_async_and_status_validation_before_cuda(L):
+    assert L.bitlinear_i2s_export_async(FAKE, FAKE, 3, 24, 0, FAKE, FAKE, 256, None) == 2
+    assert L.bitlinear_i2s_export_async(FAKE, FAKE, 3, 48, 0, FAKE + 4, FAKE, 256, None) == 3
+    assert L.bitlinear_i2s_import_async(FAKE, 3, 48, 7, FAKE, FAKE, FAKE, 256, None) == 2
+    assert L.bitlinear_i2s_import_async(FAKE, 3, 48, 0, FAKE, FAKE, FAKE, 0, None) == 4
+    assert L.bitlinear_i2s_status(None, 256, None) == 1
+    assert L.bitlinear_i2s_status(FAKE + 16, 256, None) == 3
+    assert L.bitlinear_i2s_status(FAKE, 16, None) == 4

@@ -735,3 +735,26 @@ def test_i2s_rejects_invalid_buffers(B):
     # the context still works, and a good buffer still imports
     packed, D = B.i2s_import(dev(good), N, K)
     assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)
+
+
+def test_i2s_async_conversions_share_one_status_word(B):
+    """Several asynchronous conversions with one status check; a bad buffer
+    among them sets the word, the read clears it."""
+    ws = B.i2s_workspace("cuda")
+    outs = []
+    for i, (N, K) in enumerate([(3, 48), (64, 1152), (5, 4304)]):
+        W = WL.weight(N, K, "normal", 1600 + i)
+        p_ref, D_ref = O.pack_weights(W)
+        for layout in ("consecutive", "quarters"):
+            buf = B.i2s_export(dev(p_ref.view(np.int32)), dev(D_ref), layout, ws=ws, sync=False)
+            outs.append((B.i2s_import(buf, N, K, layout, ws=ws, sync=False), buf, p_ref, D_ref, K, layout))
+    assert B.i2s_status(ws) == 0
+    for (packed, D), buf, p_ref, D_ref, K, layout in outs:
+        assert np.array_equal(buf.cpu().numpy(), O.i2s_export(p_ref, D_ref, K, layout))
+        assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)
+    bad = outs[0][1].clone()
+    bad[0] = 0xFF
+    B.i2s_import(bad, 3, 48, ws=ws, sync=False)
+    B.i2s_import(outs[0][1], 3, 48, ws=ws, sync=False)
+    assert B.i2s_status(ws) == 9
+    assert B.i2s_status(ws) == 0
