@@ -66,6 +66,9 @@ def parse_args(argv=None):
                     help="one layer of a workload, M tokens, for profiler captures (e.g. embed_batch:0:32768)")
     ap.add_argument("--ncu-i2s", action="store_true",
                     help="I2_S export/import only (stacked gate_up weights), for profiler captures")
+    ap.add_argument("--only", default=None, metavar="PARTS",
+                    help="run only these parts (comma-separated: prefill, configs, bf16, rmsnorm, pack, i2s) "
+                         "and print their results; no headline line")
     ap.add_argument("--i2s-layouts", default="consecutive,quarters",
                     help="byte groupings timed by the I2_S part (comma-separated)")
     a = ap.parse_args(argv)
@@ -285,6 +288,43 @@ def run_ours(a):
     i8_sust = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])) * INT8_PER_BF16
     stream = torch.cuda.Stream(device=dev)
 
+    def capture(fn, n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n):
+                fn(i)
+        return g
+
+    def time_graph(g):
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):  # replay() launches on the current stream
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        return e0.elapsed_time(e1)
+
+    if a.only:
+        parts = {
+            "prefill": lambda: bench_prefill(a, B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak,
+                                             i8_burst, i8_sust, rank),
+            "configs": lambda: bench_configs(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak,
+                                             i8_burst, rank),
+            "bf16": lambda: bench_bf16(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, rank),
+            "rmsnorm": lambda: bench_rmsnorm(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak,
+                                             i8_burst),
+            "pack": lambda: bench_pack(B, torch, dev, stream, hbm_peak),
+            "i2s": lambda: bench_i2s(B, torch, dev, stream, hbm_peak, layouts=tuple(a.i2s_layouts.split(","))),
+        }
+        res = {name: parts[name]() for name in a.only.split(",")}
+        if rank == 0:
+            print(json.dumps({"only": res}))
+        return 0
+
     # ---------------------------------------------------------------- decode setup
     wl = WL.WORKLOADS[HEADLINE]
     M = 1
@@ -326,26 +366,6 @@ def run_ours(a):
         r = i % rot
         B.forward_batch([(xs[r][li], packs[r][li][0], packs[r][li][1], ys[r][li]) for li in range(len(layers))],
                         flags=EARLY, ws=wss[3])
-
-    def capture(fn, n):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            for i in range(n):
-                fn(i)
-        return g
-
-    def time_graph(g):
-        barrier()
-        torch.cuda.synchronize(dev)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):  # replay() launches on the current stream
-            e0.record(stream)
-            g.replay()
-            e1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier()
-        return e0.elapsed_time(e1)
 
     # warm-up: eager W steps, then the graph once
     with torch.cuda.stream(stream):
@@ -569,6 +589,15 @@ def load_traffic(kernel):
         return None
 
 
+L2_FLUSH_BYTES = 256 << 20  # twice the 126 MB L2: a rotation through this much traffic evicts it
+
+
+def rotation(bytes_per_call, cap=16):
+    """Copies of a call's buffers to cycle through so that the data one call
+    touches was last touched at least L2_FLUSH_BYTES of traffic earlier."""
+    return int(min(cap, max(2, -(-L2_FLUSH_BYTES // max(1, bytes_per_call)))))
+
+
 def bench_prefill(a, B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, i8_burst, i8_sust, rank):
     wl = WL.WORKLOADS[PREFILL]
     M = PREFILL_M
@@ -584,7 +613,7 @@ def bench_prefill(a, B, torch, dev, stream, capture, time_graph, max_ranks, hbm_
         ys = [torch.empty((M, l.N), dtype=torch.float32, device=dev) for l in layers]
         wss = [torch.zeros(B.workspace_size(M, l.N, l.K), dtype=torch.uint8, device=dev) for l in layers]
     torch.cuda.synchronize(dev)
-    n = max(3, min(a.steps, 30))
+    n = max(16, min(a.steps, 32))
 
     def whole(i):
         for li, l in enumerate(layers):
@@ -607,13 +636,27 @@ def bench_prefill(a, B, torch, dev, stream, capture, time_graph, max_ranks, hbm_
     gemm_ops, gemm_ms = 0, 0.0
     for li, l in enumerate(layers):
         p, D = pk[li]
-        B.prepare_act(xs[li], wss[li])
+        # GEMM inputs (prepared codes in a workspace, packed weights) and outputs
+        # rotate over copies, and so do ActQuant's x and workspace, so that
+        # every call reads its inputs from HBM.
+        rg = rotation(M * l.K + l.N * l.K // 4 + 4 * M * l.N)
+        with torch.cuda.stream(stream):
+            gitems = []
+            for _ in range(rg):
+                wsc = torch.zeros_like(wss[li])
+                B.prepare_act(xs[li], wsc)
+                gitems.append((p.clone(), D.clone(), wsc, torch.empty_like(ys[li])))
+            rq = rotation(5 * M * l.K)
+            qitems = [(xs[li].clone(), torch.zeros_like(wss[li])) for _ in range(rq)]
+        torch.cuda.synchronize(dev)
 
-        def gemm(i, li=li, p=p, D=D, l=l):
-            B.forward_prepared(M, l.K, p, D, wss[li], out=ys[li])
+        def gemm(i, l=l, gitems=gitems):
+            pp, DD, wsc, yy = gitems[i % len(gitems)]
+            B.forward_prepared(M, l.K, pp, DD, wsc, out=yy)
 
-        def quant(i, li=li):
-            B.prepare_act(xs[li], wss[li])
+        def quant(i, qitems=qitems):
+            xx, wsc = qitems[i % len(qitems)]
+            B.prepare_act(xx, wsc)
 
         gg = capture(gemm, n)
         with torch.cuda.stream(stream):
@@ -635,10 +678,12 @@ def bench_prefill(a, B, torch, dev, stream, capture, time_graph, max_ranks, hbm_
             "layer": l.name, "K": l.K, "N": l.N, "gemm_us": round(tg * 1e3, 2), "TOPS": round(tops, 1),
             "frac_int8_peak": round(tops / i8_burst, 4),
             "frac_true_roofline": round(max(t_mem, t_cmp) / (tg * 1e-3), 4),
-            "actquant_us": round(tq * 1e3, 2), "actquant_GBps": round(q_bytes / (tq * 1e-3) / 1e9, 1)})
+            "actquant_us": round(tq * 1e3, 2), "actquant_GBps": round(q_bytes / (tq * 1e-3) / 1e9, 1),
+            "actquant_frac_hbm": round(q_bytes / (tq * 1e-3) / 1e9 / hbm_peak, 4),
+            "l2": f"GEMM rotates over {rg} copies, ActQuant over {rq}"})
         gemm_ops += o
         gemm_ms += tg
-        del gg, gq
+        del gg, gq, gitems, qitems
     tops = gemm_ops / (gemm_ms * 1e-3) / 1e12
     res["roofline"] = {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 kind::i8, TMEM A + TMEM accumulators)",
                        "achieved": round(tops, 1), "peak": round(i8_burst, 1), "unit": "TOPS",
@@ -742,37 +787,44 @@ def bench_bf16(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, 
     M = PREFILL_M
     aq = []
     for K in (2560, 6912):
+        qb = 2 * M * K + M * K + 12 * M
+        r = rotation(qb)
         with torch.cuda.stream(stream):
-            xb = torch.from_numpy(WL.activations(M, K, "normal", 3, layer=K)).to(dev).to(torch.bfloat16)
+            xb0 = torch.from_numpy(WL.activations(M, K, "normal", 3, layer=K)).to(dev).to(torch.bfloat16)
+            xbs = [xb0.clone() for _ in range(r)]
+            del xb0
         torch.cuda.synchronize(dev)
-        g = capture(lambda i, xb=xb: B.quant_act(xb), 20)
+        g = capture(lambda i, xbs=xbs: B.quant_act(xbs[i % len(xbs)]), 32)
         with torch.cuda.stream(stream):
             g.replay()
-        t = max_ranks(time_graph(g)) / 20 * 1e-3
-        qb = 2 * M * K + M * K + 12 * M
+        t = max_ranks(time_graph(g)) / 32 * 1e-3
         aq.append({"M": M, "K": K, "us": round(t * 1e6, 2), "GB/s": round(qb / t / 1e9, 1),
-                   "frac_hbm": round(qb / t / 1e9 / hbm_peak, 4)})
-        del g, xb
+                   "frac_hbm": round(qb / t / 1e9 / hbm_peak, 4), "l2": f"rotates over {r} copies"})
+        del g, xbs
     out["actquant"] = aq
     l = layers[2]
     with torch.cuda.stream(stream):
-        Wb = torch.from_numpy(WL.weight(l.N, l.K, "normal", 5)).to(dev).to(torch.bfloat16)
+        Wb0 = torch.from_numpy(WL.weight(l.N, l.K, "normal", 5)).to(dev).to(torch.bfloat16)
+        Wbs = [Wb0.clone() for _ in range(4)]  # 4 x 71 MB: each call's W was last read 212 MB earlier
+        del Wb0
         ws = torch.zeros(4096, dtype=torch.uint8, device=dev)
-        B.pack_weights(Wb, ws=ws)
+        B.pack_weights(Wbs[0], ws=ws)
         torch.cuda.synchronize(dev)
         ts = []
-        for _ in range(5):
+        for it in range(8):
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            B.pack_weights(Wb, ws=ws)
+            B.pack_weights(Wbs[(it + 1) % len(Wbs)], ws=ws)
             e1.record(stream)
             torch.cuda.synchronize(dev)
             ts.append(e0.elapsed_time(e1))
     t = statistics.median(ts) * 1e-3
     alg = 2 * l.N * l.K + l.N * l.K // 4 + 4 * l.N
     out["pack"] = {"layer": f"gate_up {l.K}->{l.N}", "ms": round(t * 1e3, 4),
-                   "GB/s_algorithmic": round(alg / t / 1e9, 1), "frac_hbm": round(alg / t / 1e9 / hbm_peak, 4)}
+                   "GB/s_algorithmic": round(alg / t / 1e9, 1), "frac_hbm": round(alg / t / 1e9 / hbm_peak, 4),
+                   "l2": "rotates over 4 weight copies"}
+    del Wbs
     torch.cuda.empty_cache()
     return out
 
@@ -783,19 +835,23 @@ def bench_rmsnorm(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_pea
     fused norm on the first C5 layer, against its true roofline."""
     out = {"actquant": []}
     for (M, K) in ((32768, 1024), (32768, 3072), (4096, 2560), (4096, 6912)):
+        nb = 4 * M * K + 4 * K + M * K + 12 * M
+        r = rotation(nb)
         with torch.cuda.stream(stream):
-            x = torch.from_numpy(WL.activations(M, K, "outlier_tokens", 7, layer=K,
-                                                meta={"frac": 0.01, "scale": 20.0, "df": 3.0})).to(dev)
+            x0 = torch.from_numpy(WL.activations(M, K, "outlier_tokens", 7, layer=K,
+                                                 meta={"frac": 0.01, "scale": 20.0, "df": 3.0})).to(dev)
+            xs_r = [x0.clone() for _ in range(r)]
+            del x0
             g = torch.from_numpy(WL.weight(1, K, "normal", 8).reshape(-1) + np.float32(1.0)).to(dev)
         torch.cuda.synchronize(dev)
-        g_ = capture(lambda i, x=x, g=g: B.rmsnorm_quant_act(x, g), 10)
+        nrep = 16
+        g_ = capture(lambda i, xs_r=xs_r, g=g: B.rmsnorm_quant_act(xs_r[i % len(xs_r)], g), nrep)
         with torch.cuda.stream(stream):
             g_.replay()
-        t = max_ranks(time_graph(g_)) / 10 * 1e-3
-        nb = 4 * M * K + 4 * K + M * K + 12 * M
+        t = max_ranks(time_graph(g_)) / nrep * 1e-3
         out["actquant"].append({"M": M, "K": K, "us": round(t * 1e6, 2), "GB/s": round(nb / t / 1e9, 1),
-                                "frac_hbm": round(nb / t / 1e9 / hbm_peak, 4)})
-        del g_, x, g
+                                "frac_hbm": round(nb / t / 1e9 / hbm_peak, 4), "l2": f"rotates over {r} copies"})
+        del g_, xs_r, g
     wl = WL.WORKLOADS["embed_batch"]
     l = wl.layers[2]  # 3072 -> 1024, compute-bound
     M = 32768
@@ -825,16 +881,17 @@ def bench_rmsnorm(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_pea
 def bench_pack(B, torch, dev, stream, hbm_peak):
     l = WL.WORKLOADS[HEADLINE].layers[2]  # gate_up, the largest weight
     with torch.cuda.stream(stream):
-        W = torch.from_numpy(WL.weight(l.N, l.K, "normal", 5)).to(dev)
+        W0 = torch.from_numpy(WL.weight(l.N, l.K, "normal", 5)).to(dev)
+        Ws = [W0, W0.clone()]  # 2 x 142 MB: each call's W was last read 283 MB earlier
         ws = torch.zeros(4096, dtype=torch.uint8, device=dev)
-        B.pack_weights(W, ws=ws)
+        B.pack_weights(Ws[0], ws=ws)
         torch.cuda.synchronize(dev)
         ts = []
-        for _ in range(5):
+        for it in range(6):
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            B.pack_weights(W, ws=ws)
+            B.pack_weights(Ws[(it + 1) % 2], ws=ws)
             e1.record(stream)
             torch.cuda.synchronize(dev)
             ts.append(e0.elapsed_time(e1))
@@ -842,7 +899,8 @@ def bench_pack(B, torch, dev, stream, hbm_peak):
     alg = 4 * l.N * l.K + l.N * l.K // 4 + 4 * l.N
     return {"layer": f"gate_up {l.K}->{l.N}", "ms": round(t, 4), "GB/s_algorithmic": round(alg / (t * 1e-3) / 1e9, 1),
             "frac_hbm": round(alg / (t * 1e-3) / 1e9 / hbm_peak, 4),
-            "note": "two passes over W (exact integer mean, then ternarise+pack); synchronous call"}
+            "note": "two passes over W (exact integer mean, then ternarise+pack); synchronous call; "
+                    "rotates over 2 weight copies"}
 
 
 def bench_i2s(B, torch, dev, stream, hbm_peak, copies=16, reps=10, layouts=("consecutive", "quarters")):

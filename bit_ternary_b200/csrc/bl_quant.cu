@@ -15,6 +15,17 @@
 
 namespace bl {
 
+// int8 activation code clamp(rint(RN(x * s_x)), -128, 127) for a token scale
+// s_x = RN(127 / max(max|x|, floor)) and |x| <= max|x|: then |RN(x * s_x)| is at
+// most 127 * (1 + 2^-23), far below 2^22. In that range adding 1.5 * 2^23
+// rounds to an integer with the fp32 rounding (half to even) and leaves it in
+// the low significand bits: the same value as the conversion instruction,
+// with one FADD and one integer subtract instead.
+__device__ __forceinline__ int quant_code(float x, float s_x) {
+  const int v = __float_as_int(__fadd_rn(__fmul_rn(x, s_x), 12582912.0f)) - 0x4B400000;
+  return v < -128 ? -128 : (v > 127 ? 127 : v);
+}
+
 // ------------------------------------------------------------------ pack --
 constexpr int kBinThreads = 256;
 constexpr int kBinWarps = kBinThreads / 32;
@@ -272,10 +283,10 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const void* __restrict__
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const float4 f = load4<kBf16>(x, xr + 4 * g + j);
-      v[4 * j + 0] = quant_i8(f.x, sx);
-      v[4 * j + 1] = quant_i8(f.y, sx);
-      v[4 * j + 2] = quant_i8(f.z, sx);
-      v[4 * j + 3] = quant_i8(f.w, sx);
+      v[4 * j + 0] = quant_code(f.x, sx);
+      v[4 * j + 1] = quant_code(f.y, sx);
+      v[4 * j + 2] = quant_code(f.z, sx);
+      v[4 * j + 3] = quant_code(f.w, sx);
     }
     uint32_t w4[4];
 #pragma unroll
@@ -332,10 +343,11 @@ __global__ void __launch_bounds__(256) act_quant_reg_kernel(const void* __restri
                                                             int32_t* __restrict__ rowsum_out,
                                                             uint32_t* __restrict__ err_reset) {
   __shared__ float red_f[8];
-  __shared__ int red_i[8];
   if (err_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err_reset = 0u;
   const int64_t m = blockIdx.x;
   const int64_t xr = m * (K >> 2);  // first float4 (group of 4 elements) of the row
+  // Cleared before the block barrier below; the warps add their sums after it.
+  if (rowsum_out != nullptr && threadIdx.x == 0) rowsum_out[m] = 0;
   const int ngroups = (int)(K >> 4);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
@@ -369,10 +381,10 @@ __global__ void __launch_bounds__(256) act_quant_reg_kernel(const void* __restri
     int v[16];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      v[4 * j + 0] = quant_i8(f[i][j].x, sx);
-      v[4 * j + 1] = quant_i8(f[i][j].y, sx);
-      v[4 * j + 2] = quant_i8(f[i][j].z, sx);
-      v[4 * j + 3] = quant_i8(f[i][j].w, sx);
+      v[4 * j + 0] = quant_code(f[i][j].x, sx);
+      v[4 * j + 1] = quant_code(f[i][j].y, sx);
+      v[4 * j + 2] = quant_code(f[i][j].z, sx);
+      v[4 * j + 3] = quant_code(f[i][j].w, sx);
     }
     uint32_t w4[4];
 #pragma unroll
@@ -389,15 +401,11 @@ __global__ void __launch_bounds__(256) act_quant_reg_kernel(const void* __restri
     for (int j = 0; j < 16; ++j) rsum += v[j];
     *reinterpret_cast<uint4*>(qr + 16 * (int64_t)g) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
   }
+  if (threadIdx.x == 0) s_out[m] = sx;
+  if (rowsum_out != nullptr) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) rsum += __shfl_xor_sync(0xFFFFFFFFu, rsum, o);
-  if (lane == 0) red_i[warp] = rsum;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int tot = 0;
-    for (int w = 0; w < nwarps; ++w) tot += red_i[w];
-    s_out[m] = sx;
-    if (rowsum_out != nullptr) rowsum_out[m] = tot;
+    for (int o = 16; o > 0; o >>= 1) rsum += __shfl_xor_sync(0xFFFFFFFFu, rsum, o);
+    if (lane == 0) atomicAdd(rowsum_out + m, rsum);
   }
 }
 
@@ -405,7 +413,9 @@ __global__ void __launch_bounds__(256) act_quant_reg_kernel(const void* __restri
 // Per-projection RMSNorm before ActQuant ("BitNet-Embeddings I2_S guide",
 // section 3.1; rms_norm_eps 1e-6): n = RN(RN(x*r)*g) with
 // r = RN(1/RN(sqrt(RN(ms + eps)))) and ms = mean(x^2) correctly rounded once
-// from the exact sum. One CTA per token, x and g held in registers.
+// from the exact sum. One CTA per token, x and g held in registers; the row
+// sum goes out by one atomic per warp onto a word that thread 0 cleared before
+// the first block barrier.
 //
 // ms: each x^2 is exact in fp64, so the fp64 sum S' of the K squares, in any
 // order, is within gamma_(K-1) = (K-1)u/(1-(K-1)u) of the exact S (u = 2^-53,
@@ -478,7 +488,6 @@ __global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restr
                                                             uint32_t* __restrict__ err_reset) {
   __shared__ double red_d[8];
   __shared__ float red_f[8];
-  __shared__ int red_i[8];
   __shared__ float s_ms;
   __shared__ int s_exact;
   __shared__ unsigned long long bins[kRmsBins];
@@ -488,6 +497,8 @@ __global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restr
   const int ngroups = (int)(K >> 4);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
+  // Cleared before the first block barrier; the warps add their sums at the end.
+  if (rowsum_out != nullptr && threadIdx.x == 0) rowsum_out[m] = 0;
   // g is loaded with x when it fits in registers (kG == 1), so its latency
   // overlaps the load of x instead of following the mean-square barrier.
   constexpr bool kGEarly = kG == 1;
@@ -582,10 +593,10 @@ __global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restr
     int v[16];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      v[4 * j + 0] = quant_i8(f[i][j].x, sx);
-      v[4 * j + 1] = quant_i8(f[i][j].y, sx);
-      v[4 * j + 2] = quant_i8(f[i][j].z, sx);
-      v[4 * j + 3] = quant_i8(f[i][j].w, sx);
+      v[4 * j + 0] = quant_code(f[i][j].x, sx);
+      v[4 * j + 1] = quant_code(f[i][j].y, sx);
+      v[4 * j + 2] = quant_code(f[i][j].z, sx);
+      v[4 * j + 3] = quant_code(f[i][j].w, sx);
     }
     uint32_t w4[4];
 #pragma unroll
@@ -602,15 +613,11 @@ __global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restr
     for (int j = 0; j < 16; ++j) rsum += v[j];
     *reinterpret_cast<uint4*>(qr + 16 * (int64_t)gi) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
   }
+  if (threadIdx.x == 0) s_out[m] = sx;
+  if (rowsum_out != nullptr) {
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) rsum += __shfl_xor_sync(0xFFFFFFFFu, rsum, o);
-  if (lane == 0) red_i[warp] = rsum;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int tot = 0;
-    for (int w = 0; w < nwarps; ++w) tot += red_i[w];
-    s_out[m] = sx;
-    if (rowsum_out != nullptr) rowsum_out[m] = tot;
+    for (int o = 16; o > 0; o >>= 1) rsum += __shfl_xor_sync(0xFFFFFFFFu, rsum, o);
+    if (lane == 0) atomicAdd(rowsum_out + m, rsum);
   }
 }
 
