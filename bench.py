@@ -67,7 +67,8 @@ def parse_args(argv=None):
     ap.add_argument("--ncu-i2s", action="store_true",
                     help="I2_S export/import only (stacked gate_up weights), for profiler captures")
     ap.add_argument("--only", default=None, metavar="PARTS",
-                    help="run only these parts (comma-separated: prefill, configs, bf16, rmsnorm, pack, i2s) "
+                    help="run only these parts (comma-separated: prefill, configs, bf16, rmsnorm, pack, "
+                         "decode_stream, i2s) "
                          "and print their results; no headline line")
     ap.add_argument("--i2s-layouts", default="consecutive,quarters",
                     help="byte groupings timed by the I2_S part (comma-separated)")
@@ -318,6 +319,8 @@ def run_ours(a):
             "rmsnorm": lambda: bench_rmsnorm(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak,
                                              i8_burst),
             "pack": lambda: bench_pack(B, torch, dev, stream, hbm_peak),
+            "decode_stream": lambda: bench_decode_stream(B, torch, dev, stream, capture, time_graph, max_ranks,
+                                                         hbm_peak),
             "i2s": lambda: bench_i2s(B, torch, dev, stream, hbm_peak, layouts=tuple(a.i2s_layouts.split(","))),
         }
         res = {name: parts[name]() for name in a.only.split(",")}
@@ -531,8 +534,9 @@ def run_ours(a):
         configs = bench_configs(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, i8_burst, rank)
 
     # --------------------------------------------------------------------- pack
-    pack = i2s = None
+    pack = i2s = dstream = None
     if not a.ncu_small:
+        dstream = bench_decode_stream(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak)
         pack = bench_pack(B, torch, dev, stream, hbm_peak)
         i2s = bench_i2s(B, torch, dev, stream, hbm_peak, layouts=tuple(a.i2s_layouts.split(",")))
 
@@ -587,6 +591,7 @@ def run_ours(a):
         "clocks": clk,
         "prefill": prefill,
         "configs": configs,
+        "decode_streaming": dstream,
         "pack": pack,
         "i2s": i2s,
         "bf16_inputs": bf16,
@@ -900,6 +905,40 @@ def bench_rmsnorm(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_pea
                       "TOPS": round(ops / t / 1e12, 1),
                       "frac_true_roofline": round(max(nb / (hbm_peak * 1e9), ops / (i8_burst * 1e12)) / t, 4)}
     del gg, x, y, ws
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_decode_stream(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, copies=16):
+    """The decode kernel's streaming ceiling: one call over `copies` stacked
+    gate_up weights (2560 -> 13824 x copies, 141 MB packed), so launch and
+    dependency latency are small against the weight stream. Two weight copies
+    alternate, so every call reads its weights from HBM."""
+    l = WL.WORKLOADS[HEADLINE].layers[2]
+    with torch.cuda.stream(stream):
+        W = torch.from_numpy(WL.weight(l.N, l.K, "normal", 11)).to(dev)
+        p1, D1 = B.pack_weights(W)
+        del W
+        items = [(p1.repeat(copies, 1).contiguous(), D1.repeat(copies, 1).contiguous()) for _ in range(2)]
+        del p1, D1
+    N, K = items[0][0].shape[0], l.K
+    out = {"weights": f"{copies} x gate_up stacked: [{N}, {K}], {N * K // 4 / 1e6:.1f} MB packed", "cases": []}
+    for M in (1, 8):
+        with torch.cuda.stream(stream):
+            x = torch.from_numpy(WL.activations(M, K, "normal", 12)).to(dev)
+            y = torch.empty((M, N), dtype=torch.float32, device=dev)
+            ws = torch.zeros(max(256, B.workspace_size(M, N, K)), dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize(dev)
+        nrep = 20
+        g = capture(lambda i, x=x, y=y, ws=ws: B.forward(x, items[i % 2][0], items[i % 2][1], out=y, ws=ws), nrep)
+        with torch.cuda.stream(stream):
+            g.replay()
+        t = max_ranks(time_graph(g)) / nrep * 1e-3
+        nb = N * K // 4 + 4 * N + 4 * M * K + 4 * M * N
+        out["cases"].append({"M": M, "us": round(t * 1e6, 2), "GB/s": round(nb / t / 1e9, 1),
+                             "frac_hbm": round(nb / t / 1e9 / hbm_peak, 4)})
+        del g, x, y, ws
+    del items
     torch.cuda.empty_cache()
     return out
 

@@ -758,3 +758,19 @@ def test_i2s_async_conversions_share_one_status_word(B):
     B.i2s_import(outs[0][1], 3, 48, ws=ws, sync=False)
     assert B.i2s_status(ws) == 9
     assert B.i2s_status(ws) == 0
+
+
+@pytest.mark.parametrize("M", [1, 3])
+def test_decode_stacked_weights_stream(B, M):
+    """The decode kernel over 16 stacked copies of the gate_up weight (221184
+    rows, the streaming measurement's shape): every block of 13824 rows equals
+    the oracle's output for one copy, bit for bit."""
+    W = WL.weight(13824, 2560, "normal", 1700)
+    x = WL.activations(M, 2560, "normal", 1701)
+    p_ref, D_ref = O.pack_weights(W)
+    ref = O.bitlinear_forward(x, p_ref, D_ref, 2560)
+    packed = dev(p_ref.view(np.int32)).repeat(16, 1).contiguous()
+    D = dev(D_ref).repeat(16, 1).contiguous()
+    y = B.forward(dev(x), packed, D)
+    torch.cuda.synchronize()
+    assert_y_close(y.cpu().numpy(), np.tile(ref, (1, 16)))
