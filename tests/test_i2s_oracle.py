@@ -202,3 +202,19 @@ def test_planted_twos_complement_codes_are_caught(monkeypatch, golden_dir):
     monkeypatch.setattr(O, "i2s_encode_codes", twos_complement)
     with pytest.raises(AssertionError):
         test_golden_hand_block(golden_dir, "consecutive")
+
+
+def test_round_trip_property_random_shapes():
+    """Random shapes (K % 16 == 0, any N, tails of every length mod 128) and
+    random codes: decode(encode(c)) == c in both groupings, and the encoded
+    bytes agree with the bit-string construction."""
+    rng = np.random.default_rng(20261202)
+    for _ in range(60):
+        N = int(rng.integers(1, 9))
+        K = 16 * int(rng.integers(1, 40))
+        codes = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+        for layout in O.I2S_LAYOUTS:
+            blocks = O.i2s_encode_codes(codes, layout)
+            assert blocks.size == 32 * (-(-(N * K) // 128))
+            assert np.array_equal(O.i2s_decode_codes(blocks, N * K, layout), codes.reshape(-1))
+            assert np.array_equal(blocks, _bitstring_encode(codes, layout))
