@@ -105,6 +105,8 @@ def test_batch_validation_before_cuda(L):
     assert L.bitlinear_forward_batch(calls, 2, 0, FAKE, 1 << 20, None) == 1
     calls[1] = _lib.LinearCall(FAKE, 1, 8, 64, FAKE, FAKE, FAKE)
     assert L.bitlinear_forward_batch(calls, 2, 0x80, FAKE, 1 << 20, None) == 2  # unknown flag
+    assert L.bitlinear_forward_batch(calls, 2, 0x4, FAKE, 1 << 20, None) == 2  # first undefined bit
+    assert _lib.BL_FLAG_STREAM_WEIGHTS_EARLY == 1 and _lib.BL_FLAG_ONE_LAUNCH_PER_CALL == 2
     assert L.bitlinear_forward_batch(calls, 0, 0, None, 0, None) == 0
     assert L.bitlinear_batch_workspace_size(calls, 2) == 256 + 256 + 256 + 256  # header, s_x, sums, q
 
