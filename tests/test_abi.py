@@ -195,3 +195,15 @@ def test_i2s_async_and_status_validation_before_cuda(L):
     assert L.bitlinear_i2s_status(None, 256, None) == 1
     assert L.bitlinear_i2s_status(FAKE + 16, 256, None) == 3
     assert L.bitlinear_i2s_status(FAKE, 16, None) == 4
+
+
+def test_python_constants_match_header_defines():
+    with open(os.path.join(ROOT, "include", "bitlinear.h")) as f:
+        text = f.read()
+    defines = {k: int(v) for k, v in re.findall(r"#define\s+(BL_\w+)\s+(\d+)u?\b", text)}
+    for name in ("BL_FLAG_STREAM_WEIGHTS_EARLY", "BL_FLAG_ONE_LAUNCH_PER_CALL", "BL_I2S_CONSECUTIVE",
+                 "BL_I2S_QUARTERS"):
+        assert getattr(_lib, name) == defines[name], name
+    statuses = dict((k, int(v)) for k, v in re.findall(r"(BL_(?:OK|ERR_\w+))\s*=\s*(\d+)", text))
+    for code, name in _lib.STATUS_NAMES.items():
+        assert statuses[name] == code, name
