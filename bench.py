@@ -559,7 +559,7 @@ def run_ours(a):
         dist.destroy_process_group()
     if rank != 0:
         return 0
-    traffic = load_traffic("gemv_kernel")
+    traffic = load_traffic("bl_ternary_decode_kernel")
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True, "scaling": "weak",
@@ -573,7 +573,7 @@ def run_ours(a):
                          f"({rot * sum(l.N * l.K // 4 for l in layers) / 1e6:.0f} MB)",
                    "parallelism": f"replica per GPU x{world} (independent decode streams)",
                    "graph": "CUDA graph of the timed steps"},
-        "roofline": {"bound": "hbm", "kernel": "gemv_kernel (fused ActQuant + packed GEMV + rescale)",
+        "roofline": {"bound": "hbm", "kernel": "bl_ternary_decode_kernel (fused ActQuant + packed-weight ring + int8 MMA + rescale)",
                      "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(achieved / hbm_peak, 4), "traffic": traffic,
                      "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured" else

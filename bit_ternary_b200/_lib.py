@@ -33,6 +33,7 @@ _I64 = ctypes.c_int64
 _SZ = ctypes.c_size_t
 SIGNATURES = {
     "bitlinear_abi_version": (ctypes.c_int, []),
+    "bitlinear_build_id": (ctypes.c_char_p, []),
     "bitlinear_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "bitlinear_device_check": (ctypes.c_int, []),
     "bitlinear_pack_workspace_size": (_SZ, [_I64, _I64]),
@@ -71,6 +72,8 @@ SIGNATURES = {
     "bitlinear_workspace_error": (ctypes.c_int, [_VP, _SZ, _VP]),
     "bitlinear_selftest_wait_timeout": (ctypes.c_int, [_VP, _SZ, ctypes.c_uint64, _VP]),
     "bitlinear_forward_noalloc": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP]),
+    "bitlinear_noalloc_error": (ctypes.c_int, [_VP]),
+    "bitlinear_noalloc_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint64, _VP]),
 }
 
 _lock = threading.Lock()
@@ -117,6 +120,13 @@ def lib() -> ctypes.CDLL:
                 f = getattr(L, name)
                 f.restype = res
                 f.argtypes = args
+            from . import build
+
+            built = L.bitlinear_build_id().decode()
+            if built != build.sources_sha():
+                raise RuntimeError(
+                    f"{LIB_PATH} was built from other sources (build id {built}, sources "
+                    f"{build.sources_sha()}): rebuild it with `python -m bit_ternary_b200.build --force`")
             _lib = L
     return _lib
 

@@ -60,7 +60,7 @@ def sources_sha() -> str:
 
 
 KERNEL_SOURCES = {
-    "gemv_kernel": ["bl_gemv.cu", "bl_device.cuh"],
+    "bl_ternary_decode_kernel": ["bl_decode.cu", "bl_device.cuh"],
     "gemm_kernel": ["bl_gemm.cu", "bl_device.cuh"],
 }
 
@@ -78,18 +78,27 @@ def kernel_sha(kernel: str) -> str:
     return h.hexdigest()[:16]
 
 
+ID_PATH = LIB_PATH + ".id"  # sources_sha() of the sources the library was built from
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB_PATH):
+    """True when the library exists and was built from the current sources
+    (compared by content hash, not by file times)."""
+    if not (os.path.exists(LIB_PATH) and os.path.exists(ID_PATH)):
         return False
-    t = os.path.getmtime(LIB_PATH)
-    return all(os.path.getmtime(f) <= t for f in _inputs())
+    with open(ID_PATH) as f:
+        return f.read().strip() == sources_sha()
 
 
 def build_library(force: bool = False, verbose: bool = False) -> str:
-    """Compile every .cu under csrc/ into libbitlinear.so. Returns the path."""
+    """Compile every .cu under csrc/ into libbitlinear.so. Returns the path.
+    The sources' hash is compiled in (bitlinear_build_id) and recorded beside
+    the library, so a library built from other sources is rebuilt here and
+    refused by the loader."""
     if not force and up_to_date():
         return LIB_PATH
-    cmd = [_nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, f"-I{INCLUDE}", f"-I{CSRC}"]
+    sha = sources_sha()
+    cmd = [_nvcc(), *ARCH_FLAGS, *NVCC_FLAGS, f"-I{INCLUDE}", f"-I{CSRC}", f'-DBL_BUILD_ID="{sha}"']
     if verbose:
         cmd += ["-Xptxas", "-v"]
     tmp = LIB_PATH + ".tmp"
@@ -100,6 +109,8 @@ def build_library(force: bool = False, verbose: bool = False) -> str:
     if verbose:
         sys.stderr.write(res.stdout + res.stderr)
     os.replace(tmp, LIB_PATH)
+    with open(ID_PATH, "w") as f:
+        f.write(sha + "\n")
     return LIB_PATH
 
 

@@ -1,6 +1,6 @@
 // bl_api.cu - the extern "C" entry points of libbitlinear (see include/bitlinear.h).
 // Host-side validation and dispatch only; all arithmetic of the path runs in
-// the kernels of bl_quant.cu, bl_gemv.cu and bl_gemm.cu.
+// the kernels of bl_quant.cu, bl_decode.cu, bl_gemm.cu and bl_i2s.cu.
 #include "bitlinear.h"
 #include "bl_internal.h"
 
@@ -11,6 +11,10 @@
 namespace {
 
 constexpr int kAbiVersion = 1;
+
+#ifndef BL_BUILD_ID
+#define BL_BUILD_ID "unknown"
+#endif
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool aligned256(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
@@ -64,9 +68,10 @@ int forward_impl(const void* x, bool bf16, int64_t M, int64_t N, int64_t K, cons
   if (sms <= 0) return BL_ERR_CUDA;
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint32_t* err = reinterpret_cast<uint32_t*>(base);
-  if (bl::gemv_group_fits(M, K)) {
-    const bl::GemvCall call{x, packed, D, y, acc, M, N, K, bf16};
-    return cuda_status(bl::launch_gemv_group(&call, 1, err, false, stream, sms));
+  if (bl::decode_fits(M, K, false)) {
+    const bl::DecCall call{x, nullptr, nullptr, packed, D, y, acc, M, N, K};
+    return cuda_status(
+        bl::launch_decode(&call, 1, bf16 ? bl::kDecBf16 : bl::kDecF32, nullptr, 0.0f, err, false, stream, sms));
   }
   cudaError_t e = bl::launch_act_quant(x, bf16, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
                                        reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
@@ -75,11 +80,29 @@ int forward_impl(const void* x, bool bf16, int64_t M, int64_t N, int64_t K, cons
   return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, acc, ws, stream, sms));
 }
 
+// Contraction + rescale from prepared activations in the forward workspace
+// (private-order codes, s_x, row sums): the decode kernel for M <= 16 when it
+// fits, the tensor-core kernel otherwise.
+int prepared_contraction(int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D, float* y, void* ws,
+                         cudaStream_t stream, int sms) {
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  if (bl::decode_fits(M, K, false)) {
+    const bl::DecCall call{base + bl::ws_q_off(M), reinterpret_cast<const float*>(base + bl::ws_sx_off(M)),
+                           reinterpret_cast<const int32_t*>(base + bl::ws_rowsum_off(M)), packed, D, y, nullptr,
+                           M, N, K};
+    return cuda_status(bl::launch_decode(&call, 1, bl::kDecPrepared, nullptr, 0.0f, reinterpret_cast<uint32_t*>(base),
+                                         false, stream, sms));
+  }
+  return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, nullptr, ws, stream, sms));
+}
+
 }  // namespace
 
 extern "C" {
 
 int bitlinear_abi_version(void) { return kAbiVersion; }
+
+const char* bitlinear_build_id(void) { return BL_BUILD_ID; }
 
 const char* bitlinear_status_string(int status) {
   switch (status) {
@@ -218,7 +241,7 @@ int bitlinear_forward_prepared(int64_t M, int64_t N, int64_t K, const uint32_t* 
   if (ws_bytes < bl::ws_forward_bytes(M, K)) return BL_ERR_WORKSPACE;
   const int sms = num_sms_current();
   if (sms <= 0) return BL_ERR_CUDA;
-  return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, nullptr, ws, reinterpret_cast<cudaStream_t>(stream), sms));
+  return prepared_contraction(M, N, K, packed, D, y, ws, reinterpret_cast<cudaStream_t>(stream), sms);
 }
 
 int bitlinear_forward_q(const int8_t* q, const float* s_x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
@@ -241,7 +264,7 @@ int bitlinear_forward_q(const int8_t* q, const float* s_x, int64_t M, int64_t N,
                                         reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), s,
                                         reinterpret_cast<uint32_t*>(base)));
   if (st != BL_OK) return st;
-  return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, nullptr, ws, s, sms));
+  return prepared_contraction(M, N, K, packed, D, y, ws, s, sms);
 }
 
 int bitlinear_rmsnorm_quant_act(const float* x, const float* g, float eps, int64_t M, int64_t K, int8_t* q,
@@ -278,6 +301,12 @@ int bitlinear_forward_rmsnorm(const float* x, const float* g, float eps, int64_t
   if (sms <= 0) return BL_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
+  if (bl::decode_fits(M, K, true)) {
+    // Decode sizes: the norm and the quantiser run inside the decode kernel.
+    const bl::DecCall call{x, nullptr, nullptr, packed, D, y, nullptr, M, N, K};
+    return cuda_status(
+        bl::launch_decode(&call, 1, bl::kDecRms, g, eps, reinterpret_cast<uint32_t*>(base), false, s, sms));
+  }
   st = cuda_status(bl::launch_rms_act_quant(x, g, eps, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
                                             reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
                                             reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), true, s,
@@ -320,31 +349,33 @@ int bitlinear_forward_batch(const bl_linear_call* calls, int count, uint32_t fla
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint32_t* err = static_cast<uint32_t*>(ws);
   const bool early = (flags & BL_FLAG_STREAM_WEIGHTS_EARLY) != 0;
-  const int max_group = (flags & BL_FLAG_ONE_LAUNCH_PER_CALL) ? 1 : bl::kGemvMaxGroup;
+  const int max_group = (flags & BL_FLAG_ONE_LAUNCH_PER_CALL) ? 1 : bl::kDecodeMaxGroup;
   // Decode-sized calls are grouped, in order, into launches of up to
   // max_group; every other call runs on its own.
-  bl::GemvCall group[bl::kGemvMaxGroup];
+  bl::DecCall group[bl::kDecodeMaxGroup];
   int ng = 0;
-  int64_t gM = 0, gK = 0;
   auto flush = [&]() -> int {
     if (ng == 0) return BL_OK;
-    const cudaError_t e = bl::launch_gemv_group(group, ng, err, early, s, sms);
+    const cudaError_t e = bl::launch_decode(group, ng, bl::kDecF32, nullptr, 0.0f, err, early, s, sms);
     ng = 0;
-    gM = gK = 0;
     return cuda_status(e);
   };
   for (int i = 0; i < count; ++i) {
     const bl_linear_call& c = calls[i];
     if (c.M == 0 || c.N == 0) continue;
-    const int64_t nM = c.M > gM ? c.M : gM, nK = c.K > gK ? c.K : gK;
-    if (bl::gemv_group_fits(c.M, c.K)) {
-      if (ng == max_group || !bl::gemv_group_fits(nM, nK)) {
+    const bl::DecCall dc{c.x, nullptr, nullptr, c.packed, c.D, c.y, nullptr, c.M, c.N, c.K};
+    if (bl::decode_group_fits(&dc, 1)) {
+      if (ng == max_group) {
         const int st = flush();
         if (st != BL_OK) return st;
       }
-      group[ng++] = bl::GemvCall{c.x, c.packed, c.D, c.y, nullptr, c.M, c.N, c.K, false};
-      gM = c.M > gM ? c.M : gM;
-      gK = c.K > gK ? c.K : gK;
+      group[ng] = dc;
+      if (!bl::decode_group_fits(group, ng + 1)) {
+        const int st = flush();
+        if (st != BL_OK) return st;
+        group[0] = dc;
+      }
+      ++ng;
       continue;
     }
     int st = flush();

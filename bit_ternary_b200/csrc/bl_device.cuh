@@ -275,6 +275,91 @@ __device__ __forceinline__ int quant_i8(float x, float s_x) {
   return v < -128 ? -128 : (v > 127 ? 127 : v);
 }
 
+// int8 activation code clamp(rint(RN(x * s_x)), -128, 127) for a token scale
+// s_x = RN(127 / max(max|x|, floor)) and |x| <= max|x|: then |RN(x * s_x)| is at
+// most 127 * (1 + 2^-23), far below 2^22. In that range adding 1.5 * 2^23
+// rounds to an integer with the fp32 rounding (half to even) and leaves it in
+// the low significand bits: the same value as the conversion instruction,
+// with one FADD and one integer subtract instead.
+__device__ __forceinline__ int quant_code(float x, float s_x) {
+  const int v = __float_as_int(__fadd_rn(__fmul_rn(x, s_x), 12582912.0f)) - 0x4B400000;
+  return v < -128 ? -128 : (v > 127 ? 127 : v);
+}
+
+// ------------------------------------------------------- exact mean square
+// Bins of the exact sum of squares of fp32 values, used by the RMSNorm
+// quantisers when the fp64 sum cannot decide the fp32 rounding of mean(x^2):
+constexpr int kRmsBins = 544;  // x^2 = m^2 * 2^(2(ee-1)) units of 2^-298; m^2 split in 24-bit halves
+
+// Correctly rounded fp32 of (sum_b bins[b] * 2^b) / K * 2^-298, by long
+// division on 32-bit limbs (one thread). bins[b] < 2^41.
+static __device__ __noinline__ float mean_square_exact_f32(const unsigned long long* bins, uint32_t K) {
+  constexpr int L = 19;  // 608 bits: bins below 2^41 at shifts < 544
+  uint32_t S[L];
+  for (int i = 0; i < L; ++i) S[i] = 0u;
+  for (int b = 0; b < kRmsBins; ++b) {
+    const unsigned long long v = bins[b];
+    if (v == 0ull) continue;
+    const int limb = b >> 5, bit = b & 31;
+    uint32_t parts[3];
+    parts[0] = (uint32_t)(v << bit);
+    parts[1] = bit == 0 ? (uint32_t)(v >> 32) : (uint32_t)(v >> (32 - bit));
+    parts[2] = bit == 0 ? 0u : (uint32_t)((v >> 32) >> (32 - bit));
+    unsigned long long carry = 0ull;
+    for (int i = limb; i < L; ++i) {
+      const unsigned long long add = (i - limb < 3 ? parts[i - limb] : 0u);
+      const unsigned long long t = (unsigned long long)S[i] + add + carry;
+      S[i] = (uint32_t)t;
+      carry = t >> 32;
+      if (i - limb >= 2 && carry == 0ull) break;
+    }
+  }
+  // Q = floor(S / K), remainder r (K < 2^18, so r * 2^32 + limb fits 64 bits).
+  uint32_t Q[L];
+  unsigned long long r = 0ull;
+  for (int i = L - 1; i >= 0; --i) {
+    const unsigned long long cur = (r << 32) | S[i];
+    Q[i] = (uint32_t)(cur / K);
+    r = cur % K;
+  }
+  int lead = -1;
+  for (int i = L - 1; i >= 0 && lead < 0; --i)
+    if (Q[i]) lead = 32 * i + 31 - __clz(Q[i]);
+  if (lead < 0) return 0.0f;  // below 2^-298: rounds to zero
+  auto qbit = [&](int i) -> uint32_t { return (Q[i >> 5] >> (i & 31)) & 1u; };
+  const int E = lead - 298;                    // value = 1.xxx * 2^E
+  const int qe = E - 23 > -149 ? E - 23 : -149;  // exponent of the last significand bit
+  const int p = qe + 298;                      // its bit position in Q (>= 149)
+  uint32_t sig = 0u;
+  for (int i = lead; i >= p; --i) sig = (sig << 1) | qbit(i);
+  const uint32_t round_bit = qbit(p - 1);
+  uint32_t sticky = r != 0ull ? 1u : 0u;
+  for (int i = p - 2; i >= 0 && !sticky; --i) sticky |= qbit(i);
+  if (round_bit && (sticky || (sig & 1u))) ++sig;
+  // sig * 2^qe: subnormal when qe == -149 and sig < 2^23; a carry to 2^24 moves up one binade.
+  if (qe == -149 && sig < (1u << 23)) return __uint_as_float(sig);
+  int e2 = qe + 23;
+  if (sig == (1u << 24)) {
+    sig >>= 1;
+    ++e2;
+  }
+  return __uint_as_float(((uint32_t)(e2 + 127) << 23) | (sig & 0x7FFFFFu));
+}
+
+// Adds x^2 to the bins, exactly: |x| = m * 2^(ee-1) units of 2^-149 (ee the
+// biased exponent, at least 1), so x^2 = m^2 * 2^(2(ee-1)) units of 2^-298,
+// and m^2 < 2^48 goes in as two 24-bit halves.
+__device__ __forceinline__ void rms_bins_add(unsigned long long* bins, float x) {
+  const uint32_t b = __float_as_uint(x) & 0x7FFFFFFFu;
+  const uint32_t e = b >> 23;
+  const unsigned long long mm = (b & 0x7FFFFFu) | (e != 0 ? 0x800000u : 0u);
+  if (mm == 0ull) return;
+  const int sh = 2 * ((int)(e > 1 ? e : 1) - 1);
+  const unsigned long long sq = mm * mm;
+  atomicAdd(&bins[sh], sq & 0xFFFFFFull);
+  atomicAdd(&bins[sh + 24], sq >> 24);
+}
+
 // The 4x4 byte transpose used for the kernel-private activation order: inside
 // every group of 16 columns, position 4*c + b holds column 4*b + c. This is
 // the order in which `(word >> 2c) & 0x03030303` presents the codes of a

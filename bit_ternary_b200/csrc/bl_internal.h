@@ -16,12 +16,14 @@ constexpr int kPackBins = 320;
 constexpr int kPackNonFiniteBin = kPackBins - 1;
 constexpr size_t kPackWsBytes = kHeaderBytes + kPackBins * sizeof(unsigned long long);
 
-// Decode path (fused quantise + GEMV): at most 16 tokens, and the quantised
-// activations plus two ring stages of packed weights must fit in shared memory.
-constexpr int64_t kGemvMaxM = 16;
-constexpr int kGemvMaxGroup = 8;                   // BitLinears per grouped launch
-constexpr int64_t kGemvSmemTarget = 100 * 1024;    // leaves room for a CTA of the next launch
-constexpr int64_t kGemvMaxSmem = 200 * 1024;
+// Decode path (bl_decode.cu): at most 16 tokens per BitLinear, up to 8
+// BitLinears per launch; their activation codes and a ring of at least two
+// 16-row weight tiles must fit in shared memory.
+constexpr int64_t kDecodeMaxM = 16;
+constexpr int kDecodeMaxGroup = 8;                     // BitLinears per grouped launch
+constexpr int kDecodeSlots = 16;                       // weight tiles tracked per CTA
+constexpr int64_t kDecodeSmemShared = 110 * 1024;   // two CTAs per SM (room for the next launch)
+constexpr int64_t kDecodeSmemMax = 225 * 1024;      // one CTA per SM
 
 // I2_S conversion (bl_i2s.cu): to_i2s packs `in` (BitLinear words, D_in)
 // into I2_S words at `out`; otherwise unpacks I2_S words at `in` into packed
@@ -31,25 +33,33 @@ constexpr int64_t kGemvMaxSmem = 200 * 1024;
 cudaError_t launch_i2s(bool to_i2s, bool quarters, const void* in, void* out, const float* D_in, float* D_out,
                        int64_t N, int64_t K, uint32_t* err, cudaStream_t stream, int sms);
 
-inline int64_t gemv_q_stride(int64_t K) { return ((K + 255) / 256) * 256 + 16; }
-
-struct GemvCall {
-  const void* x;   // fp32 [M, K], or bf16 bit patterns when bf16
+// One decode BitLinear. x: fp32 [M,K], bf16 bit patterns, or (prepared
+// input) int8 codes in the forward workspace's private order with s_x (sx)
+// and row sums (rs). y fp32 [M,N], or acc int32 [M,N] when acc is non-null.
+struct DecCall {
+  const void* x;
+  const float* sx;
+  const int32_t* rs;
   const uint32_t* packed;
   const float* D;
-  float* y;        // fp32 output, or
-  int32_t* acc;    // int32 accumulators (when non-null)
+  float* y;
+  int32_t* acc;
   int64_t M, N, K;
-  bool bf16;
 };
 
-int64_t gemv_stage_bytes(int64_t K);
-bool gemv_group_fits(int64_t maxM, int64_t maxK);
-// One launch over up to kGemvMaxGroup independent calls (all y or all acc).
-// pdl: launch with programmatic stream serialization (weights may be read
-// before the previous kernel in the stream has finished).
-cudaError_t launch_gemv_group(const GemvCall* calls, int n, uint32_t* err, bool pdl, cudaStream_t stream,
-                              int num_sms);
+enum DecInput : int { kDecF32 = 0, kDecBf16 = 1, kDecPrepared = 2, kDecRms = 3 };
+
+// Whether one call of M tokens and K columns (rms: with the RMSNorm input
+// mode) fits the decode kernel, and whether a group of calls fits one launch.
+bool decode_fits(int64_t M, int64_t K, bool rms);
+bool decode_group_fits(const DecCall* calls, int n);
+// One launch over n calls (all y or all acc). input: a DecInput; prepared and
+// RMSNorm inputs take one call (g: norm weight [K], eps). pdl: launch with
+// programmatic stream serialization (the packed weights and D may be read
+// before the previous kernel in the stream has finished; activations are read
+// after it). err: the workspace error word, cleared by the launch.
+cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g, float eps, uint32_t* err, bool pdl,
+                          cudaStream_t stream, int num_sms);
 
 // W is fp32, or bf16 bit patterns when bf16 (widened exactly).
 cudaError_t launch_pack(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,

@@ -16,40 +16,38 @@
 namespace {
 
 // The scratch: one copy per GPU that loads this library, held until the
-// process exits. It is laid out like the workspace of bitlinear_forward.
+// process exits. It is laid out like the workspace of bitlinear_forward; its
+// first word is the device error word of the calls that use it.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[BITLINEAR_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
 
-struct ScratchSlot {
-  std::once_flag once;
-  void* ptr = nullptr;
-  cudaError_t err = cudaSuccess;
-};
-
-ScratchSlot g_slots[kMaxDevices];
+std::mutex g_lookup_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of g_noalloc_scratch on the current device. In host code the
-// symbol's name is only a host-side stand-in, never a device address, so it
-// is looked up once per device (with that device current) and cached.
+// symbol's name is only a host-side stand-in, never a device address, so the
+// address is looked up with that device current and cached. Only a successful
+// lookup is cached: after a failure (for example a first call made during
+// stream capture) the runtime's error is cleared and the next call tries again.
 void* scratch_on_current_device(int* status) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
     *status = BL_ERR_CUDA;
     return nullptr;
   }
-  ScratchSlot& slot = g_slots[dev];
-  std::call_once(slot.once, [&slot] {
+  std::lock_guard<std::mutex> lock(g_lookup_mutex);
+  if (g_scratch_ptr[dev] == nullptr) {
     void* p = nullptr;
-    slot.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    slot.ptr = (slot.err == cudaSuccess) ? p : nullptr;
-  });
-  if (slot.err != cudaSuccess || slot.ptr == nullptr) {
-    *status = BL_ERR_CUDA;
-    return nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      (void)cudaGetLastError();
+      *status = BL_ERR_CUDA;
+      return nullptr;
+    }
+    g_scratch_ptr[dev] = p;
   }
   *status = BL_OK;
-  return slot.ptr;
+  return g_scratch_ptr[dev];
 }
 
 }  // namespace
@@ -67,4 +65,18 @@ extern "C" int bitlinear_forward_noalloc(const float* x, int64_t M, int64_t N, i
   // forward clears the error word, and the quantised activations, scales
   // and row sums are written in full before they are read.
   return bitlinear_forward(x, M, N, K, packed, D, y, scratch, (size_t)BITLINEAR_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" int bitlinear_noalloc_error(bl_stream_t stream) {
+  int st = BL_OK;
+  void* scratch = scratch_on_current_device(&st);
+  if (st != BL_OK) return st;
+  return bitlinear_workspace_error(scratch, (size_t)BITLINEAR_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+extern "C" int bitlinear_noalloc_selftest_wait_timeout(uint64_t limit_ns, bl_stream_t stream) {
+  int st = BL_OK;
+  void* scratch = scratch_on_current_device(&st);
+  if (st != BL_OK) return st;
+  return bitlinear_selftest_wait_timeout(scratch, (size_t)BITLINEAR_NOALLOC_SCRATCH_BYTES, limit_ns, stream);
 }

@@ -29,8 +29,11 @@
  *
  * Conventions for every entry point:
  *   - All pointers named "device" are device pointers on the current CUDA
- *     device; the caller owns every buffer (this library allocates nothing and
- *     keeps no state beyond cached device attributes).
+ *     device; the caller owns every buffer. This library allocates nothing and
+ *     keeps no state beyond cached device attributes, with one exception: the
+ *     fixed scratch array of bitlinear_forward_noalloc (16 MiB in the device
+ *     image of every GPU that loads the library) and its cached device
+ *     address per GPU.
  *   - Matrices are dense row-major with no padding: x [M,K] fp32, W [N,K] fp32,
  *     packed [N, K/16] uint32, D [N] fp32 (a torch [N,1] tensor), y [M,N] fp32.
  *   - Device buffers must be 16-byte aligned, the workspace 256-byte aligned.
@@ -78,6 +81,10 @@ typedef enum {
 
 /* Version of this ABI (incremented on any incompatible change). */
 BL_API int bitlinear_abi_version(void);
+
+/* Static string identifying the sources this library was built from (a hash
+ * of the kernel sources and this header, set by the build); never NULL. */
+BL_API const char* bitlinear_build_id(void);
 
 /* Static string for a status code; never NULL. */
 BL_API const char* bitlinear_status_string(int status);
@@ -142,9 +149,10 @@ BL_API size_t bitlinear_workspace_size(int64_t M, int64_t N, int64_t K);
  *   D       device fp32 [N] per-row scale.
  *   y       device fp32 [M, N], fully overwritten; nothing outside it is written.
  *   ws      device scratch, ws_bytes >= bitlinear_workspace_size(M, N, K).
- * M <= 16 runs a fused quantise + GEMV kernel that streams the packed weights
- * once; larger M quantises into ws and runs the tcgen05 tensor-core GEMM.
- * Asynchronous. */
+ * M <= 16 runs the decode kernel: every CTA quantises x itself and the packed
+ * weights stream once through a shared-memory ring (K up to about 13000 for
+ * M <= 8; wider rows take the tensor-core path). Larger M quantises into ws
+ * and runs the tcgen05 tensor-core GEMM. Asynchronous. */
 BL_API int bitlinear_forward(const float* x, int64_t M, int64_t N, int64_t K,
                       const uint32_t* packed, const float* D, float* y,
                       void* ws, size_t ws_bytes, bl_stream_t stream);
@@ -171,10 +179,10 @@ BL_API int bitlinear_prepare_act(const float* x, int64_t M, int64_t K,
                                  void* ws, size_t ws_bytes, bl_stream_t stream);
 
 /* Contraction + rescale from a workspace filled by bitlinear_prepare_act with
- * the same M and K: y [M,N] = RN(RN(acc/s_x) * D). Runs the tcgen05
- * tensor-core kernel for every M (the fused GEMV of bitlinear_forward
- * quantises x itself). The workspace is only read (and its error word reset),
- * so several calls may follow one prepare. Asynchronous. */
+ * the same M and K: y [M,N] = RN(RN(acc/s_x) * D). Runs the decode kernel
+ * (prepared codes copied into shared memory) for M <= 16 and the tcgen05
+ * tensor-core kernel otherwise. The workspace is only read (and its error
+ * word reset), so several calls may follow one prepare. Asynchronous. */
 BL_API int bitlinear_forward_prepared(int64_t M, int64_t N, int64_t K,
                                       const uint32_t* packed, const float* D, float* y,
                                       void* ws, size_t ws_bytes, bl_stream_t stream);
@@ -185,7 +193,7 @@ BL_API int bitlinear_forward_prepared(int64_t M, int64_t N, int64_t K,
  * acc = sum_k q*code exactly. Any int8 codes are accepted (-128 included).
  * q, packed, D and y must be 16-byte aligned, ws 256-byte aligned with
  * ws_bytes >= bitlinear_workspace_size(M, N, K). Reorders q into ws, then runs
- * the tensor-core kernel (every M). Asynchronous. */
+ * the contraction of bitlinear_forward_prepared. Asynchronous. */
 BL_API int bitlinear_forward_q(const int8_t* q, const float* s_x, int64_t M, int64_t N, int64_t K,
                                const uint32_t* packed, const float* D, float* y,
                                void* ws, size_t ws_bytes, bl_stream_t stream);
@@ -200,10 +208,11 @@ BL_API int bitlinear_forward_q(const int8_t* q, const float* s_x, int64_t M, int
 BL_API int bitlinear_rmsnorm_quant_act(const float* x, const float* g, float eps, int64_t M, int64_t K,
                                        int8_t* q, float* s_x, int32_t* rowsum, bl_stream_t stream);
 
-/* y = F.linear(ActQuant(RMSNorm(x, g)), WeightQuant(W)) from packed weights:
- * the fused norm + quantiser writes the codes into ws, then the tensor-core
- * kernel runs (every M). Same arguments as bitlinear_forward plus g and eps;
- * K <= 16384. Asynchronous. */
+/* y = F.linear(ActQuant(RMSNorm(x, g)), WeightQuant(W)) from packed weights.
+ * M <= 16: one decode-kernel launch whose CTAs normalise and quantise x
+ * themselves. Larger M: the fused norm + quantiser writes the codes into ws,
+ * then the tensor-core kernel runs. Same arguments as bitlinear_forward plus g
+ * and eps; K <= 16384. Asynchronous. */
 BL_API int bitlinear_forward_rmsnorm(const float* x, const float* g, float eps, int64_t M, int64_t N,
                                      int64_t K, const uint32_t* packed, const float* D, float* y,
                                      void* ws, size_t ws_bytes, bl_stream_t stream);
@@ -309,11 +318,25 @@ BL_API int bitlinear_workspace_error(void* ws, size_t ws_bytes, bl_stream_t stre
  * stream capture. Every call shares the one array per device, and the array
  * keeps the last call's contents. Calls that can overlap on the same GPU
  * (other streams, other host threads) race on it and must be serialised by the
- * caller. The device error word of these calls lives in that array and is not
- * readable through bitlinear_workspace_error. Asynchronous. */
+ * caller. The device error word of these calls is the first word of that
+ * array; bitlinear_noalloc_error reads it. Asynchronous. */
 BL_API int bitlinear_forward_noalloc(const float* x, int64_t M, int64_t N, int64_t K,
                                      const uint32_t* packed, const float* D, float* y,
                                      bl_stream_t stream);
+
+/* The device error word of bitlinear_forward_noalloc, as
+ * bitlinear_workspace_error reads it for a caller workspace: synchronises
+ * `stream`, then reads and clears the word at the start of the fixed scratch
+ * of the current device. BL_OK if no call recorded a failure since the last
+ * read, BL_ERR_DEVICE if a kernel's bounded wait expired (its y is then
+ * incomplete), BL_ERR_CUDA if the scratch's address cannot be found. Allocates
+ * nothing. */
+BL_API int bitlinear_noalloc_error(bl_stream_t stream);
+
+/* Diagnostic: bitlinear_selftest_wait_timeout on the fixed scratch of
+ * bitlinear_forward_noalloc, so that bitlinear_noalloc_error then reports
+ * BL_ERR_DEVICE. No fault, trap or hang is involved. Asynchronous. */
+BL_API int bitlinear_noalloc_selftest_wait_timeout(uint64_t limit_ns, bl_stream_t stream);
 
 /* ---------------------------------------------------------------- I2_S --- */
 

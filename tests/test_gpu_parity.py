@@ -301,7 +301,8 @@ def test_forward_host_async_shared_workspace(B):
         B.forward_host(torch.zeros(1, 16), calls[0][1][:, :1].contiguous(), calls[0][2], sync=False)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 300, 2560), (37, 257, 528), (300, 700, 1152)])
+@pytest.mark.parametrize("M,N,K", [(1, 300, 2560), (16, 257, 6912), (5, 33, 4304), (37, 257, 528),
+                                   (300, 700, 1152)])
 def test_forward_q_from_quant_act(B, M, N, K):
     """forward_q on quant_act's natural-order codes equals the oracle's
     contraction and rescale of the same codes; arbitrary codes (-128 included)
@@ -384,12 +385,12 @@ def _sample_rows(M, extra=()):
 
 
 @pytest.mark.parametrize("li", range(3))
-@pytest.mark.parametrize("M", [512, 4096])
+@pytest.mark.parametrize("M", [512, 2048, 4096])
 def test_prefill_sweep_sampled(B, li, M):
     _layer_case(B, "prefill_sweep", li, M, rows=_sample_rows(M))
 
 
-@pytest.mark.parametrize("li", [0, 2, 3, 5])
+@pytest.mark.parametrize("li", range(6))
 def test_embed_batch_sampled(B, li):
     M = 32768
     seed = WL.WORKLOADS["embed_batch"].seed
@@ -633,7 +634,8 @@ def test_rmsnorm_exact_path_on_rounding_ties_and_zero_row(B):
     assert np.array_equal(s_x.cpu().numpy(), s_ref)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 3840, 2560), (37, 700, 1024), (300, 1024, 3072), (16, 129, 528)])
+@pytest.mark.parametrize("M,N,K", [(1, 3840, 2560), (1, 2560, 6912), (8, 300, 4304), (37, 700, 1024),
+                                   (300, 1024, 3072), (16, 129, 528), (9, 64, 16384)])
 def test_forward_rmsnorm(B, M, N, K):
     W = WL.weight(N, K, "normal", 90 + N)
     x = WL.activations(M, K, "outlier_tokens", 91 + M, meta={"df": 3.0, "frac": 0.02, "scale": 20.0})
@@ -642,6 +644,49 @@ def test_forward_rmsnorm(B, M, N, K):
     p_ref, D_ref = O.pack_weights(W)
     y = B.forward_rmsnorm(dev(x), dev(g), packed, D).cpu().numpy()
     assert_y_close(y, O.bitlinear_forward_rmsnorm(x, g, p_ref, D_ref, K))
+
+
+def test_forward_rmsnorm_decode_exact_path(B):
+    """The decode kernel's own RMSNorm: rows whose mean square sits on (or a
+    hair from) an fp32 rounding tie take the exact integer path, a zero row
+    gives ms = 0, a tiny row a subnormal ms; outputs equal the oracle's."""
+    K, N = 64, 40
+    rows = [np.full(K, 1 + 2.0 ** -12, np.float32), np.full(K, 1 + 3 * 2.0 ** -12, np.float32),
+            np.full(K, 1 + 2.0 ** -12 + 2.0 ** -23, np.float32), np.zeros(K, np.float32),
+            np.full(K, 3.0 * 2.0 ** -70, np.float32)]
+    x = np.stack(rows)
+    x[:, ::3] *= -1.0
+    g = np.linspace(0.5, 1.5, K).astype(np.float32)
+    W = WL.weight(N, K, "normal", 95)
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    y = B.forward_rmsnorm(dev(x), dev(g), packed, D).cpu().numpy()
+    assert_y_close(y, O.bitlinear_forward_rmsnorm(x, g, p_ref, D_ref, K))
+
+
+@pytest.mark.parametrize("M,K", [(1, 2560), (16, 6912), (3, 528), (300, 1152)])
+def test_forward_prepared_shares_one_quantisation(B, M, K):
+    """prepare_act once, then forward_prepared with three weights (decode
+    kernel for M <= 16, tensor-core kernel above): each equals the oracle."""
+    x = WL.activations(M, K, "student_t", 110 + M, meta={"df": 3.0})
+    ws = torch.zeros(B.workspace_size(M, 1, K), dtype=torch.uint8, device="cuda")
+    B.prepare_act(dev(x), ws)
+    for i, N in enumerate([300, 17, 2560]):
+        W = WL.weight(N, K, "laplace", 120 + i)
+        packed, D = B.pack_weights(dev(W))
+        p_ref, D_ref = O.pack_weights(W)
+        y = B.forward_prepared(M, K, packed, D, ws).cpu().numpy()
+        assert_y_close(y, O.bitlinear_forward(x, p_ref, D_ref, K))
+    assert B.workspace_error(ws) == 0
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 16, 16), (1, 1, 4304), (2, 15, 64), (7, 4305, 1152), (16, 16, 16),
+                                   (1, 65536, 256), (3, 97, 16384)])
+def test_decode_ring_shapes(B, M, N, K):
+    """Decode kernel edge shapes: single words, one-row problems with a row
+    that is not 16-byte aligned, N tails, many small tiles per CTA (a ring of
+    many tiles that wraps), and tiles of 64 KB (K = 16384)."""
+    run_case(B, M, N, K, xdist="student_t", seed=3 * M + N + K)
 
 
 # ------------------------------------------------------------ I2_S import/export

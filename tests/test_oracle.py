@@ -465,6 +465,57 @@ def test_mean_square_exact_tie_rounds_to_even():
     assert O.mean_square_exact(np.full(16, c, np.float32)) == np.float32(1 + 12292 * 2.0 ** -23)
 
 
+def _sqrt_rn_f32(v: Fraction) -> np.float32:
+    """Nearest fp32 to sqrt(v), decided by exact squares of the midpoints
+    between neighbouring fp32 values (sqrt of an fp32 is never a midpoint)."""
+    c = np.float32(math.sqrt(float(v)))
+    cands = sorted({np.nextafter(np.nextafter(c, np.float32(0)), np.float32(0)), np.nextafter(c, np.float32(0)), c,
+                    np.nextafter(c, np.float32(np.inf)),
+                    np.nextafter(np.nextafter(c, np.float32(np.inf)), np.float32(np.inf))})
+    for i in range(1, len(cands) - 1):
+        lo = (exact(cands[i - 1]) + exact(cands[i])) / 2
+        hi = (exact(cands[i]) + exact(cands[i + 1])) / 2
+        if lo * lo <= v < hi * hi:
+            return np.float32(cands[i])
+    raise AssertionError("no candidate brackets sqrt(v)")
+
+
+def test_rmsnorm_hand_row_exact_rationals():
+    """Reading 11's rounding order, re-derived step by step with rationals on
+    a hand row: x = the primes 2..19 with alternating signs, so sum x^2 = 1027
+    and ms = 1027/8 = 128.375 exactly; eps = 1e-6 is below half an ulp of
+    128.375 (2^-16), so RN(ms + eps) = ms. Then RN(sqrt), RN(1/.), RN(x*r),
+    RN(.*g). The row is chosen so that the reading is pinned to the bit: one
+    rounding of 1/sqrt(v) instead of two gives another r, and scaling by
+    RN(r*g) instead of x*r first changes two of the eight outputs."""
+    x = np.array([2, -3, 5, -7, 11, -13, 17, -19], np.float32)
+    g = np.array([0.125, 1.0, 0.75, 1.125, 1.25, 1.125, 0.25, 1.625], np.float32)
+    eps = O.RMS_EPS
+    ms_exact = sum(Fraction(int(v)) ** 2 for v in x) / 8
+    assert ms_exact == Fraction(1027, 8)
+    ms = rn_f32(ms_exact)
+    assert exact(ms) == ms_exact
+    v = rn_f32(exact(ms) + exact(eps))
+    assert v == ms  # eps is below half an ulp of 128.375
+    sq = _sqrt_rn_f32(exact(v))
+    r = rn_f32(1 / exact(sq))
+    n = [rn_f32(exact(rn_f32(exact(a) * exact(r))) * exact(b)) for a, b in zip(x, g)]
+    got = O.rmsnorm(x[None, :], g, eps)[0]
+    assert [int(t) for t in got.view(np.uint32)] == [int(np.float32(t).view(np.uint32)) for t in n]
+    # the pin discriminates: the alternatives give other bits
+    # one rounding of 1/sqrt(v): the fp32 c with 1/hi^2 < v <= 1/lo^2 for the
+    # midpoints lo < c < hi around it
+    c0 = np.float32(1.0 / math.sqrt(float(exact(v))))
+    cands = sorted({np.nextafter(c0, np.float32(0)), c0, np.nextafter(c0, np.float32(1))})
+    r_once = [cands[i] for i in range(1, len(cands) - 1)
+              if 1 / ((exact(cands[i]) + exact(cands[i + 1])) / 2) ** 2 < exact(v)
+              <= 1 / ((exact(cands[i - 1]) + exact(cands[i])) / 2) ** 2]
+    assert [hex(int(np.float32(t).view(np.uint32))) for t in r_once] == ["0x3db4c137"]
+    alt = [rn_f32(exact(a) * exact(rn_f32(exact(r) * exact(b)))) for a, b in zip(x, g)]
+    assert sum(np.float32(p) != np.float32(q) for p, q in zip(alt, n)) == 2
+    assert hex(int(np.float32(r).view(np.uint32))) == "0x3db4c138"
+
+
 def test_rmsnorm_act_quant_constant_row_and_g_scaling():
     x = np.full((2, 64), 3.0, np.float32)
     g = np.ones(64, np.float32)
