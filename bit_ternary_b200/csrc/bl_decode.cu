@@ -1,34 +1,38 @@
 // bl_decode.cu - decode BitLinear (M <= 16 tokens) for one or several
 // independent BitLinears per launch: ActQuant (or RMSNorm + ActQuant) of the
 // activations inside every CTA, the packed ternary weights streamed once from
-// HBM through a shared-memory ring, an exact int32 contraction and the fp32
-// rescale in the epilogue.
+// HBM straight into registers, an exact int32 contraction and the fp32 rescale
+// in the epilogue.
 //
 // The operation is the BitLinear product of "Core AI model zoo - BitVLA",
 // section 2 (M=1 decode, arbitrary K with K % 16 == 0, any N, per-row scale
 // D [N,1]), with the wrapper's ActQuant (section 1) done inside the kernel.
 //
 // Streaming. The packed weights are the only large stream (2 bits per weight).
-// The unit of the stream is a tile: 16 consecutive rows, i.e. 16 * K/4
-// contiguous bytes. Every CTA owns a contiguous, byte-balanced range of tiles
-// over all problems of the launch (one CTA per SM). A producer warp keeps that
-// range flowing through a byte ring in shared memory: one thread allocates a
-// tile's bytes in the ring (first fit after the newest tile, wrapping to the
-// start when the end is too short), issues one cp.async.bulk for it and hands
-// it to the consumers through the tile's "full" mbarrier. A tile's bytes are
-// given back when its "done" mbarrier fires, so up to the whole ring (about
-// 90 KB, or 200 KB when one CTA holds the SM) is in flight at any time. The
-// producer never reads activations, so it starts before griddepcontrol.wait:
-// when launches are chained with programmatic dependent launch, a launch's
-// weights stream while the previous launch still runs.
+// Work is cut into tiles of 16 consecutive rows, and a tile into tasks: the
+// whole tile when every warp of a CTA gets two or more tiles, else chunks of a
+// few 256-code units so that all warps share a short launch (chunk j of tile i
+// is one task). Every CTA owns a contiguous, byte-balanced range of tiles over
+// all problems of the launch; its 8 warps take every 8th task in (tile, chunk)
+// order, and walk each task in groups of up to 4 units. Each lane copies
+// exactly the words it will contract (words 4t..4t+3 of rows g and g+8 of
+// every unit) with 16-byte cp.async into its warp's own pipeline stages in
+// shared memory, so a warp waits only on its own copies (cp.async.wait_group)
+// and needs no barrier with other warps; the in-flight bytes take no
+// registers. The first groups of every warp are issued before
+// griddepcontrol.wait (weights never depend on the previous kernel), so under
+// programmatic dependent launch a launch's weights stream while the previous
+// launch still runs. (One bulk-copy engine per SM moves only about 20-25 GB/s,
+// far below a B200 SM's share of HBM bandwidth, so the stream goes through the
+// load/store units of all warps instead.)
 //
-// Tasks. A tile is split into chunks of a few 256-code units; chunk j of tile i
-// is one task, and consumer warp w takes every 8th task in (tile, chunk) order.
-// A task's partial sums go to the tile's accumulator block in shared memory
-// with shared atomics (exact integers, so the order does not matter); the warp
-// that adds the tile's last chunk writes the outputs and releases the tile.
+// Accumulation. A chunk's partial sums go to its tile's block in shared
+// memory (one of 16 slots, by tile index) with shared atomics: exact integers,
+// so the order does not matter. The warp that adds the tile's last chunk
+// writes the outputs, clears the block and hands the slot to tile i + 16. A
+// warp that holds a whole tile writes its outputs directly from registers.
 //
-// Math. Lane (g, t) = (lane/4, lane%4) reads words 4t..4t+3 of each unit for
+// Math. Lane (g, t) = (lane/4, lane%4) holds words 4t..4t+3 of each unit for
 // rows g and g+8 of the tile. For class c in 0..3, word & (0x03030303 << 2c)
 // leaves in byte b the value (code[4b+c]+1) << 2c: one AND gives four u8
 // operands of mma.sync.m16n8k32 (u8 weights x s8 activations). One accumulator
@@ -48,13 +52,18 @@
 
 namespace bl {
 
-constexpr int kDecConsumerWarps = 8;
-constexpr int kDecConsumers = 32 * kDecConsumerWarps;
-constexpr int kDecThreads = kDecConsumers + 32;  // + the producer warp
-constexpr int kDecMaxGrid = 256;
+constexpr int kDecWarps = 8;
+constexpr int kDecThreads = 32 * kDecWarps;
+constexpr int kDecMaxGrid = 3 * 160;
 constexpr int kDecRegGroups = 2;  // 16-column groups per thread held in registers by the quantiser
-constexpr int kDecMaxUnitsPerTask = 5;
 constexpr int kDecTok = kDecodeMaxGroup * 16;  // per-token state entries: problem * 16 + token
+
+// Units per task (the register buffer of one task): eight 32-bit registers
+// per unit, two tasks in flight.
+template <int MT>
+__host__ __device__ constexpr int dec_upt() { return 4; }
+// Pipeline stages per warp (S - 1 groups of copies in flight).
+constexpr int kDecStages = 2;
 
 struct DecProblem {
   const void* x;        // fp32 / bf16 activations [M, K]; prepared mode: int8 codes, private order, [M, K]
@@ -83,45 +92,45 @@ struct DecLaunch {
   float eps;
   int nprob;
   int total_tiles;
-  int ring_bytes;
   int q_bytes;
   uint32_t* err;
   int cta_start[kDecMaxGrid + 1];  // CTA c owns launch tiles [cta_start[c], cta_start[c+1])
 };
 
-// Shared memory past the ring and the activation codes.
+// Shared memory past the activation codes.
 __host__ __device__ constexpr int dec_fixed_bytes(int MT) {
-  return kDecodeSlots * 16 * 8 * MT * 4   // s_acc
-         + kDecodeSlots * 16 * 4          // s_D
-         + 3 * kDecTok * 4              // s_sx, s_rs, s_amax
-         + 2 * kDecodeSlots * 4           // s_cnt, s_off
-         + 2 * kDecodeSlots * 8           // full, done
-         + 16 * (8 + 4 + 4)             // RMSNorm: sums of squares, mean squares, flags
-         + 16;                          // abort flag
+  return kDecTok * 8                     // s_inv
+         + kDecodeSlots * 16 * 8 * MT * 4  // s_acc
+         + kDecodeSlots * 16 * 4         // s_D
+         + 3 * kDecTok * 4               // s_sx, s_rs, s_amax
+         + 2 * kDecodeSlots * 4          // s_cnt, s_gen
+         + 16 * (8 + 4 + 4)              // RMSNorm: sums of squares, mean squares, flags
+         + 64                            // abort flag
+         + kDecWarps * kDecStages * 16;  // records of the groups in flight
 }
 
 __device__ __forceinline__ void dec_mma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                                         uint32_t b1) {
-  asm(
-      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void dec_bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
-      : "memory");
+// 16-byte load of streamed weights: read once, not kept in L1.
+__device__ __forceinline__ uint4 ldg_stream(const uint32_t* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(__cvta_generic_to_global(p)));
 }
 
-// Named barrier of the 8 consumer warps (the producer warp never joins it).
-__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers) : "memory"); }
+// Barrier of the CTA's 8 warps (named, so that its count is explicit).
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kDecThreads) : "memory"); }
 
 __device__ __forceinline__ int dec_problem_of(const DecLaunch& L, int gt) {
   int p = 0;
@@ -187,6 +196,204 @@ __device__ __forceinline__ int dec_quant_group(const float4 (&f)[4], float sx, u
   return sum;
 }
 
+// What the contraction of a group in flight needs, packed in four words (the
+// same for every lane): the activation offset of its first unit (token 0),
+// the tile's CTA-local index, and
+// problem | chunk << 3 | units << 20 | first << 24 | last << 25 | valid << 26.
+struct __align__(16) DecRun {
+  int qoff, i, meta, pad;
+  __device__ __forceinline__ int p() const { return meta & 7; }
+  __device__ __forceinline__ int j() const { return (meta >> 3) & 0x1FFFF; }
+  __device__ __forceinline__ int n() const { return (meta >> 20) & 15; }
+  __device__ __forceinline__ bool first() const { return (meta >> 24) & 1; }
+  __device__ __forceinline__ bool last() const { return (meta >> 25) & 1; }
+  __device__ __forceinline__ bool valid() const { return (meta >> 26) & 1; }
+};
+
+// Asynchronous copies of 16 or 4 bytes global -> shared. With src_bytes == 0
+// the destination is zero-filled; the source address must still lie inside
+// an allocation (callers pass the buffer's first element).
+__device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)),
+               "l"(__cvta_generic_to_global(src)), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(__cvta_generic_to_global(src))
+               : "memory");
+}
+__device__ __forceinline__ void cp_async4_zfill(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)),
+               "l"(__cvta_generic_to_global(src)), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Bytes of one pipeline stage of a warp: per unit, 512 bytes of row-g words
+// and 512 of row-(g+8) words (16 per lane), then two row scales per lane.
+template <int UPT>
+__host__ __device__ constexpr int dec_stage_bytes() { return UPT * 1024 + 256; }
+
+// A warp's position in its work: tasks warp, warp + 8, warp + 16, ... in
+// (tile, chunk) order (chunk j of the CTA's tile i, in problem p), each task
+// cut into groups of at most UPT units. The current problem's fields are kept
+// in registers, so stepping reads the launch parameters only when the
+// problem changes.
+template <int UPT, bool kAccOut>
+struct DecCursor {
+  // task position
+  int p, C, i, j, pend;
+  bool valid;
+  // the current problem
+  const uint32_t* packed;
+  const float* D;
+  int wpr, N, tile0, upt, nu, q_off;
+  // the current task
+  const uint32_t* rowa;  // row g, word 16*u + 4t of the next unit u
+  int w0;                // word 16*u + 4t
+  int left;              // units of the task not yet issued
+  int qoff;              // activation offset of unit u (token 0)
+  int row0;
+  bool aon, bon, fast, first;
+
+  __device__ __forceinline__ void load_problem(const DecLaunch& L, int t0) {
+    const DecProblem& P = L.pr[p];
+    packed = P.packed;
+    D = P.D;
+    wpr = P.wpr;
+    N = P.N;
+    tile0 = P.tile0;
+    upt = P.upt;
+    nu = P.nu;
+    q_off = P.q_off;
+    C = P.nchunk;
+    pend = P.tile0 + P.tiles - t0;
+  }
+  // Move (i, j) onto a task: whole tiles are skipped at once, one problem at
+  // a time.
+  __device__ __forceinline__ void normalise(const DecLaunch& L, int t0, int nt) {
+    while (j >= C && i < nt) {
+      const int adv = C == 1 ? j : j / C;
+      if (i + adv < pend) {
+        i += adv;
+        j -= adv * C;
+      } else {
+        j -= (pend - i) * C;
+        i = pend;
+        if (i < nt && p + 1 < L.nprob) {
+          ++p;
+          load_problem(L, t0);
+        }
+      }
+    }
+  }
+  // Set up the task at (i, j).
+  __device__ __forceinline__ void open(int t0, int nt, int lane) {
+    valid = i < nt;
+    if (!valid) return;
+    const int g = lane >> 2, t = lane & 3;
+    row0 = (t0 + i - tile0) * 16;
+    const int rv = N - row0 < 16 ? N - row0 : 16;
+    const int ua = j * upt;
+    const int ue = ua + upt < nu ? ua + upt : nu;
+    w0 = 16 * ua + 4 * t;
+    rowa = packed + (int64_t)(row0 + g) * wpr + w0;
+    qoff = q_off + 256 * ua;
+    left = ue - ua;
+    first = true;
+    aon = g < rv;
+    bon = g + 8 < rv;
+    fast = rv == 16 && (wpr & 3) == 0 && 16 * ue <= wpr;
+  }
+  __device__ __forceinline__ void init(const DecLaunch& L, int t0, int nt, int warp, int lane) {
+    p = dec_problem_of(L, t0);
+    load_problem(L, t0);
+    i = 0;
+    j = warp;
+    normalise(L, t0, nt);
+    open(t0, nt, lane);
+  }
+  // Start the copies of the next group into `stage` and return what its
+  // contraction needs (valid() == false past the warp's last task; nothing
+  // is copied then, but the caller still commits a copy group). Each lane
+  // copies exactly the words it contracts: words 4t..4t+3 of rows g and g+8
+  // of every unit; rows past N and words past the row are zero-filled. A
+  // group that opens its task also brings row scales: D[row0 + lane] (lanes
+  // 0..15, chunked tiles) or D[row0 + g] and D[row0 + g + 8] (whole tiles).
+  __device__ __forceinline__ DecRun issue(const DecLaunch& L, int t0, int nt, uint8_t* stage, int lane) {
+    DecRun r;
+    r.pad = 0;
+    if (!valid) {
+      r.qoff = r.i = r.meta = 0;
+      return r;
+    }
+    const int n = left < UPT ? left : UPT;
+    uint8_t* da = stage + 16 * lane;
+    const uint32_t* rowb = rowa + (int64_t)8 * wpr;
+    if (fast) {
+#pragma unroll
+      for (int k = 0; k < UPT; ++k)
+        if (k < n) {
+          cp_async16(da + 1024 * k, rowa + 16 * k);
+          cp_async16(da + 1024 * k + 512, rowb + 16 * k);
+        }
+    } else if ((wpr & 3) == 0) {
+      // Rows start 16-byte aligned; a 4-word group is wholly in the row or past it.
+#pragma unroll
+      for (int k = 0; k < UPT; ++k)
+        if (k < n) {
+          const bool in = w0 + 16 * k < wpr;
+          cp_async16_zfill(da + 1024 * k, in && aon ? rowa + 16 * k : packed, in && aon ? 16u : 0u);
+          cp_async16_zfill(da + 1024 * k + 512, in && bon ? rowb + 16 * k : packed, in && bon ? 16u : 0u);
+        }
+    } else {
+      // Rows not 16-byte aligned: 4-byte copies.
+#pragma unroll
+      for (int k = 0; k < UPT; ++k)
+        if (k < n) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const bool in = w0 + 16 * k + e < wpr;
+            cp_async4_zfill(da + 1024 * k + 4 * e, in && aon ? rowa + 16 * k + e : packed, in && aon ? 4u : 0u);
+            cp_async4_zfill(da + 1024 * k + 512 + 4 * e, in && bon ? rowb + 16 * k + e : packed,
+                            in && bon ? 4u : 0u);
+          }
+        }
+    }
+    if (!kAccOut && first) {
+      const int g = lane >> 2;
+      float* dd = reinterpret_cast<float*>(stage + UPT * 1024) + 2 * lane;
+      if (C > 1) {
+        const bool in = j == 0 && lane < 16 && row0 + lane < N;
+        cp_async4_zfill(dd, in ? D + row0 + lane : D, in ? 4u : 0u);
+      } else {
+        cp_async4_zfill(dd, aon ? D + row0 + g : D, aon ? 4u : 0u);
+        cp_async4_zfill(dd + 1, bon ? D + row0 + g + 8 : D, bon ? 4u : 0u);
+      }
+    }
+    const bool last = left == n;
+    r.qoff = qoff;
+    r.i = i;
+    r.meta = p | ((j & 0x1FFFF) << 3) | (n << 20) | ((int)first << 24) | ((int)last << 25) | (1 << 26);
+    if (last) {
+      j += kDecWarps;
+      normalise(L, t0, nt);
+      open(t0, nt, lane);
+    } else {
+      left -= n;
+      first = false;
+      rowa += 16 * n;
+      w0 += 16 * n;
+      qoff += 256 * n;
+    }
+    return r;
+  }
+};
+
 // Problems [pa, pb] of this CTA, flattened into 16-column groups: group gg
 // belongs to problem p with pre[p - pa] <= gg < pre[p - pa + 1].
 struct DecGroups {
@@ -225,7 +432,7 @@ __device__ void dec_quantise(const DecLaunch& L, const DecGroups& G, uint8_t* sq
   float4 f[kDecRegGroups][4];
 #pragma unroll
   for (int r = 0; r < kDecRegGroups; ++r) {
-    const int gg = tid + r * kDecConsumers;
+    const int gg = tid + r * kDecThreads;
     if (gg < G.total) {
       int p, m, gi;
       G.locate(L, gg, p, m, gi);
@@ -234,7 +441,7 @@ __device__ void dec_quantise(const DecLaunch& L, const DecGroups& G, uint8_t* sq
   }
 #pragma unroll
   for (int r = 0; r < kDecRegGroups; ++r) {
-    const int gg = tid + r * kDecConsumers;
+    const int gg = tid + r * kDecThreads;
     int tok = -1;
     float a = 0.0f;
     if (gg < G.total) {
@@ -246,7 +453,7 @@ __device__ void dec_quantise(const DecLaunch& L, const DecGroups& G, uint8_t* sq
     dec_amax(s_amax, tok, a);
   }
   // Groups beyond the registers: loaded now for the maximum, again for the codes.
-  for (int base = kDecRegGroups * kDecConsumers; base < G.total; base += kDecConsumers) {
+  for (int base = kDecRegGroups * kDecThreads; base < G.total; base += kDecThreads) {
     const int gg = base + tid;
     int tok = -1;
     float a = 0.0f;
@@ -263,7 +470,7 @@ __device__ void dec_quantise(const DecLaunch& L, const DecGroups& G, uint8_t* sq
   consumers_sync();  // every token's max|x| is complete
 #pragma unroll
   for (int r = 0; r < kDecRegGroups; ++r) {
-    const int gg = tid + r * kDecConsumers;
+    const int gg = tid + r * kDecThreads;
     int tok = -1, sum = 0;
     if (gg < G.total) {
       int p, m, gi;
@@ -275,7 +482,7 @@ __device__ void dec_quantise(const DecLaunch& L, const DecGroups& G, uint8_t* sq
     }
     dec_rowsum(s_rs, tok, sum);
   }
-  for (int base = kDecRegGroups * kDecConsumers; base < G.total; base += kDecConsumers) {
+  for (int base = kDecRegGroups * kDecThreads; base < G.total; base += kDecThreads) {
     const int gg = base + tid;
     int tok = -1, sum = 0;
     if (gg < G.total) {
@@ -296,14 +503,14 @@ __device__ void dec_quantise(const DecLaunch& L, const DecGroups& G, uint8_t* sq
 // group order, row stride K; s_x and row sums): copied into the shared layout.
 __device__ void dec_load_prepared(const DecLaunch& L, const DecGroups& G, uint8_t* sq, float* s_sx, int32_t* s_rs) {
   const int tid = threadIdx.x;
-  for (int gg = tid; gg < G.total; gg += kDecConsumers) {
+  for (int gg = tid; gg < G.total; gg += kDecThreads) {
     int p, m, gi;
     G.locate(L, gg, p, m, gi);
     const DecProblem& P = L.pr[p];
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const int8_t*>(P.x) + (int64_t)m * P.K) + gi);
     *reinterpret_cast<uint4*>(dec_q_group(sq, P, m, gi)) = v;
   }
-  for (int i = tid; i < G.np * 16; i += kDecConsumers) {
+  for (int i = tid; i < G.np * 16; i += kDecThreads) {
     const int p = G.pa + (i >> 4), m = i & 15;
     if (m < L.pr[p].M) {
       s_sx[p * 16 + m] = __ldg(L.pr[p].sx_in + m);
@@ -331,8 +538,8 @@ __device__ void dec_rms_quantise(const DecLaunch& L, const DecGroups& G, uint8_t
   const float4* g4 = reinterpret_cast<const float4*>(L.g);
   float4 f[kDecRegGroups][4];
   // Sum of squares per token.
-  for (int base = 0; base < G.total; base += kDecConsumers) {
-    const int r = base / kDecConsumers;
+  for (int base = 0; base < G.total; base += kDecThreads) {
+    const int r = base / kDecThreads;
     const int gg = base + tid;
     int tok = -1;
     double ss = 0.0;
@@ -372,10 +579,10 @@ __device__ void dec_rms_quantise(const DecLaunch& L, const DecGroups& G, uint8_t
   consumers_sync();
   for (int m = 0; m < P.M; ++m) {
     if (!s_flag[m]) continue;  // uniform over the consumers
-    for (int b = tid; b < kRmsBins; b += kDecConsumers) bins[b] = 0ull;
+    for (int b = tid; b < kRmsBins; b += kDecThreads) bins[b] = 0ull;
     consumers_sync();
     const float4* xr = reinterpret_cast<const float4*>(P.x) + ((int64_t)m * P.K >> 2);
-    for (int i4 = tid; i4 < (P.K >> 2); i4 += kDecConsumers) {
+    for (int i4 = tid; i4 < (P.K >> 2); i4 += kDecThreads) {
       const float4 v = __ldg(xr + i4);
       rms_bins_add(bins, v.x);
       rms_bins_add(bins, v.y);
@@ -396,8 +603,8 @@ __device__ void dec_rms_quantise(const DecLaunch& L, const DecGroups& G, uint8_t
                          __fmul_rn(__fmul_rn(v[j].z, rr), gw.z), __fmul_rn(__fmul_rn(v[j].w, rr), gw.w));
     }
   };
-  for (int base = 0; base < G.total; base += kDecConsumers) {
-    const int r = base / kDecConsumers;
+  for (int base = 0; base < G.total; base += kDecThreads) {
+    const int r = base / kDecThreads;
     const int gg = base + tid;
     int tok = -1;
     float a = 0.0f;
@@ -429,8 +636,8 @@ __device__ void dec_rms_quantise(const DecLaunch& L, const DecGroups& G, uint8_t
     dec_amax(s_amax, tok, a);
   }
   consumers_sync();
-  for (int base = 0; base < G.total; base += kDecConsumers) {
-    const int r = base / kDecConsumers;
+  for (int base = 0; base < G.total; base += kDecThreads) {
+    const int r = base / kDecThreads;
     const int gg = base + tid;
     int tok = -1, sum = 0;
     if (gg < G.total) {
@@ -456,24 +663,26 @@ __device__ void dec_rms_quantise(const DecLaunch& L, const DecGroups& G, uint8_t
   }
 }
 
+
 template <int MT, bool kAccOut, int kX>
 __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decode_kernel(const __grid_constant__ DecLaunch L) {
+  constexpr int UPT = dec_upt<MT>();
   extern __shared__ __align__(128) uint8_t smem[];
-  uint8_t* ring = smem;
-  uint8_t* sq = smem + L.ring_bytes;
-  int32_t* s_acc = reinterpret_cast<int32_t*>(sq + L.q_bytes);        // [slot][16 rows][8*MT tokens]
+  uint8_t* stages = smem;                                                      // [warp][stage]
+  uint8_t* sq = smem + kDecWarps * kDecStages * dec_stage_bytes<UPT>();
+  double* s_inv = reinterpret_cast<double*>(sq + L.q_bytes);                   // [problem * 16 + token] RN64(1/s_x)
+  int32_t* s_acc = reinterpret_cast<int32_t*>(s_inv + kDecTok);               // [slot][16 rows][8*MT tokens]
   float* s_D = reinterpret_cast<float*>(s_acc + kDecodeSlots * 16 * 8 * MT);  // [slot][16]
-  float* s_sx = s_D + kDecodeSlots * 16;                                 // [problem * 16 + token]
+  float* s_sx = s_D + kDecodeSlots * 16;                                       // [problem * 16 + token]
   int32_t* s_rs = reinterpret_cast<int32_t*>(s_sx + kDecTok);
   uint32_t* s_amax = reinterpret_cast<uint32_t*>(s_rs + kDecTok);
-  int32_t* s_cnt = reinterpret_cast<int32_t*>(s_amax + kDecTok);      // chunks added per slot
-  uint32_t* s_off = reinterpret_cast<uint32_t*>(s_cnt + kDecodeSlots);  // ring offset per slot
-  uint64_t* full = reinterpret_cast<uint64_t*>(s_off + kDecodeSlots);
-  uint64_t* done = full + kDecodeSlots;
-  double* s_ss = reinterpret_cast<double*>(done + kDecodeSlots);  // RMSNorm: [16] sums of squares
-  float* s_ms = reinterpret_cast<float*>(s_ss + 16);              // [16] mean squares
-  int* s_flag = reinterpret_cast<int*>(s_ms + 16);                // [16] exact path needed
+  int32_t* s_cnt = reinterpret_cast<int32_t*>(s_amax + kDecTok);  // chunks added per slot
+  int32_t* s_gen = s_cnt + kDecodeSlots;                           // slot s holds tile s + 16 * s_gen[s]
+  double* s_ss = reinterpret_cast<double*>(s_gen + kDecodeSlots);  // RMSNorm: [16] sums of squares
+  float* s_ms = reinterpret_cast<float*>(s_ss + 16);               // [16] mean squares
+  int* s_flag = reinterpret_cast<int*>(s_ms + 16);                 // [16] exact path needed
   volatile int* abort_flag = reinterpret_cast<volatile int*>(s_flag + 16);
+  int* s_rec = s_flag + 32;  // [warp][stage] records of the groups in flight (3 ints each, 16-byte slots)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -483,99 +692,36 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
 
   // Dependents may be scheduled as soon as every CTA of this grid is running.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  if (tid == 0) {
-    for (int s = 0; s < kDecodeSlots; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&done[s], 1);
-    }
-    *abort_flag = 0;
-    fence_barrier_init();
+  if (nt <= 0) return;
+
+  // The first two groups' weights are requested at once: they never depend on
+  // the grid this launch waits for.
+  constexpr int S = kDecStages;
+  constexpr int SB = dec_stage_bytes<UPT>();
+  uint8_t* wstage = stages + (size_t)warp * S * SB;  // this warp's S stages
+  DecCursor<UPT, kAccOut> cur;
+  cur.init(L, t0, nt, warp, lane);
+  // What each stage's contraction needs, by stage (every lane writes and
+  // reads the same values).
+  DecRun* rec = reinterpret_cast<DecRun*>(s_rec) + warp * S;
+#pragma unroll 1
+  for (int k = 0; k < S - 1; ++k) {
+    rec[k] = cur.issue(L, t0, nt, wstage + k * SB, lane);
+    cp_async_commit();
   }
+
   for (int i = tid; i < kDecodeSlots * 16 * 8 * MT; i += kDecThreads) s_acc[i] = 0;
-  if (tid < kDecodeSlots) s_cnt[tid] = 0;
+  if (tid < kDecodeSlots) {
+    s_cnt[tid] = 0;
+    s_gen[tid] = 0;
+  }
   if (tid < kDecTok) {
     s_amax[tid] = 0u;
     s_rs[tid] = 0;
   }
   if (tid < 16) s_ss[tid] = 0.0;
-  __syncthreads();
-  if (nt <= 0) return;
+  if (tid == 0) *abort_flag = 0;
 
-  if (warp == kDecConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    if (lane != 0) return;
-    const uint32_t R = (uint32_t)L.ring_bytes;
-    uint32_t head = 0;  // end of the newest tile in the ring
-    int tail = 0;       // oldest tile not yet seen released
-    int issued = 0;
-    bool ok = true;
-    int p = dec_problem_of(L, t0);
-    for (int i = 0; i < nt && ok; ++i) {
-      const int gt = t0 + i;
-      while (p + 1 < L.nprob && gt >= L.pr[p + 1].tile0) ++p;
-      const DecProblem& P = L.pr[p];
-      const int row0 = (gt - P.tile0) * 16;
-      const int rows = P.N - row0 < 16 ? P.N - row0 : 16;
-      const uint32_t bytes = (uint32_t)rows * (uint32_t)P.wpr * 4u;
-      const uint32_t sz = (bytes + 127u) & ~127u;
-      uint32_t off = 0;
-      // First fit after the newest tile; otherwise wait for the oldest tile.
-      for (;;) {
-        if (tail == i) {
-          off = 0;
-          break;
-        }
-        if (i - tail < kDecodeSlots) {
-          const uint32_t o = s_off[tail % kDecodeSlots];
-          if (head > o) {  // live bytes [o, head)
-            if (head + sz <= R) {
-              off = head;
-              break;
-            }
-            if (sz <= o) {
-              off = 0;
-              break;
-            }
-          } else if (head + sz <= o) {  // live bytes [o, R) and [0, head)
-            off = head;
-            break;
-          }
-        }
-        if (!mbar_wait(&done[tail % kDecodeSlots], (uint32_t)(tail / kDecodeSlots) & 1u, abort_flag, L.err,
-                       kDevTimeoutProducer)) {
-          ok = false;
-          break;
-        }
-        ++tail;
-      }
-      if (!ok) break;
-      head = off + sz;
-      const int s = i % kDecodeSlots;
-      s_off[s] = off;
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(P.packed + (int64_t)row0 * P.wpr);
-      const uint32_t bulk = bytes & ~15u;
-      if (bulk != bytes) {
-        // 4..12 trailing bytes (a problem's last tile only): plain copies,
-        // ordered for the readers by the barrier arrival below and for later
-        // bulk writes to the same bytes by the proxy fence.
-        for (uint32_t o = bulk; o < bytes; o += 4)
-          *reinterpret_cast<uint32_t*>(ring + off + o) = __ldg(reinterpret_cast<const uint32_t*>(src + o));
-        fence_proxy_async_smem();
-      }
-      mbar_arrive_expect_tx(&full[s], bulk);
-      if (bulk) dec_bulk_g2s(ring + off, src, bulk, &full[s]);
-      issued = i + 1;
-    }
-    if (!ok) {
-      // Let the copies still in flight land before the CTA exits.
-      for (int j = issued - kDecodeSlots > 0 ? issued - kDecodeSlots : 0; j < issued; ++j)
-        mbar_wait(&full[j % kDecodeSlots], (uint32_t)(j / kDecodeSlots) & 1u, nullptr, L.err, kDevTimeoutDrain,
-                  100000000ull);
-    }
-    return;
-  }
-
-  // -------------------------------------------------------------- consumers
   DecGroups G;
   G.pa = dec_problem_of(L, t0);
   G.np = dec_problem_of(L, t0 + nt - 1) - G.pa + 1;
@@ -592,12 +738,13 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
     for (int i = 0; i < G.np; ++i) {
       const DecProblem& P = L.pr[G.pa + i];
       const int64_t bytes = (int64_t)P.M * P.K * esz;
-      for (int64_t o = (int64_t)tid * 128; o < bytes; o += (int64_t)kDecConsumers * 128)
+      for (int64_t o = (int64_t)tid * 128; o < bytes; o += (int64_t)kDecThreads * 128)
         prefetch_l2(static_cast<const uint8_t*>(P.x) + o);
     }
   }
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0 && c == 0 && L.err != nullptr) *L.err = 0u;
+  consumers_sync();  // shared state initialised
 
   if (kX == kDecPrepared)
     dec_load_prepared(L, G, sq, s_sx, s_rs);
@@ -606,83 +753,64 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
                      reinterpret_cast<unsigned long long*>(sq + L.q_bytes - kRmsBins * 8));
   else
     dec_quantise<kX>(L, G, sq, s_sx, s_rs, s_amax);
-  consumers_sync();  // codes, scales and row sums visible to every consumer warp
+  consumers_sync();  // codes, scales and row sums visible to every warp
+  // Per-token fp64 reciprocal for the exact rescale of the epilogues.
+  if (tid < kDecTok) s_inv[tid] = __drcp_rn((double)s_sx[tid]);
+  consumers_sync();
 
   const int g = lane >> 2, t = lane & 3;
-  int p = G.pa;
-  int task = 0;
-  for (int i = 0; i < nt; ++i) {
-    const int gt = t0 + i;
-    while (p + 1 < L.nprob && gt >= L.pr[p + 1].tile0) ++p;
-    const DecProblem& P = L.pr[p];
-    const int C = P.nchunk;
-    const int s = i % kDecodeSlots;
-    const int row0 = (gt - P.tile0) * 16;
-    const int rv = P.N - row0 < 16 ? P.N - row0 : 16;
-    for (int j = (warp - task) & (kDecConsumerWarps - 1); j < C; j += kDecConsumerWarps) {
-      if (!mbar_wait(&full[s], (uint32_t)(i / kDecodeSlots) & 1u, abort_flag, L.err, kDevTimeoutMma)) return;
-      if (!kAccOut && j == 0 && lane < 16) s_D[s * 16 + lane] = lane < rv ? __ldg(P.D + row0 + lane) : 0.0f;
-      const uint32_t* tile = reinterpret_cast<const uint32_t*>(ring + s_off[s]);
-      const int wpr = P.wpr;
-      // Rows past N are not in the ring: lanes on them read nothing.
-      const bool aon = g < rv, bon = g + 8 < rv;
-      const uint32_t* rowa = tile + (aon ? g : 0) * wpr + 4 * t;
-      const uint32_t* rowb = tile + (bon ? g + 8 : 0) * wpr + 4 * t;
-      const bool al = (wpr & 3) == 0;
-      // Only lanes of existing tokens read activations (the other MMA
-      // columns are never used).
-      const uint8_t* qb[MT];
-      bool qon[MT];
+  int acc[4][MT][4];
+  float dg0 = 0.0f, dg1 = 0.0f;  // row scales of the current task
+  auto zero_acc = [&]() {
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) acc[cc][mt][k] = 0;
+  };
+  zero_acc();
+  int qp = -1, qlane[MT];  // the lane's token-row offset, for problem qp
+  // Contract one group from its registers into acc; at the end of its task,
+  // write the task's result. False if a wait gave up.
+  auto run = [&](const DecRun& Gr, const uint8_t* stage) -> bool {
+    const struct {
+      int p, i, j;
+    } T{Gr.p(), Gr.i, Gr.j()};
+    const DecProblem& P = L.pr[T.p];
+    if (!kAccOut && Gr.first()) {
+      const float2 dd = *reinterpret_cast<const float2*>(stage + UPT * 1024 + 8 * lane);
+      dg0 = dd.x;
+      dg1 = dd.y;
+    }
+    // Lanes of token columns past M read the last token's codes (their MMA
+    // columns are never used).
+    if (T.p != qp) {
+      qp = T.p;
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        qon[mt] = g + 8 * mt < P.M;
-        qb[mt] = sq + P.q_off + (qon[mt] ? g + 8 * mt : 0) * P.q_stride + 32 * t;
+        const int m = g + 8 * mt < P.M ? g + 8 * mt : P.M - 1;
+        qlane[mt] = m * P.q_stride + 32 * t;
       }
-      int acc[4][MT][4];
+    }
+    const uint8_t* qb[MT];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc)
+    for (int mt = 0; mt < MT; ++mt) qb[mt] = sq + Gr.qoff + qlane[mt];
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-          for (int k = 0; k < 4; ++k) acc[cc][mt][k] = 0;
-      const int ua = j * P.upt;
-      const int ub = ua + P.upt < P.nu ? ua + P.upt : P.nu;
-#pragma unroll 2
-      for (int u = ua; u < ub; ++u) {
-        uint32_t wa[4], wb[4];
-        const int w0 = 16 * u + 4 * t;
-        if (al && w0 + 4 <= wpr) {
-          uint4 va = make_uint4(0u, 0u, 0u, 0u), vb = make_uint4(0u, 0u, 0u, 0u);
-          if (aon) va = *reinterpret_cast<const uint4*>(rowa + 16 * u);
-          if (bon) vb = *reinterpret_cast<const uint4*>(rowb + 16 * u);
-          wa[0] = va.x;
-          wa[1] = va.y;
-          wa[2] = va.z;
-          wa[3] = va.w;
-          wb[0] = vb.x;
-          wb[1] = vb.y;
-          wb[2] = vb.z;
-          wb[3] = vb.w;
-        } else {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const bool in = w0 + k < wpr;  // words past the row belong to the next row: zero
-            wa[k] = in && aon ? rowa[16 * u + k] : 0u;
-            wb[k] = in && bon ? rowb[16 * u + k] : 0u;
-          }
-        }
+    for (int k = 0; k < UPT; ++k) {
+      if (k < Gr.n()) {
+        const uint4 va = *reinterpret_cast<const uint4*>(stage + 1024 * k + 16 * lane);
+        const uint4 vb = *reinterpret_cast<const uint4*>(stage + 1024 * k + 512 + 16 * lane);
+        const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
+        const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint4 Q[MT][2];
 #pragma unroll
           for (int mt = 0; mt < MT; ++mt) {
-            Q[mt][0] = make_uint4(0u, 0u, 0u, 0u);
-            Q[mt][1] = make_uint4(0u, 0u, 0u, 0u);
-            if (qon[mt]) {
-              const uint8_t* qp = qb[mt] + 256 * u + 128 * h;
-              Q[mt][0] = *reinterpret_cast<const uint4*>(qp);
-              Q[mt][1] = *reinterpret_cast<const uint4*>(qp + 16);
-            }
+            const uint8_t* qp = qb[mt] + 256 * k + 128 * h;
+            Q[mt][0] = *reinterpret_cast<const uint4*>(qp);
+            Q[mt][1] = *reinterpret_cast<const uint4*>(qp + 16);
           }
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
@@ -698,131 +826,175 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
           }
         }
       }
-      // Partial sums of this chunk into the tile's block: class c holds
-      // 4^c * sum q*(code+1), an exact multiple of 4^c.
-      int32_t* blk = s_acc + s * 16 * 8 * MT;
+    }
+    if (!Gr.last()) return true;
+    const int gt = t0 + T.i;
+    const int row0 = (gt - P.tile0) * 16;
+    const int rv = P.N - row0 < 16 ? P.N - row0 : 16;
+    // Slot s serves tiles s, s + 16, s + 32, ... in turn; a tile may use it
+    // once the tile 16 before it has finished (s_gen counts finished turns).
+    const int s = T.i % kDecodeSlots;
+    const int gen = T.i / kDecodeSlots;
+    if (*reinterpret_cast<volatile int32_t*>(&s_gen[s]) != gen) {
+      const uint64_t w0 = globaltimer_ns();
+      while (*reinterpret_cast<volatile int32_t*>(&s_gen[s]) != gen) {
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - w0 > kWaitLimitNs) {
+          *abort_flag = 1;
+          if (L.err != nullptr) atomicCAS(L.err, 0u, (uint32_t)kDevTimeoutMma);
+          return false;
+        }
+      }
+      __threadfence_block();
+    }
+    if (P.nchunk == 1) {
+      // The warp holds the whole tile: lane (g, t) has rows g and g+8 for
+      // tokens 2t, 2t+1 (+ 8 per token group). Class c holds 4^c * sum
+      // q*(code+1), an exact multiple of 4^c. y = RN(RN(a / s_x) * D) with
+      // RN(a / s_x) taken as RN32(RN64(a * RN64(1 / s_x))), which is the
+      // correctly rounded quotient for |a| < 2^24 (double rounding is
+      // innocuous here, Figueroa 1995).
+      const int M = P.M;
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
+          if (M == 1 && (k & 1)) continue;  // one token: only the even columns exist
           const int tok = 8 * mt + 2 * t + (k & 1);
-          if (tok < P.M) {
-            const int v = acc[0][mt][k] + (acc[1][mt][k] >> 2) + (acc[2][mt][k] >> 4) + (acc[3][mt][k] >> 6);
-            atomicAdd(blk + (g + 8 * (k >> 1)) * 8 * MT + tok, v);
-          }
-        }
-      __syncwarp();
-      __threadfence_block();
-      int last = 0;
-      if (lane == 0) last = atomicAdd(&s_cnt[s], 1) == C - 1;
-      last = __shfl_sync(0xFFFFFFFFu, last, 0);
-      if (last) {
-        // Every chunk of the tile is in: outputs, then release the tile.
-        __threadfence_block();
-        for (int idx = lane; idx < 16 * P.M; idx += 32) {
-          const int tok = idx >> 4, r = idx & 15;
-          if (r < rv) {
-            const int a = blk[r * 8 * MT + tok] - s_rs[p * 16 + tok];
+          const int r = g + 8 * (k >> 1);
+          if (tok < M && r < rv) {
+            const int a = acc[0][mt][k] + (acc[1][mt][k] >> 2) + (acc[2][mt][k] >> 4) + (acc[3][mt][k] >> 6) -
+                          s_rs[T.p * 16 + tok];
             const int64_t o = (int64_t)tok * P.N + row0 + r;
             if (kAccOut)
               P.acc[o] = a;
             else
-              P.y[o] = rescale(a, s_sx[p * 16 + tok], s_D[s * 16 + r]);
+              P.y[o] = __fmul_rn(div_by_scale(a, s_inv[T.p * 16 + tok]), (k >> 1) ? dg1 : dg0);
           }
         }
-        __syncwarp();
-        for (int k = lane; k < 16 * 8 * MT; k += 32) blk[k] = 0;
-        if (lane == 0) s_cnt[s] = 0;
-        __syncwarp();
-        __threadfence_block();
-        if (lane == 0) mbar_arrive(&done[s]);
-      }
+      zero_acc();
+      // The slot was not used: pass its turn on (no shared data to order).
+      __syncwarp();
+      if (lane == 0) *reinterpret_cast<volatile int32_t*>(&s_gen[s]) = gen + 1;
+      return true;
     }
-    task += C;
+    // Chunked tile: partial sums through the slot's block.
+    if (!kAccOut && T.j == 0 && lane < 16) s_D[s * 16 + lane] = dg0;
+    // Partial sums of this chunk into the tile's block.
+    int32_t* blk = s_acc + s * 16 * 8 * MT;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int tok = 8 * mt + 2 * t + (k & 1);
+        if (tok < P.M) {
+          const int v = acc[0][mt][k] + (acc[1][mt][k] >> 2) + (acc[2][mt][k] >> 4) + (acc[3][mt][k] >> 6);
+          atomicAdd(blk + (g + 8 * (k >> 1)) * 8 * MT + tok, v);
+        }
+      }
+    zero_acc();
+    __syncwarp();
+    __threadfence_block();
+    int last = 0;
+    if (lane == 0) last = atomicAdd(&s_cnt[s], 1) == P.nchunk - 1;
+    last = __shfl_sync(0xFFFFFFFFu, last, 0);
+    if (last) {
+      // Every chunk of the tile is in: outputs, then hand the slot on.
+      __threadfence_block();
+      for (int idx = lane; idx < 16 * P.M; idx += 32) {
+        const int tok = idx >> 4, r = idx & 15;
+        if (r < rv) {
+          const int a = blk[r * 8 * MT + tok] - s_rs[T.p * 16 + tok];
+          const int64_t o = (int64_t)tok * P.N + row0 + r;
+          if (kAccOut)
+            P.acc[o] = a;
+          else
+            P.y[o] = __fmul_rn(div_by_scale(a, s_inv[T.p * 16 + tok]), s_D[s * 16 + r]);
+        }
+      }
+      __syncwarp();
+      for (int k = lane; k < 16 * 8 * MT; k += 32) blk[k] = 0;
+      if (lane == 0) s_cnt[s] = 0;
+      __syncwarp();
+      __threadfence_block();
+      if (lane == 0) *reinterpret_cast<volatile int32_t*>(&s_gen[s]) = gen + 1;
+    }
+    return true;
+  };
+  // S - 1 groups in flight: start the next group in the stage freed by the
+  // last contraction, wait for the oldest, contract it.
+  int st = 0;
+#pragma unroll 1
+  for (;;) {
+    const int sti = st == 0 ? S - 1 : st - 1;
+    rec[sti] = cur.issue(L, t0, nt, wstage + sti * SB, lane);
+    cp_async_commit();
+    cp_async_wait<S - 1>();
+    const DecRun R = rec[st];
+    if (!R.valid() || !run(R, wstage + st * SB)) break;
+    st = st + 1 == S ? 0 : st + 1;
   }
+  cp_async_wait<0>();  // no copy is left in flight when the warp exits
 }
 
+using DecKernel = void (*)(const DecLaunch);
+
+// The decode kernel for (MT, output kind, input mode), with its dynamic
+// shared-memory limit raised (once per device).
 template <int MT, bool kAccOut, int kX>
-static cudaError_t launch_decode_t(const DecLaunch& L, int grid, size_t smem, bool pdl, cudaStream_t stream) {
-  auto kern = bl_ternary_decode_kernel<MT, kAccOut, kX>;
-  // The shared-memory limit is raised once per device for each instantiation.
-  static std::atomic<int> raised[64];
+static cudaError_t decode_kernel(DecKernel* out) {
+  static std::atomic<bool> raised[64];
+  DecKernel kern = bl_ternary_decode_kernel<MT, kAccOut, kX>;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64 || raised[dev].load(std::memory_order_relaxed) < (int)smem) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDecodeSmemMax);
+  if (dev < 0 || dev >= 64 || !raised[dev].load(std::memory_order_acquire)) {
+    e = cudaFuncSetAttribute(reinterpret_cast<const void*>(kern), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)kDecodeSmemMax);
     if (e != cudaSuccess) return e;
-    if (dev >= 0 && dev < 64) raised[dev].store((int)kDecodeSmemMax, std::memory_order_relaxed);
+    if (dev >= 0 && dev < 64) raised[dev].store(true, std::memory_order_release);
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kDecThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, L);
+  *out = kern;
+  return cudaSuccess;
 }
 
 int64_t decode_q_stride(int64_t K) { return ((K + 255) / 256) * 256 + 16; }
 
 static int64_t round128(int64_t v) { return (v + 127) / 128 * 128; }
 
-static int64_t tile_bytes_max(int64_t K) { return round128(16 * (K / 4)); }
-
-// Shared-memory plan of a launch: ring bytes and total, or false when the
-// calls do not fit (then they take the tensor-core path).
-// q_total includes the RMSNorm mode's exact-sum bins, which follow the codes.
-static bool decode_plan(int64_t q_total, int64_t tile_max, int MT, int64_t* ring, int64_t* total) {
-  const int64_t fixed = dec_fixed_bytes(MT);
-  // Two CTAs per SM when three tiles fit beside the codes (a launch's CTAs
-  // then leave room on every SM for the next launch's), else one.
-  const int64_t budgets[2] = {kDecodeSmemShared, kDecodeSmemMax};
-  const int64_t want_tiles[2] = {3, 2};
-  for (int b = 0; b < 2; ++b) {
-    const int64_t r = (budgets[b] - q_total - fixed) / 128 * 128;
-    if (r >= want_tiles[b] * tile_max) {
-      *ring = r;
-      *total = r + q_total + fixed;
-      return true;
-    }
-  }
-  return false;
+// Shared-memory bytes of a launch (q_total includes the RMSNorm mode's
+// exact-sum bins, which follow the codes), or -1 when it does not fit.
+static int64_t decode_smem(int64_t q_total, int MT) {
+  const int64_t stages = (int64_t)kDecWarps * kDecStages * dec_stage_bytes<dec_upt<1>()>();
+  const int64_t total = stages + q_total + dec_fixed_bytes(MT);
+  return total <= kDecodeSmemMax ? total : -1;
 }
 
 bool decode_group_fits(const DecCall* calls, int n) {
   if (n < 1 || n > kDecodeMaxGroup) return false;
-  int64_t q = 0, tmax = 0, maxM = 0;
+  int64_t q = 0, maxM = 0;
   for (int i = 0; i < n; ++i) {
     if (calls[i].M < 1 || calls[i].M > kDecodeMaxM) return false;
     q += round128(calls[i].M * decode_q_stride(calls[i].K));
-    const int64_t tb = tile_bytes_max(calls[i].K);
-    tmax = tb > tmax ? tb : tmax;
     maxM = calls[i].M > maxM ? calls[i].M : maxM;
   }
-  int64_t ring = 0, total = 0;
-  return decode_plan(q, tmax, maxM <= 8 ? 1 : 2, &ring, &total);
+  return decode_smem(q, maxM <= 8 ? 1 : 2) >= 0;
 }
 
 bool decode_fits(int64_t M, int64_t K, bool rms) {
   if (M < 1 || M > kDecodeMaxM) return false;
-  int64_t ring = 0, total = 0;
   const int64_t q = round128(M * decode_q_stride(K)) + (rms ? kRmsBins * 8 : 0);
-  return decode_plan(q, tile_bytes_max(K), M <= 8 ? 1 : 2, &ring, &total);
+  return decode_smem(q, M <= 8 ? 1 : 2) >= 0;
 }
 
-// Bytes of launch tile gt (rows x K/4, rounded up to 128).
+// Bytes of launch tile gt (rows x K/4).
 static int64_t host_tile_bytes(const DecLaunch& L, int gt) {
   int p = 0;
   while (p + 1 < L.nprob && gt >= L.pr[p + 1].tile0) ++p;
   const DecProblem& P = L.pr[p];
   const int64_t row0 = (int64_t)(gt - P.tile0) * 16;
   const int64_t rows = P.N - row0 < 16 ? P.N - row0 : 16;
-  return round128(rows * P.wpr * 4);
+  return rows * P.wpr * 4;
 }
 
 // Split the launch's tiles into `grid` contiguous ranges of about equal bytes,
@@ -851,9 +1023,10 @@ cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g
   if ((input == kDecRms || input == kDecPrepared) && n != 1) return cudaErrorInvalidValue;
   DecLaunch L;
   std::memset(&L, 0, sizeof(L));
-  int64_t maxM = 0, q = 0, tmax = 0;
+  int64_t maxM = 0, q = 0;
   int tiles = 0;
   for (int i = 0; i < n; ++i) {
+    if (calls[i].M < 1 || calls[i].M > kDecodeMaxM || calls[i].N < 1) return cudaErrorInvalidValue;
     DecProblem& P = L.pr[i];
     P.x = calls[i].x;
     P.sx_in = calls[i].sx;
@@ -874,40 +1047,24 @@ cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g
     q += round128((int64_t)P.M * P.q_stride);
     tiles += P.tiles;
     maxM = calls[i].M > maxM ? calls[i].M : maxM;
-    const int64_t tb = tile_bytes_max(calls[i].K);
-    tmax = tb > tmax ? tb : tmax;
-    if (calls[i].M < 1 || calls[i].M > kDecodeMaxM || calls[i].N < 1) return cudaErrorInvalidValue;
   }
   const int MT = maxM <= 8 ? 1 : 2;
   if (input == kDecRms) q += kRmsBins * 8;  // exact-sum bins after the codes
-  int64_t ring = 0, total = 0;
-  if (!decode_plan(q, tmax, MT, &ring, &total)) return cudaErrorInvalidValue;
+  const int64_t smem = decode_smem(q, MT);
+  if (smem < 0) return cudaErrorInvalidValue;
   L.nprob = n;
   L.total_tiles = tiles;
-  L.ring_bytes = (int)ring;
   L.q_bytes = (int)q;
   L.err = err;
   L.g = g;
   L.eps = eps;
-  int grid = tiles < num_sms ? tiles : num_sms;
-  if (grid > kDecMaxGrid) grid = kDecMaxGrid;
-  partition_by_bytes(L, grid);
-  // Units per task: about eight tasks per warp-sized share of a CTA's tiles
-  // for short launches (latency), up to kDecMaxUnitsPerTask for long ones.
-  const double tiles_per_cta = (double)tiles / grid;
-  for (int i = 0; i < n; ++i) {
-    DecProblem& P = L.pr[i];
-    int upt = (int)((P.nu * tiles_per_cta + kDecConsumerWarps - 1) / kDecConsumerWarps);
-    upt = upt < 1 ? 1 : (upt > kDecMaxUnitsPerTask ? kDecMaxUnitsPerTask : upt);
-    if (upt > P.nu) upt = P.nu;
-    P.upt = upt;
-    P.nchunk = (P.nu + upt - 1) / upt;
-  }
   const bool accout = calls[0].acc != nullptr;
   for (int i = 1; i < n; ++i)
     if ((calls[i].acc != nullptr) != accout) return cudaErrorInvalidValue;  // one output kind per launch
+  DecKernel kern = nullptr;
+  cudaError_t e = cudaErrorInvalidValue;
 #define BL_DEC(MTV, AO, XM) \
-  if (MT == MTV && accout == AO && input == XM) return launch_decode_t<MTV, AO, XM>(L, grid, (size_t)total, pdl, stream);
+  if (MT == MTV && accout == AO && input == XM) e = decode_kernel<MTV, AO, XM>(&kern);
   BL_DEC(1, false, kDecF32)
   BL_DEC(1, true, kDecF32)
   BL_DEC(2, false, kDecF32)
@@ -921,7 +1078,45 @@ cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g
   BL_DEC(1, false, kDecRms)
   BL_DEC(2, false, kDecRms)
 #undef BL_DEC
-  return cudaErrorInvalidValue;
+  if (e != cudaSuccess) return e;
+  // One CTA per SM leaves room on every SM for a CTA of the next launch
+  // (programmatic dependent launch). Long streams launched without it take
+  // as many CTAs per SM as fit (more copies in flight).
+  int per_sm = 1;
+  if (!pdl && tiles >= 8 * num_sms) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, (size_t)smem);
+    if (e != cudaSuccess) return e;
+    per_sm = per_sm < 1 ? 1 : (per_sm > 3 ? 3 : per_sm);
+  }
+  int grid = per_sm * num_sms;
+  if (grid > tiles) grid = tiles;
+  if (grid > kDecMaxGrid) grid = kDecMaxGrid;
+  partition_by_bytes(L, grid);
+  // Tasks: whole tiles when every warp gets two or more of them (a warp then
+  // writes its tiles' outputs itself); otherwise chunks of about
+  // nu * tiles_per_cta / 8 units, so that all 8 warps share a short launch.
+  const double tiles_per_cta = (double)tiles / grid;
+  for (int i = 0; i < n; ++i) {
+    DecProblem& P = L.pr[i];
+    int upt = P.nu;
+    if (tiles_per_cta < 2.0 * kDecWarps) {
+      upt = (int)((P.nu * tiles_per_cta + kDecWarps - 1) / kDecWarps);
+      upt = upt < 1 ? 1 : (upt > P.nu ? P.nu : upt);
+    }
+    P.upt = upt;
+    P.nchunk = (P.nu + upt - 1) / upt;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, L);
 }
 
 }  // namespace bl

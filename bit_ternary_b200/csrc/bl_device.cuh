@@ -102,6 +102,41 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// As mbar_try_wait, but a thread whose phase is not complete is suspended
+// until it completes or `suspend_ns` elapses, instead of returning at once:
+// waiting warps then take no issue slots from the warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// mbar_wait with suspended waiting (the abort flag and the time limit are
+// checked each time the suspension ends).
+constexpr uint32_t kSuspendNs = 50000;  // 50 us: a waiting warp wakes at the phase or after this
+
+__device__ __forceinline__ bool mbar_wait_suspend(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                  uint32_t* err_word, uint32_t code,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity, kSuspendNs)) return true;
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) {
+      if (abort_flag != nullptr) *abort_flag = 1;
+      if (err_word != nullptr) atomicCAS(err_word, 0u, code);
+      return false;
+    }
+  }
+}
+
 // ----------------------------------------------------------------- TMA ---
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");

@@ -424,7 +424,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ------------------------------------------------------------------ host --
-static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -451,7 +451,7 @@ cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                         int32_t* acc_out, void* ws, cudaStream_t stream, int num_sms) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   int8_t* q = reinterpret_cast<int8_t*>(base + ws_q_off(M));
-  PFN_cuTensorMapEncodeTiled_v12000 encode = get_encode_fn();
+  PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
   CUtensorMap tmap_q, tmap_out;
   {

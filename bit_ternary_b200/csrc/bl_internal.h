@@ -7,6 +7,8 @@
 
 #include "bl_device.cuh"
 
+#include <cudaTypedefs.h>
+
 namespace bl {
 
 // Pack workspace: header (status word at 0, mean_c and s at 16/20) + bins:
@@ -60,6 +62,9 @@ bool decode_group_fits(const DecCall* calls, int n);
 // after it). err: the workspace error word, cleared by the launch.
 cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g, float eps, uint32_t* err, bool pdl,
                           cudaStream_t stream, int num_sms);
+
+// The driver's cuTensorMapEncodeTiled (looked up once), or nullptr.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // W is fp32, or bf16 bit patterns when bf16 (widened exactly).
 cudaError_t launch_pack(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
