@@ -39,12 +39,15 @@
 // set per class, recombined exactly as acc0 + acc1/4 + acc2/16 + acc3/64, gives
 // sum q*(code+1); subtracting sum q gives the signed result.
 //
-// Activations in shared memory. A token's codes are stored per 256-code unit;
-// inside a unit, the 16 bytes of word w = 4t + 2h + j (codes 16w..16w+15, in
-// the private order where position 4c+b holds column 4b+c) sit at byte
-// 128h + 32t + 16j. Lane (g, t) then reads its 32 bytes of half h at 128h + 32t:
-// the four lanes of a token cover 128 distinct bytes, and the row stride of
-// 16 (mod 128) bytes moves the next token onto the other banks.
+// Activations in shared memory. A token's codes are stored per 256-code unit.
+// Word w = 4t + 2h + j of a unit (codes 16w..16w+15) splits into four class
+// words: class c holds the codes of columns {c, 4+c, 8+c, 12+c}, the order in
+// which a masked weight word presents them. Inside the 32-byte chunk
+// 128h + 32t, class c of word j sits at 8c + 4j, so one 16-byte load gives the
+// B operands (words 2h and 2h+1) of two classes as aligned register pairs.
+// Lane (g, t) reads its 32 bytes of half h at 128h + 32t: the four lanes of a
+// token cover 128 distinct bytes, and the row stride of 16 (mod 128) bytes
+// moves the next token onto the other banks.
 #include "bl_internal.h"
 
 #include <atomic>
@@ -139,12 +142,24 @@ __device__ __forceinline__ int dec_problem_of(const DecLaunch& L, int gt) {
   return p;
 }
 
-// Byte offset, inside a unit, of the 16 codes of word w (see the file header).
-__device__ __forceinline__ int dec_group_slot(int w) { return 128 * ((w >> 1) & 1) + 32 * (w >> 2) + 16 * (w & 1); }
+// Byte offset, inside a unit, of the codes of word w = 4t + 2h + j (see the
+// file header): the 32-byte chunk 128h + 32t, where class c of word j (its
+// 4 codes for columns {c, 4+c, 8+c, 12+c}) sits at 8c + 4j.
+__device__ __forceinline__ int dec_group_slot(int w) { return 128 * ((w >> 1) & 1) + 32 * (w >> 2) + 4 * (w & 1); }
 
-// Shared-memory address of the 16 codes of group gi (columns 16gi..16gi+15) of token m.
+// Shared-memory address of the codes of group gi (columns 16gi..16gi+15) of
+// token m; its class c word goes to this address + 8c.
 __device__ __forceinline__ uint8_t* dec_q_group(uint8_t* sq, const DecProblem& P, int m, int gi) {
   return sq + P.q_off + m * P.q_stride + 256 * (gi >> 4) + dec_group_slot(gi & 15);
+}
+
+// Store a group's four class words (w[c]: the codes of columns {c, 4+c, 8+c,
+// 12+c}) at dec_q_group's address.
+__device__ __forceinline__ void dec_store_group(uint8_t* dst, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+  *reinterpret_cast<uint32_t*>(dst) = w0;
+  *reinterpret_cast<uint32_t*>(dst + 8) = w1;
+  *reinterpret_cast<uint32_t*>(dst + 16) = w2;
+  *reinterpret_cast<uint32_t*>(dst + 24) = w3;
 }
 
 // Warp-aggregated shared atomics on per-token state; tok < 0 marks an idle
@@ -192,7 +207,7 @@ __device__ __forceinline__ int dec_quant_group(const float4 (&f)[4], float sx, u
   for (int r = 0; r < 4; ++r)
     w[r] = (uint32_t)(q[0][r] & 0xFF) | ((uint32_t)(q[1][r] & 0xFF) << 8) | ((uint32_t)(q[2][r] & 0xFF) << 16) |
            ((uint32_t)(q[3][r] & 0xFF) << 24);
-  *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  dec_store_group(dst, w[0], w[1], w[2], w[3]);
   return sum;
 }
 
@@ -233,10 +248,13 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// Bytes of one pipeline stage of a warp: per unit, 512 bytes of row-g words
-// and 512 of row-(g+8) words (16 per lane), then two row scales per lane.
+// One pipeline stage of a warp holds a group's 16 rows, UPT * 64 bytes each,
+// at a row stride of UPT * 64 + 64 bytes (rows g and g+1, read by the same
+// quarter-warp, then fall on different banks), then two row scales per lane.
 template <int UPT>
-__host__ __device__ constexpr int dec_stage_bytes() { return UPT * 1024 + 256; }
+__host__ __device__ constexpr int dec_row_stride() { return UPT * 64 + 64; }
+template <int UPT>
+__host__ __device__ constexpr int dec_stage_bytes() { return 16 * dec_row_stride<UPT>() + 256; }
 
 // A warp's position in its work: tasks warp, warp + 8, warp + 16, ... in
 // (tile, chunk) order (chunk j of the CTA's tile i, in problem p), each task
@@ -253,12 +271,12 @@ struct DecCursor {
   const float* D;
   int wpr, N, tile0, upt, nu, q_off;
   // the current task
-  const uint32_t* rowa;  // row g, word 16*u + 4t of the next unit u
-  int w0;                // word 16*u + 4t
-  int left;              // units of the task not yet issued
-  int qoff;              // activation offset of unit u (token 0)
-  int row0;
-  bool aon, bon, fast, first;
+  const uint32_t* src;  // the lane's first copy source: row lane / CPR, chunk lane % CPR of unit u
+  int w0;               // word of that chunk in its row: 16*u + 4*(lane % CPR)
+  int left;             // units of the task not yet issued
+  int qoff;             // activation offset of unit u (token 0)
+  int row0, rv;
+  bool first;
 
   __device__ __forceinline__ void load_problem(const DecLaunch& L, int t0) {
     const DecProblem& P = L.pr[p];
@@ -292,22 +310,23 @@ struct DecCursor {
     }
   }
   // Set up the task at (i, j).
+  // Copies: a group's 16 rows x (4 * UPT) 16-byte chunks are spread over the
+  // lanes so that one copy instruction covers whole rows (full 128-byte
+  // lines): chunk lane + 32m is row m * RPM + lane / CPR, chunk lane % CPR.
+  static constexpr int CPR = 4 * UPT;  // chunks per row
+  static constexpr int RPM = 32 / CPR;  // rows per copy instruction
   __device__ __forceinline__ void open(int t0, int nt, int lane) {
     valid = i < nt;
     if (!valid) return;
-    const int g = lane >> 2, t = lane & 3;
     row0 = (t0 + i - tile0) * 16;
-    const int rv = N - row0 < 16 ? N - row0 : 16;
+    rv = N - row0 < 16 ? N - row0 : 16;
     const int ua = j * upt;
     const int ue = ua + upt < nu ? ua + upt : nu;
-    w0 = 16 * ua + 4 * t;
-    rowa = packed + (int64_t)(row0 + g) * wpr + w0;
+    w0 = 16 * ua + 4 * (lane % CPR);
+    src = packed + (int64_t)(row0 + lane / CPR) * wpr + w0;
     qoff = q_off + 256 * ua;
     left = ue - ua;
     first = true;
-    aon = g < rv;
-    bon = g + 8 < rv;
-    fast = rv == 16 && (wpr & 3) == 0 && 16 * ue <= wpr;
   }
   __device__ __forceinline__ void init(const DecLaunch& L, int t0, int nt, int warp, int lane) {
     p = dec_problem_of(L, t0);
@@ -319,11 +338,11 @@ struct DecCursor {
   }
   // Start the copies of the next group into `stage` and return what its
   // contraction needs (valid() == false past the warp's last task; nothing
-  // is copied then, but the caller still commits a copy group). Each lane
-  // copies exactly the words it contracts: words 4t..4t+3 of rows g and g+8
-  // of every unit; rows past N and words past the row are zero-filled. A
+  // is copied then, but the caller still commits a copy group). Rows past N
+  // and words past the row (or past the group's units) are zero-filled. A
   // group that opens its task also brings row scales: D[row0 + lane] (lanes
   // 0..15, chunked tiles) or D[row0 + g] and D[row0 + g + 8] (whole tiles).
+  // The copies land only for this lane: the warp synchronises before reading.
   __device__ __forceinline__ DecRun issue(const DecLaunch& L, int t0, int nt, uint8_t* stage, int lane) {
     DecRun r;
     r.pad = 0;
@@ -331,48 +350,41 @@ struct DecCursor {
       r.qoff = r.i = r.meta = 0;
       return r;
     }
+    constexpr int RS = dec_row_stride<UPT>();
     const int n = left < UPT ? left : UPT;
-    uint8_t* da = stage + 16 * lane;
-    const uint32_t* rowb = rowa + (int64_t)8 * wpr;
-    if (fast) {
+    const int lr = lane / CPR, lc = lane % CPR;
+    uint8_t* dst = stage + lr * RS + 16 * lc;
+    const int64_t rstep = (int64_t)RPM * wpr;  // words between a lane's rows
+    if (rv == 16 && n == UPT && (wpr & 3) == 0 && w0 - 4 * lc + 16 * UPT <= wpr) {
+      // Every row present and every unit whole.
 #pragma unroll
-      for (int k = 0; k < UPT; ++k)
-        if (k < n) {
-          cp_async16(da + 1024 * k, rowa + 16 * k);
-          cp_async16(da + 1024 * k + 512, rowb + 16 * k);
-        }
+      for (int m = 0; m < 16 / RPM; ++m) cp_async16(dst + m * RPM * RS, src + m * rstep);
     } else if ((wpr & 3) == 0) {
-      // Rows start 16-byte aligned; a 4-word group is wholly in the row or past it.
+      // Rows start 16-byte aligned; a chunk is wholly in the row or past it.
 #pragma unroll
-      for (int k = 0; k < UPT; ++k)
-        if (k < n) {
-          const bool in = w0 + 16 * k < wpr;
-          cp_async16_zfill(da + 1024 * k, in && aon ? rowa + 16 * k : packed, in && aon ? 16u : 0u);
-          cp_async16_zfill(da + 1024 * k + 512, in && bon ? rowb + 16 * k : packed, in && bon ? 16u : 0u);
-        }
+      for (int m = 0; m < 16 / RPM; ++m) {
+        const bool in = m * RPM + lr < rv && lc < 4 * n && w0 < wpr;
+        cp_async16_zfill(dst + m * RPM * RS, in ? src + m * rstep : packed, in ? 16u : 0u);
+      }
     } else {
       // Rows not 16-byte aligned: 4-byte copies.
 #pragma unroll
-      for (int k = 0; k < UPT; ++k)
-        if (k < n) {
+      for (int m = 0; m < 16 / RPM; ++m)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const bool in = w0 + 16 * k + e < wpr;
-            cp_async4_zfill(da + 1024 * k + 4 * e, in && aon ? rowa + 16 * k + e : packed, in && aon ? 4u : 0u);
-            cp_async4_zfill(da + 1024 * k + 512 + 4 * e, in && bon ? rowb + 16 * k + e : packed,
-                            in && bon ? 4u : 0u);
-          }
+        for (int e = 0; e < 4; ++e) {
+          const bool in = m * RPM + lr < rv && lc < 4 * n && w0 + e < wpr;
+          cp_async4_zfill(dst + m * RPM * RS + 4 * e, in ? src + m * rstep + e : packed, in ? 4u : 0u);
         }
     }
     if (!kAccOut && first) {
       const int g = lane >> 2;
-      float* dd = reinterpret_cast<float*>(stage + UPT * 1024) + 2 * lane;
+      float* dd = reinterpret_cast<float*>(stage + 16 * RS) + 2 * lane;
       if (C > 1) {
         const bool in = j == 0 && lane < 16 && row0 + lane < N;
         cp_async4_zfill(dd, in ? D + row0 + lane : D, in ? 4u : 0u);
       } else {
-        cp_async4_zfill(dd, aon ? D + row0 + g : D, aon ? 4u : 0u);
-        cp_async4_zfill(dd + 1, bon ? D + row0 + g + 8 : D, bon ? 4u : 0u);
+        cp_async4_zfill(dd, g < rv ? D + row0 + g : D, g < rv ? 4u : 0u);
+        cp_async4_zfill(dd + 1, g + 8 < rv ? D + row0 + g + 8 : D, g + 8 < rv ? 4u : 0u);
       }
     }
     const bool last = left == n;
@@ -386,7 +398,7 @@ struct DecCursor {
     } else {
       left -= n;
       first = false;
-      rowa += 16 * n;
+      src += 16 * n;
       w0 += 16 * n;
       qoff += 256 * n;
     }
@@ -508,7 +520,7 @@ __device__ void dec_load_prepared(const DecLaunch& L, const DecGroups& G, uint8_
     G.locate(L, gg, p, m, gi);
     const DecProblem& P = L.pr[p];
     const uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const int8_t*>(P.x) + (int64_t)m * P.K) + gi);
-    *reinterpret_cast<uint4*>(dec_q_group(sq, P, m, gi)) = v;
+    dec_store_group(dec_q_group(sq, P, m, gi), v.x, v.y, v.z, v.w);
   }
   for (int i = tid; i < G.np * 16; i += kDecThreads) {
     const int p = G.pa + (i >> 4), m = i & 15;
@@ -698,6 +710,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
   // the grid this launch waits for.
   constexpr int S = kDecStages;
   constexpr int SB = dec_stage_bytes<UPT>();
+  constexpr int RS = dec_row_stride<UPT>();
   uint8_t* wstage = stages + (size_t)warp * S * SB;  // this warp's S stages
   DecCursor<UPT, kAccOut> cur;
   cur.init(L, t0, nt, warp, lane);
@@ -779,7 +792,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
     } T{Gr.p(), Gr.i, Gr.j()};
     const DecProblem& P = L.pr[T.p];
     if (!kAccOut && Gr.first()) {
-      const float2 dd = *reinterpret_cast<const float2*>(stage + UPT * 1024 + 8 * lane);
+      const float2 dd = *reinterpret_cast<const float2*>(stage + 16 * RS + 8 * lane);
       dg0 = dd.x;
       dg1 = dd.y;
     }
@@ -799,8 +812,8 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
 #pragma unroll
     for (int k = 0; k < UPT; ++k) {
       if (k < Gr.n()) {
-        const uint4 va = *reinterpret_cast<const uint4*>(stage + 1024 * k + 16 * lane);
-        const uint4 vb = *reinterpret_cast<const uint4*>(stage + 1024 * k + 512 + 16 * lane);
+        const uint4 va = *reinterpret_cast<const uint4*>(stage + g * RS + 64 * k + 16 * t);
+        const uint4 vb = *reinterpret_cast<const uint4*>(stage + (g + 8) * RS + 64 * k + 16 * t);
         const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
         const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
@@ -819,8 +832,9 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
             const uint32_t a1 = wb[2 * h] & mask, a3 = wb[2 * h + 1] & mask;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-              const uint32_t b0 = cc == 0 ? Q[mt][0].x : (cc == 1 ? Q[mt][0].y : (cc == 2 ? Q[mt][0].z : Q[mt][0].w));
-              const uint32_t b1 = cc == 0 ? Q[mt][1].x : (cc == 1 ? Q[mt][1].y : (cc == 2 ? Q[mt][1].z : Q[mt][1].w));
+              // class cc of words 2h (b0) and 2h+1 (b1): an aligned register pair
+              const uint32_t b0 = cc == 0 ? Q[mt][0].x : (cc == 1 ? Q[mt][0].z : (cc == 2 ? Q[mt][1].x : Q[mt][1].z));
+              const uint32_t b1 = cc == 0 ? Q[mt][0].y : (cc == 1 ? Q[mt][0].w : (cc == 2 ? Q[mt][1].y : Q[mt][1].w));
               dec_mma(acc[cc][mt], a0, a1, a2, a3, b0, b1);
             }
           }
@@ -930,6 +944,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
     rec[sti] = cur.issue(L, t0, nt, wstage + sti * SB, lane);
     cp_async_commit();
     cp_async_wait<S - 1>();
+    __syncwarp();  // every lane's copies of this stage have landed
     const DecRun R = rec[st];
     if (!R.valid() || !run(R, wstage + st * SB)) break;
     st = st + 1 == S ? 0 : st + 1;
