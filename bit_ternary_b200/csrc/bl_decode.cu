@@ -1,8 +1,8 @@
 // bl_decode.cu - decode BitLinear (M <= 16 tokens) for one or several
 // independent BitLinears per launch: ActQuant (or RMSNorm + ActQuant) of the
 // activations inside every CTA, the packed ternary weights streamed once from
-// HBM straight into registers, an exact int32 contraction and the fp32 rescale
-// in the epilogue.
+// HBM through per-warp shared-memory stages, an exact int32 contraction and
+// the fp32 rescale in the epilogue.
 //
 // The operation is the BitLinear product of "Core AI model zoo - BitVLA",
 // section 2 (M=1 decode, arbitrary K with K % 16 == 0, any N, per-row scale
@@ -10,21 +10,23 @@
 //
 // Streaming. The packed weights are the only large stream (2 bits per weight).
 // Work is cut into tiles of 16 consecutive rows, and a tile into tasks: the
-// whole tile when every warp of a CTA gets two or more tiles, else chunks of a
-// few 256-code units so that all warps share a short launch (chunk j of tile i
-// is one task). Every CTA owns a contiguous, byte-balanced range of tiles over
-// all problems of the launch; its 8 warps take every 8th task in (tile, chunk)
-// order, and walk each task in groups of up to 4 units. Each lane copies
-// exactly the words it will contract (words 4t..4t+3 of rows g and g+8 of
-// every unit) with 16-byte cp.async into its warp's own pipeline stages in
-// shared memory, so a warp waits only on its own copies (cp.async.wait_group)
-// and needs no barrier with other warps; the in-flight bytes take no
-// registers. The first groups of every warp are issued before
-// griddepcontrol.wait (weights never depend on the previous kernel), so under
-// programmatic dependent launch a launch's weights stream while the previous
-// launch still runs. (One bulk-copy engine per SM moves only about 20-25 GB/s,
-// far below a B200 SM's share of HBM bandwidth, so the stream goes through the
-// load/store units of all warps instead.)
+// whole tile when every warp of a CTA gets two or more tiles, else chunks of
+// units so that all warps share a short launch (chunk j of tile i is one
+// task). Every CTA owns a contiguous, byte-balanced range of tiles over all
+// problems of the launch; its 8 warps take every 8th task in (tile, chunk)
+// order, and walk each task in groups of up to 4 256-code units. A warp
+// copies each group (16 rows x 256 bytes) with 16-byte cp.async into one of
+// its two shared-memory stages, each copy instruction covering whole
+// 128-byte lines, and contracts one stage while the next group lands; it
+// waits only on its own copies (cp.async.wait_group + __syncwarp). The copies
+// carry an L2 evict-first policy: the weights are read once. The first group
+// of every warp is issued before griddepcontrol.wait (weights never depend on
+// the previous kernel), so under programmatic dependent launch a launch's
+// weights stream while the previous launch still runs; without that
+// dependency the activations are loaded first, ahead of the weight stream.
+// (One bulk-copy engine per SM moves only about 20-25 GB/s, far below a
+// B200 SM's share of HBM bandwidth, so the stream goes through the load/store
+// units of all warps instead.)
 //
 // Accumulation. A chunk's partial sums go to its tile's block in shared
 // memory (one of 16 slots, by tile index) with shared atomics: exact integers,
@@ -89,27 +91,34 @@ struct DecProblem {
   int q_stride;  // bytes per token row there (K rounded up to 256, + 16)
 };
 
-struct DecLaunch {
+// The launch's problems and common arguments.
+struct DecHead {
   DecProblem pr[kDecodeMaxGroup];
   const float* g;  // RMSNorm mode: norm weight [K] (one problem per launch)
   float eps;
   int nprob;
   int total_tiles;
   int q_bytes;
+  int pdl;       // launched as a programmatic dependent of the previous work in the stream
+  int acc_cols;  // token columns of a slot's partial-sum block: the largest M
   uint32_t* err;
+};
+
+struct DecLaunch {
+  DecHead h;
   int cta_start[kDecMaxGrid + 1];  // CTA c owns launch tiles [cta_start[c], cta_start[c+1])
 };
 
 // Shared memory past the activation codes.
-__host__ __device__ constexpr int dec_fixed_bytes(int MT) {
+__host__ __device__ constexpr int dec_fixed_bytes(int acc_cols, int S) {
   return kDecTok * 8                     // s_inv
-         + kDecodeSlots * 16 * 8 * MT * 4  // s_acc
+         + kDecodeSlots * 16 * acc_cols * 4  // s_acc
          + kDecodeSlots * 16 * 4         // s_D
          + 3 * kDecTok * 4               // s_sx, s_rs, s_amax
          + 2 * kDecodeSlots * 4          // s_cnt, s_gen
          + 16 * (8 + 4 + 4)              // RMSNorm: sums of squares, mean squares, flags
          + 64                            // abort flag
-         + kDecWarps * kDecStages * 16;  // records of the groups in flight
+         + kDecWarps * S * 16;  // records of the groups in flight
 }
 
 __device__ __forceinline__ void dec_mma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -135,7 +144,7 @@ __device__ __forceinline__ void prefetch_l2(const void* p) {
 // Barrier of the CTA's 8 warps (named, so that its count is explicit).
 __device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kDecThreads) : "memory"); }
 
-__device__ __forceinline__ int dec_problem_of(const DecLaunch& L, int gt) {
+__device__ __forceinline__ int dec_problem_of(const DecHead& L, int gt) {
   int p = 0;
 #pragma unroll 1
   while (p + 1 < L.nprob && gt >= L.pr[p + 1].tile0) ++p;
@@ -237,6 +246,22 @@ __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(__cvta_generic_to_global(src))
                : "memory");
 }
+// The same with an L2 cache policy (the streamed weights are read once).
+__device__ __forceinline__ void cp_async16_zfill_pol(void* dst, const void* src, uint32_t src_bytes, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(smem_u32(dst)),
+               "l"(__cvta_generic_to_global(src)), "r"(src_bytes), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async16_pol(void* dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)),
+               "l"(__cvta_generic_to_global(src)), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
 __device__ __forceinline__ void cp_async4_zfill(void* dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)),
                "l"(__cvta_generic_to_global(src)), "r"(src_bytes)
@@ -248,13 +273,20 @@ __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-// One pipeline stage of a warp holds a group's 16 rows, UPT * 64 bytes each,
-// at a row stride of UPT * 64 + 64 bytes (rows g and g+1, read by the same
-// quarter-warp, then fall on different banks), then two row scales per lane.
+// One pipeline stage of a warp holds a group's 16 rows, UPT * 64 bytes each
+// and unpadded, then two row scales per lane. Lanes (g, t) and (g + 1, t) read
+// in the same quarter-warp, so rows g and g + 1 must use different halves of
+// the 128-byte bank window: with an even UPT (row stride 0 mod 128) the
+// 64-byte halves of every odd row are swapped (16-byte chunk c is stored at
+// position c ^ 4); with an odd UPT the stride alone offsets them.
 template <int UPT>
-__host__ __device__ constexpr int dec_row_stride() { return UPT * 64 + 64; }
+__host__ __device__ constexpr int dec_row_stride() { return UPT * 64; }
 template <int UPT>
 __host__ __device__ constexpr int dec_stage_bytes() { return 16 * dec_row_stride<UPT>() + 256; }
+template <int UPT>
+__device__ __forceinline__ int dec_chunk_pos(int row, int chunk) {
+  return (UPT & 1) ? chunk : chunk ^ (4 * (row & 1));
+}
 
 // A warp's position in its work: tasks warp, warp + 8, warp + 16, ... in
 // (tile, chunk) order (chunk j of the CTA's tile i, in problem p), each task
@@ -274,11 +306,12 @@ struct DecCursor {
   const uint32_t* src;  // the lane's first copy source: row lane / CPR, chunk lane % CPR of unit u
   int w0;               // word of that chunk in its row: 16*u + 4*(lane % CPR)
   int left;             // units of the task not yet issued
+  uint64_t pol;         // L2 policy of the weight copies: evict first
   int qoff;             // activation offset of unit u (token 0)
   int row0, rv;
   bool first;
 
-  __device__ __forceinline__ void load_problem(const DecLaunch& L, int t0) {
+  __device__ __forceinline__ void load_problem(const DecHead& L, int t0) {
     const DecProblem& P = L.pr[p];
     packed = P.packed;
     D = P.D;
@@ -293,7 +326,7 @@ struct DecCursor {
   }
   // Move (i, j) onto a task: whole tiles are skipped at once, one problem at
   // a time.
-  __device__ __forceinline__ void normalise(const DecLaunch& L, int t0, int nt) {
+  __device__ __forceinline__ void normalise(const DecHead& L, int t0, int nt) {
     while (j >= C && i < nt) {
       const int adv = C == 1 ? j : j / C;
       if (i + adv < pend) {
@@ -315,6 +348,7 @@ struct DecCursor {
   // lines): chunk lane + 32m is row m * RPM + lane / CPR, chunk lane % CPR.
   static constexpr int CPR = 4 * UPT;  // chunks per row
   static constexpr int RPM = 32 / CPR;  // rows per copy instruction
+  static_assert(32 % CPR == 0 && 16 % RPM == 0, "a copy instruction covers whole rows");
   __device__ __forceinline__ void open(int t0, int nt, int lane) {
     valid = i < nt;
     if (!valid) return;
@@ -328,9 +362,10 @@ struct DecCursor {
     left = ue - ua;
     first = true;
   }
-  __device__ __forceinline__ void init(const DecLaunch& L, int t0, int nt, int warp, int lane) {
+  __device__ __forceinline__ void init(const DecHead& L, int t0, int nt, int warp, int lane) {
     p = dec_problem_of(L, t0);
     load_problem(L, t0);
+    pol = l2_policy_evict_first();
     i = 0;
     j = warp;
     normalise(L, t0, nt);
@@ -343,7 +378,7 @@ struct DecCursor {
   // group that opens its task also brings row scales: D[row0 + lane] (lanes
   // 0..15, chunked tiles) or D[row0 + g] and D[row0 + g + 8] (whole tiles).
   // The copies land only for this lane: the warp synchronises before reading.
-  __device__ __forceinline__ DecRun issue(const DecLaunch& L, int t0, int nt, uint8_t* stage, int lane) {
+  __device__ __forceinline__ DecRun issue(const DecHead& L, int t0, int nt, uint8_t* stage, int lane) {
     DecRun r;
     r.pad = 0;
     if (!valid) {
@@ -353,18 +388,19 @@ struct DecCursor {
     constexpr int RS = dec_row_stride<UPT>();
     const int n = left < UPT ? left : UPT;
     const int lr = lane / CPR, lc = lane % CPR;
-    uint8_t* dst = stage + lr * RS + 16 * lc;
+    // destination of the lane's chunk in row m * RPM + lr
+    auto dst = [&](int m) { return stage + (m * RPM + lr) * RS + 16 * dec_chunk_pos<UPT>(m * RPM + lr, lc); };
     const int64_t rstep = (int64_t)RPM * wpr;  // words between a lane's rows
     if (rv == 16 && n == UPT && (wpr & 3) == 0 && w0 - 4 * lc + 16 * UPT <= wpr) {
       // Every row present and every unit whole.
 #pragma unroll
-      for (int m = 0; m < 16 / RPM; ++m) cp_async16(dst + m * RPM * RS, src + m * rstep);
+      for (int m = 0; m < 16 / RPM; ++m) cp_async16_pol(dst(m), src + m * rstep, pol);
     } else if ((wpr & 3) == 0) {
       // Rows start 16-byte aligned; a chunk is wholly in the row or past it.
 #pragma unroll
       for (int m = 0; m < 16 / RPM; ++m) {
         const bool in = m * RPM + lr < rv && lc < 4 * n && w0 < wpr;
-        cp_async16_zfill(dst + m * RPM * RS, in ? src + m * rstep : packed, in ? 16u : 0u);
+        cp_async16_zfill_pol(dst(m), in ? src + m * rstep : packed, in ? 16u : 0u, pol);
       }
     } else {
       // Rows not 16-byte aligned: 4-byte copies.
@@ -373,7 +409,7 @@ struct DecCursor {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const bool in = m * RPM + lr < rv && lc < 4 * n && w0 + e < wpr;
-          cp_async4_zfill(dst + m * RPM * RS + 4 * e, in ? src + m * rstep + e : packed, in ? 4u : 0u);
+          cp_async4_zfill(dst(m) + 4 * e, in ? src + m * rstep + e : packed, in ? 4u : 0u);
         }
     }
     if (!kAccOut && first) {
@@ -411,7 +447,7 @@ struct DecCursor {
 struct DecGroups {
   int pa, np, total;
   int pre[kDecodeMaxGroup + 1];
-  __device__ __forceinline__ void locate(const DecLaunch& L, int gg, int& p, int& m, int& gi) const {
+  __device__ __forceinline__ void locate(const DecHead& L, int gg, int& p, int& m, int& gi) const {
     int k = 0, base = 0;
 #pragma unroll
     for (int i = 1; i < kDecodeMaxGroup; ++i)
@@ -435,13 +471,17 @@ __device__ __forceinline__ void dec_load_group(const DecProblem& P, int m, int g
 }
 
 // ActQuant of every token of the CTA's problems into shared memory (fp32 or
-// bf16 activations): per-token max|x| by shared atomics, then the codes, the
-// scale s_x and the row sums. Run by the 256 consumer threads.
+// bf16 activations), in two parts. dec_quant_load reads the first
+// kDecRegGroups 16-column groups of each thread into registers (a launch
+// without a dependency issues it before any weight copy, so that these loads
+// do not queue behind the weight stream); dec_quant_rest finishes: per-token
+// max|x| by shared atomics, then the codes, s_x, RN64(1/s_x) and the row sums.
+// Groups beyond the registers are read twice (for the maximum, then for the
+// codes), two at a time so that their loads are in flight together. Run by
+// the 256 consumer threads.
 template <int kX>
-__device__ void dec_quantise(const DecLaunch& L, const DecGroups& G, uint8_t* sq, float* s_sx, int32_t* s_rs,
-                             uint32_t* s_amax) {
+__device__ __forceinline__ void dec_quant_load(const DecHead& L, const DecGroups& G, float4 (&f)[kDecRegGroups][4]) {
   const int tid = threadIdx.x;
-  float4 f[kDecRegGroups][4];
 #pragma unroll
   for (int r = 0; r < kDecRegGroups; ++r) {
     const int gg = tid + r * kDecThreads;
@@ -451,6 +491,16 @@ __device__ void dec_quantise(const DecLaunch& L, const DecGroups& G, uint8_t* sq
       dec_load_group<kX>(L.pr[p], m, gi, f[r]);
     }
   }
+}
+
+template <int kX>
+__device__ void dec_quant_rest(const DecHead& L, const DecGroups& G, float4 (&f)[kDecRegGroups][4], uint8_t* sq,
+                               float* s_sx, double* s_inv, int32_t* s_rs, uint32_t* s_amax) {
+  const int tid = threadIdx.x;
+  constexpr int B = 2;  // groups beyond the registers loaded together
+  auto absmax16 = [](const float4 (&v)[4]) {
+    return fmaxf(fmaxf(dec_absmax4(v[0]), dec_absmax4(v[1])), fmaxf(dec_absmax4(v[2]), dec_absmax4(v[3])));
+  };
 #pragma unroll
   for (int r = 0; r < kDecRegGroups; ++r) {
     const int gg = tid + r * kDecThreads;
@@ -460,60 +510,64 @@ __device__ void dec_quantise(const DecLaunch& L, const DecGroups& G, uint8_t* sq
       int p, m, gi;
       G.locate(L, gg, p, m, gi);
       tok = p * 16 + m;
-      a = fmaxf(fmaxf(dec_absmax4(f[r][0]), dec_absmax4(f[r][1])), fmaxf(dec_absmax4(f[r][2]), dec_absmax4(f[r][3])));
+      a = absmax16(f[r]);
     }
     dec_amax(s_amax, tok, a);
   }
-  // Groups beyond the registers: loaded now for the maximum, again for the codes.
-  for (int base = kDecRegGroups * kDecThreads; base < G.total; base += kDecThreads) {
-    const int gg = base + tid;
-    int tok = -1;
-    float a = 0.0f;
-    if (gg < G.total) {
-      int p, m, gi;
-      G.locate(L, gg, p, m, gi);
-      float4 v[4];
-      dec_load_group<kX>(L.pr[p], m, gi, v);
-      tok = p * 16 + m;
-      a = fmaxf(fmaxf(dec_absmax4(v[0]), dec_absmax4(v[1])), fmaxf(dec_absmax4(v[2]), dec_absmax4(v[3])));
+  for (int base = kDecRegGroups * kDecThreads; base < G.total; base += B * kDecThreads) {
+    float4 v[B][4];
+    int tok[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int gg = base + b * kDecThreads + tid;
+      tok[b] = -1;
+      if (gg < G.total) {
+        int p, m, gi;
+        G.locate(L, gg, p, m, gi);
+        dec_load_group<kX>(L.pr[p], m, gi, v[b]);
+        tok[b] = p * 16 + m;
+      }
     }
-    dec_amax(s_amax, tok, a);
+#pragma unroll
+    for (int b = 0; b < B; ++b) dec_amax(s_amax, tok[b], tok[b] >= 0 ? absmax16(v[b]) : 0.0f);
   }
   consumers_sync();  // every token's max|x| is complete
-#pragma unroll
-  for (int r = 0; r < kDecRegGroups; ++r) {
-    const int gg = tid + r * kDecThreads;
+  auto codes = [&](const float4 (&v)[4], int gg) {
     int tok = -1, sum = 0;
     if (gg < G.total) {
       int p, m, gi;
       G.locate(L, gg, p, m, gi);
-      tok = p * 16 + m;
-      const float sx = __fdiv_rn(kQmax, fmaxf(__uint_as_float(s_amax[tok]), kFloor));
-      sum = dec_quant_group(f[r], sx, dec_q_group(sq, L.pr[p], m, gi));
-      if (gi == 0) s_sx[tok] = sx;
-    }
-    dec_rowsum(s_rs, tok, sum);
-  }
-  for (int base = kDecRegGroups * kDecThreads; base < G.total; base += kDecThreads) {
-    const int gg = base + tid;
-    int tok = -1, sum = 0;
-    if (gg < G.total) {
-      int p, m, gi;
-      G.locate(L, gg, p, m, gi);
-      float4 v[4];
-      dec_load_group<kX>(L.pr[p], m, gi, v);
       tok = p * 16 + m;
       const float sx = __fdiv_rn(kQmax, fmaxf(__uint_as_float(s_amax[tok]), kFloor));
       sum = dec_quant_group(v, sx, dec_q_group(sq, L.pr[p], m, gi));
-      if (gi == 0) s_sx[tok] = sx;
+      if (gi == 0) {
+        s_sx[tok] = sx;
+        s_inv[tok] = __drcp_rn((double)sx);
+      }
     }
     dec_rowsum(s_rs, tok, sum);
+  };
+#pragma unroll
+  for (int r = 0; r < kDecRegGroups; ++r) codes(f[r], tid + r * kDecThreads);
+  for (int base = kDecRegGroups * kDecThreads; base < G.total; base += B * kDecThreads) {
+    float4 v[B][4];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int gg = base + b * kDecThreads + tid;
+      if (gg < G.total) {
+        int p, m, gi;
+        G.locate(L, gg, p, m, gi);
+        dec_load_group<kX>(L.pr[p], m, gi, v[b]);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < B; ++b) codes(v[b], base + b * kDecThreads + tid);
   }
 }
 
 // Prepared activations (int8 codes already in the private order, natural
 // group order, row stride K; s_x and row sums): copied into the shared layout.
-__device__ void dec_load_prepared(const DecLaunch& L, const DecGroups& G, uint8_t* sq, float* s_sx, int32_t* s_rs) {
+__device__ void dec_load_prepared(const DecHead& L, const DecGroups& G, uint8_t* sq, float* s_sx, int32_t* s_rs) {
   const int tid = threadIdx.x;
   for (int gg = tid; gg < G.total; gg += kDecThreads) {
     int p, m, gi;
@@ -541,7 +595,7 @@ __device__ void dec_load_prepared(const DecLaunch& L, const DecGroups& G, uint8_
 // ends round to different fp32 values (a rounding boundary inside the
 // interval: a few tokens in a million) the token is summed again exactly in
 // integer bins and divided with one correct rounding.
-__device__ void dec_rms_quantise(const DecLaunch& L, const DecGroups& G, uint8_t* sq, float* s_sx, int32_t* s_rs,
+__device__ void dec_rms_quantise(const DecHead& L, const DecGroups& G, uint8_t* sq, float* s_sx, int32_t* s_rs,
                                  uint32_t* s_amax, double* s_ss, float* s_ms, int* s_flag,
                                  unsigned long long* bins) {
   const int tid = threadIdx.x;
@@ -677,14 +731,16 @@ __device__ void dec_rms_quantise(const DecLaunch& L, const DecGroups& G, uint8_t
 
 
 template <int MT, bool kAccOut, int kX>
-__global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decode_kernel(const __grid_constant__ DecLaunch L) {
+__global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decode_kernel(const __grid_constant__ DecLaunch LP) {
   constexpr int UPT = dec_upt<MT>();
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;                                                      // [warp][stage]
-  uint8_t* sq = smem + kDecWarps * kDecStages * dec_stage_bytes<UPT>();
-  double* s_inv = reinterpret_cast<double*>(sq + L.q_bytes);                   // [problem * 16 + token] RN64(1/s_x)
-  int32_t* s_acc = reinterpret_cast<int32_t*>(s_inv + kDecTok);               // [slot][16 rows][8*MT tokens]
-  float* s_D = reinterpret_cast<float*>(s_acc + kDecodeSlots * 16 * 8 * MT);  // [slot][16]
+  constexpr int S = kDecStages;
+  uint8_t* sq = smem + kDecWarps * S * dec_stage_bytes<UPT>();
+  double* s_inv = reinterpret_cast<double*>(sq + LP.h.q_bytes);                   // [problem * 16 + token] RN64(1/s_x)
+  int32_t* s_acc = reinterpret_cast<int32_t*>(s_inv + kDecTok);               // [slot][16 rows][acc_cols tokens]
+  const int AC = LP.h.acc_cols;
+  float* s_D = reinterpret_cast<float*>(s_acc + kDecodeSlots * 16 * AC);      // [slot][16]
   float* s_sx = s_D + kDecodeSlots * 16;                                       // [problem * 16 + token]
   int32_t* s_rs = reinterpret_cast<int32_t*>(s_sx + kDecTok);
   uint32_t* s_amax = reinterpret_cast<uint32_t*>(s_rs + kDecTok);
@@ -699,16 +755,33 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const int c = blockIdx.x;
-  const int t0 = L.cta_start[c];
-  const int nt = L.cta_start[c + 1] - t0;
 
   // Dependents may be scheduled as soon as every CTA of this grid is running.
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const DecHead& L = LP.h;
+  const int t0 = LP.cta_start[c];
+  const int nt = LP.cta_start[c + 1] - t0;
   if (nt <= 0) return;
 
-  // The first two groups' weights are requested at once: they never depend on
+  DecGroups G;
+  G.pa = dec_problem_of(L, t0);
+  G.np = dec_problem_of(L, t0 + nt - 1) - G.pa + 1;
+  G.pre[0] = 0;
+#pragma unroll
+  for (int i = 0; i < kDecodeMaxGroup; ++i)
+    G.pre[i + 1] = G.pre[i] + (i < G.np ? L.pr[G.pa + i].M * (L.pr[G.pa + i].K >> 4) : 0);
+  G.total = G.pre[kDecodeMaxGroup];
+
+  // Without a programmatic dependency nothing this launch reads is still
+  // being written, and the activations' loads go first, ahead of the weight
+  // stream in the memory queues.
+  constexpr bool kRegQuant = kX == kDecF32 || kX == kDecBf16;
+  const bool early_x = kRegQuant && !L.pdl;
+  float4 f[kDecRegGroups][4];
+  if (early_x) dec_quant_load<kX>(L, G, f);
+
+  // The first groups' weights are requested at once: they never depend on
   // the grid this launch waits for.
-  constexpr int S = kDecStages;
   constexpr int SB = dec_stage_bytes<UPT>();
   constexpr int RS = dec_row_stride<UPT>();
   uint8_t* wstage = stages + (size_t)warp * S * SB;  // this warp's S stages
@@ -723,7 +796,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
     cp_async_commit();
   }
 
-  for (int i = tid; i < kDecodeSlots * 16 * 8 * MT; i += kDecThreads) s_acc[i] = 0;
+  for (int i = tid; i < kDecodeSlots * 16 * AC; i += kDecThreads) s_acc[i] = 0;
   if (tid < kDecodeSlots) {
     s_cnt[tid] = 0;
     s_gen[tid] = 0;
@@ -735,18 +808,9 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
   if (tid < 16) s_ss[tid] = 0.0;
   if (tid == 0) *abort_flag = 0;
 
-  DecGroups G;
-  G.pa = dec_problem_of(L, t0);
-  G.np = dec_problem_of(L, t0 + nt - 1) - G.pa + 1;
-  G.pre[0] = 0;
-#pragma unroll
-  for (int i = 0; i < kDecodeMaxGroup; ++i)
-    G.pre[i + 1] = G.pre[i] + (i < G.np ? L.pr[G.pa + i].M * (L.pr[G.pa + i].K >> 4) : 0);
-  G.total = G.pre[kDecodeMaxGroup];
-
   // The activations may be written by the grid this launch depends on: only
   // an L2 prefetch (no data is consumed) before the dependency wait.
-  {
+  if (!early_x) {
     const int esz = kX == kDecBf16 ? 2 : (kX == kDecPrepared ? 1 : 4);
     for (int i = 0; i < G.np; ++i) {
       const DecProblem& P = L.pr[G.pa + i];
@@ -764,12 +828,16 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
   else if (kX == kDecRms)
     dec_rms_quantise(L, G, sq, s_sx, s_rs, s_amax, s_ss, s_ms, s_flag,
                      reinterpret_cast<unsigned long long*>(sq + L.q_bytes - kRmsBins * 8));
-  else
-    dec_quantise<kX>(L, G, sq, s_sx, s_rs, s_amax);
+  if (kRegQuant) {
+    if (!early_x) dec_quant_load<kX>(L, G, f);
+    dec_quant_rest<kX>(L, G, f, sq, s_sx, s_inv, s_rs, s_amax);
+  }
   consumers_sync();  // codes, scales and row sums visible to every warp
-  // Per-token fp64 reciprocal for the exact rescale of the epilogues.
-  if (tid < kDecTok) s_inv[tid] = __drcp_rn((double)s_sx[tid]);
-  consumers_sync();
+  if (!kRegQuant) {
+    // Per-token fp64 reciprocal for the exact rescale of the epilogues.
+    if (tid < kDecTok) s_inv[tid] = __drcp_rn((double)s_sx[tid]);
+    consumers_sync();
+  }
 
   const int g = lane >> 2, t = lane & 3;
   int acc[4][MT][4];
@@ -812,8 +880,10 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
 #pragma unroll
     for (int k = 0; k < UPT; ++k) {
       if (k < Gr.n()) {
-        const uint4 va = *reinterpret_cast<const uint4*>(stage + g * RS + 64 * k + 16 * t);
-        const uint4 vb = *reinterpret_cast<const uint4*>(stage + (g + 8) * RS + 64 * k + 16 * t);
+        // rows g and g + 8 have the same parity, hence the same chunk order
+        const int cpos = 16 * dec_chunk_pos<UPT>(g, 4 * k + t);
+        const uint4 va = *reinterpret_cast<const uint4*>(stage + g * RS + cpos);
+        const uint4 vb = *reinterpret_cast<const uint4*>(stage + (g + 8) * RS + cpos);
         const uint32_t wa[4] = {va.x, va.y, va.z, va.w};
         const uint32_t wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
@@ -895,7 +965,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
     // Chunked tile: partial sums through the slot's block.
     if (!kAccOut && T.j == 0 && lane < 16) s_D[s * 16 + lane] = dg0;
     // Partial sums of this chunk into the tile's block.
-    int32_t* blk = s_acc + s * 16 * 8 * MT;
+    int32_t* blk = s_acc + s * 16 * AC;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -903,7 +973,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
         const int tok = 8 * mt + 2 * t + (k & 1);
         if (tok < P.M) {
           const int v = acc[0][mt][k] + (acc[1][mt][k] >> 2) + (acc[2][mt][k] >> 4) + (acc[3][mt][k] >> 6);
-          atomicAdd(blk + (g + 8 * (k >> 1)) * 8 * MT + tok, v);
+          atomicAdd(blk + (g + 8 * (k >> 1)) * AC + tok, v);
         }
       }
     zero_acc();
@@ -918,7 +988,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
       for (int idx = lane; idx < 16 * P.M; idx += 32) {
         const int tok = idx >> 4, r = idx & 15;
         if (r < rv) {
-          const int a = blk[r * 8 * MT + tok] - s_rs[T.p * 16 + tok];
+          const int a = blk[r * AC + tok] - s_rs[T.p * 16 + tok];
           const int64_t o = (int64_t)tok * P.N + row0 + r;
           if (kAccOut)
             P.acc[o] = a;
@@ -927,7 +997,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
         }
       }
       __syncwarp();
-      for (int k = lane; k < 16 * 8 * MT; k += 32) blk[k] = 0;
+      for (int k = lane; k < 16 * AC; k += 32) blk[k] = 0;
       if (lane == 0) s_cnt[s] = 0;
       __syncwarp();
       __threadfence_block();
@@ -979,9 +1049,9 @@ static int64_t round128(int64_t v) { return (v + 127) / 128 * 128; }
 
 // Shared-memory bytes of a launch (q_total includes the RMSNorm mode's
 // exact-sum bins, which follow the codes), or -1 when it does not fit.
-static int64_t decode_smem(int64_t q_total, int MT) {
+static int64_t decode_smem(int64_t q_total, int64_t maxM) {
   const int64_t stages = (int64_t)kDecWarps * kDecStages * dec_stage_bytes<dec_upt<1>()>();
-  const int64_t total = stages + q_total + dec_fixed_bytes(MT);
+  const int64_t total = stages + q_total + dec_fixed_bytes((int)maxM, kDecStages);
   return total <= kDecodeSmemMax ? total : -1;
 }
 
@@ -993,17 +1063,17 @@ bool decode_group_fits(const DecCall* calls, int n) {
     q += round128(calls[i].M * decode_q_stride(calls[i].K));
     maxM = calls[i].M > maxM ? calls[i].M : maxM;
   }
-  return decode_smem(q, maxM <= 8 ? 1 : 2) >= 0;
+  return decode_smem(q, maxM) >= 0;
 }
 
 bool decode_fits(int64_t M, int64_t K, bool rms) {
   if (M < 1 || M > kDecodeMaxM) return false;
   const int64_t q = round128(M * decode_q_stride(K)) + (rms ? kRmsBins * 8 : 0);
-  return decode_smem(q, M <= 8 ? 1 : 2) >= 0;
+  return decode_smem(q, M) >= 0;
 }
 
 // Bytes of launch tile gt (rows x K/4).
-static int64_t host_tile_bytes(const DecLaunch& L, int gt) {
+static int64_t host_tile_bytes(const DecHead& L, int gt) {
   int p = 0;
   while (p + 1 < L.nprob && gt >= L.pr[p + 1].tile0) ++p;
   const DecProblem& P = L.pr[p];
@@ -1014,30 +1084,33 @@ static int64_t host_tile_bytes(const DecLaunch& L, int gt) {
 
 // Split the launch's tiles into `grid` contiguous ranges of about equal bytes,
 // at least one tile each.
-static void partition_by_bytes(DecLaunch& L, int grid) {
+static void partition_by_bytes(DecLaunch& LP, int grid) {
+  const DecHead& L = LP.h;
+  int* cta_start = LP.cta_start;
   int64_t total = 0;
   for (int gt = 0; gt < L.total_tiles; ++gt) total += host_tile_bytes(L, gt);
   int64_t acc = 0;
   int cta = 0, start = 0;
-  L.cta_start[0] = 0;
+  cta_start[0] = 0;
   for (int gt = 0; gt < L.total_tiles; ++gt) {
     const int64_t tb = host_tile_bytes(L, gt);
     const int64_t target = total * (cta + 1) / grid;
     if (cta + 1 < grid && gt > start && acc + tb / 2 > target && L.total_tiles - gt >= grid - cta - 1) {
-      L.cta_start[++cta] = gt;
+      cta_start[++cta] = gt;
       start = gt;
     }
     acc += tb;
   }
-  for (int k = cta + 1; k <= grid; ++k) L.cta_start[k] = L.total_tiles;
+  for (int k = cta + 1; k <= grid; ++k) cta_start[k] = L.total_tiles;
 }
 
 cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g, float eps, uint32_t* err, bool pdl,
                           cudaStream_t stream, int num_sms) {
   if (n < 1 || n > kDecodeMaxGroup) return cudaErrorInvalidValue;
   if ((input == kDecRms || input == kDecPrepared) && n != 1) return cudaErrorInvalidValue;
-  DecLaunch L;
-  std::memset(&L, 0, sizeof(L));
+  DecLaunch LP;
+  std::memset(&LP, 0, sizeof(LP));
+  DecHead& L = LP.h;
   int64_t maxM = 0, q = 0;
   int tiles = 0;
   for (int i = 0; i < n; ++i) {
@@ -1065,8 +1138,9 @@ cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g
   }
   const int MT = maxM <= 8 ? 1 : 2;
   if (input == kDecRms) q += kRmsBins * 8;  // exact-sum bins after the codes
-  const int64_t smem = decode_smem(q, MT);
+  int64_t smem = decode_smem(q, maxM);
   if (smem < 0) return cudaErrorInvalidValue;
+  L.acc_cols = (int)maxM;
   L.nprob = n;
   L.total_tiles = tiles;
   L.q_bytes = (int)q;
@@ -1106,16 +1180,19 @@ cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g
   int grid = per_sm * num_sms;
   if (grid > tiles) grid = tiles;
   if (grid > kDecMaxGrid) grid = kDecMaxGrid;
-  partition_by_bytes(L, grid);
-  // Tasks: whole tiles when every warp gets two or more of them (a warp then
-  // writes its tiles' outputs itself); otherwise chunks of about
-  // nu * tiles_per_cta / 8 units, so that all 8 warps share a short launch.
+  partition_by_bytes(LP, grid);
+  // Tasks: whole tiles when every warp of a CTA gets two or more of them (a
+  // warp then writes its tiles' outputs itself); otherwise chunks. A launch
+  // of one problem cuts its tiles into chunks of one group of units, which
+  // spreads a CTA's share evenly over its warps; a launch of several problems
+  // uses chunks of about nu * tiles_per_cta / 8 units (on the B200, measured
+  // faster there: fewer chunks to combine through shared memory).
   const double tiles_per_cta = (double)tiles / grid;
   for (int i = 0; i < n; ++i) {
     DecProblem& P = L.pr[i];
     int upt = P.nu;
     if (tiles_per_cta < 2.0 * kDecWarps) {
-      upt = (int)((P.nu * tiles_per_cta + kDecWarps - 1) / kDecWarps);
+      upt = n == 1 ? dec_upt<1>() : (int)((P.nu * tiles_per_cta + kDecWarps - 1) / kDecWarps);
       upt = upt < 1 ? 1 : (upt > P.nu ? P.nu : upt);
     }
     P.upt = upt;
@@ -1131,7 +1208,8 @@ cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kern, L);
+  L.pdl = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, LP);
 }
 
 }  // namespace bl
