@@ -111,7 +111,7 @@ struct DecLaunch {
 
 // Shared memory past the activation codes.
 __host__ __device__ constexpr int dec_fixed_bytes(int acc_cols, int S) {
-  return kDecTok * 8                     // s_inv
+  return 0
          + kDecodeSlots * 16 * acc_cols * 4  // s_acc
          + kDecodeSlots * 16 * 4         // s_D
          + 3 * kDecTok * 4               // s_sx, s_rs, s_amax
@@ -475,7 +475,7 @@ __device__ __forceinline__ void dec_load_group(const DecProblem& P, int m, int g
 // kDecRegGroups 16-column groups of each thread into registers (a launch
 // without a dependency issues it before any weight copy, so that these loads
 // do not queue behind the weight stream); dec_quant_rest finishes: per-token
-// max|x| by shared atomics, then the codes, s_x, RN64(1/s_x) and the row sums.
+// max|x| by shared atomics, then the codes, s_x and the row sums.
 // Groups beyond the registers are read twice (for the maximum, then for the
 // codes), two at a time so that their loads are in flight together. Run by
 // the 256 consumer threads.
@@ -495,7 +495,7 @@ __device__ __forceinline__ void dec_quant_load(const DecHead& L, const DecGroups
 
 template <int kX>
 __device__ void dec_quant_rest(const DecHead& L, const DecGroups& G, float4 (&f)[kDecRegGroups][4], uint8_t* sq,
-                               float* s_sx, double* s_inv, int32_t* s_rs, uint32_t* s_amax) {
+                               float* s_sx, int32_t* s_rs, uint32_t* s_amax) {
   const int tid = threadIdx.x;
   constexpr int B = 2;  // groups beyond the registers loaded together
   auto absmax16 = [](const float4 (&v)[4]) {
@@ -540,10 +540,7 @@ __device__ void dec_quant_rest(const DecHead& L, const DecGroups& G, float4 (&f)
       tok = p * 16 + m;
       const float sx = __fdiv_rn(kQmax, fmaxf(__uint_as_float(s_amax[tok]), kFloor));
       sum = dec_quant_group(v, sx, dec_q_group(sq, L.pr[p], m, gi));
-      if (gi == 0) {
-        s_sx[tok] = sx;
-        s_inv[tok] = __drcp_rn((double)sx);
-      }
+      if (gi == 0) s_sx[tok] = sx;
     }
     dec_rowsum(s_rs, tok, sum);
   };
@@ -737,8 +734,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
   uint8_t* stages = smem;                                                      // [warp][stage]
   constexpr int S = kDecStages;
   uint8_t* sq = smem + kDecWarps * S * dec_stage_bytes<UPT>();
-  double* s_inv = reinterpret_cast<double*>(sq + LP.h.q_bytes);                   // [problem * 16 + token] RN64(1/s_x)
-  int32_t* s_acc = reinterpret_cast<int32_t*>(s_inv + kDecTok);               // [slot][16 rows][acc_cols tokens]
+  int32_t* s_acc = reinterpret_cast<int32_t*>(sq + LP.h.q_bytes);             // [slot][16 rows][acc_cols tokens]
   const int AC = LP.h.acc_cols;
   float* s_D = reinterpret_cast<float*>(s_acc + kDecodeSlots * 16 * AC);      // [slot][16]
   float* s_sx = s_D + kDecodeSlots * 16;                                       // [problem * 16 + token]
@@ -830,14 +826,9 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
                      reinterpret_cast<unsigned long long*>(sq + L.q_bytes - kRmsBins * 8));
   if (kRegQuant) {
     if (!early_x) dec_quant_load<kX>(L, G, f);
-    dec_quant_rest<kX>(L, G, f, sq, s_sx, s_inv, s_rs, s_amax);
+    dec_quant_rest<kX>(L, G, f, sq, s_sx, s_rs, s_amax);
   }
   consumers_sync();  // codes, scales and row sums visible to every warp
-  if (!kRegQuant) {
-    // Per-token fp64 reciprocal for the exact rescale of the epilogues.
-    if (tid < kDecTok) s_inv[tid] = __drcp_rn((double)s_sx[tid]);
-    consumers_sync();
-  }
 
   const int g = lane >> 2, t = lane & 3;
   int acc[4][MT][4];
@@ -934,10 +925,8 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
     if (P.nchunk == 1) {
       // The warp holds the whole tile: lane (g, t) has rows g and g+8 for
       // tokens 2t, 2t+1 (+ 8 per token group). Class c holds 4^c * sum
-      // q*(code+1), an exact multiple of 4^c. y = RN(RN(a / s_x) * D) with
-      // RN(a / s_x) taken as RN32(RN64(a * RN64(1 / s_x))), which is the
-      // correctly rounded quotient for |a| < 2^24 (double rounding is
-      // innocuous here, Figueroa 1995).
+      // q*(code+1), an exact multiple of 4^c. y = RN(RN(a / s_x) * D), the
+      // quotient by the IEEE fp32 division of the exact float(a).
       const int M = P.M;
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt)
@@ -953,7 +942,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
             if (kAccOut)
               P.acc[o] = a;
             else
-              P.y[o] = __fmul_rn(div_by_scale(a, s_inv[T.p * 16 + tok]), (k >> 1) ? dg1 : dg0);
+              P.y[o] = rescale(a, s_sx[T.p * 16 + tok], (k >> 1) ? dg1 : dg0);
           }
         }
       zero_acc();
@@ -993,7 +982,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
           if (kAccOut)
             P.acc[o] = a;
           else
-            P.y[o] = __fmul_rn(div_by_scale(a, s_inv[T.p * 16 + tok]), s_D[s * 16 + r]);
+            P.y[o] = rescale(a, s_sx[T.p * 16 + tok], s_D[s * 16 + r]);
         }
       }
       __syncwarp();

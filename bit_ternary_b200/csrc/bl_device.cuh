@@ -259,27 +259,11 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 
 // ------------------------------------------------------------ epilogue ---
 // y = RN(RN(float(acc) / s_x) * d), the two-step rescale of the definition.
+// float(acc) is exact for |acc| <= 2^24 (the library's K <= 131072 keeps every
+// accumulator within that) and the IEEE division __fdiv_rn is correctly
+// rounded, so both steps are the single fp32 roundings the definition names.
 __device__ __forceinline__ float rescale(int32_t acc, float s_x, float d) {
   return __fmul_rn(__fdiv_rn(__int2float_rn(acc), s_x), d);
-}
-
-// Exact int32 -> double without the conversion unit: the bit pattern
-// 0x43300000:(a ^ 0x80000000) is 2^52 + 2^31 + a, so one fp64 subtraction
-// recovers a exactly.
-__device__ __forceinline__ double int_to_double_exact(int32_t a) {
-  return __hiloint2double(0x43300000, a ^ (int32_t)0x80000000) - 4503601774854144.0;
-}
-
-// RN(float(a) / s_x) computed as RN_f32(RN_f64(a * inv)), with inv = RN_f64(1/s_x)
-// precomputed per token (__drcp_rn). This equals the correctly rounded fp32
-// quotient for every |a| < 2^24 and normal s_x. The fp64 value carries a
-// relative error below 2^-51.9. A quotient of a 24-bit integer by a 24-bit
-// significand is either an fp32 midpoint's distant neighbour or lies more than
-// 2^-49 (relative) away from every fp32 rounding midpoint, so the final
-// rounding to fp32 cannot differ (the same argument as S. A. Figueroa, "When
-// is double rounding innocuous?", SIGNUM Newsletter 30(3), 1995, for 53 >= 2*24+2).
-__device__ __forceinline__ float div_by_scale(int32_t a, double inv) {
-  return __double2float_rn(int_to_double_exact(a) * inv);
 }
 
 // Inputs are fp32, or bf16 given as 16-bit patterns. A bf16 is the upper half

@@ -19,7 +19,7 @@
 //       kernel), loaded by TMA as 128 tokens x 128 bytes with 128-byte swizzle.
 //   D = int32 accumulators in TMEM, two buffers of 128 columns.
 // Warp roles: 0 TMA producer, 1 MMA issuer (TMEM owner), 2 per-token
-// constants (1/s_x in fp64 and sum_k q) into a shared ring, 4..7 unpack,
+// constants (s_x and sum_k q) into a shared ring, 4..7 unpack,
 // 8..15 epilogue. An epilogue warp reads its 32 rows x 64 tokens of the
 // accumulator, releases the TMEM buffer at once, rescales
 // y = RN(RN(acc/s_x)*D), stages the block in shared memory and writes it with
@@ -41,8 +41,9 @@ constexpr int kBK = 256;   // codes per stage
 constexpr int kStages = 4;
 constexpr int kStageWords = kBK / 16;          // packed words per row per stage
 constexpr int kACols = kBK / 4;                // TMEM columns of one A stage
-constexpr uint32_t kBHalfBytes = kBN * 128;    // one TMA box: 128 tokens x 128 codes
-constexpr uint32_t kBStageBytes = 2 * kBHalfBytes;
+constexpr uint32_t kBBoxBytes = kBN * 128;     // one TMA box: 128 tokens x 128 codes
+constexpr int kBBoxes = kBK / 128;             // boxes per stage
+constexpr uint32_t kBStageBytes = kBBoxes * kBBoxBytes;
 constexpr uint32_t kTmemCols = 512;
 constexpr int kAccCol = 0;                     // accumulator b at column 128*b
 constexpr int kACol = 256;                     // A stage s at column 256 + 64*s
@@ -59,9 +60,8 @@ constexpr int kConstRing = 4;                  // tiles of per-token constants i
 constexpr uint32_t kYSliceBytes = kEpiTokens * 32 * 4;  // one epilogue warp's output block
 
 struct TokConst {
-  double inv;  // RN_f64(1 / s_x)
+  float sx;    // s_x = 127 / max|x|
   int32_t rs;  // sum_k q[m, k]
-  int32_t pad;
 };
 
 struct GemmSmem {
@@ -209,10 +209,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int k0 = c.kb * kBK;
         // A box lying wholly past K is not loaded: its A codes are zero, so
         // whatever the stage buffer holds there contributes nothing.
-        const bool second = k0 + 128 < p.K;
-        mbar_arrive_expect_tx(&S.full[s], second ? kBStageBytes : kBHalfBytes);
-        tma_load_2d(sB + (size_t)s * kBStageBytes, &tmap_q, k0, m0, &S.full[s]);
-        if (second) tma_load_2d(sB + (size_t)s * kBStageBytes + kBHalfBytes, &tmap_q, k0 + 128, m0, &S.full[s]);
+        int nbox = (p.K - k0 + 127) / 128;
+        nbox = nbox > kBBoxes ? kBBoxes : nbox;
+        mbar_arrive_expect_tx(&S.full[s], (uint32_t)nbox * kBBoxBytes);
+        for (int b = 0; b < nbox; ++b)
+          tma_load_2d(sB + (size_t)s * kBStageBytes + b * kBBoxBytes, &tmap_q, k0 + 128 * b, m0, &S.full[s]);
         ++issued;
         c.next(p.kblocks);
         if (++s == kStages) {
@@ -251,7 +252,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
           for (int k8 = 0; k8 < kBK / 32; ++k8) {
             if (k8 < steps) {
-              const uint64_t bdesc = bdesc0 + (uint64_t)((s * kBStageBytes + (k8 >> 2) * kBHalfBytes) >> 4) +
+              const uint64_t bdesc = bdesc0 + (uint64_t)((s * kBStageBytes + (k8 >> 2) * kBBoxBytes) >> 4) +
                                      2 * (k8 & 3);
               umma_i8_ts(d_tmem, a_tmem + 8 * k8, bdesc, idesc, (kb | k8) != 0 ? 1u : 0u);
             }
@@ -275,19 +276,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int lt = 0; lt < my_tiles; ++lt) {
       const int tile = blockIdx.x + lt * gridDim.x;
       const int m0 = (tile / p.tiles_n) * kBN;
-      double inv[kBN / 32];
+      float sx[kBN / 32];
       int32_t rs[kBN / 32];
 #pragma unroll
       for (int h = 0; h < kBN / 32; ++h) {
         const int m = m0 + 32 * h + lane;
         const bool ok = m < p.M;
-        inv[h] = ok ? __drcp_rn((double)__ldg(p.s_x + m)) : 0.0;
+        sx[h] = ok ? __ldg(p.s_x + m) : 1.0f;
         rs[h] = ok ? __ldg(p.rowsum + m) : 0;
       }
       if (!warp_wait(&S.cst_empty[r], ph ^ 1, abort_flag, p.err, kDevTimeoutEpilogue)) break;
 #pragma unroll
       for (int h = 0; h < kBN / 32; ++h) {
-        S.cst[r][32 * h + lane].inv = inv[h];
+        S.cst[r][32 * h + lane].sx = sx[h];
         S.cst[r][32 * h + lane].rs = rs[h];
       }
       __syncwarp();
@@ -381,7 +382,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int t = 0; t < kEpiTokens; ++t) {
         const TokConst kc = cst[t];
         const int a = (int)(t < 32 ? v0[t] : v1[t - 32]) - kc.rs;
-        const uint32_t out = kAccOut ? (uint32_t)a : __float_as_uint(__fmul_rn(div_by_scale(a, kc.inv), dn));
+        const uint32_t out = kAccOut ? (uint32_t)a : __float_as_uint(rescale(a, kc.sx, dn));
         if (kTmaStore) {
           sy[t * 32 + lane] = out;
         } else {
