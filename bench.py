@@ -64,6 +64,8 @@ def parse_args(argv=None):
                     help="small prefill-only run for profiler captures (gate_up layer, M=4096)")
     ap.add_argument("--ncu-layer", default=None, metavar="WORKLOAD:LAYER:M",
                     help="one layer of a workload, M tokens, for profiler captures (e.g. embed_batch:0:32768)")
+    ap.add_argument("--ncu-rms", action="store_true",
+                    help="with --ncu-layer: the RMSNorm + BitLinear forward (norm weight of ones)")
     ap.add_argument("--ncu-i2s", action="store_true",
                     help="I2_S export/import only (stacked gate_up weights), for profiler captures")
     ap.add_argument("--only", default=None, metavar="PARTS",
@@ -1044,11 +1046,16 @@ def run_prefill_small(a, B, torch, dev):
     x = torch.from_numpy(WL.activations(M, l.K, wl.x_dist, wl.seed, layer=li, meta=wl.meta)).to(dev)
     y = torch.empty((M, l.N), dtype=torch.float32, device=dev)
     ws = torch.zeros(B.workspace_size(M, l.N, l.K), dtype=torch.uint8, device=dev)
+    g = torch.ones(l.K, dtype=torch.float32, device=dev)
     for _ in range(a.warmup + a.steps):
-        B.forward(x, p, D, out=y, ws=ws)
+        if a.ncu_rms:
+            B.forward_rmsnorm(x, g, p, D, out=y, ws=ws)
+        else:
+            B.forward(x, p, D, out=y, ws=ws)
     torch.cuda.synchronize(dev)
     assert B.workspace_error(ws) == 0
-    print(json.dumps({"prefill_small": "ok", "M": M, "K": l.K, "N": l.N, "calls": a.warmup + a.steps}))
+    print(json.dumps({"prefill_small": "ok", "rmsnorm": bool(a.ncu_rms), "M": M, "K": l.K, "N": l.N,
+                      "calls": a.warmup + a.steps}))
     return 0
 
 
