@@ -203,19 +203,73 @@ def prepare_oracle_inputs(key, M):
     return wl, packs, xs
 
 
-def cpu_baseline(seconds):
-    wl, packs, xs = prepare_oracle_inputs(HEADLINE, 1)
+def _oracle_worker(args):
+    """One host process of the all-core oracle timing: whole layer-set forwards for `seconds`."""
+    seconds, layers, packs, xs = args
     t0 = time.perf_counter()
     nbytes, steps = 0, 0
     while True:
-        nbytes += oracle_decode_step(wl.layers, packs, xs)
+        nbytes += oracle_decode_step(layers, packs, xs)
         steps += 1
         if time.perf_counter() - t0 >= seconds:
             break
-    dt = time.perf_counter() - t0
-    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-            "sample": f"{steps} full layer-set forwards (M=1, all 4 layers, all rows) in {dt:.1f} s; "
-                      "numpy int64 matmul, single thread"}
+    return nbytes, steps, time.perf_counter() - t0
+
+
+def _oracle_processes():
+    """Host processes for the all-core timing: one per core available to this process, capped
+    so that their working sets (~0.6 GB each: the oracle unpacks a layer's codes to int64) fit
+    in half of the host memory."""
+    ncores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    try:
+        mem = os.sysconf("SC_PAGE_SIZE") * os.sysconf("SC_PHYS_PAGES")
+        ncores = max(1, min(ncores, int(mem * 0.5 // (0.6 * 2**30))))
+    except (ValueError, OSError, AttributeError):
+        pass
+    return ncores
+
+
+def cpu_baseline(seconds):
+    """The oracle on the host cores: one process (the plain single-thread figure), then one
+    process per core over the same workload (processes started by spawn, after the GPU work:
+    a forked child of a CUDA process can hang), then a sampled-token prefill layer."""
+    import multiprocessing as mp
+
+    wl, packs, xs = prepare_oracle_inputs(HEADLINE, 1)
+    nbytes, steps, dt = _oracle_worker((seconds, wl.layers, packs, xs))
+    one = nbytes / dt / 1e9
+    nproc = _oracle_processes()
+    all_cores = None
+    if nproc > 1:
+        with mp.get_context("spawn").Pool(nproc) as pool:
+            res = pool.map(_oracle_worker, [(seconds, wl.layers, packs, xs)] * nproc)
+        tot_bytes = sum(r[0] for r in res)
+        tot_steps = sum(r[1] for r in res)
+        wall = max(r[2] for r in res)
+        all_cores = {"value": tot_bytes / wall / 1e9, "unit": "GB/s", "cores": nproc,
+                     "sample": f"{nproc} processes x ~{seconds:.0f} s: {tot_steps} full layer-set forwards"}
+    # Prefill (C4 gate_up at M=4096) on a sample of tokens: the oracle's cost is linear in M.
+    import oracle as O
+
+    pw = WL.WORKLOADS[PREFILL]
+    li = 1
+    l = pw.layers[li]
+    p_ref, D_ref = O.pack_weights(WL.weight(l.N, l.K, pw.w_dist, pw.seed, layer=li))
+    ms = 8
+    x = WL.activations(ms, l.K, pw.x_dist, pw.seed, layer=li, meta=pw.meta)
+    t0 = time.perf_counter()
+    O.bitlinear_forward(x, p_ref, D_ref, l.K)
+    tp = time.perf_counter() - t0
+    prefill = {"value": 2.0 * ms * l.N * l.K / tp / 1e12, "unit": "TOPS", "cores": 1,
+               "sample": f"{PREFILL} gate_up {l.K}->{l.N}: {ms} of the {PREFILL_M} tokens, all rows, "
+                         f"{tp:.2f} s (cost linear in tokens)"}
+    out = {"value": one, "unit": "GB/s", "cores": 1, "kind": "oracle",
+           "sample": f"{steps} full layer-set forwards (M=1, all 4 layers, all rows) in {dt:.1f} s; "
+                     "numpy int64 matmul, single thread",
+           "prefill_sample": prefill}
+    if all_cores is not None:
+        out["all_cores"] = all_cores
+    return out
 
 
 def run_reference(a):
