@@ -6,24 +6,29 @@
 // M=1 decode kernel; a prefill of many tokens is a dense int8 contraction, so
 // it runs on tcgen05.mma kind::i8 with int32 accumulators in tensor memory.
 //
-// Tile: 128 weight rows (MMA M) x 128 tokens (MMA N); 256 codes per pipeline
+// Tile: 128 weight rows (MMA M) x 192 tokens (MMA N); 256 codes per pipeline
 // stage (8 MMAs of K=32 per barrier round trip, so the single issuing thread
-// keeps the tensor pipe fed), 4 stages.
+// keeps the tensor pipe fed). Larger MMAs carry the pipe's per-instruction
+// cost over more work: measured on gate_up (M=4096), a 128x192x32 MMA issues
+// every ~155-185 cycles against ~144 for 128x128x32.
 //
 // Operand placement (chosen for shared-memory bandwidth):
 //   A = unpacked ternary weights, written by four unpack warps straight from
 //       registers into TMEM (tcgen05.st). `(w >> 2c) & 0x03030303` yields
 //       code+1 for columns {c, 4+c, 8+c, 12+c} of a packed word, so TMEM
-//       holds each 16-column group in the order 4c+b <- 4b+c.
+//       holds each 16-column group in the order 4c+b <- 4b+c. Two stages.
 //   B = int8 activations in the same order (written so by the ActQuant
-//       kernel), loaded by TMA as 128 tokens x 128 bytes with 128-byte swizzle.
-//   D = int32 accumulators in TMEM, two buffers of 128 columns.
+//       kernel), loaded by TMA as 192 tokens x 128 bytes with 128-byte
+//       swizzle; three stages, a ring of its own.
+//   D = int32 accumulators in TMEM, two buffers of 192 columns
+//       (2*192 + 2*64 = 512 columns with the A stages).
 // Warp roles: 0 TMA producer, 1 MMA issuer (TMEM owner), 2 per-token
-// constants (s_x and sum_k q) into a shared ring, 4..7 unpack,
-// 8..15 epilogue. An epilogue warp reads its 32 rows x 64 tokens of the
-// accumulator, releases the TMEM buffer at once, rescales
-// y = RN(RN(acc/s_x)*D), stages the block in shared memory and writes it with
-// one TMA bulk store (or plain stores when N % 4 != 0).
+// constants (s_x and sum_k q) into a shared ring, 4..7 unpack, 8..15
+// epilogue. An epilogue warp owns 32 rows x 96 tokens of the accumulator and
+// walks it in chunks of 32 tokens: TMEM load, rescale y = RN(RN(acc/s_x)*D),
+// a 4 KB staging buffer (two per warp, alternating) and one TMA bulk store
+// per chunk (plain stores when N % 4 != 0); the TMEM buffer is released once
+// its last chunk is in registers.
 // Every barrier wait is bounded in time; a timeout sets a shared abort flag
 // and the error word in the workspace, and all roles drain and exit.
 #include "bl_internal.h"
@@ -36,37 +41,54 @@
 namespace bl {
 
 constexpr int kBM = 128;   // weight rows per tile (MMA M)
-constexpr int kBN = 128;   // tokens per tile (MMA N)
 constexpr int kBK = 256;   // codes per stage
-constexpr int kStages = 4;
 constexpr int kStageWords = kBK / 16;          // packed words per row per stage
 constexpr int kACols = kBK / 4;                // TMEM columns of one A stage
-constexpr uint32_t kBBoxBytes = kBN * 128;     // one TMA box: 128 tokens x 128 codes
-constexpr int kBBoxes = kBK / 128;             // boxes per stage
-constexpr uint32_t kBStageBytes = kBBoxes * kBBoxBytes;
+constexpr int kBBoxes = kBK / 128;             // TMA boxes per B stage
 constexpr uint32_t kTmemCols = 512;
-constexpr int kAccCol = 0;                     // accumulator b at column 128*b
-constexpr int kACol = 256;                     // A stage s at column 256 + 64*s
-static_assert(kACol + kStages * kACols <= (int)kTmemCols, "TMEM budget");
+constexpr int kAccCol = 0;                     // accumulator b at column BN*b
+
+// Tile shapes: BN tokens per tile (MMA N). 192 tokens carry the pipe's
+// per-instruction cost over more work; 128 tokens waste less on launches of
+// one or two tiles per CTA, whose pipeline fill and last epilogue are not
+// overlapped. TMEM holds the two accumulators and the A stages.
+template <int BN>
+struct GemmShape {
+  static constexpr int kBN = BN;
+  static constexpr int kAStages = BN == 128 ? 4 : 2;  // ring of A stages in TMEM
+  static constexpr int kBStages = BN == 128 ? 4 : 3;  // ring of B stages in shared memory
+  static constexpr uint32_t kBBoxBytes = BN * 128;    // one TMA box: BN tokens x 128 codes
+  static constexpr uint32_t kBStageBytes = kBBoxes * kBBoxBytes;
+  static constexpr int kACol = 2 * BN;                // A stage s at column 2*BN + kACols*s
+  static constexpr int kEpiTokens = BN / 2;           // tokens per epilogue warp
+  static_assert(kACol + kAStages * kACols <= (int)kTmemCols, "TMEM budget");
+  static_assert(BN % 16 == 0 && BN <= 256, "MMA N for M = 128");
+  static_assert(kBBoxBytes % 1024 == 0, "128-byte swizzle atoms");
+};
 
 constexpr int kWarpConst = 2;
 constexpr int kUnpackWarp0 = 4;                // 4..7: one per TMEM lane quarter
 constexpr int kEpiWarp0 = 8;                   // 8..15: two per lane quarter
 constexpr int kEpiWarps = 8;
-constexpr int kEpiTokens = kBN / 2;            // tokens per epilogue warp
+constexpr int kEpiChunk = 32;                  // accumulator columns per TMEM load
 constexpr int kGemmThreads = 32 * (kEpiWarp0 + kEpiWarps);  // 512
 constexpr int kUnpackPrefetch = 2;             // stages of packed words in flight
 constexpr int kConstRing = 4;                  // tiles of per-token constants in flight
-constexpr uint32_t kYSliceBytes = kEpiTokens * 32 * 4;  // one epilogue warp's output block
+constexpr uint32_t kYChunkBytes = kEpiChunk * 32 * 4;  // one epilogue chunk: 32 tokens x 32 rows fp32
 
 struct TokConst {
   float sx;    // s_x = 127 / max|x|
   int32_t rs;  // sum_k q[m, k]
 };
 
+template <int BN>
 struct GemmSmem {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
+  static constexpr int kAStages = GemmShape<BN>::kAStages;
+  static constexpr int kBStages = GemmShape<BN>::kBStages;
+  uint64_t full_b[kBStages];   // activation stage landed (TMA bytes)
+  uint64_t empty_b[kBStages];  // activation stage consumed (MMA commit)
+  uint64_t full_a[kAStages];   // weight stage written to TMEM (4 unpack warps)
+  uint64_t empty_a[kAStages];  // weight stage consumed (MMA commit)
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t cst_full[kConstRing];
@@ -74,7 +96,7 @@ struct GemmSmem {
   uint64_t drain;
   uint32_t tmem_base;
   int abort_flag;
-  TokConst cst[kConstRing][kBN];
+  TokConst cst[kConstRing][BN];
 };
 
 struct GemmParams {
@@ -94,11 +116,16 @@ struct GemmParams {
   int num_tiles;
 };
 
-// Smem: [B stages | Y slices | GemmSmem], 1024-aligned; one CTA per SM (each
-// CTA owns all 512 TMEM columns).
-constexpr size_t kSmemB = (size_t)kStages * kBStageBytes;
-constexpr size_t kSmemY = (size_t)kEpiWarps * kYSliceBytes;
-constexpr size_t kGemmSmemBytes = 1024 + kSmemB + kSmemY + ((sizeof(GemmSmem) + 127) & ~size_t(127));
+// Smem: [B stages | Y chunks (two per epilogue warp) | GemmSmem], 1024-aligned;
+// one CTA per SM (each CTA owns all 512 TMEM columns).
+constexpr size_t kSmemY = (size_t)kEpiWarps * 2 * kYChunkBytes;
+template <int BN>
+constexpr size_t gemm_smem_b() { return (size_t)GemmShape<BN>::kBStages * GemmShape<BN>::kBStageBytes; }
+template <int BN>
+constexpr size_t gemm_smem_bytes() {
+  return 1024 + gemm_smem_b<BN>() + kSmemY + ((sizeof(GemmSmem<BN>) + 127) & ~size_t(127));
+}
+static_assert(gemm_smem_bytes<128>() <= 227 * 1024 && gemm_smem_bytes<192>() <= 227 * 1024, "shared memory");
 
 // Warp-uniform bounded wait: lane 0 polls, the whole warp gets the outcome, so
 // the warp stays converged for the .sync.aligned tcgen05 instructions.
@@ -152,24 +179,37 @@ __device__ __forceinline__ void unpack_load(const GemmParams& p, const JobCursor
   }
 }
 
-template <bool kAligned, bool kAccOut, bool kTmaStore>
+template <int BN, bool kAligned, bool kAccOut, bool kTmaStore>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_out,
                 const GemmParams p) {
+  using Shape = GemmShape<BN>;
+  constexpr int kBN = Shape::kBN;
+  constexpr int kAStages = Shape::kAStages;
+  constexpr int kBStages = Shape::kBStages;
+  constexpr uint32_t kBBoxBytes = Shape::kBBoxBytes;
+  constexpr uint32_t kBStageBytes = Shape::kBStageBytes;
+  constexpr int kACol = Shape::kACol;
+  constexpr int kEpiTokens = Shape::kEpiTokens;
+  static_assert(kEpiTokens % kEpiChunk == 0, "epilogue chunks");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sB = smem;
-  uint8_t* sY = smem + kSmemB;
-  GemmSmem& S = *reinterpret_cast<GemmSmem*>(smem + kSmemB + kSmemY);
+  uint8_t* sY = smem + gemm_smem_b<BN>();
+  GemmSmem<BN>& S = *reinterpret_cast<GemmSmem<BN>*>(smem + gemm_smem_b<BN>() + kSmemY);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int my_tiles = p.num_tiles > (int)blockIdx.x ? (p.num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
   const int jobs = my_tiles * p.kblocks;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&S.full[s], 1 + 4);  // TMA producer + one unpack warp per lane quarter
-      mbar_init(&S.empty[s], 1);
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&S.full_b[s], 1);   // the TMA producer's expect-tx arrival
+      mbar_init(&S.empty_b[s], 1);
+    }
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&S.full_a[s], 4);   // one unpack warp per TMEM lane quarter
+      mbar_init(&S.empty_a[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&S.acc_full[b], 1);
@@ -203,7 +243,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       JobCursor c{0, 0};
       int issued = 0;
       for (int j = 0; j < jobs; ++j) {
-        if (!mbar_wait(&S.empty[s], ph ^ 1, abort_flag, p.err, kDevTimeoutProducer)) break;
+        if (!mbar_wait(&S.empty_b[s], ph ^ 1, abort_flag, p.err, kDevTimeoutProducer)) break;
         const int tile = blockIdx.x + c.tile_local * gridDim.x;
         const int m0 = (tile / p.tiles_n) * kBN;
         const int k0 = c.kb * kBK;
@@ -211,56 +251,62 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // whatever the stage buffer holds there contributes nothing.
         int nbox = (p.K - k0 + 127) / 128;
         nbox = nbox > kBBoxes ? kBBoxes : nbox;
-        mbar_arrive_expect_tx(&S.full[s], (uint32_t)nbox * kBBoxBytes);
+        mbar_arrive_expect_tx(&S.full_b[s], (uint32_t)nbox * kBBoxBytes);
         for (int b = 0; b < nbox; ++b)
-          tma_load_2d(sB + (size_t)s * kBStageBytes + b * kBBoxBytes, &tmap_q, k0 + 128 * b, m0, &S.full[s]);
+          tma_load_2d(sB + (size_t)s * kBStageBytes + b * kBBoxBytes, &tmap_q, k0 + 128 * b, m0, &S.full_b[s]);
         ++issued;
         c.next(p.kblocks);
-        if (++s == kStages) {
+        if (++s == kBStages) {
           s = 0;
           ph ^= 1;
         }
       }
       // Let every issued copy land before the CTA can exit.
-      const int first = issued > kStages ? issued - kStages : 0;
+      const int first = issued > kBStages ? issued - kBStages : 0;
       for (int j = first; j < issued; ++j)
-        mbar_wait(&S.full[j % kStages], (j / kStages) & 1, nullptr, p.err, kDevTimeoutDrain, 100000000ull);
+        mbar_wait(&S.full_b[j % kBStages], (j / kBStages) & 1, nullptr, p.err, kDevTimeoutDrain, 100000000ull);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_i8(kBM, kBN);
       const uint64_t bdesc0 = umma_sdesc_sw128(sB);
-      int s = 0;
-      uint32_t ph = 0;
+      int sb = 0, sa = 0;
+      uint32_t phb = 0, pha = 0;
       bool ok = true;
       for (int lt = 0; lt < my_tiles && ok; ++lt) {
         const int b = lt & 1;
         if (!mbar_wait(&S.acc_empty[b], ((lt >> 1) & 1) ^ 1, abort_flag, p.err, kDevTimeoutMma)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + kAccCol + 128 * b;
+        const uint32_t d_tmem = tmem + kAccCol + kBN * b;
         for (int kb = 0; kb < p.kblocks; ++kb) {
-          if (!mbar_wait(&S.full[s], ph, abort_flag, p.err, kDevTimeoutMma)) {
+          if (!mbar_wait(&S.full_a[sa], pha, abort_flag, p.err, kDevTimeoutMma) ||
+              !mbar_wait(&S.full_b[sb], phb, abort_flag, p.err, kDevTimeoutMma)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_tmem = tmem + kACol + kACols * s;
+          const uint32_t a_tmem = tmem + kACol + kACols * sa;
           // K=32 steps of this stage that hold real codes (the rest are zero).
           const int rem = p.K - kb * kBK;
           const int steps = rem >= kBK ? kBK / 32 : (rem + 31) / 32;
 #pragma unroll
           for (int k8 = 0; k8 < kBK / 32; ++k8) {
             if (k8 < steps) {
-              const uint64_t bdesc = bdesc0 + (uint64_t)((s * kBStageBytes + (k8 >> 2) * kBBoxBytes) >> 4) +
+              const uint64_t bdesc = bdesc0 + (uint64_t)((sb * kBStageBytes + (k8 >> 2) * kBBoxBytes) >> 4) +
                                      2 * (k8 & 3);
               umma_i8_ts(d_tmem, a_tmem + 8 * k8, bdesc, idesc, (kb | k8) != 0 ? 1u : 0u);
             }
           }
-          tc_commit(&S.empty[s]);
-          if (++s == kStages) {
-            s = 0;
-            ph ^= 1;
+          tc_commit(&S.empty_a[sa]);
+          tc_commit(&S.empty_b[sb]);
+          if (++sa == kAStages) {
+            sa = 0;
+            pha ^= 1;
+          }
+          if (++sb == kBStages) {
+            sb = 0;
+            phb ^= 1;
           }
         }
         if (ok) tc_commit(&S.acc_full[b]);
@@ -318,7 +364,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int q = 0; q < kUnpackPrefetch; ++q) {
         const int j = j0 + q;
         if (j >= jobs) break;
-        if (!warp_wait(&S.empty[s], ph ^ 1, abort_flag, p.err, kDevTimeoutUnpack)) {
+        if (!warp_wait(&S.empty_a[s], ph ^ 1, abort_flag, p.err, kDevTimeoutUnpack)) {
           ok = false;
           break;
         }
@@ -337,20 +383,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&S.full[s]);
-        if (++s == kStages) {
+        if (lane == 0) mbar_arrive(&S.full_a[s]);
+        if (++s == kAStages) {
           s = 0;
           ph ^= 1;
         }
       }
     }
   } else if (warp >= kEpiWarp0) {
-    // ------------------------------------------------ epilogue: 32 weight rows x 64 tokens per warp
+    // ------------------------------------------------ epilogue: 32 weight rows x kEpiTokens tokens per warp
     const int ew = warp - kEpiWarp0;
     const int quarter = warp & 3;
     const int half = ew >> 2;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    uint32_t* sy = reinterpret_cast<uint32_t*>(sY + (size_t)ew * kYSliceBytes);
+    uint32_t* sy0 = reinterpret_cast<uint32_t*>(sY + (size_t)ew * 2 * kYChunkBytes);
+    int ybuf = 0;  // which of the warp's two staging chunks the next chunk uses
     int r = 0;
     uint32_t rph = 0;
     for (int lt = 0; lt < my_tiles; ++lt) {
@@ -363,36 +410,55 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const float dn = (!kAccOut && nvalid) ? __ldg(p.D + n) : 0.0f;
       if (!warp_wait(&S.acc_full[b], (lt >> 1) & 1, abort_flag, p.err, kDevTimeoutEpilogue)) break;
       tc_fence_after();
-      uint32_t v0[32], v1[32];
-      tmem_ld_32x32b_x32(lane_base + kAccCol + 128 * b + kEpiTokens * half, v0);
-      tmem_ld_32x32b_x32(lane_base + kAccCol + 128 * b + kEpiTokens * half + 32, v1);
-      tmem_wait_ld();
-      // The accumulator is in registers: hand the TMEM buffer back to the MMA.
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.acc_empty[b]);
       if (!warp_wait(&S.cst_full[r], rph, abort_flag, p.err, kDevTimeoutEpilogue)) break;
       const TokConst* cst = &S.cst[r][kEpiTokens * half];
-      if (kTmaStore) {
-        // The previous block's bulk store must have read this slice.
-        if (lane == 0) bulk_wait_group_read0();
-        __syncwarp();
-      }
-#pragma unroll
-      for (int t = 0; t < kEpiTokens; ++t) {
-        const TokConst kc = cst[t];
-        const int a = (int)(t < 32 ? v0[t] : v1[t - 32]) - kc.rs;
-        const uint32_t out = kAccOut ? (uint32_t)a : __float_as_uint(rescale(a, kc.sx, dn));
+      // Chunks of 32 accumulator columns: load, rescale, store. Lane `lane`
+      // holds row n of the chunk's 32 tokens. With TMA stores the chunk is
+      // staged in one of the warp's two shared buffers and written as one
+      // 32 x 32 box (rows past M or N are clipped); otherwise a warp's store
+      // of one token covers 32 consecutive outputs (128 bytes).
+#pragma unroll 1
+      for (int c0 = 0; c0 < kEpiTokens; c0 += kEpiChunk) {
+        uint32_t v[kEpiChunk];
+        tmem_ld_32x32b_x32(lane_base + kAccCol + kBN * b + kEpiTokens * half + c0, v);
+        tmem_wait_ld();
+        if (c0 + kEpiChunk == kEpiTokens) {
+          // The whole accumulator is in registers: hand the TMEM buffer back.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.acc_empty[b]);
+        }
+        uint32_t* sy = sy0 + ybuf * (kYChunkBytes / 4);
         if (kTmaStore) {
-          sy[t * 32 + lane] = out;
-        } else {
-          const int m = m0 + t;
-          if (m < p.M && nvalid) {
-            if (kAccOut)
-              p.acc_out[(int64_t)m * p.N + n] = (int32_t)out;
-            else
-              __stcs(p.y + (int64_t)m * p.N + n, __uint_as_float(out));
+          // The store that used this buffer two chunks ago must have read it.
+          if (lane == 0) bulk_wait_group_read1();
+          __syncwarp();
+        }
+#pragma unroll
+        for (int t = 0; t < kEpiChunk; ++t) {
+          const TokConst kc = cst[c0 + t];
+          const int a = (int)v[t] - kc.rs;
+          const uint32_t out = kAccOut ? (uint32_t)a : __float_as_uint(rescale(a, kc.sx, dn));
+          if (kTmaStore) {
+            sy[t * 32 + lane] = out;
+          } else {
+            const int m = m0 + c0 + t;
+            if (m < p.M && nvalid) {
+              if (kAccOut)
+                p.acc_out[(int64_t)m * p.N + n] = (int32_t)out;
+              else
+                __stcs(p.y + (int64_t)m * p.N + n, __uint_as_float(out));
+            }
           }
+        }
+        if (kTmaStore) {
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmap_out, n0, m0 + c0, sy);
+            bulk_commit_group();
+          }
+          ybuf ^= 1;
         }
       }
       __syncwarp();
@@ -400,14 +466,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       if (++r == kConstRing) {
         r = 0;
         rph ^= 1;
-      }
-      if (kTmaStore) {
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          tma_store_2d(&tmap_out, n0, m0, sy);
-          bulk_commit_group();
-        }
       }
     }
     if (kTmaStore) {
@@ -438,14 +496,26 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-template <bool kAligned, bool kAccOut, bool kTmaStore>
+template <int BN, bool kAligned, bool kAccOut, bool kTmaStore>
 static cudaError_t launch_gemm_t(const CUtensorMap& tq, const CUtensorMap& to, const GemmParams& p, int grid,
                                  cudaStream_t stream) {
-  auto kern = gemm_kernel<kAligned, kAccOut, kTmaStore>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kGemmSmemBytes);
+  auto kern = gemm_kernel<BN, kAligned, kAccOut, kTmaStore>;
+  constexpr size_t smem = gemm_smem_bytes<BN>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(tq, to, p);
+  kern<<<grid, kGemmThreads, smem, stream>>>(tq, to, p);
   return cudaGetLastError();
+}
+
+// Estimated time of a launch with BN-token tiles, in units of 10 ns on the
+// B200 (fitted to timings of the prefill and SigLIP shapes): the waves of
+// tiles times a tile's k-blocks at the measured cost of one k-block, plus
+// the launch's fixed cost (pipeline fill and the last tile's epilogue, which
+// nothing overlaps; larger for 192-token tiles).
+static int64_t gemm_estimate(int BN, int64_t M, int64_t tiles_n, int64_t kblocks, int grid) {
+  const int64_t tiles = (M + BN - 1) / BN * tiles_n;
+  const int64_t waves = (tiles + grid - 1) / grid;
+  return BN == 128 ? waves * kblocks * 80 + 750 : waves * kblocks * 95 + 1390;
 }
 
 cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D, float* y,
@@ -454,11 +524,18 @@ cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed,
   int8_t* q = reinterpret_cast<int8_t*>(base + ws_q_off(M));
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
+  // Token-tile width: whichever the cost model puts first.
+  const int64_t tiles_n = (N + kBM - 1) / kBM;
+  const int64_t kblocks = (K + kBK - 1) / kBK;
+  const int est_grid = num_sms;
+  const int BN = gemm_estimate(192, M, tiles_n, kblocks, est_grid) < gemm_estimate(128, M, tiles_n, kblocks, est_grid)
+                     ? 192
+                     : 128;
   CUtensorMap tmap_q, tmap_out;
   {
     const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
     const cuuint64_t gstride[1] = {(cuuint64_t)K};
-    const cuuint32_t box[2] = {128u, (cuuint32_t)kBN};
+    const cuuint32_t box[2] = {128u, (cuuint32_t)BN};
     const cuuint32_t estride[2] = {1, 1};
     if (encode(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, gdim, gstride, box, estride,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -472,7 +549,7 @@ cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed,
   if (tma_store) {
     const cuuint64_t gdim[2] = {(cuuint64_t)N, (cuuint64_t)M};
     const cuuint64_t gstride[1] = {(cuuint64_t)N * 4};
-    const cuuint32_t box[2] = {32u, (cuuint32_t)kEpiTokens};
+    const cuuint32_t box[2] = {32u, (cuuint32_t)kEpiChunk};
     const cuuint32_t estride[2] = {1, 1};
     if (encode(&tmap_out, acc_out != nullptr ? CU_TENSOR_MAP_DATA_TYPE_INT32 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
                out, gdim, gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -492,17 +569,19 @@ cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed,
   p.N = (int)N;
   p.K = (int)K;
   p.wpr = (int)(K / 16);
-  p.kblocks = (int)((K + kBK - 1) / kBK);
-  p.tiles_n = (int)((N + kBM - 1) / kBM);
-  const int64_t tiles_m = (M + kBN - 1) / kBN;
+  p.kblocks = (int)kblocks;
+  p.tiles_n = (int)tiles_n;
+  const int64_t tiles_m = (M + BN - 1) / BN;
   const int64_t nt = tiles_m * p.tiles_n;
   if (nt > 0x7FFFFFFF) return cudaErrorInvalidValue;
   p.num_tiles = (int)nt;
   const int grid = (int)(nt < num_sms ? nt : num_sms);
   const bool aligned = (p.wpr % 4) == 0;
   const bool accout = acc_out != nullptr;
-#define BL_GEMM_CASE(AL, AO, TS) \
-  if (aligned == AL && accout == AO && tma_store == TS) return launch_gemm_t<AL, AO, TS>(tmap_q, tmap_out, p, grid, stream);
+#define BL_GEMM_CASE(AL, AO, TS)                                                                     \
+  if (aligned == AL && accout == AO && tma_store == TS)                                              \
+    return BN == 192 ? launch_gemm_t<192, AL, AO, TS>(tmap_q, tmap_out, p, grid, stream)               \
+                     : launch_gemm_t<128, AL, AO, TS>(tmap_q, tmap_out, p, grid, stream);
   BL_GEMM_CASE(true, false, true)
   BL_GEMM_CASE(true, false, false)
   BL_GEMM_CASE(false, false, true)
