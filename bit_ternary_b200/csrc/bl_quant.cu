@@ -101,87 +101,98 @@ __global__ void __launch_bounds__(kBinThreads) absum_bins_kernel(const void* __r
 // bin is below 2^60 and S below 2^313.
 __global__ void absmean_finalize_kernel(const unsigned long long* __restrict__ gbins, uint64_t n,
                                         float* __restrict__ scal, uint32_t* __restrict__ status) {
-  // The warp stages the bins in shared memory (parallel loads); one thread
-  // then does the exact arithmetic.
+  // S = sum_e bins[e] * 2^(max(e,1)-1) as 11 little-endian 32-bit limbs (used
+  // bins < 2^60 at indices <= 258: S < 2^318). The block adds every bin's
+  // (up to three) limb parts into 64-bit per-limb sums with shared atomics
+  // (at most ~260 parts of < 2^32 per limb: no overflow); one thread then
+  // propagates the carries and divides.
+  constexpr int L = 11;
   __shared__ unsigned long long bins[kPackBins];
+  __shared__ unsigned long long limb_sum[L + 3];
+  __shared__ uint32_t sS[L];
   if (blockIdx.x != 0) return;
   for (int i = threadIdx.x; i < kPackBins; i += blockDim.x) bins[i] = gbins[i];
+  for (int i = threadIdx.x; i < L + 3; i += blockDim.x) limb_sum[i] = 0ull;
+  __syncthreads();
+  const bool nonfinite = bins[kPackNonFiniteBin] != 0ull;
+  if (!nonfinite) {
+    for (int e = threadIdx.x; e < kPackNonFiniteBin; e += blockDim.x) {
+      const unsigned long long v = bins[e];
+      if (v == 0ull) continue;
+      const int sh = (e > 1 ? e : 1) - 1;
+      const int limb = sh >> 5, bit = sh & 31;
+      // v << bit spans up to three limbs.
+      const uint32_t p0 = (uint32_t)(v << bit);
+      const uint32_t p1 = bit == 0 ? (uint32_t)(v >> 32) : (uint32_t)(v >> (32 - bit));
+      const uint32_t p2 = bit == 0 ? 0u : (uint32_t)((v >> 32) >> (32 - bit));
+      atomicAdd(&limb_sum[limb], (unsigned long long)p0);
+      atomicAdd(&limb_sum[limb + 1], (unsigned long long)p1);
+      if (p2 != 0u) atomicAdd(&limb_sum[limb + 2], (unsigned long long)p2);
+    }
+  }
   __syncthreads();
   if (threadIdx.x != 0) return;
-  if (bins[kPackNonFiniteBin] != 0ull) {
+  if (nonfinite) {
     *status = 1u;  // non-finite input
     scal[0] = __int_as_float(0x7FC00000);
     scal[1] = __int_as_float(0x7FC00000);
     return;
   }
-  // S as 11 little-endian 32-bit limbs (used bins < 2^60 at indices <= 258:
-  // S < 2^318).
-  constexpr int L = 11;
-  uint32_t S[L];
-#pragma unroll
-  for (int i = 0; i < L; ++i) S[i] = 0u;
-  for (int e = 0; e < kPackNonFiniteBin; ++e) {
-    const unsigned long long v = bins[e];
-    if (v == 0ull) continue;
-    const int sh = (e > 1 ? e : 1) - 1;
-    const int limb = sh >> 5, bit = sh & 31;
-    // v << bit spans up to three limbs.
-    const uint32_t p0 = (uint32_t)(v << bit);
-    const uint32_t p1 = (uint32_t)((v >> (32 - bit)) >> 0);
-    uint32_t parts[3];
-    parts[0] = p0;
-    if (bit == 0) {
-      parts[1] = (uint32_t)(v >> 32);
-      parts[2] = 0u;
-    } else {
-      parts[1] = (uint32_t)(v >> (32 - bit));
-      parts[2] = (uint32_t)((v >> 32) >> (32 - bit));
-    }
-    (void)p1;
+  {
     unsigned long long carry = 0ull;
-    for (int i = limb; i < L; ++i) {
-      const unsigned long long add = (i - limb < 3 ? parts[i - limb] : 0u);
-      const unsigned long long t = (unsigned long long)S[i] + add + carry;
-      S[i] = (uint32_t)t;
+#pragma unroll
+    for (int i = 0; i < L; ++i) {
+      const unsigned long long t = limb_sum[i] + carry;
+      sS[i] = (uint32_t)t;
       carry = t >> 32;
-      if (i - limb >= 2 && carry == 0ull) break;
     }
   }
   // Long division of S * 2^F by n (n < 2^48), 16-bit digits MSB first: the
   // remainder stays below n, so remainder * 2^16 + digit fits in 64 bits.
+  // Digit d covers bits [32L + F - 16(d+1), +16) of S * 2^F.
   constexpr int F = 32;
   constexpr int kDigits = (32 * L + F) / 16;  // 24
-  uint16_t qd[kDigits];
-  unsigned long long rem = 0ull;
-  for (int d = 0; d < kDigits; ++d) {
-    const int bit = 32 * L + F - 16 * (d + 1);  // weight of this digit's lowest bit in S * 2^F
-    uint32_t digit = 0u;
-    if (bit >= F) {
-      const int j = bit - F;
-      digit = (S[j >> 5] >> (j & 31)) & 0xFFFFu;
-    }
-    const unsigned long long cur = (rem << 16) | digit;
-    qd[d] = (uint16_t)(cur / n);
+  auto digit = [&](int d) -> uint32_t {
+    const int bit = 32 * L + F - 16 * (d + 1);
+    if (bit < F) return 0u;
+    const int j = bit - F;
+    return (sS[j >> 5] >> (j & 31)) & 0xFFFFu;
+  };
+  // Leading zero digits of S * 2^F give zero quotient digits and leave the
+  // remainder at 0. From the first nonzero quotient digit on, four digits
+  // hold the leading 24 bits, the round bit and the start of the sticky bits;
+  // every bit below them is nonzero exactly when the remainder or a digit of
+  // S * 2^F not yet taken is.
+  int d = 0;
+  while (d < kDigits && digit(d) == 0u) ++d;
+  unsigned long long rem = 0ull, w = 0ull;
+  uint32_t q_lead = 0u;
+  int dl = -1, got = 0;
+  for (; d < kDigits && got < 4; ++d) {
+    const unsigned long long cur = (rem << 16) | digit(d);
+    const uint32_t qd = (uint32_t)(cur / n);
     rem = cur % n;
+    if (dl < 0 && qd != 0u) {
+      dl = d;
+      q_lead = qd;
+    }
+    if (dl >= 0) {
+      w = (w << 16) | qd;
+      ++got;
+    }
   }
-  // Leading 24 bits of the quotient, the next (round) bit, and a sticky bit
-  // for every lower bit and the final remainder. The leading 25 bits lie in
-  // the first four nonzero-led digits, read as one 64-bit window.
+  bool rest = rem != 0ull;
+  for (int dd = d; dd < kDigits && !rest; ++dd) rest = digit(dd) != 0u;
   float mean = 0.0f;
-  int dl = 0;
-  while (dl < kDigits && qd[dl] == 0) ++dl;
-  if (dl < kDigits) {
-    unsigned long long w = 0ull;
-#pragma unroll
-    for (int k = 0; k < 4; ++k) w = (w << 16) | (dl + k < kDigits ? qd[dl + k] : 0u);
-    const int lb = 31 - __clz((uint32_t)qd[dl]);          // leading bit inside digit dl
+  if (dl >= 0) {
+    w <<= 16 * (4 - got);                                 // digits past the last one are zero
+    const int lb = 31 - __clz(q_lead);                    // leading bit inside digit dl
     const int lead = 16 * (kDigits - 1 - dl) + lb;        // its index from the quotient's LSB
     if (lead >= 24) {
       const int top = 48 + lb;                            // the leading bit's index in w
       uint32_t sig = (uint32_t)(w >> (top - 23)) & 0xFFFFFFu;
       const uint32_t round_bit = (uint32_t)(w >> (top - 24)) & 1u;
-      uint32_t sticky = (rem != 0ull || (w & ((1ull << (top - 24)) - 1ull)) != 0ull) ? 1u : 0u;
-      for (int d = dl + 4; d < kDigits && !sticky; ++d) sticky |= qd[d] != 0 ? 1u : 0u;
+      const uint32_t sticky = (rest || (w & ((1ull << (top - 24)) - 1ull)) != 0ull) ? 1u : 0u;
       int E = lead - 149 - F;  // value = 1.xxx * 2^E
       if (round_bit && (sticky || (sig & 1u))) {
         ++sig;
