@@ -11,6 +11,9 @@
 namespace {
 
 constexpr int kAbiVersion = 1;
+// From this many tokens on, a decode forward quantises x once into the
+// workspace instead of in every CTA of the decode kernel.
+constexpr int64_t kDecodeQuantiseOnceM = 4;
 
 #ifndef BL_BUILD_ID
 #define BL_BUILD_ID "unknown"
@@ -69,6 +72,22 @@ int forward_impl(const void* x, bool bf16, int64_t M, int64_t N, int64_t K, cons
   uint8_t* base = static_cast<uint8_t*>(ws);
   uint32_t* err = reinterpret_cast<uint32_t*>(base);
   if (bl::decode_fits(M, K, false)) {
+    if (M >= kDecodeQuantiseOnceM && acc == nullptr) {
+      // Several tokens: quantise them once into the workspace, then the
+      // decode kernel copies the codes (a quarter of x's bytes) into every
+      // CTA instead of each CTA reading and quantising all of x. The decode
+      // launch depends on the quantiser programmatically: its weights start
+      // streaming while the quantiser runs.
+      cudaError_t e = bl::launch_act_quant(x, bf16, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
+                                           reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
+                                           reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), true, stream,
+                                           err);
+      if (e != cudaSuccess) return BL_ERR_CUDA;
+      const bl::DecCall call{base + bl::ws_q_off(M), reinterpret_cast<const float*>(base + bl::ws_sx_off(M)),
+                             reinterpret_cast<const int32_t*>(base + bl::ws_rowsum_off(M)), packed, D, y, nullptr,
+                             M, N, K};
+      return cuda_status(bl::launch_decode(&call, 1, bl::kDecPrepared, nullptr, 0.0f, err, true, stream, sms));
+    }
     const bl::DecCall call{x, nullptr, nullptr, packed, D, y, acc, M, N, K};
     return cuda_status(
         bl::launch_decode(&call, 1, bf16 ? bl::kDecBf16 : bl::kDecF32, nullptr, 0.0f, err, false, stream, sms));

@@ -566,12 +566,25 @@ __device__ void dec_quant_rest(const DecHead& L, const DecGroups& G, float4 (&f)
 // group order, row stride K; s_x and row sums): copied into the shared layout.
 __device__ void dec_load_prepared(const DecHead& L, const DecGroups& G, uint8_t* sq, float* s_sx, int32_t* s_rs) {
   const int tid = threadIdx.x;
-  for (int gg = tid; gg < G.total; gg += kDecThreads) {
-    int p, m, gi;
-    G.locate(L, gg, p, m, gi);
-    const DecProblem& P = L.pr[p];
-    const uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const int8_t*>(P.x) + (int64_t)m * P.K) + gi);
-    dec_store_group(dec_q_group(sq, P, m, gi), v.x, v.y, v.z, v.w);
+  constexpr int B = 4;  // groups per thread whose loads are in flight together
+  for (int base = 0; base < G.total; base += B * kDecThreads) {
+    uint4 v[B];
+    uint8_t* dst[B];
+#pragma unroll
+    for (int b = 0; b < B; ++b) {
+      const int gg = base + b * kDecThreads + tid;
+      dst[b] = nullptr;
+      if (gg < G.total) {
+        int p, m, gi;
+        G.locate(L, gg, p, m, gi);
+        const DecProblem& P = L.pr[p];
+        v[b] = __ldg(reinterpret_cast<const uint4*>(static_cast<const int8_t*>(P.x) + (int64_t)m * P.K) + gi);
+        dst[b] = dec_q_group(sq, P, m, gi);
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < B; ++b)
+      if (dst[b] != nullptr) dec_store_group(dst[b], v[b].x, v[b].y, v[b].z, v[b].w);
   }
   for (int i = tid; i < G.np * 16; i += kDecThreads) {
     const int p = G.pa + (i >> 4), m = i & 15;
@@ -1158,10 +1171,10 @@ cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g
 #undef BL_DEC
   if (e != cudaSuccess) return e;
   // One CTA per SM leaves room on every SM for a CTA of the next launch
-  // (programmatic dependent launch). Long streams launched without it take
-  // as many CTAs per SM as fit (more copies in flight).
+  // (programmatic dependent launch), which matters for short launches. Long
+  // streams take as many CTAs per SM as fit (more copies in flight).
   int per_sm = 1;
-  if (!pdl && tiles >= 8 * num_sms) {
+  if (tiles >= 8 * num_sms) {
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kDecThreads, (size_t)smem);
     if (e != cudaSuccess) return e;
     per_sm = per_sm < 1 ? 1 : (per_sm > 3 ? 3 : per_sm);

@@ -251,6 +251,8 @@ __global__ void __launch_bounds__(256) act_quant_kernel(const void* __restrict__
                                                         int8_t* __restrict__ q, float* __restrict__ s_out,
                                                         int32_t* __restrict__ rowsum_out,
                                                         uint32_t* __restrict__ err_reset) {
+  // A decode launch that waits on these codes may start streaming its weights.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (err_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err_reset = 0u;
   __shared__ float red_f[8];
   __shared__ int red_i[8];
@@ -342,6 +344,8 @@ __global__ void __launch_bounds__(256) act_quant_reg_kernel(const void* __restri
                                                             int8_t* __restrict__ q, float* __restrict__ s_out,
                                                             int32_t* __restrict__ rowsum_out,
                                                             uint32_t* __restrict__ err_reset) {
+  // A decode launch that waits on these codes may start streaming its weights.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   __shared__ float red_f[8];
   if (err_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err_reset = 0u;
   const int64_t m = blockIdx.x;
