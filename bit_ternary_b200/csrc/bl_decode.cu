@@ -789,8 +789,8 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
   float4 f[kDecRegGroups][4];
   if (early_x) dec_quant_load<kX>(L, G, f);
 
-  // The first groups' weights are requested at once: they never depend on
-  // the grid this launch waits for.
+  // The first groups' weights (one per stage) are requested at once: they
+  // never depend on the grid this launch waits for.
   constexpr int SB = dec_stage_bytes<UPT>();
   constexpr int RS = dec_row_stride<UPT>();
   uint8_t* wstage = stages + (size_t)warp * S * SB;  // this warp's S stages
@@ -800,7 +800,7 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
   // reads the same values).
   DecRun* rec = reinterpret_cast<DecRun*>(s_rec) + warp * S;
 #pragma unroll 1
-  for (int k = 0; k < S - 1; ++k) {
+  for (int k = 0; k < S; ++k) {
     rec[k] = cur.issue(L, t0, nt, wstage + k * SB, lane);
     cp_async_commit();
   }
@@ -828,9 +828,9 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
         prefetch_l2(static_cast<const uint8_t*>(P.x) + o);
     }
   }
+  consumers_sync();  // shared state initialised (before the wait, where it costs nothing)
   asm volatile("griddepcontrol.wait;" ::: "memory");
   if (tid == 0 && c == 0 && L.err != nullptr) *L.err = 0u;
-  consumers_sync();  // shared state initialised
 
   if (kX == kDecPrepared)
     dec_load_prepared(L, G, sq, s_sx, s_rs);
@@ -1007,18 +1007,20 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
     }
     return true;
   };
-  // S - 1 groups in flight: start the next group in the stage freed by the
-  // last contraction, wait for the oldest, contract it.
+  // All S stages were filled before the quantiser ran. Wait for the oldest,
+  // contract it, refill its stage with the next group: S - 1 groups stay in
+  // flight during each contraction. (The stage's shared loads have all been
+  // consumed by the MMAs of the contraction before the refill is issued.)
   int st = 0;
 #pragma unroll 1
   for (;;) {
-    const int sti = st == 0 ? S - 1 : st - 1;
-    rec[sti] = cur.issue(L, t0, nt, wstage + sti * SB, lane);
-    cp_async_commit();
     cp_async_wait<S - 1>();
     __syncwarp();  // every lane's copies of this stage have landed
     const DecRun R = rec[st];
     if (!R.valid() || !run(R, wstage + st * SB)) break;
+    __syncwarp();
+    rec[st] = cur.issue(L, t0, nt, wstage + st * SB, lane);
+    cp_async_commit();
     st = st + 1 == S ? 0 : st + 1;
   }
   cp_async_wait<0>();  // no copy is left in flight when the warp exits
