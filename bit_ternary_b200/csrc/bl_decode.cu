@@ -54,6 +54,7 @@
 
 #include <atomic>
 #include <cstring>
+#include <utility>
 
 namespace bl {
 
@@ -117,8 +118,7 @@ __host__ __device__ constexpr int dec_fixed_bytes(int acc_cols, int S) {
          + 3 * kDecTok * 4               // s_sx, s_rs, s_amax
          + 2 * kDecodeSlots * 4          // s_cnt, s_gen
          + 16 * (8 + 4 + 4)              // RMSNorm: sums of squares, mean squares, flags
-         + 64                            // abort flag
-         + kDecWarps * S * 16;  // records of the groups in flight
+         + 64;                           // abort flag
 }
 
 __device__ __forceinline__ void dec_mma(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
@@ -257,6 +257,14 @@ __device__ __forceinline__ void cp_async16_pol(void* dst, const void* src, uint6
                "l"(__cvta_generic_to_global(src)), "l"(pol)
                : "memory");
 }
+// As cp_async16_pol, with the destination given as a 32-bit shared address
+// plus a compile-time offset (folded into the instruction).
+template <int OFF>
+__device__ __forceinline__ void cp_async16_pol_at(uint32_t dst, const void* src, uint64_t pol) {
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0+%3], [%1], 16, %2;" ::"r"(dst),
+               "l"(__cvta_generic_to_global(src)), "l"(pol), "n"(OFF)
+               : "memory");
+}
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
@@ -271,6 +279,14 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// The fast path's copies: copy m goes to d0 + m * ROWB (a compile-time offset)
+// from s0 + m * rstep words.
+template <int ROWB, int... Ms>
+__device__ __forceinline__ void dec_fast_copies(uint32_t d0, const uint32_t* s0, int64_t rstep, uint64_t pol,
+                                                std::integer_sequence<int, Ms...>) {
+  (cp_async16_pol_at<Ms * ROWB>(d0, s0 + Ms * rstep, pol), ...);
 }
 
 // One pipeline stage of a warp holds a group's 16 rows, UPT * 64 bytes each
@@ -392,9 +408,17 @@ struct DecCursor {
     auto dst = [&](int m) { return stage + (m * RPM + lr) * RS + 16 * dec_chunk_pos<UPT>(m * RPM + lr, lc); };
     const int64_t rstep = (int64_t)RPM * wpr;  // words between a lane's rows
     if (rv == 16 && n == UPT && (wpr & 3) == 0 && w0 - 4 * lc + 16 * UPT <= wpr) {
-      // Every row present and every unit whole.
+      // Every row present and every unit whole. With an even number of rows
+      // per copy instruction every row of this lane has the parity of lr, so
+      // the destinations are one base plus constant offsets.
+      if constexpr (RPM % 2 == 0 || (UPT & 1)) {
+        const uint32_t d0 = smem_u32(dst(0));
+        const uint32_t* s0 = src;
+        dec_fast_copies<RPM * RS>(d0, s0, rstep, pol, std::make_integer_sequence<int, 16 / RPM>{});
+      } else {
 #pragma unroll
-      for (int m = 0; m < 16 / RPM; ++m) cp_async16_pol(dst(m), src + m * rstep, pol);
+        for (int m = 0; m < 16 / RPM; ++m) cp_async16_pol(dst(m), src + m * rstep, pol);
+      }
     } else if ((wpr & 3) == 0) {
       // Rows start 16-byte aligned; a chunk is wholly in the row or past it.
 #pragma unroll
@@ -759,7 +783,6 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
   float* s_ms = reinterpret_cast<float*>(s_ss + 16);               // [16] mean squares
   int* s_flag = reinterpret_cast<int*>(s_ms + 16);                 // [16] exact path needed
   volatile int* abort_flag = reinterpret_cast<volatile int*>(s_flag + 16);
-  int* s_rec = s_flag + 32;  // [warp][stage] records of the groups in flight (3 ints each, 16-byte slots)
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -796,14 +819,13 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
   uint8_t* wstage = stages + (size_t)warp * S * SB;  // this warp's S stages
   DecCursor<UPT, kAccOut> cur;
   cur.init(L, t0, nt, warp, lane);
-  // What each stage's contraction needs, by stage (every lane writes and
-  // reads the same values).
-  DecRun* rec = reinterpret_cast<DecRun*>(s_rec) + warp * S;
-#pragma unroll 1
-  for (int k = 0; k < S; ++k) {
-    rec[k] = cur.issue(L, t0, nt, wstage + k * SB, lane);
-    cp_async_commit();
-  }
+  // What each stage's contraction needs, in registers (two stages: the
+  // stage index selects one of two records).
+  static_assert(S == 2, "one register record per stage");
+  DecRun rec0 = cur.issue(L, t0, nt, wstage, lane);
+  cp_async_commit();
+  DecRun rec1 = cur.issue(L, t0, nt, wstage + SB, lane);
+  cp_async_commit();
 
   for (int i = tid; i < kDecodeSlots * 16 * AC; i += kDecThreads) s_acc[i] = 0;
   if (tid < kDecodeSlots) {
@@ -1016,12 +1038,13 @@ __global__ void __launch_bounds__(kDecThreads, MT == 1 ? 2 : 1) bl_ternary_decod
   for (;;) {
     cp_async_wait<S - 1>();
     __syncwarp();  // every lane's copies of this stage have landed
-    const DecRun R = rec[st];
+    const DecRun R = st ? rec1 : rec0;
     if (!R.valid() || !run(R, wstage + st * SB)) break;
     __syncwarp();
-    rec[st] = cur.issue(L, t0, nt, wstage + st * SB, lane);
+    const DecRun Rn = cur.issue(L, t0, nt, wstage + st * SB, lane);
     cp_async_commit();
-    st = st + 1 == S ? 0 : st + 1;
+    if (st) rec1 = Rn; else rec0 = Rn;
+    st ^= 1;
   }
   cp_async_wait<0>();  // no copy is left in flight when the warp exits
 }
