@@ -238,6 +238,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------ TMA producer (x)
     if (lane == 0) {
+      // The quantised activations come from the launch this one may overlap
+      // (programmatic dependent launch): wait for it before the first load.
+      asm volatile("griddepcontrol.wait;" ::: "memory");
       int s = 0;
       uint32_t ph = 0;
       JobCursor c{0, 0};
@@ -317,6 +320,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
   } else if (warp == kWarpConst) {
     // ------------------------------------------------ per-token constants, ahead of the epilogue
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // s_x and row sums come from the same launch
     int r = 0;
     uint32_t ph = 0;
     for (int lt = 0; lt < my_tiles; ++lt) {
@@ -503,8 +507,21 @@ static cudaError_t launch_gemm_t(const CUtensorMap& tq, const CUtensorMap& to, c
   constexpr size_t smem = gemm_smem_bytes<BN>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, kGemmThreads, smem, stream>>>(tq, to, p);
-  return cudaGetLastError();
+  // Programmatic dependent launch: TMEM allocation, barrier setup and the
+  // weight unpack (which needs nothing from the previous launch) overlap the
+  // quantiser that precedes this launch; the activation loads and the
+  // per-token constants wait for it (griddepcontrol.wait).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tq, to, p);
 }
 
 // Estimated time of a launch with BN-token tiles, in units of 10 ns on the
