@@ -390,6 +390,31 @@ def test_prefill_sweep_sampled(B, li, M):
     _layer_case(B, "prefill_sweep", li, M, rows=_sample_rows(M))
 
 
+@pytest.mark.parametrize("kind", ["acc", "n_tail"])
+def test_gemm_wide_tiles_output_paths(B, kind):
+    """Launches large enough for the 192-token tiles, through the two output
+    paths the prefill sweep does not reach: the exact int32 accumulators
+    (bitlinear_forward_acc), and y rows that do not start on a 16-byte
+    boundary (N % 4 != 0: plain stores instead of TMA stores). Sampled token
+    rows, every output column."""
+    M, K = 4096, 2560
+    N = 13824 if kind == "acc" else 3843
+    W = WL.weight(N, K, "laplace", 71)
+    x = WL.activations(M, K, "normal", 72)
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    rows = _sample_rows(M, extra=(4095 - 64, 191, 192))  # either side of a 192-token tile edge
+    if kind == "acc":
+        acc = B.forward_acc(dev(x), packed).cpu().numpy()
+        q, _ = O.act_quant(x[rows])
+        acc_ref = O.int_matmul(q, O.unpack_codes(p_ref, K))
+        assert np.array_equal(acc[rows].astype(np.int64), acc_ref)
+    else:
+        y = B.forward(dev(x), packed, D).cpu().numpy()
+        y_ref = O.bitlinear_forward_rows(x, p_ref, D_ref, K, rows)
+        assert_y_close(y[rows], y_ref)
+
+
 @pytest.mark.parametrize("li", range(6))
 def test_embed_batch_sampled(B, li):
     M = 32768
