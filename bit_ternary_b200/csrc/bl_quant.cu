@@ -429,40 +429,74 @@ __global__ void __launch_bounds__(256) act_quant_reg_kernel(const void* __restri
 // interval: a few tokens in a million) the block sums the squares exactly in
 // integers and divides by K.
 template <bool kPerm, int kG>
-__global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restrict__ x, const float* __restrict__ g,
+__global__ void __launch_bounds__(256, kG == 1 ? 3 : (kG == 2 ? 4 : 1)) rms_act_quant_kernel(const float* __restrict__ x, const float* __restrict__ g,
                                                             float eps, int64_t K, int8_t* __restrict__ q,
                                                             float* __restrict__ s_out, int32_t* __restrict__ rowsum_out,
-                                                            uint32_t* __restrict__ err_reset) {
+                                                            uint32_t* __restrict__ err_reset, int64_t M) {
   __shared__ double red_d[8];
   __shared__ float red_f[8];
   __shared__ float s_ms;
   __shared__ int s_exact;
   __shared__ unsigned long long bins[kRmsBins];
   if (err_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err_reset = 0u;
-  const int64_t m = blockIdx.x;
-  const int64_t xr = m * (K >> 2);
   const int ngroups = (int)(K >> 4);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
-  // Cleared before the first block barrier; the warps add their sums at the end.
-  if (rowsum_out != nullptr && threadIdx.x == 0) rowsum_out[m] = 0;
-  // g is loaded with x when it fits in registers (kG == 1), so its latency
-  // overlaps the load of x instead of following the mean-square barrier.
+  // A CTA walks tokens blockIdx.x, blockIdx.x + gridDim.x, ... With one
+  // 16-column group per thread (kG == 1) the next token's row is loaded into
+  // registers while the current one is normalised and quantised, so the row
+  // loads of successive tokens overlap the per-token reductions and barriers,
+  // and g (the same for every token) is loaded once. Wider rows launch one
+  // CTA per token (a second row copy would cost occupancy).
   constexpr bool kGEarly = kG == 1;
-  float4 f[kG][4];
+  constexpr bool kPrefetch = kG == 1;
+  float4 fn[kPrefetch ? kG : 1][4];  // the next token's row (prefetch form only)
   float4 gw[kGEarly ? kG : 1][4];
-  double ss = 0.0;
+  auto load_row = [&](int64_t mm, float4 (&dst)[kG][4]) {
+    const int64_t xr = mm * (K >> 2);
 #pragma unroll
-  for (int i = 0; i < kG; ++i) {
-    const int gi = threadIdx.x + i * blockDim.x;
+    for (int i = 0; i < kG; ++i) {
+      const int gi = threadIdx.x + i * blockDim.x;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      f[i][j] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (gi < ngroups) f[i][j] = __ldg(reinterpret_cast<const float4*>(x) + xr + 4 * gi + j);
-      if (kGEarly) {
+      for (int j = 0; j < 4; ++j) {
+        dst[i][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (gi < ngroups) dst[i][j] = __ldg(reinterpret_cast<const float4*>(x) + xr + 4 * gi + j);
+      }
+    }
+  };
+  if (kGEarly) {
+#pragma unroll
+    for (int i = 0; i < kG; ++i) {
+      const int gi = threadIdx.x + i * blockDim.x;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
         gw[kGEarly ? i : 0][j] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (gi < ngroups) gw[kGEarly ? i : 0][j] = __ldg(reinterpret_cast<const float4*>(g) + 4 * gi + j);
       }
+    }
+  }
+  if constexpr (kPrefetch) {
+    if ((int64_t)blockIdx.x < M) load_row(blockIdx.x, fn);
+  }
+#pragma unroll 1
+  for (int64_t m = blockIdx.x; m < M; m += gridDim.x) {
+  float4 f[kG][4];
+  if constexpr (kPrefetch) {
+#pragma unroll
+    for (int i = 0; i < kG; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) f[i][j] = fn[i][j];
+    if (m + gridDim.x < M) load_row(m + gridDim.x, fn);
+  } else {
+    load_row(m, f);
+  }
+  // Cleared before the first block barrier; the warps add their sums at the end.
+  if (rowsum_out != nullptr && threadIdx.x == 0) rowsum_out[m] = 0;
+  double ss = 0.0;
+#pragma unroll
+  for (int i = 0; i < kG; ++i) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
       ss += (double)f[i][j].x * f[i][j].x + (double)f[i][j].y * f[i][j].y;
       ss += (double)f[i][j].z * f[i][j].z + (double)f[i][j].w * f[i][j].w;
     }
@@ -558,6 +592,7 @@ __global__ void __launch_bounds__(256) rms_act_quant_kernel(const float* __restr
     for (int o = 16; o > 0; o >>= 1) rsum += __shfl_xor_sync(0xFFFFFFFFu, rsum, o);
     if (lane == 0) atomicAdd(rowsum_out + m, rsum);
   }
+  }  // token loop
 }
 
 // ------------------------------------------------------------ launchers --
@@ -678,8 +713,19 @@ cudaError_t launch_rms_act_quant(const float* x, const float* g, float eps, int6
   kg = kg <= 1 ? 1 : (kg <= 2 ? 2 : 4);
   int threads = (int)(((ngroups + kg - 1) / kg + 31) / 32 * 32);
   if (threads < 32) threads = 32;
-#define BL_RQ(P, G) \
-  rms_act_quant_kernel<P, G><<<(unsigned)M, threads, 0, stream>>>(x, g, eps, K, q, s_x, rowsum, err_reset)
+  // Persistent CTAs (as many as fit, up to one per token), each walking tokens.
+  int dev = 0, sms = 0, per_sm = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+#define BL_RQ(P, G)                                                                                            \
+  do {                                                                                                         \
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rms_act_quant_kernel<P, G>, threads, 0);      \
+    if (e != cudaSuccess) return e;                                                                            \
+    int64_t grid = (int64_t)sms * (per_sm < 1 ? 1 : per_sm);                                                  \
+    if (G > 1 || grid > M) grid = M; /* one CTA per token unless the row prefetch runs */                    \
+    rms_act_quant_kernel<P, G><<<(unsigned)grid, threads, 0, stream>>>(x, g, eps, K, q, s_x, rowsum, err_reset, M); \
+  } while (0)
   if (permuted) {
     if (kg == 1) BL_RQ(true, 1); else if (kg == 2) BL_RQ(true, 2); else BL_RQ(true, 4);
   } else {
