@@ -629,6 +629,22 @@ def test_forward_bf16(B, M, N, K):
 
 
 # --------------------------------------------------- RMSNorm + ActQuant
+@pytest.mark.parametrize("K", [1024, 2560])
+def test_rmsnorm_quant_act_many_tokens_per_cta(B, K):
+    """Enough tokens that every persistent CTA of the RMSNorm quantiser walks
+    many of them (the next row's loads in flight while the current one is
+    quantised): sampled tokens, including both ends, bit for bit."""
+    M = 20000
+    x = WL.activations(M, K, "outlier_tokens", 90 + K, meta={"frac": 0.02, "scale": 20.0})
+    g = np.random.default_rng(91 + K).uniform(0.5, 2.0, K).astype(np.float32)
+    q, s_x, rs = B.rmsnorm_quant_act(dev(x), dev(g))
+    rows = _sample_rows(M, extra=(1, 147, 148, 149, 1775, 1776, 1777, M - 2))
+    q_ref, s_ref = O.rmsnorm_act_quant(x[rows], g)
+    assert np.array_equal(q.cpu().numpy()[rows], q_ref)
+    assert np.array_equal(s_x.cpu().numpy()[rows], s_ref)
+    assert np.array_equal(rs.cpu().numpy()[rows], q_ref.astype(np.int64).sum(axis=1))
+
+
 @pytest.mark.parametrize("M,K,xdist", [(1, 2560, "student_t"), (5, 1024, "outlier_tokens"), (64, 3072, "normal"),
                                        (300, 640, "student_t"), (17, 16384, "normal")])
 def test_rmsnorm_quant_act_bitexact(B, M, K, xdist):
