@@ -1099,36 +1099,37 @@ bool decode_fits(int64_t M, int64_t K, bool rms) {
   return decode_smem(q, M) >= 0;
 }
 
-// Bytes of launch tile gt (rows x K/4).
-static int64_t host_tile_bytes(const DecHead& L, int gt) {
-  int p = 0;
-  while (p + 1 < L.nprob && gt >= L.pr[p + 1].tile0) ++p;
-  const DecProblem& P = L.pr[p];
-  const int64_t row0 = (int64_t)(gt - P.tile0) * 16;
-  const int64_t rows = P.N - row0 < 16 ? P.N - row0 : 16;
-  return rows * P.wpr * 4;
-}
-
 // Split the launch's tiles into `grid` contiguous ranges of about equal bytes,
-// at least one tile each.
+// at least one tile each. A problem's tiles all hold 16 rows of the same
+// length (its last tile possibly fewer rows), so the boundary nearest to each
+// 1/grid of the bytes is computed directly, problem by problem: O(grid +
+// problems) host work per launch.
 static void partition_by_bytes(DecLaunch& LP, int grid) {
   const DecHead& L = LP.h;
   int* cta_start = LP.cta_start;
   int64_t total = 0;
-  for (int gt = 0; gt < L.total_tiles; ++gt) total += host_tile_bytes(L, gt);
-  int64_t acc = 0;
-  int cta = 0, start = 0;
-  cta_start[0] = 0;
-  for (int gt = 0; gt < L.total_tiles; ++gt) {
-    const int64_t tb = host_tile_bytes(L, gt);
-    const int64_t target = total * (cta + 1) / grid;
-    if (cta + 1 < grid && gt > start && acc + tb / 2 > target && L.total_tiles - gt >= grid - cta - 1) {
-      cta_start[++cta] = gt;
-      start = gt;
-    }
-    acc += tb;
+  int64_t pre[kDecodeMaxGroup + 1];
+  pre[0] = 0;
+  for (int p = 0; p < L.nprob; ++p) {
+    pre[p + 1] = pre[p] + (int64_t)L.pr[p].N * L.pr[p].wpr * 4;
+    total = pre[p + 1];
   }
-  for (int k = cta + 1; k <= grid; ++k) cta_start[k] = L.total_tiles;
+  cta_start[0] = 0;
+  int p = 0;
+  for (int c = 1; c < grid; ++c) {
+    const int64_t target = total * c / grid;
+    while (p + 1 < L.nprob && pre[p + 1] <= target) ++p;
+    const DecProblem& P = L.pr[p];
+    const int64_t tb = 64 * (int64_t)P.wpr;  // bytes of a full tile
+    int64_t k = tb > 0 ? (target - pre[p] + tb / 2) / tb : 0;
+    if (k > P.tiles) k = P.tiles;
+    int gt = P.tile0 + (int)k;
+    // Strictly increasing, and enough tiles left for the CTAs after this one.
+    if (gt <= cta_start[c - 1]) gt = cta_start[c - 1] + 1;
+    if (gt > L.total_tiles - (grid - c)) gt = L.total_tiles - (grid - c);
+    cta_start[c] = gt;
+  }
+  cta_start[grid] = L.total_tiles;
 }
 
 cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g, float eps, uint32_t* err, bool pdl,
