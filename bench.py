@@ -378,6 +378,8 @@ def run_ours(a):
             "decode_stream": lambda: bench_decode_stream(B, torch, dev, stream, capture, time_graph, max_ranks,
                                                          hbm_peak),
             "i2s": lambda: bench_i2s(B, torch, dev, stream, hbm_peak, layouts=tuple(a.i2s_layouts.split(","))),
+            "block_scale": lambda: bench_block_scale(B, torch, dev, stream, capture, time_graph, max_ranks,
+                                                     hbm_peak, i8_burst, rank),
         }
         res = {name: parts[name]() for name in a.only.split(",")}
         if rank == 0:
@@ -606,6 +608,11 @@ def run_ours(a):
     if not a.no_prefill and not a.ncu_small:
         bf16 = bench_bf16(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, rank)
 
+    # ------------------------------------------------- per-256-block scale variant
+    blk = None
+    if not a.no_prefill and not a.ncu_small:
+        blk = bench_block_scale(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, i8_burst, rank)
+
     # --------------------------------------------------------------- cpu baseline
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline and not a.ncu_small:
@@ -652,6 +659,7 @@ def run_ours(a):
         "i2s": i2s,
         "bf16_inputs": bf16,
         "rmsnorm_actquant": rms,
+        "block_scale": blk,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)
@@ -912,6 +920,130 @@ def bench_bf16(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, 
                    "GB/s_algorithmic": round(alg / t / 1e9, 1), "frac_hbm": round(alg / t / 1e9 / hbm_peak, 4),
                    "l2": "rotates over 4 weight copies"}
     del Wbs
+    torch.cuda.empty_cache()
+    return out
+
+
+def bench_block_scale(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_peak, i8_burst, rank):
+    """The per-256-block scale variant (D [N, ceil(K/256)]): the decode layer set at M=1, the
+    forward kernel's streaming rate on 16 stacked gate_up weights, a prefill-sized call on the
+    CUDA-core path, and the per-block pack. Bytes per call: NK/4 packed + 4*N*nb scales + 4MK x
+    + 4MN y."""
+    out = {}
+    wl = WL.WORKLOADS[HEADLINE]
+    layers = list(wl.layers)
+    rot = 16
+
+    def nbytes(l, M):
+        nb = (l.K + 255) // 256
+        return l.N * l.K // 4 + 4 * l.N * nb + 4 * M * l.K + 4 * M * l.N
+
+    with torch.cuda.stream(stream):
+        base = []
+        for li, l in enumerate(layers):
+            W = torch.from_numpy(WL.weight(l.N, l.K, wl.w_dist, wl.seed + 17 * rank, layer=li)).to(dev)
+            base.append(B.pack_weights_blocks(W))
+            del W
+        packs = [[(p.clone(), D.clone()) for (p, D) in base] for _ in range(rot)]
+        xs = [[torch.from_numpy(WL.activations(1, l.K, wl.x_dist, wl.seed + r, layer=li, meta=wl.meta)).to(dev)
+               for li, l in enumerate(layers)] for r in range(rot)]
+        ys = [torch.empty((1, l.N), dtype=torch.float32, device=dev) for l in layers]
+        wss = [torch.zeros(max(256, B.workspace_size(1, l.N, l.K)), dtype=torch.uint8, device=dev) for l in layers]
+    torch.cuda.synchronize(dev)
+
+    def step(i):
+        r = i % rot
+        for li in range(len(layers)):
+            p, D = packs[r][li]
+            B.forward_blocks(xs[r][li], p, D, out=ys[li], ws=wss[li])
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i)
+    torch.cuda.synchronize(dev)
+    n = 64
+    g = capture(step, n)
+    with torch.cuda.stream(stream):
+        g.replay()
+    t = max_ranks(time_graph(g)) / n * 1e-3
+    tot = sum(nbytes(l, 1) for l in layers)
+    out["decode_layer_set"] = {"us_per_step": round(t * 1e6, 2), "GB/s": round(tot / t / 1e9, 1),
+                               "frac_hbm": round(tot / t / 1e9 / hbm_peak, 4), "bytes_per_step": tot,
+                               "note": "four bitlinear_forward_blocks calls per step (ActQuant launch + "
+                                       f"block-scale kernel each), M=1, weights rotating over {rot} copies"}
+    del g, packs, xs, base
+    torch.cuda.empty_cache()
+
+    # Streaming rate: one call over 16 stacked gate_up weights (141.6 MB packed).
+    l = layers[2]
+    Nst = 16 * l.N
+    with torch.cuda.stream(stream):
+        W1 = torch.from_numpy(WL.weight(l.N, l.K, wl.w_dist, wl.seed, layer=2)).to(dev)
+        p1, D1 = B.pack_weights_blocks(W1)
+        del W1
+        pst, Dst = p1.repeat(16, 1).contiguous(), D1.repeat(16, 1).contiguous()
+        copies = 2
+        pk = [(pst.clone(), Dst.clone()) for _ in range(copies)]
+        del pst, Dst
+        x1 = torch.from_numpy(WL.activations(1, l.K, wl.x_dist, wl.seed, layer=2, meta=wl.meta)).to(dev)
+        y1 = torch.empty((1, Nst), dtype=torch.float32, device=dev)
+        ws1 = torch.zeros(max(256, B.workspace_size(1, Nst, l.K)), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize(dev)
+    g = capture(lambda i: B.forward_blocks(x1, pk[i % copies][0], pk[i % copies][1], out=y1, ws=ws1), 16)
+    with torch.cuda.stream(stream):
+        g.replay()
+    t = max_ranks(time_graph(g)) / 16 * 1e-3
+    sb = Nst * l.K // 4 + 4 * Nst * ((l.K + 255) // 256) + 4 * l.K + 4 * Nst
+    out["streaming_m1"] = {"rows": Nst, "K": l.K, "us": round(t * 1e6, 2), "GB/s": round(sb / t / 1e9, 1),
+                           "frac_hbm": round(sb / t / 1e9 / hbm_peak, 4),
+                           "note": f"16 stacked gate_up weights, {copies} copies alternating (each 150 MB)"}
+    del g, pk
+    torch.cuda.empty_cache()
+
+    # Prefill size on the CUDA-core path: gate_up at M=512.
+    M = 512
+    with torch.cuda.stream(stream):
+        W1 = torch.from_numpy(WL.weight(l.N, l.K, "laplace", 9)).to(dev)
+        pp, DD = B.pack_weights_blocks(W1)
+        del W1
+        xp = torch.from_numpy(WL.activations(M, l.K, "normal", 9)).to(dev)
+        yp = torch.empty((M, l.N), dtype=torch.float32, device=dev)
+        wsp = torch.zeros(max(256, B.workspace_size(M, l.N, l.K)), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize(dev)
+    g = capture(lambda i: B.forward_blocks(xp, pp, DD, out=yp, ws=wsp), 8)
+    with torch.cuda.stream(stream):
+        g.replay()
+    t = max_ranks(time_graph(g)) / 8 * 1e-3
+    ops = 2.0 * M * l.N * l.K
+    out["prefill_m512_gate_up"] = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 2),
+                                   "frac_int8_peak": round(ops / t / 1e12 / (i8_burst), 4),
+                                   "note": "CUDA-core dp4a path (no tensor-core kernel for this variant)"}
+    del g, pp, DD, xp, yp
+    torch.cuda.empty_cache()
+
+    # Per-block pack of gate_up (offline).
+    with torch.cuda.stream(stream):
+        W0 = torch.from_numpy(WL.weight(l.N, l.K, "normal", 5)).to(dev)
+        Ws = [W0.clone() for _ in range(4)]
+        del W0
+        ws = torch.zeros(4096, dtype=torch.uint8, device=dev)
+        B.pack_weights_blocks(Ws[0], ws=ws)
+        torch.cuda.synchronize(dev)
+        ts = []
+        for it in range(8):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            B.pack_weights_blocks(Ws[(it + 1) % len(Ws)], ws=ws)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(e0.elapsed_time(e1))
+    t = statistics.median(ts) * 1e-3
+    alg = 4 * l.N * l.K + l.N * l.K // 4 + 4 * l.N * ((l.K + 255) // 256)
+    out["pack"] = {"layer": f"gate_up {l.K}->{l.N}", "ms": round(t * 1e3, 4),
+                   "GB/s_algorithmic": round(alg / t / 1e9, 1), "frac_hbm": round(alg / t / 1e9 / hbm_peak, 4),
+                   "note": "synchronous call (includes the status read-back); W rotates over 4 copies"}
+    del Ws
     torch.cuda.empty_cache()
     return out
 

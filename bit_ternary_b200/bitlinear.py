@@ -27,6 +27,9 @@ __all__ = [
     "forward_q",
     "rmsnorm_quant_act",
     "forward_rmsnorm",
+    "block_scales",
+    "pack_weights_blocks",
+    "forward_blocks",
     "workspace_size",
     "workspace_error",
     "BitLinear",
@@ -217,6 +220,47 @@ def forward_rmsnorm(x: torch.Tensor, g: torch.Tensor, packed: torch.Tensor, D: t
         ws = _alloc_ws(workspace_size(M, N, K), x.device)
     _lib.call("bitlinear_forward_rmsnorm", x.data_ptr(), g.data_ptr(), float(eps), M, N, K, packed.data_ptr(),
               D.data_ptr(), y.data_ptr(), ws.data_ptr(), ws.numel(), _stream_handle(x.device))
+    return y
+
+
+def block_scales(K: int) -> int:
+    """nb = ceil(K / 256): scale blocks per row of the per-256-block variant."""
+    nb = int(_lib.lib().bitlinear_block_scales(K))
+    if nb <= 0:
+        raise ValueError(f"invalid K = {K}")
+    return nb
+
+
+def pack_weights_blocks(W: torch.Tensor, ws: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Per-256-block WeightQuant + pack: fp32 W [N, K] -> (packed int32 [N, K/16], D fp32 [N, nb])."""
+    _need_cuda(W, "W", torch.float32)
+    N, K = W.shape
+    nb = block_scales(K)
+    packed = torch.empty((N, K // 16), dtype=torch.int32, device=W.device)
+    D = torch.empty((N, nb), dtype=torch.float32, device=W.device)
+    L = _lib.lib()
+    if ws is None:
+        ws = _alloc_ws(L.bitlinear_pack_workspace_size(N, K), W.device)
+    _lib.call("bitlinear_pack_weights_blocks", W.data_ptr(), N, K, packed.data_ptr(), D.data_ptr(),
+              ws.data_ptr(), ws.numel(), _stream_handle(W.device))
+    return packed, D
+
+
+def forward_blocks(x: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,
+                   out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y [M, N] from per-256-block scaled weights (D fp32 [N, ceil(K/256)])."""
+    K = x.shape[-1]
+    M, N = _fwd_args(x, packed, K)
+    nb = block_scales(K)
+    if tuple(D.shape) != (N, nb):
+        raise ValueError(f"D must have shape [N, nb] = [{N}, {nb}], got {list(D.shape)}")
+    _need_cuda(D, "D", torch.float32)
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _need_cuda(y, "out", torch.float32)
+    if ws is None:
+        ws = _alloc_ws(workspace_size(M, N, K), x.device)
+    _lib.call("bitlinear_forward_blocks", x.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(), y.data_ptr(),
+              ws.data_ptr(), ws.numel(), _stream_handle(x.device))
     return y
 
 

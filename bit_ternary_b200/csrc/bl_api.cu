@@ -334,6 +334,53 @@ int bitlinear_forward_rmsnorm(const float* x, const float* g, float eps, int64_t
   return cuda_status(bl::launch_gemm(M, N, K, packed, D, y, nullptr, ws, s, sms));
 }
 
+int64_t bitlinear_block_scales(int64_t K) {
+  if (check_k(K) != BL_OK) return 0;
+  return bl::scale_blocks(K);
+}
+
+int bitlinear_pack_weights_blocks(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
+                                  size_t ws_bytes, bl_stream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  if (N <= 0 || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
+  if (W == nullptr || packed == nullptr || D == nullptr || ws == nullptr) return BL_ERR_NULL;
+  if (!aligned16(W) || !aligned16(packed) || !aligned16(D) || !aligned256(ws)) return BL_ERR_ALIGN;
+  if (ws_bytes < bl::kPackWsBytes) return BL_ERR_WORKSPACE;
+  const int sms = num_sms_current();
+  if (sms <= 0) return BL_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* word = static_cast<uint32_t*>(ws);
+  if (cudaMemsetAsync(word, 0, sizeof(uint32_t), s) != cudaSuccess) return BL_ERR_CUDA;
+  if (bl::launch_pack_blocks(W, N, K, packed, D, word, s, sms) != cudaSuccess) return BL_ERR_CUDA;
+  uint32_t status = 0;
+  if (cudaMemcpyAsync(&status, word, sizeof(status), cudaMemcpyDeviceToHost, s) != cudaSuccess) return BL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
+  return status == 0u ? BL_OK : BL_ERR_NONFINITE;
+}
+
+int bitlinear_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                             const float* D, float* y, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  int st = check_k(K);
+  if (st != BL_OK) return st;
+  st = check_mn(M, N);
+  if (st != BL_OK) return st;
+  if (M == 0 || N == 0) return BL_OK;
+  if (x == nullptr || packed == nullptr || D == nullptr || y == nullptr || ws == nullptr) return BL_ERR_NULL;
+  if (!aligned16(x) || !aligned16(packed) || !aligned16(D) || !aligned16(y) || !aligned256(ws)) return BL_ERR_ALIGN;
+  if (ws_bytes < bitlinear_workspace_size(M, N, K)) return BL_ERR_WORKSPACE;
+  const int sms = num_sms_current();
+  if (sms <= 0) return BL_ERR_CUDA;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  st = cuda_status(bl::launch_act_quant(x, false, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
+                                        reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
+                                        reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), true, s,
+                                        reinterpret_cast<uint32_t*>(base)));
+  if (st != BL_OK) return st;
+  return cuda_status(bl::launch_forward_blocks(M, N, K, packed, D, y, ws, s, sms));
+}
+
 size_t bitlinear_batch_workspace_size(const bl_linear_call* calls, int count) {
   size_t need = bl::kHeaderBytes;
   if (calls == nullptr || count < 0) return 0;

@@ -87,6 +87,23 @@ cudaError_t launch_q_prepare(const int8_t* q, const float* s_x, int64_t M, int64
 cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D, float* y,
                         int32_t* acc_out, void* ws, cudaStream_t stream, int num_sms);
 
+// Per-256-block scale variant (bl_block.cu): blocks of 256 consecutive
+// columns within a row, D fp32 [N, scale_blocks(K)].
+constexpr int kScaleBlock = 256;
+inline int64_t scale_blocks(int64_t K) { return (K + kScaleBlock - 1) / kScaleBlock; }
+constexpr size_t kBlockFwdSmemMax = 200 * 1024;
+// status: a device word that gets bit 0 OR-ed in for a block holding a
+// non-finite weight (that block's words and scale are left unwritten).
+cudaError_t launch_pack_blocks(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, uint32_t* status,
+                               cudaStream_t stream, int num_sms);
+// Tokens per CTA tile of the block forward (its activation codes fit in
+// kBlockFwdSmemMax of shared memory); always >= 1 for K <= kMaxK.
+int block_forward_tile(int64_t M, int64_t K);
+// Expects the permuted activation codes and s_x in the forward workspace
+// (launch_act_quant with permuted = true).
+cudaError_t launch_forward_blocks(int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D, float* y,
+                                  const void* ws, cudaStream_t stream, int num_sms);
+
 cudaError_t launch_selftest_wait(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);
 
 }  // namespace bl

@@ -217,6 +217,47 @@ BL_API int bitlinear_forward_rmsnorm(const float* x, const float* g, float eps, 
                                      int64_t K, const uint32_t* packed, const float* D, float* y,
                                      void* ws, size_t ws_bytes, bl_stream_t stream);
 
+/* ------------------------------------------- per-256-block scale variant --- */
+
+/* "Core AI model zoo - BitVLA" section 2 contrasts BitNet's per-row scale
+ * D [N, 1] with BitCPM's per-256-block scale, which it names without defining.
+ * Reading implemented here: a block is 256 consecutive columns of one row
+ * (the last block of a row holds K % 256 columns when that is not zero); each
+ * block is quantised with the per-tensor formula above applied to the block
+ * alone (exact mean of |W| over the block, floor 1e-5, s = RN(1/mean_c),
+ * code = clamp(rint(RN(W*s)), -1, 1)); the packed words are the same format;
+ * D is fp32 [N, nb] row-major with nb = ceil(K / 256), D[n,b] = mean_c of
+ * block (n, b). The product, per token m and row n:
+ *   acc_b = sum over block b's columns of q[m,k] * code[n,k]   (exact)
+ *   t_b   = RN( RN(float(acc_b) / s_x[m]) * D[n,b] )
+ *   y     = t_0, then y = RN(y + t_b) for b = 1 .. nb-1 (ascending order). */
+
+/* nb = ceil(K / 256), the number of scale blocks per row; 0 for an invalid K. */
+BL_API int64_t bitlinear_block_scales(int64_t K);
+
+/* WeightQuant per 256-column block + 2-bit pack.
+ *   W       device fp32 [N, K], read only.
+ *   packed  device uint32 [N, K/16], fully overwritten.
+ *   D       device fp32 [N, nb], fully overwritten.
+ *   ws      device scratch of ws_bytes >= bitlinear_pack_workspace_size().
+ * Synchronous (it reads back the status word). BL_ERR_NONFINITE if a block
+ * holds Inf or NaN; that block's words and scale are then left unwritten and
+ * every other block is packed. N >= 1 is required. */
+BL_API int bitlinear_pack_weights_blocks(const float* W, int64_t N, int64_t K,
+                                         uint32_t* packed, float* D,
+                                         void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* y [M, N] from per-block scaled weights (packed and D from
+ * bitlinear_pack_weights_blocks): ActQuant of x into ws (as bitlinear_forward
+ * does), then a CUDA-core kernel that contracts each 256-column block with
+ * dp4a and adds the block terms in ascending order. Any M (tiles of up to 16
+ * tokens per CTA; there is no tensor-core path for this variant). Same
+ * workspace as bitlinear_forward (bitlinear_workspace_size(M, N, K)); every
+ * device pointer 16-byte aligned, ws 256-byte aligned. Asynchronous. */
+BL_API int bitlinear_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K,
+                                    const uint32_t* packed, const float* D, float* y,
+                                    void* ws, size_t ws_bytes, bl_stream_t stream);
+
 /* ---------------------------------------------------------------- batch --- */
 
 /* One BitLinear of a batch: y [M,N] = F.linear(ActQuant(x [M,K]), W) from
