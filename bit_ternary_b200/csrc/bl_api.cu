@@ -371,14 +371,8 @@ int bitlinear_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, co
   if (ws_bytes < bitlinear_workspace_size(M, N, K)) return BL_ERR_WORKSPACE;
   const int sms = num_sms_current();
   if (sms <= 0) return BL_ERR_CUDA;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  uint8_t* base = static_cast<uint8_t*>(ws);
-  st = cuda_status(bl::launch_act_quant(x, false, M, K, reinterpret_cast<int8_t*>(base + bl::ws_q_off(M)),
-                                        reinterpret_cast<float*>(base + bl::ws_sx_off(M)),
-                                        reinterpret_cast<int32_t*>(base + bl::ws_rowsum_off(M)), true, s,
-                                        reinterpret_cast<uint32_t*>(base)));
-  if (st != BL_OK) return st;
-  return cuda_status(bl::launch_forward_blocks(M, N, K, packed, D, y, ws, s, sms));
+  return cuda_status(
+      bl::launch_forward_blocks(x, M, N, K, packed, D, y, ws, reinterpret_cast<cudaStream_t>(stream), sms));
 }
 
 size_t bitlinear_batch_workspace_size(const bl_linear_call* calls, int count) {

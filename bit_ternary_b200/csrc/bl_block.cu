@@ -170,6 +170,24 @@ __host__ __device__ inline size_t block_fwd_smem(int tm, int64_t K, int nb) {
   return (size_t)tm * (size_t)K + 4 * (size_t)tm * (size_t)nb + 4 * (size_t)tm;
 }
 
+// One warp step: the packed words of columns [16*w0, 16*w0 + 4096) of a row
+// (8 per lane) and this lane's block scale after the reduction.
+struct BlockStep {
+  uint32_t w[8];
+  float d;
+};
+
+__device__ __forceinline__ void load_step(BlockStep& st, const uint32_t* __restrict__ prow,
+                                          const float* __restrict__ drow, int w0, int KW, int nb, int lane, int jl) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int idx = w0 + lane + 32 * i;
+    st.w[i] = idx < KW ? __ldg(prow + idx) : 0u;
+  }
+  const int bb = (w0 >> 4) + jl;
+  st.d = bb < nb ? __ldg(drow + bb) : 0.0f;
+}
+
 template <int TM>
 __global__ void __launch_bounds__(256) bl_block_scale_forward_kernel(BlockFwdArgs a) {
   extern __shared__ __align__(16) uint8_t smem[];
@@ -183,13 +201,33 @@ __global__ void __launch_bounds__(256) bl_block_scale_forward_kernel(BlockFwdArg
   int32_t* bsum = reinterpret_cast<int32_t*>(smem + (size_t)a.tm * K);
   float* sxs = reinterpret_cast<float*>(smem + (size_t)a.tm * K + 4 * (size_t)a.tm * nb);
 
+  // This warp's rows are row0 + warp + 8*j; each is `steps` warp steps long.
+  // The (row, step) units run in order with the next unit's loads in flight.
+  // After the reduce-scatter below, lane L holds the sum of block
+  // j = 2 * ((L >> 1) & 7) + (L >> 4) of a step; block j is read back from
+  // lane 16 * (j & 1) + 2 * (j >> 1).
+  const int jl = 2 * ((lane >> 1) & 7) + (lane >> 4);
+  const int64_t row0 = tile_n * a.rows_per_cta;
+  const int64_t row_end = std::min<int64_t>(row0 + a.rows_per_cta, a.N);
+  const int64_t first = row0 + warp;
+  const int nrows = first < row_end ? (int)((row_end - first + kFwdWarps - 1) / kFwdWarps) : 0;
+  const int steps = (KW + kStepWords - 1) / kStepWords;
+  BlockStep nxt;
+  if (nrows > 0) load_step(nxt, a.packed + first * KW, a.D + first * nb, 0, KW, nb, lane, jl);
+
+  // The weights above do not depend on the previous kernel in the stream (the
+  // activation quantiser); its codes and scales are read only after it is done.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+
   // The tile's activation codes (tm rows of K bytes, contiguous) and scales.
+  // Plain loads: a read-only-path load (__ldg) counts as invariant memory and
+  // may be hoisted above the wait, before the quantiser has written it.
   {
     const uint4* src = reinterpret_cast<const uint4*>(a.q + t0 * a.K);
     uint4* dst = reinterpret_cast<uint4*>(qs);
     const int n16 = tm * KW;
-    for (int i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = __ldg(src + i);
-    if (threadIdx.x < tm) sxs[threadIdx.x] = __ldg(a.sx + t0 + threadIdx.x);
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) dst[i] = src[i];
+    if (threadIdx.x < tm) sxs[threadIdx.x] = a.sx[t0 + threadIdx.x];
   }
   __syncthreads();
   // Per-token block sums of q (the codes are stored as code + 1).
@@ -207,79 +245,340 @@ __global__ void __launch_bounds__(256) bl_block_scale_forward_kernel(BlockFwdArg
   }
   __syncthreads();
 
-  // After the reduce-scatter below, lane L holds the sum of block
-  // j = 2 * ((L >> 1) & 7) + (L >> 4) of the step; block j is read back from
-  // lane 16 * (j & 1) + 2 * (j >> 1).
-  const int jl = 2 * ((lane >> 1) & 7) + (lane >> 4);
   const bool b3 = (lane & 8) != 0, b2 = (lane & 4) != 0, b1 = (lane & 2) != 0;
-  const int64_t row0 = tile_n * a.rows_per_cta;
-  const int64_t row_end = std::min<int64_t>(row0 + a.rows_per_cta, a.N);
-  for (int64_t r = row0 + warp; r < row_end; r += kFwdWarps) {
-    const uint32_t* prow = a.packed + r * KW;
-    const float* drow = a.D + r * nb;
-    float yr[TM];
+  float yr[TM];
 #pragma unroll
-    for (int m = 0; m < TM; ++m) yr[m] = -0.0f;  // -0 + t == t for every t
-    for (int w0 = 0; w0 < KW; w0 += kStepWords) {
-      uint32_t wv[8];
+  for (int m = 0; m < TM; ++m) yr[m] = -0.0f;  // -0 + t == t for every t
+  int j = 0, st = 0;                              // current row index (of this warp) and step
+  const int units = nrows * steps;
+  for (int u = 0; u < units; ++u) {
+    const BlockStep cur = nxt;
+    const int64_t r = first + (int64_t)kFwdWarps * j;
+    const int w0 = st * kStepWords;
+    if (u + 1 < units) {
+      const int jn = st + 1 == steps ? j + 1 : j, sn = st + 1 == steps ? 0 : st + 1;
+      const int64_t rn = first + (int64_t)kFwdWarps * jn;
+      load_step(nxt, a.packed + rn * KW, a.D + rn * nb, sn * kStepWords, KW, nb, lane, jl);
+    }
+    const int bb = (w0 >> 4) + jl;              // this lane's block after the reduction
+    const int nblk = min(16, nb - (w0 >> 4));   // blocks present in this step
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int idx = w0 + lane + 32 * i;
-        wv[i] = idx < KW ? __ldg(prow + idx) : 0u;
-      }
-      const int bb = (w0 >> 4) + jl;  // this lane's block after the reduction
-      const float dv = bb < nb ? __ldg(drow + bb) : 0.0f;
-      const int nblk = min(16, nb - (w0 >> 4));  // blocks present in this step
+    for (int m = 0; m < TM; ++m) {
+      if (m < tm) {
+        const int8_t* qrow = qs + (size_t)m * K;
+        int av[8];
 #pragma unroll
-      for (int m = 0; m < TM; ++m) {
-        if (m < tm) {
-          const int8_t* qrow = qs + (size_t)m * K;
-          int av[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int idx = w0 + lane + 32 * i;
-            int s = 0;
-            if (idx < KW) {
-              const uint4 qq = *reinterpret_cast<const uint4*>(qrow + 16 * idx);
-              const uint32_t w = wv[i];
-              s = __dp4a((int)(w & 0x03030303u), (int)qq.x, s);
-              s = __dp4a((int)((w >> 2) & 0x03030303u), (int)qq.y, s);
-              s = __dp4a((int)((w >> 4) & 0x03030303u), (int)qq.z, s);
-              s = __dp4a((int)((w >> 6) & 0x03030303u), (int)qq.w, s);
-            }
-            av[i] = s;
+        for (int i = 0; i < 8; ++i) {
+          const int idx = w0 + lane + 32 * i;
+          int s = 0;
+          if (idx < KW) {
+            const uint4 qq = *reinterpret_cast<const uint4*>(qrow + 16 * idx);
+            const uint32_t w = cur.w[i];
+            s = __dp4a((int)(w & 0x03030303u), (int)qq.x, s);
+            s = __dp4a((int)((w >> 2) & 0x03030303u), (int)qq.y, s);
+            s = __dp4a((int)((w >> 4) & 0x03030303u), (int)qq.z, s);
+            s = __dp4a((int)((w >> 6) & 0x03030303u), (int)qq.w, s);
           }
-          // Reduce-scatter over the 16 lanes of each half-warp: 8 shuffles
-          // leave lane L with the sum of av[(L >> 1) & 7] over its half.
-          int c4[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int send = b3 ? av[k] : av[k + 4];
-            const int keep = b3 ? av[k + 4] : av[k];
-            c4[k] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 8);
-          }
-          int c2[2];
-#pragma unroll
-          for (int k = 0; k < 2; ++k) {
-            const int send = b2 ? c4[k] : c4[k + 2];
-            const int keep = b2 ? c4[k + 2] : c4[k];
-            c2[k] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 4);
-          }
-          int c1 = (b1 ? c2[1] : c2[0]) + __shfl_xor_sync(0xFFFFFFFFu, b1 ? c2[0] : c2[1], 2);
-          c1 += __shfl_xor_sync(0xFFFFFFFFu, c1, 1);
-          float t = 0.0f;
-          if (bb < nb) t = rescale(c1 - bsum[m * nb + bb], sxs[m], dv);
-          float yv = yr[m];
-          for (int j = 0; j < nblk; ++j) yv = __fadd_rn(yv, __shfl_sync(0xFFFFFFFFu, t, 16 * (j & 1) + 2 * (j >> 1)));
-          yr[m] = yv;
+          av[i] = s;
         }
+        // Reduce-scatter over the 16 lanes of each half-warp: 8 shuffles
+        // leave lane L with the sum of av[(L >> 1) & 7] over its half.
+        int c4[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int send = b3 ? av[k] : av[k + 4];
+          const int keep = b3 ? av[k + 4] : av[k];
+          c4[k] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 8);
+        }
+        int c2[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const int send = b2 ? c4[k] : c4[k + 2];
+          const int keep = b2 ? c4[k + 2] : c4[k];
+          c2[k] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, 4);
+        }
+        int c1 = (b1 ? c2[1] : c2[0]) + __shfl_xor_sync(0xFFFFFFFFu, b1 ? c2[0] : c2[1], 2);
+        c1 += __shfl_xor_sync(0xFFFFFFFFu, c1, 1);
+        float t = 0.0f;
+        if (bb < nb) t = rescale(c1 - bsum[m * nb + bb], sxs[m], cur.d);
+        float yv = yr[m];
+        for (int jb = 0; jb < nblk; ++jb) yv = __fadd_rn(yv, __shfl_sync(0xFFFFFFFFu, t, 16 * (jb & 1) + 2 * (jb >> 1)));
+        yr[m] = yv;
       }
     }
-    if (lane == 0) {
+    if (++st == steps) {
+      if (lane == 0) {
 #pragma unroll
-      for (int m = 0; m < TM; ++m)
-        if (m < tm) a.y[(t0 + m) * a.N + r] = yr[m];
+        for (int m = 0; m < TM; ++m)
+          if (m < tm) a.y[(t0 + m) * a.N + r] = yr[m];
+      }
+#pragma unroll
+      for (int m = 0; m < TM; ++m) yr[m] = -0.0f;
+      st = 0;
+      ++j;
     }
+  }
+}
+
+// K % 256 == 0: every block is 16 whole words and block g of the flattened
+// [N, nb] grid is the 64 bytes at word 16*g, so one lane owns one block (four
+// 16-byte loads, no cross-lane reduction). A warp walks the blocks of its
+// contiguous rows 32 at a time, with the next 32 blocks' loads in flight, and
+// adds the terms of each row in order with shuffles. The activation codes sit
+// in shared memory with block b's 16-byte chunk k at slot (k + b) mod 16, so
+// that lanes on neighbouring blocks read different banks.
+struct AlignedStep {
+  uint4 w[4];
+  float d;
+};
+
+__device__ __forceinline__ void load_aligned(AlignedStep& st, const uint32_t* __restrict__ packed,
+                                             const float* __restrict__ D, int64_t g, bool ok) {
+  const uint4* p = reinterpret_cast<const uint4*>(packed) + 4 * g;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) st.w[i] = ok ? __ldg(p + i) : make_uint4(0u, 0u, 0u, 0u);
+  st.d = ok ? __ldg(D + g) : 0.0f;
+}
+
+__device__ __forceinline__ int dot16(uint32_t w, const uint4& q, int acc) {
+  acc = __dp4a((int)(w & 0x03030303u), (int)q.x, acc);
+  acc = __dp4a((int)((w >> 2) & 0x03030303u), (int)q.y, acc);
+  acc = __dp4a((int)((w >> 4) & 0x03030303u), (int)q.z, acc);
+  return __dp4a((int)((w >> 6) & 0x03030303u), (int)q.w, acc);
+}
+
+template <int TM>
+__global__ void __launch_bounds__(256) bl_block_scale_forward_aligned_kernel(BlockFwdArgs a) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t tile_m = (int64_t)blockIdx.x / a.tiles_n;
+  const int64_t tile_n = (int64_t)blockIdx.x - tile_m * a.tiles_n;
+  const int64_t t0 = tile_m * a.tm;
+  const int tm = (int)std::min<int64_t>(a.tm, a.M - t0);
+  const int K = (int)a.K, nb = a.nb;
+  int8_t* qs = reinterpret_cast<int8_t*>(smem);
+  int32_t* bsum = reinterpret_cast<int32_t*>(smem + (size_t)a.tm * K);
+  float* sxs = reinterpret_cast<float*>(smem + (size_t)a.tm * K + 4 * (size_t)a.tm * nb);
+
+  const int rpw = a.rows_per_cta / kFwdWarps;
+  const int64_t wr0 = tile_n * a.rows_per_cta + (int64_t)warp * rpw;
+  const int64_t wr1 = std::min<int64_t>(wr0 + rpw, a.N);
+  const int64_t g0 = wr0 * nb, g1 = wr0 < wr1 ? wr1 * nb : g0;
+  AlignedStep nxt;
+  if (g0 < g1) load_aligned(nxt, a.packed, a.D, g0 + lane, g0 + lane < g1);
+
+  // Weights and scales do not depend on the previous kernel in the stream
+  // (the activation quantiser); its codes and scales are read after it is
+  // done, with plain loads (a read-only-path load may be hoisted above this).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(a.q + t0 * a.K);
+    uint4* dst = reinterpret_cast<uint4*>(qs);
+    const int per_row = K >> 4;  // 16-byte chunks per token row
+    const int n16 = tm * per_row;
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) {
+      const int m = i / per_row, c = i - m * per_row;
+      const int b = c >> 4, k = c & 15;
+      dst[m * per_row + 16 * b + ((k + b) & 15)] = src[i];
+    }
+    if (threadIdx.x < tm) sxs[threadIdx.x] = a.sx[t0 + threadIdx.x];
+  }
+  __syncthreads();
+  for (int p = warp; p < tm * nb; p += kFwdWarps) {
+    const int m = p / nb, b = p - m * nb;
+    const uint2 qq = *reinterpret_cast<const uint2*>(qs + (size_t)m * K + 256 * b + 8 * lane);
+    int s = __dp4a((int)qq.x, 0x01010101, 0);
+    s = __dp4a((int)qq.y, 0x01010101, s);
+    s = __reduce_add_sync(0xFFFFFFFFu, s);
+    if (lane == 0) bsum[p] = s;
+  }
+  __syncthreads();
+
+  float yr[TM];
+#pragma unroll
+  for (int m = 0; m < TM; ++m) yr[m] = -0.0f;  // -0 + t == t for every t
+  int64_t n = wr0;                                // row of the next block to be added
+  for (int64_t gb = g0; gb < g1; gb += 32) {
+    const AlignedStep cur = nxt;
+    if (gb + 32 < g1) load_aligned(nxt, a.packed, a.D, gb + 32 + lane, gb + 32 + lane < g1);
+    const int nval = (int)std::min<int64_t>(32, g1 - gb);
+    const int bl = (int)((gb % nb + lane) % nb);  // this lane's block within its row
+    const unsigned ends = __ballot_sync(0xFFFFFFFFu, lane < nval && bl == nb - 1);
+    const int sw = bl & 15;
+#pragma unroll
+    for (int m = 0; m < TM; ++m) {
+      if (m < tm) {
+        const uint4* qb = reinterpret_cast<const uint4*>(qs + (size_t)m * K + 256 * bl);
+        int acc = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t wi[4] = {cur.w[i].x, cur.w[i].y, cur.w[i].z, cur.w[i].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc = dot16(wi[j], qb[(4 * i + j + sw) & 15], acc);
+        }
+        const float t = lane < nval ? rescale(acc - bsum[m * nb + bl], sxs[m], cur.d) : 0.0f;
+        float yv = yr[m];
+        int64_t nn = n;
+        for (int l = 0; l < nval; ++l) {
+          yv = __fadd_rn(yv, __shfl_sync(0xFFFFFFFFu, t, l));
+          if ((ends >> l) & 1u) {
+            if (lane == 0) a.y[(t0 + m) * a.N + nn] = yv;
+            yv = -0.0f;
+            ++nn;
+          }
+        }
+        yr[m] = yv;
+      }
+    }
+    n += __popc(ends);
+  }
+}
+
+template <int TM>
+cudaError_t launch_block_forward_aligned_t(const BlockFwdArgs& a, unsigned grid, size_t smem, cudaStream_t stream) {
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(bl_block_scale_forward_aligned_kernel<TM>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBlockFwdSmemMax);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kFwdWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, bl_block_scale_forward_aligned_kernel<TM>, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// One token (M == 1), K % 256 == 0 and nb <= 32, in one launch: every CTA
+// quantises the token itself (it is at most 32 KB of fp32). Lane l owns block l % nb of
+// row l / nb of each warp step (floor(32 / nb) rows per step), so it keeps
+// that block's 256 activation codes in registers for the whole launch and
+// reads no shared memory. Each packed word is split into its four 2-bit
+// classes by masks alone: byte j of (w & (3 << 2c) per byte) holds
+// (code + 1) << 2c of column 4j + c, which the private activation order puts
+// in byte j of the word c of the same 16-byte chunk. An unsigned x signed
+// dp4a per class accumulates 4^c times the class sum; the four sums are
+// recombined exactly by arithmetic shifts (each is an exact multiple).
+struct BlockDecArgs {
+  const float* x;   // [1, K] fp32, quantised by every CTA
+  const uint32_t* packed;
+  const float* D;   // [N, nb]
+  float* y;         // [1, N]
+  int64_t N;
+  int K, nb, rows_per_warp;
+};
+
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__global__ void __launch_bounds__(256, 2) bl_block_scale_decode_kernel(BlockDecArgs a) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nb = a.nb, R = 32 / nb;
+  const int r = lane / nb, b = lane - r * nb;
+  const bool active = r < R;
+  const int64_t row0 = ((int64_t)blockIdx.x * kFwdWarps + warp) * a.rows_per_warp;
+  const int64_t row1 = std::min<int64_t>(row0 + a.rows_per_warp, a.N);
+
+  AlignedStep nxt;  // the first step's weights, requested before the quantiser runs
+  {
+    const int64_t row = row0 + r;
+    const bool ok = active && row < row1;
+    load_aligned(nxt, a.packed, a.D, ok ? row * nb + b : 0, ok);
+  }
+  // ActQuant of the token in every CTA (BitVLA section 1): max|x| over the
+  // row, s_x = RN(127 / max(max|x|, 1e-5)), q = clamp(rint(RN(x * s_x))), the
+  // codes stored in the private order (position 4c + j of each 16 holds
+  // column 4j + c) in shared memory.
+  __shared__ float red[kFwdWarps];
+  __shared__ __align__(16) int8_t qs[kBlockDecMaxK];
+  const float4* x4 = reinterpret_cast<const float4*>(a.x);
+  const int K4 = a.K >> 2;
+  float amax = 0.0f;
+  for (int i = threadIdx.x; i < K4; i += blockDim.x) {
+    const float4 v = __ldg(x4 + i);
+    amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if (lane == 0) red[warp] = amax;
+  __syncthreads();
+  amax = red[0];
+#pragma unroll
+  for (int w = 1; w < kFwdWarps; ++w) amax = fmaxf(amax, red[w]);
+  const float sx = __fdiv_rn(kQmax, fmaxf(amax, kFloor));
+  for (int g = threadIdx.x; g < (a.K >> 4); g += blockDim.x) {
+    int v[16];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 f = __ldg(x4 + 4 * g + j);
+      v[4 * j + 0] = quant_code(f.x, sx);
+      v[4 * j + 1] = quant_code(f.y, sx);
+      v[4 * j + 2] = quant_code(f.z, sx);
+      v[4 * j + 3] = quant_code(f.w, sx);
+    }
+    uint32_t w4[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t word = 0u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) word |= (uint32_t)(v[4 * j + c] & 0xFF) << (8 * j);
+      w4[c] = word;
+    }
+    *reinterpret_cast<uint4*>(qs + 16 * g) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
+  __syncthreads();
+  uint4 qv[16];
+  const uint4* qb = reinterpret_cast<const uint4*>(qs + 256 * b);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) qv[k] = qb[k];
+  int bsum = 0;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    bsum = __dp4a((int)qv[k].x, 0x01010101, bsum);
+    bsum = __dp4a((int)qv[k].y, 0x01010101, bsum);
+    bsum = __dp4a((int)qv[k].z, 0x01010101, bsum);
+    bsum = __dp4a((int)qv[k].w, 0x01010101, bsum);
+  }
+
+  for (int64_t base = row0; base < row1; base += R) {
+    const AlignedStep cur = nxt;
+    if (base + R < row1) {
+      const int64_t row = base + R + r;
+      const bool ok = active && row < row1;
+      load_aligned(nxt, a.packed, a.D, ok ? row * nb + b : 0, ok);
+    }
+    int c0 = 0, c1 = 0, c2 = 0, c3 = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t wi[4] = {cur.w[i].x, cur.w[i].y, cur.w[i].z, cur.w[i].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t w = wi[j];
+        const uint4& q = qv[4 * i + j];
+        c0 = dp4a_us(w & 0x03030303u, q.x, c0);
+        c1 = dp4a_us(w & 0x0C0C0C0Cu, q.y, c1);
+        c2 = dp4a_us(w & 0x30303030u, q.z, c2);
+        c3 = dp4a_us(w & 0xC0C0C0C0u, q.w, c3);
+      }
+    }
+    const int acc = c0 + (c1 >> 2) + (c2 >> 4) + (c3 >> 6) - bsum;
+    const int64_t row = base + r;
+    const bool ok = active && row < row1;
+    const float t = ok ? rescale(acc, sx, cur.d) : 0.0f;
+    float yv = -0.0f;  // -0 + t == t for every t
+    const int src = active ? r * nb : 0;
+    for (int j = 0; j < nb; ++j) yv = __fadd_rn(yv, __shfl_sync(0xFFFFFFFFu, t, src + j));
+    if (ok && b == 0) a.y[row] = yv;
   }
 }
 
@@ -290,7 +589,20 @@ cudaError_t launch_block_forward_t(const BlockFwdArgs& a, unsigned grid, size_t 
                                          (int)kBlockFwdSmemMax);
     if (e != cudaSuccess) return e;
   }
-  bl_block_scale_forward_kernel<TM><<<grid, kFwdWarps * 32, smem, stream>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kFwdWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  // Programmatic dependent launch: the weights start streaming while the
+  // activation quantiser launched just before still runs.
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, bl_block_scale_forward_kernel<TM>, a);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -312,9 +624,9 @@ int block_forward_tile(int64_t M, int64_t K) {
   return tm;
 }
 
-cudaError_t launch_forward_blocks(int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D, float* y,
-                                  const void* ws, cudaStream_t stream, int num_sms) {
-  const uint8_t* base = static_cast<const uint8_t*>(ws);
+cudaError_t launch_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                                  const float* D, float* y, void* ws, cudaStream_t stream, int num_sms) {
+  uint8_t* base = static_cast<uint8_t*>(ws);
   BlockFwdArgs a;
   a.q = reinterpret_cast<const int8_t*>(base + ws_q_off(M));
   a.sx = reinterpret_cast<const float*>(base + ws_sx_off(M));
@@ -326,17 +638,57 @@ cudaError_t launch_forward_blocks(int64_t M, int64_t N, int64_t K, const uint32_
   a.K = K;
   a.nb = (int)scale_blocks(K);
   a.tm = block_forward_tile(M, K);
+  const bool aligned = (K % kScaleBlock) == 0;
+  if (M == 1 && aligned && a.nb <= 32) {
+    BlockDecArgs d;
+    d.x = x;
+    d.K = (int)K;
+    d.packed = packed;
+    d.D = D;
+    d.y = y;
+    d.N = N;
+    d.nb = a.nb;
+    const int R = 32 / a.nb;
+    // About two CTAs of 8 warps per SM, each warp a whole number of steps.
+    int64_t rpw = (N + (int64_t)num_sms * 16 - 1) / ((int64_t)num_sms * 16);
+    rpw = (rpw + R - 1) / R * R;
+    d.rows_per_warp = (int)rpw;
+    const int64_t grid = (N + rpw * kFwdWarps - 1) / (rpw * kFwdWarps);
+    if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kFwdWarps * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, bl_block_scale_decode_kernel, d);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+  // Otherwise the activations are quantised once into the workspace (private
+  // order), and the contraction launches as a programmatic dependent of that.
+  cudaError_t eq = launch_act_quant(x, false, M, K, reinterpret_cast<int8_t*>(base + ws_q_off(M)),
+                                    reinterpret_cast<float*>(base + ws_sx_off(M)),
+                                    reinterpret_cast<int32_t*>(base + ws_rowsum_off(M)), true, stream,
+                                    reinterpret_cast<uint32_t*>(base));
+  if (eq != cudaSuccess) return eq;
   const int64_t tiles_m = (M + a.tm - 1) / a.tm;
   // Enough warps to keep every SM's loads in flight at one tile of tokens;
-  // with several token tiles, more rows per CTA amortise the tile's load.
-  int64_t rpw = (N + (int64_t)num_sms * 32 - 1) / ((int64_t)num_sms * 32);
+  // with several token tiles, more rows per CTA amortise the tile's load. The
+  // aligned kernel also wants at least 32 blocks (one per lane) per warp.
+  int64_t rpw = (N + (int64_t)num_sms * 48 - 1) / ((int64_t)num_sms * 48);
   if (tiles_m > 1) rpw = std::max<int64_t>(rpw, 4);
+  if (aligned) rpw = std::max<int64_t>(rpw, (32 + a.nb - 1) / a.nb);
   rpw = std::max<int64_t>(rpw, 1);
   a.rows_per_cta = (int)(rpw * kFwdWarps);
   a.tiles_n = (N + a.rows_per_cta - 1) / a.rows_per_cta;
   const int64_t grid = tiles_m * a.tiles_n;
   if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
   const size_t smem = block_fwd_smem(a.tm, K, a.nb);
+  if (aligned) {
+    if (a.tm == 1) return launch_block_forward_aligned_t<1>(a, (unsigned)grid, smem, stream);
+    if (a.tm <= 4) return launch_block_forward_aligned_t<4>(a, (unsigned)grid, smem, stream);
+    return launch_block_forward_aligned_t<16>(a, (unsigned)grid, smem, stream);
+  }
   if (a.tm == 1) return launch_block_forward_t<1>(a, (unsigned)grid, smem, stream);
   if (a.tm <= 4) return launch_block_forward_t<4>(a, (unsigned)grid, smem, stream);
   return launch_block_forward_t<16>(a, (unsigned)grid, smem, stream);

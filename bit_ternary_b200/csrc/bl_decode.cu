@@ -491,7 +491,7 @@ template <int kX>
 __device__ __forceinline__ void dec_load_group(const DecProblem& P, int m, int gi, float4 (&f)[4]) {
   const int64_t i4 = ((int64_t)m * P.K >> 2) + 4 * gi;
 #pragma unroll
-  for (int j = 0; j < 4; ++j) f[j] = load4<kX == kDecBf16>(P.x, i4 + j);
+  for (int j = 0; j < 4; ++j) f[j] = load4_dep<kX == kDecBf16>(P.x, i4 + j);
 }
 
 // ActQuant of every token of the CTA's problems into shared memory (fp32 or
@@ -602,7 +602,7 @@ __device__ void dec_load_prepared(const DecHead& L, const DecGroups& G, uint8_t*
         int p, m, gi;
         G.locate(L, gg, p, m, gi);
         const DecProblem& P = L.pr[p];
-        v[b] = __ldg(reinterpret_cast<const uint4*>(static_cast<const int8_t*>(P.x) + (int64_t)m * P.K) + gi);
+        v[b] = reinterpret_cast<const uint4*>(static_cast<const int8_t*>(P.x) + (int64_t)m * P.K)[gi];
         dst[b] = dec_q_group(sq, P, m, gi);
       }
     }
@@ -613,8 +613,8 @@ __device__ void dec_load_prepared(const DecHead& L, const DecGroups& G, uint8_t*
   for (int i = tid; i < G.np * 16; i += kDecThreads) {
     const int p = G.pa + (i >> 4), m = i & 15;
     if (m < L.pr[p].M) {
-      s_sx[p * 16 + m] = __ldg(L.pr[p].sx_in + m);
-      s_rs[p * 16 + m] = __ldg(L.pr[p].rs_in + m);
+      s_sx[p * 16 + m] = L.pr[p].sx_in[m];  // plain loads: written by the grid waited for
+      s_rs[p * 16 + m] = L.pr[p].rs_in[m];
     }
   }
 }
@@ -683,7 +683,7 @@ __device__ void dec_rms_quantise(const DecHead& L, const DecGroups& G, uint8_t* 
     consumers_sync();
     const float4* xr = reinterpret_cast<const float4*>(P.x) + ((int64_t)m * P.K >> 2);
     for (int i4 = tid; i4 < (P.K >> 2); i4 += kDecThreads) {
-      const float4 v = __ldg(xr + i4);
+      const float4 v = xr[i4];  // x may come from the grid waited for: no read-only path
       rms_bins_add(bins, v.x);
       rms_bins_add(bins, v.y);
       rms_bins_add(bins, v.z);

@@ -285,6 +285,19 @@ __device__ __forceinline__ float4 load4(const void* p, int64_t i4) {
   return __ldg(reinterpret_cast<const float4*>(p) + i4);
 }
 
+// As load4, with ordinary (coherent) loads, for data that the grid this
+// launch depends on may have written: a read-only-path load counts as
+// invariant memory, so the compiler may hoist it above griddepcontrol.wait.
+template <bool kBf16>
+__device__ __forceinline__ float4 load4_dep(const void* p, int64_t i4) {
+  if (kBf16) {
+    const uint2 v = reinterpret_cast<const uint2*>(p)[i4];
+    return make_float4(bf16_bits_to_float(v.x & 0xFFFFu), bf16_bits_to_float(v.x >> 16),
+                       bf16_bits_to_float(v.y & 0xFFFFu), bf16_bits_to_float(v.y >> 16));
+  }
+  return reinterpret_cast<const float4*>(p)[i4];
+}
+
 // Ternary code of one weight: clamp(rint(RN(w*s)), -1, 1) + 1, in {0, 1, 2}.
 __device__ __forceinline__ uint32_t code_plus_one(float w, float s) {
   int c = __float2int_rn(__fmul_rn(w, s));

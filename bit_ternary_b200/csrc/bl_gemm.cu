@@ -332,8 +332,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int h = 0; h < kBN / 32; ++h) {
         const int m = m0 + 32 * h + lane;
         const bool ok = m < p.M;
-        sx[h] = ok ? __ldg(p.s_x + m) : 1.0f;
-        rs[h] = ok ? __ldg(p.rowsum + m) : 0;
+        sx[h] = ok ? p.s_x[m] : 1.0f;  // plain loads: written by the grid waited for
+        rs[h] = ok ? p.rowsum[m] : 0;
       }
       if (!warp_wait(&S.cst_empty[r], ph ^ 1, abort_flag, p.err, kDevTimeoutEpilogue)) break;
 #pragma unroll

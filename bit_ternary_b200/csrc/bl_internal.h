@@ -99,10 +99,12 @@ cudaError_t launch_pack_blocks(const float* W, int64_t N, int64_t K, uint32_t* p
 // Tokens per CTA tile of the block forward (its activation codes fit in
 // kBlockFwdSmemMax of shared memory); always >= 1 for K <= kMaxK.
 int block_forward_tile(int64_t M, int64_t K);
-// Expects the permuted activation codes and s_x in the forward workspace
-// (launch_act_quant with permuted = true).
-cudaError_t launch_forward_blocks(int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D, float* y,
-                                  const void* ws, cudaStream_t stream, int num_sms);
+// One token with K % 256 == 0 and K <= kBlockDecMaxK: a single launch that
+// quantises x in every CTA. Otherwise ActQuant into the forward workspace ws
+// (private order), then the contraction as its programmatic dependent.
+constexpr int kBlockDecMaxK = 32 * kScaleBlock;
+cudaError_t launch_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                                  const float* D, float* y, void* ws, cudaStream_t stream, int num_sms);
 
 cudaError_t launch_selftest_wait(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);
 

@@ -141,6 +141,10 @@ def test_pack_blocks_nonfinite_rejected(B):
 FWD_CASES = [
     (1, 1, 16), (1, 33, 272), (3, 257, 528), (16, 100, 1152), (1, 300, 4304), (5, 64, 6912),
     (17, 65, 528), (40, 33, 2560), (1, 7, 131072), (2, 3, 4096 + 16),
+    # K % 256 == 0 (one lane per block): few blocks per row, rows across chunk edges
+    (1, 1, 256), (3, 5, 256), (2, 70, 512), (1, 33, 1024), (4, 1000, 768), (16, 45, 2048),
+    # one token, K % 256 == 0, at most 32 blocks per row (activation codes held in registers)
+    (1, 1000, 2560), (1, 77, 6912), (1, 129, 8192), (1, 5, 768), (1, 4097, 512),
 ]
 
 
