@@ -38,6 +38,8 @@ SIGNATURES = {
     "bitlinear_device_check": (ctypes.c_int, []),
     "bitlinear_pack_workspace_size": (_SZ, [_I64, _I64]),
     "bitlinear_pack_weights": (ctypes.c_int, [_VP, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
+    "bitlinear_pack_weights_async": (ctypes.c_int, [_VP, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
+    "bitlinear_pack_status": (ctypes.c_int, [_VP, _SZ, _VP]),
     "bitlinear_quant_act": (ctypes.c_int, [_VP, _I64, _I64, _VP, _VP, _VP, _VP]),
     "bitlinear_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "bitlinear_forward": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),

@@ -17,6 +17,8 @@ from . import _lib
 
 __all__ = [
     "pack_weights",
+    "pack_status",
+    "pack_workspace",
     "quant_act",
     "forward",
     "forward_acc",
@@ -73,9 +75,20 @@ def _float_input(t: torch.Tensor, name: str) -> str:
     return ""
 
 
-def pack_weights(W: torch.Tensor, ws: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """WeightQuant + pack: fp32 or bf16 W [N, K] -> (packed int32 [N, K/16], D fp32 [N, 1])."""
+def pack_weights(W: torch.Tensor, ws: Optional[torch.Tensor] = None,
+                 sync: bool = True) -> Tuple[torch.Tensor, torch.Tensor]:
+    """WeightQuant + pack: fp32 or bf16 W [N, K] -> (packed int32 [N, K/16], D fp32 [N, 1]).
+
+    sync=False (fp32 W only) enqueues the pack without waiting; a non-finite
+    weight is then recorded in ws (zero-filled before the first call) and
+    reported by pack_status(ws)."""
     sfx = _float_input(W, "W")
+    if not sync and sfx:
+        raise ValueError("the asynchronous pack takes fp32 W")
+    if not sync and ws is None:
+        raise ValueError("the asynchronous pack needs a caller workspace (zero-filled before the first call)")
+    if not sync:
+        sfx = "_async"
     N, K = W.shape
     packed = torch.empty((N, K // 16), dtype=torch.int32, device=W.device)
     D = torch.empty((N, 1), dtype=torch.float32, device=W.device)
@@ -85,6 +98,17 @@ def pack_weights(W: torch.Tensor, ws: Optional[torch.Tensor] = None) -> Tuple[to
     _lib.call("bitlinear_pack_weights" + sfx, W.data_ptr(), N, K, packed.data_ptr(), D.data_ptr(),
               ws.data_ptr(), ws.numel(), _stream_handle(W.device))
     return packed, D
+
+
+def pack_status(ws: torch.Tensor) -> int:
+    """Synchronises the stream, reads and clears the status word of a pack workspace:
+    BL_OK (0) or BL_ERR_NONFINITE (5)."""
+    return int(_lib.lib().bitlinear_pack_status(ws.data_ptr(), ws.numel(), _stream_handle(ws.device)))
+
+
+def pack_workspace(device) -> torch.Tensor:
+    """A zero-filled pack workspace, as the asynchronous pack wants it."""
+    return torch.zeros(int(_lib.lib().bitlinear_pack_workspace_size(1, 16)), dtype=torch.uint8, device=device)
 
 
 def quant_act(x: torch.Tensor):

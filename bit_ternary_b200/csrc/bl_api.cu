@@ -156,7 +156,7 @@ size_t bitlinear_pack_workspace_size(int64_t N, int64_t K) {
 }
 
 static int pack_impl(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
-                     size_t ws_bytes, bl_stream_t stream) {
+                     size_t ws_bytes, bl_stream_t stream, bool sync = true) {
   int st = check_k(K);
   if (st != BL_OK) return st;
   if (N <= 0 || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
@@ -166,7 +166,8 @@ static int pack_impl(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* p
   const int sms = num_sms_current();
   if (sms <= 0) return BL_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (bl::launch_pack(W, bf16, N, K, packed, D, ws, s, sms) != cudaSuccess) return BL_ERR_CUDA;
+  if (bl::launch_pack(W, bf16, N, K, packed, D, ws, sync, s, sms) != cudaSuccess) return BL_ERR_CUDA;
+  if (!sync) return BL_OK;
   uint32_t status = 0;
   if (cudaMemcpyAsync(&status, ws, sizeof(status), cudaMemcpyDeviceToHost, s) != cudaSuccess) return BL_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
@@ -195,6 +196,26 @@ int bitlinear_pack_weights(const float* W, int64_t N, int64_t K, uint32_t* packe
 int bitlinear_pack_weights_bf16(const uint16_t* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
                                 size_t ws_bytes, bl_stream_t stream) {
   return pack_impl(W, true, N, K, packed, D, ws, ws_bytes, stream);
+}
+
+int bitlinear_pack_weights_async(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
+                                 size_t ws_bytes, bl_stream_t stream) {
+  return pack_impl(W, false, N, K, packed, D, ws, ws_bytes, stream, false);
+}
+
+int bitlinear_pack_status(void* ws, size_t ws_bytes, bl_stream_t stream) {
+  if (ws == nullptr) return BL_ERR_NULL;
+  if (!aligned256(ws)) return BL_ERR_ALIGN;
+  if (ws_bytes < bl::kPackWsBytes) return BL_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t* word = static_cast<uint32_t*>(ws);
+  uint32_t status = 0;
+  if (cudaMemcpyAsync(&status, word, sizeof(status), cudaMemcpyDeviceToHost, s) != cudaSuccess) return BL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
+  if (status == 0u) return BL_OK;
+  if (cudaMemsetAsync(word, 0, sizeof(status), s) != cudaSuccess) return BL_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
+  return BL_ERR_NONFINITE;
 }
 
 int bitlinear_quant_act(const float* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,

@@ -11,12 +11,15 @@
 
 namespace bl {
 
-// Pack workspace: header (status word at 0, mean_c and s at 16/20) + bins:
+// Pack workspace: header (the sticky status word at 0, this call's status at
+// 4, a count of finished CTAs at 8, mean_c and s at 16/20) + bins:
 // kPackBins sums of significands by weight (bin b weighs 2^(max(b,1)-1) units
 // of 2^-149) and, at kPackNonFiniteBin, a count of non-finite weights.
 constexpr int kPackBins = 320;
 constexpr int kPackNonFiniteBin = kPackBins - 1;
-constexpr size_t kPackWsBytes = kHeaderBytes + kPackBins * sizeof(unsigned long long);
+// After the bins: one fp64 partial sum of |W| per CTA of the first pass.
+constexpr int kPackSumBlocks = 1024;
+constexpr size_t kPackWsBytes = kHeaderBytes + kPackBins * sizeof(unsigned long long) + kPackSumBlocks * sizeof(double);
 
 // Decode path (bl_decode.cu): at most 16 tokens per BitLinear, up to 8
 // BitLinears per launch; their activation codes and a ring of at least two
@@ -67,8 +70,10 @@ cudaError_t launch_decode(const DecCall* calls, int n, int input, const float* g
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // W is fp32, or bf16 bit patterns when bf16 (widened exactly).
+// clear_sticky: also zero the workspace's first word, where every call ORs in
+// its failure (asynchronous packs leave it for bitlinear_pack_status).
 cudaError_t launch_pack(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
-                        cudaStream_t stream, int num_sms);
+                        bool clear_sticky, cudaStream_t stream, int num_sms);
 // err_reset (nullable): the workspace error word, cleared by the kernel.
 // x is fp32, or bf16 bit patterns when bf16 (widened exactly).
 cudaError_t launch_act_quant(const void* x, bool bf16, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,

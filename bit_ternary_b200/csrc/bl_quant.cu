@@ -6,11 +6,14 @@
 // ActQuant (BitVLA page, section 1): per token, round(x*127/max|x|)
 // clamped to int8.
 //
-// The mean of |W| must be identical however the reduction is ordered, so it is
-// an exact integer sum: every |w| = m * 2^(max(e,1)-150), and the 24-bit
-// significands m are summed, in integers, into bins by weight (exact and order
-// independent). A single thread then forms the exact total and divides it by
-// N*K with one correct rounding to fp32.
+// The mean of |W| must be identical however the reduction is ordered: it is
+// the exact mean, correctly rounded to fp32 once. A first pass sums |w| in
+// fp64 with a known bound on its rounding error; when the two fp32 roundings
+// of the bounds agree, that is the correctly rounded mean. Otherwise (an fp32
+// rounding boundary within ~2^-44 of the mean) the exact path runs: every
+// |w| = m * 2^(max(e,1)-150), the 24-bit significands m are summed, in
+// integers, into bins by weight (exact and order independent), and a single
+// thread forms the exact total and divides it by N*K with one correct rounding.
 #include "bl_internal.h"
 
 namespace bl {
@@ -29,17 +32,18 @@ constexpr int kWindow = 38;  // binades below a batch's largest exponent summed 
 // base+42 of a per-warp shared copy. Weights below the window go to their own
 // bin. Every step is integer arithmetic, so the result does not depend on the
 // order of the reduction.
+// Run by one CTA of kBinThreads threads over every float4 of W (the rare
+// case where the fp64 pass cannot decide); sbins is its shared scratch.
 template <bool kBf16>
-__global__ void __launch_bounds__(kBinThreads) absum_bins_kernel(const void* __restrict__ W, int64_t n4,
-                                                                  unsigned long long* __restrict__ bins) {
-  __shared__ unsigned long long sbins[kBinWarps][kPackBins];
+__device__ void absum_bins_block(const void* __restrict__ W, int64_t n4, unsigned long long* __restrict__ bins,
+                                 unsigned long long (*sbins)[kPackBins]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < kBinWarps * kPackBins; i += blockDim.x) (&sbins[0][0])[i] = 0ull;
   __syncthreads();
   unsigned long long* my = sbins[warp];
-  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int64_t stride = (int64_t)blockDim.x;
   // Warp-uniform loop bound: every lane reaches the warp reductions.
-  const int64_t base0 = blockIdx.x * (int64_t)blockDim.x + (threadIdx.x & ~31);
+  const int64_t base0 = (int64_t)(threadIdx.x & ~31);
   for (int64_t wb = base0; wb < n4; wb += stride) {
     const int64_t i = wb + lane;
     uint32_t m[4], ee[4];
@@ -92,6 +96,7 @@ __global__ void __launch_bounds__(kBinThreads) absum_bins_kernel(const void* __r
     for (int w = 0; w < kBinWarps; ++w) s += sbins[w][e];
     if (s) atomicAdd(&bins[e], s);
   }
+  __syncthreads();
 }
 
 // Correctly rounded fp32 of S * 2^-149 / n, where S = sum_e bins[e] * 2^(max(e,1)-1).
@@ -99,8 +104,8 @@ __global__ void __launch_bounds__(kBinThreads) absum_bins_kernel(const void* __r
 // 1e-5 floor that is applied afterwards). One thread. n = N*K < 2^48 (N < 2^31,
 // K <= 2^17), and a tensor that fits in device memory has n < 2^36, so every
 // bin is below 2^60 and S below 2^313.
-__global__ void absmean_finalize_kernel(const unsigned long long* __restrict__ gbins, uint64_t n,
-                                        float* __restrict__ scal, uint32_t* __restrict__ status) {
+__device__ void absmean_exact_block(const unsigned long long* __restrict__ gbins, uint64_t n,
+                                    float* __restrict__ scal, uint32_t* __restrict__ status) {
   // S = sum_e bins[e] * 2^(max(e,1)-1) as 11 little-endian 32-bit limbs (used
   // bins < 2^60 at indices <= 258: S < 2^318). The block adds every bin's
   // (up to three) limb parts into 64-bit per-limb sums with shared atomics
@@ -110,7 +115,6 @@ __global__ void absmean_finalize_kernel(const unsigned long long* __restrict__ g
   __shared__ unsigned long long bins[kPackBins];
   __shared__ unsigned long long limb_sum[L + 3];
   __shared__ uint32_t sS[L];
-  if (blockIdx.x != 0) return;
   for (int i = threadIdx.x; i < kPackBins; i += blockDim.x) bins[i] = gbins[i];
   for (int i = threadIdx.x; i < L + 3; i += blockDim.x) limb_sum[i] = 0ull;
   __syncthreads();
@@ -210,9 +214,110 @@ __global__ void absmean_finalize_kernel(const unsigned long long* __restrict__ g
   *status = 0u;
 }
 
+// First pass: fp64 sums of |w|. Each thread adds its weights in sequence
+// (four float4 loads in flight), then the warp (butterfly, 5 levels) and the
+// CTA (8 warps, 3 levels) add in a fixed order; one partial per CTA. Each |w|
+// is exact in fp64. The last CTA to finish adds the partials in a fixed order
+// and decides the mean: the sum S has gone through at most `depth` roundings
+// on any path from a weight (a bound the host derives from the launch shape),
+// so with non-negative terms the exact sum lies within S * depth * 2^-52 of S
+// (twice the first-order bound). If the fp32 roundings of the two ends of that
+// interval, divided by n with directed rounding, agree, that is the correctly
+// rounded mean. Otherwise the same CTA runs the exact integer path over all of
+// W (slow, and reached only within ~2^-44 of a rounding boundary).
+constexpr int kSumThreads = kBinThreads;
+constexpr int kSumUnroll = 4;
+template <bool kBf16>
+__global__ void __launch_bounds__(kSumThreads) absum_f64_kernel(const void* __restrict__ W, int64_t n4, uint64_t n,
+                                                                int depth, double* __restrict__ partial,
+                                                                unsigned long long* __restrict__ bins,
+                                                                uint32_t* __restrict__ done,
+                                                                float* __restrict__ scal,
+                                                                uint32_t* __restrict__ status,
+                                                                uint32_t* __restrict__ sticky) {
+  __shared__ double red[kSumThreads / 32];
+  __shared__ int is_last;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  double s = 0.0;
+  uint32_t bad = 0u;
+  for (int64_t i0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i0 < n4; i0 += kSumUnroll * stride) {
+    float4 v[kSumUnroll];
+#pragma unroll
+    for (int u = 0; u < kSumUnroll; ++u) {
+      const int64_t i = i0 + u * stride;
+      v[u] = i < n4 ? load4<kBf16>(W, i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kSumUnroll; ++u) {
+      const float f[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        bad |= (__float_as_uint(f[j]) & 0x7F800000u) == 0x7F800000u;
+        s += (double)fabsf(f[j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  if (lane == 0) red[warp] = s;
+  if (__any_sync(0xFFFFFFFFu, bad != 0u) && lane == 0) atomicAdd(&bins[kPackNonFiniteBin], 1ull);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const double t0 = red[0] + red[1], t1 = red[2] + red[3], t2 = red[4] + red[5], t3 = red[6] + red[7];
+    partial[blockIdx.x] = (t0 + t1) + (t2 + t3);
+    __threadfence();
+    is_last = atomicAdd(done, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+
+  // The last CTA: every partial and non-finite count is visible.
+  const volatile double* vp = partial;
+  s = 0.0;
+  for (int i = threadIdx.x; i < (int)gridDim.x; i += blockDim.x) s += vp[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  __syncthreads();  // every warp has read red[] above
+  if (lane == 0) red[warp] = s;
+  __syncthreads();
+  const bool nonfinite = *reinterpret_cast<volatile unsigned long long*>(&bins[kPackNonFiniteBin]) != 0ull;
+  if (nonfinite) {
+    if (threadIdx.x == 0) {
+      *status = 1u;  // non-finite input: this call writes neither packed nor D
+      atomicOr(sticky, 1u);
+      scal[0] = __int_as_float(0x7FC00000);
+      scal[1] = __int_as_float(0x7FC00000);
+    }
+    return;
+  }
+  const double t0 = red[0] + red[1], t1 = red[2] + red[3], t2 = red[4] + red[5], t3 = red[6] + red[7];
+  const double S = (t0 + t1) + (t2 + t3);
+  const double rel = (double)depth * 0x1p-52;
+  const double lo = __ddiv_rd(__dmul_rd(S, 1.0 - rel), (double)n);
+  const double hi = __ddiv_ru(__dmul_ru(S, 1.0 + rel), (double)n);
+  const float c1 = __double2float_rn(lo), c2 = __double2float_rn(hi);
+  if (c1 == c2) {  // uniform over the CTA: every thread computed the same values
+    if (threadIdx.x == 0) {
+      // Below the normal range the exact path gives 0; either way the floor applies.
+      const float mean_c = fmaxf(c1, kFloor);
+      scal[0] = mean_c;
+      scal[1] = __fdiv_rn(1.0f, mean_c);
+      *status = 0u;
+    }
+    return;
+  }
+  __shared__ unsigned long long sbins[kBinWarps][kPackBins];
+  absum_bins_block<kBf16>(W, n4, bins, sbins);
+  absmean_exact_block(bins, n, scal, status);
+}
+
 // Each thread ternarises one float4 (4 codes = one byte of a packed word);
 // lanes 4j..4j+3 of a warp hold the four bytes of one word and combine them
-// with shuffles. Also writes D[n] = mean_c.
+// with shuffles. Also writes D[n] = mean_c. Warps take 32-float4 chunks from
+// the end of W backwards: the first pass read W from the start, so its tail
+// is what the L2 still holds.
 template <bool kBf16>
 __global__ void __launch_bounds__(256) ternarize_pack_kernel(const void* __restrict__ W, int64_t n4,
                                                              const float* __restrict__ scal,
@@ -225,9 +330,10 @@ __global__ void __launch_bounds__(256) ternarize_pack_kernel(const void* __restr
   const int lane = threadIdx.x & 31;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   // Loop bound is warp-uniform so every lane reaches the shuffles.
-  const int64_t warp_base0 = (blockIdx.x * (int64_t)blockDim.x + (threadIdx.x & ~31));
-  for (int64_t base = warp_base0; base < n4; base += stride) {
-    const int64_t i = base + lane;
+  const int64_t nchunks = (n4 + 31) >> 5;
+  const int64_t cstride = stride >> 5;
+  for (int64_t c = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; c < nchunks; c += cstride) {
+    const int64_t i = ((nchunks - 1 - c) << 5) + lane;
     uint32_t byte = 0u;
     if (i < n4) {
       const float4 v = load4<kBf16>(W, i);
@@ -597,21 +703,37 @@ __global__ void __launch_bounds__(256, kG == 1 ? 3 : (kG == 2 ? 4 : 1)) rms_act_
 
 // ------------------------------------------------------------ launchers --
 cudaError_t launch_pack(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
-                        cudaStream_t stream, int num_sms) {
+                        bool clear_sticky, cudaStream_t stream, int num_sms) {
   uint8_t* base = static_cast<uint8_t*>(ws);
-  uint32_t* status = reinterpret_cast<uint32_t*>(base);
+  uint32_t* sticky = reinterpret_cast<uint32_t*>(base);     // OR of every call's failure since the last read
+  uint32_t* status = reinterpret_cast<uint32_t*>(base + 4);  // this call's
+  uint32_t* done = reinterpret_cast<uint32_t*>(base + 8);  // CTAs of the fp64 pass that have finished
   float* scal = reinterpret_cast<float*>(base + 16);
   unsigned long long* bins = reinterpret_cast<unsigned long long*>(base + kHeaderBytes);
-  cudaError_t err = cudaMemsetAsync(base, 0, kPackWsBytes, stream);
+  double* partial = reinterpret_cast<double*>(base + kHeaderBytes + kPackBins * sizeof(unsigned long long));
+  const size_t keep = clear_sticky ? 0 : 4;
+  cudaError_t err = cudaMemsetAsync(base + keep, 0, kPackWsBytes - keep, stream);
   if (err != cudaSuccess) return err;
   const int64_t n4 = N * K / 4;
-  const int64_t want = (n4 + kBinThreads * 8 - 1) / (kBinThreads * 8);
-  const int grid1 = (int)(want < 4 * num_sms ? (want < 1 ? 1 : want) : 4 * num_sms);
-  if (bf16)
-    absum_bins_kernel<true><<<grid1, kBinThreads, 0, stream>>>(W, n4, bins);
-  else
-    absum_bins_kernel<false><<<grid1, kBinThreads, 0, stream>>>(W, n4, bins);
-  absmean_finalize_kernel<<<1, 32, 0, stream>>>(bins, (uint64_t)(N * K), scal, status);
+  // fp64 pass (and, in its last CTA, the mean): up to 4 CTAs per SM.
+  {
+    const int64_t want0 = (n4 + kSumThreads * kSumUnroll - 1) / (kSumThreads * kSumUnroll);
+    int64_t g0 = want0 < 4 * (int64_t)num_sms ? want0 : 4 * (int64_t)num_sms;
+    g0 = g0 < 1 ? 1 : (g0 > kPackSumBlocks ? kPackSumBlocks : g0);
+    const int64_t stride = g0 * kSumThreads;
+    // Roundings on any path: the thread's sequential adds (4 per float4), the
+    // warp's 5 and the CTA's 3 levels, then the last CTA's sequential adds of
+    // partials, its warp's 5 and its 3 levels; plus a margin.
+    const int64_t per_thread = 4 * ((n4 + stride - 1) / stride);
+    const int64_t per_final = (g0 + kSumThreads - 1) / kSumThreads;
+    const int depth = (int)(per_thread + 8 + per_final + 8 + 4);
+    if (bf16)
+      absum_f64_kernel<true><<<(unsigned)g0, kSumThreads, 0, stream>>>(W, n4, (uint64_t)(N * K), depth, partial,
+                                                                       bins, done, scal, status, sticky);
+    else
+      absum_f64_kernel<false><<<(unsigned)g0, kSumThreads, 0, stream>>>(W, n4, (uint64_t)(N * K), depth, partial,
+                                                                        bins, done, scal, status, sticky);
+  }
   const int64_t want2 = (n4 + 255) / 256;
   const int grid2 = (int)(want2 < 16 * num_sms ? (want2 < 1 ? 1 : want2) : 16 * num_sms);
   if (bf16)

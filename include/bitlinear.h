@@ -117,6 +117,21 @@ BL_API int bitlinear_pack_weights_bf16(const uint16_t* W, int64_t N, int64_t K,
                                        uint32_t* packed, float* D,
                                        void* ws, size_t ws_bytes, bl_stream_t stream);
 
+/* As bitlinear_pack_weights, without synchronising: the pack is enqueued on
+ * `stream` and a non-finite weight is OR-ed into the status word at the start
+ * of `ws` instead of being returned (that call then writes neither packed nor
+ * D; later calls are not affected). The caller zeroes that word before the
+ * first call (a zero-filled workspace); bitlinear_pack_status reads it.
+ * Calls that share `ws` must be ordered on one stream. */
+BL_API int bitlinear_pack_weights_async(const float* W, int64_t N, int64_t K,
+                                        uint32_t* packed, float* D,
+                                        void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* Synchronises `stream`, reads and clears the status word of a pack
+ * workspace: BL_OK if no asynchronous pack since the last read met a
+ * non-finite weight, else BL_ERR_NONFINITE. */
+BL_API int bitlinear_pack_status(void* ws, size_t ws_bytes, bl_stream_t stream);
+
 /* ------------------------------------------------------------ ActQuant --- */
 
 /* Per-token int8 absmax quantisation (BitVLA page section 1).

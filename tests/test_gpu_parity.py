@@ -97,6 +97,50 @@ def test_pack_special_values(B):
     assert np.array_equal(D.cpu().numpy(), D_ref)
 
 
+def test_pack_exact_path_on_mean_ties(B):
+    """Tensors whose exact mean of |W| lies on, or a hair off, the midpoint of
+    two fp32 values (and one where values 200 binades apart decide it): the
+    fp64 pass cannot round these, so the exact integer path must."""
+    one = np.ones(256, np.float32)
+    cases = []
+    for delta in (0.0, 2.0 ** -23, -(2.0 ** -23)):
+        r = one.copy()
+        r[255] = np.float32(1.0 + 2.0 ** -16 + delta)  # mean 1 + 2^-24 (+ delta / 256)
+        cases.append(r.reshape(16, 16))
+    for tiny in (2.0 ** -100, 0.0):
+        r = np.full(256, np.float32(tiny))
+        r[:128] = np.float32(2.0 ** 100)
+        r[128] = np.float32(2.0 ** 83)  # mean on the midpoint of 2^99 and 2^99 + 2^76, decided by the tiny values
+        cases.append(r.reshape(8, 32))
+    for W in cases:
+        W = W.copy()
+        W[:, 1::3] *= -1
+        packed, D = B.pack_weights(dev(W))
+        p_ref, D_ref = O.pack_weights(W)
+        assert np.array_equal(D.cpu().numpy().view(np.uint32), D_ref.view(np.uint32))
+        assert np.array_equal(packed.cpu().numpy().view(np.uint32), p_ref)
+    assert O.absmean_exact(cases[0]) == np.float32(1.0)
+
+
+def test_pack_async_back_to_back_sticky_status(B):
+    """Asynchronous packs sharing one zero-filled workspace: a non-finite
+    weight in the middle is reported once by pack_status, and the packs
+    before and after it are still bit-exact."""
+    Ws = [WL.weight(64, 528, "normal", 11), WL.weight(33, 1152, "laplace", 12), WL.weight(200, 2560, "normal", 13)]
+    Ws[1][5, 17] = np.inf
+    ws = B.pack_workspace("cuda")
+    outs = [B.pack_weights(dev(W), ws=ws, sync=False) for W in Ws]
+    assert B.pack_status(ws) == 5  # BL_ERR_NONFINITE
+    assert B.pack_status(ws) == 0  # read and cleared
+    for i in (0, 2):
+        p_ref, D_ref = O.pack_weights(Ws[i])
+        assert np.array_equal(outs[i][0].cpu().numpy().view(np.uint32), p_ref)
+        assert np.array_equal(outs[i][1].cpu().numpy(), D_ref)
+    out = B.pack_weights(dev(Ws[2]), ws=ws, sync=False)
+    assert B.pack_status(ws) == 0
+    assert np.array_equal(out[0].cpu().numpy(), outs[2][0].cpu().numpy())
+
+
 def test_pack_all_zero_uses_floor(B):
     W = np.zeros((4, 32), np.float32)
     packed, D = B.pack_weights(dev(W))
