@@ -969,8 +969,8 @@ def bench_block_scale(B, torch, dev, stream, capture, time_graph, max_ranks, hbm
     tot = sum(nbytes(l, 1) for l in layers)
     out["decode_layer_set"] = {"us_per_step": round(t * 1e6, 2), "GB/s": round(tot / t / 1e9, 1),
                                "frac_hbm": round(tot / t / 1e9 / hbm_peak, 4), "bytes_per_step": tot,
-                               "note": "four bitlinear_forward_blocks calls per step (ActQuant launch + "
-                                       f"block-scale kernel each), M=1, weights rotating over {rot} copies"}
+                               "note": "four bitlinear_forward_blocks calls per step (at M=1 one launch each: the "
+                                       f"quantiser runs in every CTA), M=1, weights rotating over {rot} copies"}
     del g, packs, xs, base
     torch.cuda.empty_cache()
 

@@ -481,9 +481,12 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
   return d;
 }
 
+// NBT != 0 fixes the number of blocks per row at compile time (the per-row
+// sum then unrolls); NBT == 0 reads it from the arguments.
+template <int NBT>
 __global__ void __launch_bounds__(256, 2) bl_block_scale_decode_kernel(BlockDecArgs a) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nb = a.nb, R = 32 / nb;
+  const int nb = NBT != 0 ? NBT : a.nb, R = 32 / nb;
   const int r = lane / nb, b = lane - r * nb;
   const bool active = r < R;
   const int64_t row0 = ((int64_t)blockIdx.x * kFwdWarps + warp) * a.rows_per_warp;
@@ -577,7 +580,12 @@ __global__ void __launch_bounds__(256, 2) bl_block_scale_decode_kernel(BlockDecA
     const float t = ok ? rescale(acc, sx, cur.d) : 0.0f;
     float yv = -0.0f;  // -0 + t == t for every t
     const int src = active ? r * nb : 0;
-    for (int j = 0; j < nb; ++j) yv = __fadd_rn(yv, __shfl_sync(0xFFFFFFFFu, t, src + j));
+    if (NBT != 0) {
+#pragma unroll
+      for (int j = 0; j < (NBT != 0 ? NBT : 1); ++j) yv = __fadd_rn(yv, __shfl_sync(0xFFFFFFFFu, t, src + j));
+    } else {
+      for (int j = 0; j < nb; ++j) yv = __fadd_rn(yv, __shfl_sync(0xFFFFFFFFu, t, src + j));
+    }
     if (ok && b == 0) a.y[row] = yv;
   }
 }
@@ -660,7 +668,16 @@ cudaError_t launch_forward_blocks(const float* x, int64_t M, int64_t N, int64_t 
     cfg.blockDim = dim3(kFwdWarps * 32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, bl_block_scale_decode_kernel, d);
+    void (*kern)(BlockDecArgs) = bl_block_scale_decode_kernel<0>;
+    switch (a.nb) {
+      case 4: kern = bl_block_scale_decode_kernel<4>; break;     // K = 1024
+      case 8: kern = bl_block_scale_decode_kernel<8>; break;     // K = 2048
+      case 10: kern = bl_block_scale_decode_kernel<10>; break;   // K = 2560
+      case 12: kern = bl_block_scale_decode_kernel<12>; break;   // K = 3072
+      case 27: kern = bl_block_scale_decode_kernel<27>; break;   // K = 6912
+      default: break;
+    }
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, d);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }

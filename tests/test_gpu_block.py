@@ -145,6 +145,7 @@ FWD_CASES = [
     (1, 1, 256), (3, 5, 256), (2, 70, 512), (1, 33, 1024), (4, 1000, 768), (16, 45, 2048),
     # one token, K % 256 == 0, at most 32 blocks per row (activation codes held in registers)
     (1, 1000, 2560), (1, 77, 6912), (1, 129, 8192), (1, 5, 768), (1, 4097, 512),
+    (1, 300, 2048), (1, 1025, 3072),
 ]
 
 
