@@ -948,7 +948,8 @@ def bench_block_scale(B, torch, dev, stream, capture, time_graph, max_ranks, hbm
         xs = [[torch.from_numpy(WL.activations(1, l.K, wl.x_dist, wl.seed + r, layer=li, meta=wl.meta)).to(dev)
                for li, l in enumerate(layers)] for r in range(rot)]
         ys = [torch.empty((1, l.N), dtype=torch.float32, device=dev) for l in layers]
-        wss = [torch.zeros(max(256, B.workspace_size(1, l.N, l.K)), dtype=torch.uint8, device=dev) for l in layers]
+        wss = [torch.zeros(max(256, B.blocks_workspace_size(1, l.N, l.K)), dtype=torch.uint8, device=dev)
+               for l in layers]
     torch.cuda.synchronize(dev)
 
     def step(i):
@@ -987,7 +988,7 @@ def bench_block_scale(B, torch, dev, stream, capture, time_graph, max_ranks, hbm
         del pst, Dst
         x1 = torch.from_numpy(WL.activations(1, l.K, wl.x_dist, wl.seed, layer=2, meta=wl.meta)).to(dev)
         y1 = torch.empty((1, Nst), dtype=torch.float32, device=dev)
-        ws1 = torch.zeros(max(256, B.workspace_size(1, Nst, l.K)), dtype=torch.uint8, device=dev)
+        ws1 = torch.zeros(max(256, B.blocks_workspace_size(1, Nst, l.K)), dtype=torch.uint8, device=dev)
     torch.cuda.synchronize(dev)
     g = capture(lambda i: B.forward_blocks(x1, pk[i % copies][0], pk[i % copies][1], out=y1, ws=ws1), 16)
     with torch.cuda.stream(stream):
@@ -1000,26 +1001,34 @@ def bench_block_scale(B, torch, dev, stream, capture, time_graph, max_ranks, hbm
     del g, pk
     torch.cuda.empty_cache()
 
-    # Prefill size on the CUDA-core path: gate_up at M=512.
-    M = 512
-    with torch.cuda.stream(stream):
-        W1 = torch.from_numpy(WL.weight(l.N, l.K, "laplace", 9)).to(dev)
-        pp, DD = B.pack_weights_blocks(W1)
-        del W1
-        xp = torch.from_numpy(WL.activations(M, l.K, "normal", 9)).to(dev)
-        yp = torch.empty((M, l.N), dtype=torch.float32, device=dev)
-        wsp = torch.zeros(max(256, B.workspace_size(M, l.N, l.K)), dtype=torch.uint8, device=dev)
-    torch.cuda.synchronize(dev)
-    g = capture(lambda i: B.forward_blocks(xp, pp, DD, out=yp, ws=wsp), 8)
-    with torch.cuda.stream(stream):
-        g.replay()
-    t = max_ranks(time_graph(g)) / 8 * 1e-3
-    ops = 2.0 * M * l.N * l.K
-    out["prefill_m512_gate_up"] = {"us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 2),
-                                   "frac_int8_peak": round(ops / t / 1e12 / (i8_burst), 4),
-                                   "note": "CUDA-core dp4a path (no tensor-core kernel for this variant)"}
-    del g, pp, DD, xp, yp
-    torch.cuda.empty_cache()
+    # Prefill sizes: gate_up at M=512 and 4096 (one tensor-core GEMM per 256-column block).
+    pre = []
+    for M in (512, 4096):
+        with torch.cuda.stream(stream):
+            W1 = torch.from_numpy(WL.weight(l.N, l.K, "laplace", 9)).to(dev)
+            pp, DD = B.pack_weights_blocks(W1)
+            del W1
+            xp = torch.from_numpy(WL.activations(M, l.K, "normal", 9)).to(dev)
+            yp = torch.empty((M, l.N), dtype=torch.float32, device=dev)
+            wsp = torch.zeros(max(256, B.blocks_workspace_size(M, l.N, l.K)), dtype=torch.uint8, device=dev)
+        torch.cuda.synchronize(dev)
+        g = capture(lambda i: B.forward_blocks(xp, pp, DD, out=yp, ws=wsp), 8)
+        with torch.cuda.stream(stream):
+            g.replay()
+        t = max_ranks(time_graph(g)) / 8 * 1e-3
+        ops = 2.0 * M * l.N * l.K
+        nbk = (l.K + 255) // 256
+        alg = 4 * M * l.K + l.N * l.K // 4 + 4 * l.N * nbk + 4 * M * l.N
+        true_t = max(alg / (hbm_peak * 1e9), ops / (i8_burst * 1e12))
+        pre.append({"M": M, "us": round(t * 1e6, 2), "TOPS": round(ops / t / 1e12, 2),
+                    "frac_int8_peak": round(ops / t / 1e12 / i8_burst, 4),
+                    "frac_true_roofline": round(true_t / t, 4)})
+        del g, pp, DD, xp, yp, wsp
+        torch.cuda.empty_cache()
+    out["prefill_gate_up"] = {"cases": pre,
+                              "note": "ActQuant, per-block row sums of the codes, then one tcgen05 GEMM per "
+                                      f"256-column block ({(l.K + 255) // 256} launches), each epilogue adding "
+                                      "its block's term to y (TMA reduce-add); the same input each call"}
 
     # Per-block pack of gate_up (offline).
     with torch.cuda.stream(stream):

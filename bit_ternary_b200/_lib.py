@@ -72,6 +72,7 @@ SIGNATURES = {
     "bitlinear_forward_rmsnorm": (ctypes.c_int, [_VP, _VP, ctypes.c_float, _I64, _I64, _I64, _VP, _VP, _VP,
                                                  _VP, _SZ, _VP]),
     "bitlinear_block_scales": (_I64, [_I64]),
+    "bitlinear_blocks_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "bitlinear_pack_weights_blocks": (ctypes.c_int, [_VP, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
     "bitlinear_forward_blocks": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "bitlinear_workspace_error": (ctypes.c_int, [_VP, _SZ, _VP]),

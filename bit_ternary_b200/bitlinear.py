@@ -32,6 +32,7 @@ __all__ = [
     "block_scales",
     "pack_weights_blocks",
     "forward_blocks",
+    "blocks_workspace_size",
     "workspace_size",
     "workspace_error",
     "BitLinear",
@@ -255,6 +256,10 @@ def block_scales(K: int) -> int:
     return nb
 
 
+def blocks_workspace_size(M: int, N: int, K: int) -> int:
+    return int(_lib.lib().bitlinear_blocks_workspace_size(M, N, K))
+
+
 def pack_weights_blocks(W: torch.Tensor, ws: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Per-256-block WeightQuant + pack: fp32 W [N, K] -> (packed int32 [N, K/16], D fp32 [N, nb])."""
     _need_cuda(W, "W", torch.float32)
@@ -282,7 +287,7 @@ def forward_blocks(x: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,
     y = out if out is not None else torch.empty((M, N), dtype=torch.float32, device=x.device)
     _need_cuda(y, "out", torch.float32)
     if ws is None:
-        ws = _alloc_ws(workspace_size(M, N, K), x.device)
+        ws = _alloc_ws(blocks_workspace_size(M, N, K), x.device)
     _lib.call("bitlinear_forward_blocks", x.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(), y.data_ptr(),
               ws.data_ptr(), ws.numel(), _stream_handle(x.device))
     return y

@@ -380,6 +380,12 @@ int bitlinear_pack_weights_blocks(const float* W, int64_t N, int64_t K, uint32_t
   return status == 0u ? BL_OK : BL_ERR_NONFINITE;
 }
 
+size_t bitlinear_blocks_workspace_size(int64_t M, int64_t N, int64_t K) {
+  (void)N;
+  if (M < 0 || K <= 0 || check_k(K) != BL_OK) return 0;
+  return bl::ws_blocks_bytes(M, K);
+}
+
 int bitlinear_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                              const float* D, float* y, void* ws, size_t ws_bytes, bl_stream_t stream) {
   int st = check_k(K);
@@ -389,7 +395,7 @@ int bitlinear_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, co
   if (M == 0 || N == 0) return BL_OK;
   if (x == nullptr || packed == nullptr || D == nullptr || y == nullptr || ws == nullptr) return BL_ERR_NULL;
   if (!aligned16(x) || !aligned16(packed) || !aligned16(D) || !aligned16(y) || !aligned256(ws)) return BL_ERR_ALIGN;
-  if (ws_bytes < bitlinear_workspace_size(M, N, K)) return BL_ERR_WORKSPACE;
+  if (ws_bytes < bl::ws_blocks_bytes(M, K)) return BL_ERR_WORKSPACE;
   const int sms = num_sms_current();
   if (sms <= 0) return BL_ERR_CUDA;
   return cuda_status(

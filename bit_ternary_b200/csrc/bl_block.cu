@@ -614,6 +614,31 @@ cudaError_t launch_block_forward_t(const BlockFwdArgs& a, unsigned grid, size_t 
   return cudaGetLastError();
 }
 
+// Row sums of the activation codes per block, for the tensor-core route:
+// bs[b * M + m] = sum of q[m, k] over block b's columns (the codes are stored
+// as code + 1, so each block's contraction subtracts its own sum). One warp
+// per (token, block); the private column order is a permutation inside
+// groups of 16 columns, which never straddle blocks.
+__global__ void __launch_bounds__(256) bl_block_scale_rowsum_kernel(const int8_t* __restrict__ q, int64_t M, int K,
+                                                                    int nb, int32_t* __restrict__ bs) {
+  const int lane = threadIdx.x & 31;
+  const int64_t total = M * nb;
+  const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t p = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); p < total; p += warps) {
+    const int64_t m = p / nb;
+    const int b = (int)(p - m * nb);
+    const int k0 = b * kScaleBlock, cnt = min(kScaleBlock, K - k0);
+    int s = 0;
+    if (8 * lane < cnt) {
+      const uint2 qq = *reinterpret_cast<const uint2*>(q + m * K + k0 + 8 * lane);
+      s = __dp4a((int)qq.x, 0x01010101, s);
+      s = __dp4a((int)qq.y, 0x01010101, s);
+    }
+    s = __reduce_add_sync(0xFFFFFFFFu, s);
+    if (lane == 0) bs[(int64_t)b * M + m] = s;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_pack_blocks(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, uint32_t* status,
@@ -688,6 +713,30 @@ cudaError_t launch_forward_blocks(const float* x, int64_t M, int64_t N, int64_t 
                                     reinterpret_cast<int32_t*>(base + ws_rowsum_off(M)), true, stream,
                                     reinterpret_cast<uint32_t*>(base));
   if (eq != cudaSuccess) return eq;
+  if (M >= kBlockGemmMinM) {
+    // Tensor-core route: one GEMM per block over its K range (a 256-code
+    // stage of the tcgen05 kernel is exactly one block), with the block's
+    // column of D; the first block stores y, the others add their terms to it
+    // in ascending order (the kernel's epilogue adds with one fp32 rounding).
+    int32_t* bs = reinterpret_cast<int32_t*>(base + ws_forward_bytes(M, K));
+    const int64_t nwarps = M * a.nb;
+    const int64_t g = std::min<int64_t>((nwarps + 7) / 8, (int64_t)num_sms * 16);
+    bl_block_scale_rowsum_kernel<<<(unsigned)g, 256, 0, stream>>>(a.q, M, (int)K, a.nb, bs);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    for (int b = 0; b < a.nb; ++b) {
+      GemmSlice sl;
+      sl.k0 = (int64_t)b * kScaleBlock;
+      sl.kfull = K;
+      sl.dstride = a.nb;
+      sl.accumulate = b > 0;
+      sl.rowsum = bs + (int64_t)b * M;
+      const int64_t kc = std::min<int64_t>(kScaleBlock, K - sl.k0);
+      e = launch_gemm_slice(M, N, kc, sl, packed, D + b, y, nullptr, ws, stream, num_sms);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   const int64_t tiles_m = (M + a.tm - 1) / a.tm;
   // Enough warps to keep every SM's loads in flight at one tile of tokens;
   // with several token tiles, more rows per CTA amortise the tile's load. The

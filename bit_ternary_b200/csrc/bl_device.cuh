@@ -160,6 +160,14 @@ __device__ __forceinline__ void tma_store_2d(const void* tmap, int32_t c0, int32
                "r"(c0), "r"(c1), "r"(smem_u32(smem_src))
                : "memory");
 }
+// As tma_store_2d, but each element is added to the one in global memory
+// (fp32: one IEEE round-to-nearest addition per element).
+__device__ __forceinline__ void tma_reduce_add_2d(const void* tmap, int32_t c0, int32_t c1, const void* smem_src) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(tmap)),
+               "r"(c0), "r"(c1), "r"(smem_u32(smem_src))
+               : "memory");
+}
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the shared-memory sources of all committed bulk stores have been read.
 __device__ __forceinline__ void bulk_wait_group_read0() {

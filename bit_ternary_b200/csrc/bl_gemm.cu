@@ -110,7 +110,10 @@ struct GemmParams {
   int M;
   int N;
   int K;
-  int wpr;
+  int wpr;         // packed words in the contracted K range of a row
+  int wstride;     // words from one row of `packed` to the next (>= wpr)
+  int dstride;     // floats from D[n] to D[n + 1]
+  int accumulate;  // add the rescaled tile to y (y = RN(y + t)) instead of storing it
   int kblocks;
   int tiles_n;
   int num_tiles;
@@ -157,7 +160,7 @@ __device__ __forceinline__ void unpack_load(const GemmParams& p, const JobCursor
   const int64_t n = (int64_t)(tile % p.tiles_n) * kBM + row_in_tile;
   const int w0 = jc.kb * kStageWords;
   if (n < p.N) {
-    const uint32_t* rp = p.packed + n * (int64_t)p.wpr + w0;
+    const uint32_t* rp = p.packed + n * (int64_t)p.wstride + w0;
     if (kAligned) {
       // wpr % 4 == 0 and w0 % 4 == 0: each group of four words is all in or all out.
 #pragma unroll
@@ -411,7 +414,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int n0 = (tile % p.tiles_n) * kBM + quarter * 32;
       const int64_t n = (int64_t)n0 + lane;
       const bool nvalid = n < p.N;
-      const float dn = (!kAccOut && nvalid) ? __ldg(p.D + n) : 0.0f;
+      const float dn = (!kAccOut && nvalid) ? __ldg(p.D + n * p.dstride) : 0.0f;
       if (!warp_wait(&S.acc_full[b], (lt >> 1) & 1, abort_flag, p.err, kDevTimeoutEpilogue)) break;
       tc_fence_after();
       if (!warp_wait(&S.cst_full[r], rph, abort_flag, p.err, kDevTimeoutEpilogue)) break;
@@ -448,10 +451,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else {
             const int m = m0 + c0 + t;
             if (m < p.M && nvalid) {
-              if (kAccOut)
+              if (kAccOut) {
                 p.acc_out[(int64_t)m * p.N + n] = (int32_t)out;
-              else
+              } else if (p.accumulate) {
+                float* py = p.y + (int64_t)m * p.N + n;  // one writer per element in this launch
+                *py = __fadd_rn(*py, __uint_as_float(out));
+              } else {
                 __stcs(p.y + (int64_t)m * p.N + n, __uint_as_float(out));
+              }
             }
           }
         }
@@ -459,7 +466,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_2d(&tmap_out, n0, m0 + c0, sy);
+            if (!kAccOut && p.accumulate)
+              tma_reduce_add_2d(&tmap_out, n0, m0 + c0, sy);
+            else
+              tma_store_2d(&tmap_out, n0, m0 + c0, sy);
             bulk_commit_group();
           }
           ybuf ^= 1;
@@ -537,8 +547,20 @@ static int64_t gemm_estimate(int BN, int64_t M, int64_t tiles_n, int64_t kblocks
 
 cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D, float* y,
                         int32_t* acc_out, void* ws, cudaStream_t stream, int num_sms) {
+  GemmSlice sl;
+  sl.k0 = 0;
+  sl.kfull = K;
+  sl.dstride = 1;
+  sl.accumulate = false;
+  sl.rowsum = nullptr;
+  return launch_gemm_slice(M, N, K, sl, packed, D, y, acc_out, ws, stream, num_sms);
+}
+
+cudaError_t launch_gemm_slice(int64_t M, int64_t N, int64_t K, const GemmSlice& sl, const uint32_t* packed,
+                              const float* D, float* y, int32_t* acc_out, void* ws, cudaStream_t stream,
+                              int num_sms) {
   uint8_t* base = static_cast<uint8_t*>(ws);
-  int8_t* q = reinterpret_cast<int8_t*>(base + ws_q_off(M));
+  int8_t* q = reinterpret_cast<int8_t*>(base + ws_q_off(M)) + sl.k0;
   PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
   if (encode == nullptr) return cudaErrorNotSupported;
   // Token-tile width: whichever the cost model puts first.
@@ -551,7 +573,7 @@ cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed,
   CUtensorMap tmap_q, tmap_out;
   {
     const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
-    const cuuint64_t gstride[1] = {(cuuint64_t)K};
+    const cuuint64_t gstride[1] = {(cuuint64_t)sl.kfull};
     const cuuint32_t box[2] = {128u, (cuuint32_t)BN};
     const cuuint32_t estride[2] = {1, 1};
     if (encode(&tmap_q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, gdim, gstride, box, estride,
@@ -575,10 +597,10 @@ cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed,
   }
 
   GemmParams p;
-  p.packed = packed;
+  p.packed = packed + sl.k0 / 16;
   p.D = D;
   p.s_x = reinterpret_cast<const float*>(base + ws_sx_off(M));
-  p.rowsum = reinterpret_cast<const int32_t*>(base + ws_rowsum_off(M));
+  p.rowsum = sl.rowsum != nullptr ? sl.rowsum : reinterpret_cast<const int32_t*>(base + ws_rowsum_off(M));
   p.y = y;
   p.acc_out = acc_out;
   p.err = reinterpret_cast<uint32_t*>(base);
@@ -586,6 +608,9 @@ cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed,
   p.N = (int)N;
   p.K = (int)K;
   p.wpr = (int)(K / 16);
+  p.wstride = (int)(sl.kfull / 16);
+  p.dstride = sl.dstride;
+  p.accumulate = sl.accumulate ? 1 : 0;
   p.kblocks = (int)kblocks;
   p.tiles_n = (int)tiles_n;
   const int64_t tiles_m = (M + BN - 1) / BN;
@@ -593,7 +618,7 @@ cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed,
   if (nt > 0x7FFFFFFF) return cudaErrorInvalidValue;
   p.num_tiles = (int)nt;
   const int grid = (int)(nt < num_sms ? nt : num_sms);
-  const bool aligned = (p.wpr % 4) == 0;
+  const bool aligned = (p.wpr % 4) == 0 && (p.wstride % 4) == 0 && (reinterpret_cast<uintptr_t>(p.packed) & 15u) == 0;
   const bool accout = acc_out != nullptr;
 #define BL_GEMM_CASE(AL, AO, TS)                                                                     \
   if (aligned == AL && accout == AO && tma_store == TS)                                              \

@@ -91,6 +91,22 @@ cudaError_t launch_q_prepare(const int8_t* q, const float* s_x, int64_t M, int64
 // workspace (launch_act_quant with permuted = true).
 cudaError_t launch_gemm(int64_t M, int64_t N, int64_t K, const uint32_t* packed, const float* D, float* y,
                         int32_t* acc_out, void* ws, cudaStream_t stream, int num_sms);
+// The same tensor-core kernel over the K range [k0, k0 + K) of rows that are
+// kfull columns long (k0 % 16 == 0): the weights' words and the workspace's
+// activation codes of that range, the row sums of the codes over it (rowsum,
+// or the workspace's when null), D[n * dstride], and with accumulate the
+// rescaled tile is added to y (one fp32 rounding per element) instead of
+// stored.
+struct GemmSlice {
+  int64_t k0;
+  int64_t kfull;
+  int dstride;
+  bool accumulate;
+  const int32_t* rowsum;
+};
+cudaError_t launch_gemm_slice(int64_t M, int64_t N, int64_t K, const GemmSlice& sl, const uint32_t* packed,
+                              const float* D, float* y, int32_t* acc_out, void* ws, cudaStream_t stream,
+                              int num_sms);
 
 // Per-256-block scale variant (bl_block.cu): blocks of 256 consecutive
 // columns within a row, D fp32 [N, scale_blocks(K)].
@@ -108,6 +124,12 @@ int block_forward_tile(int64_t M, int64_t K);
 // quantises x in every CTA. Otherwise ActQuant into the forward workspace ws
 // (private order), then the contraction as its programmatic dependent.
 constexpr int kBlockDecMaxK = 32 * kScaleBlock;
+// From this many tokens on, the block forward runs one tensor-core GEMM per
+// block; its workspace then also holds the per-block row sums of the codes.
+constexpr int64_t kBlockGemmMinM = 128;
+inline size_t ws_blocks_bytes(int64_t M, int64_t K) {
+  return ws_forward_bytes(M, K) + align256(4 * (size_t)M * (size_t)scale_blocks(K));
+}
 cudaError_t launch_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                                   const float* D, float* y, void* ws, cudaStream_t stream, int num_sms);
 

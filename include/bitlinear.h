@@ -262,13 +262,21 @@ BL_API int bitlinear_pack_weights_blocks(const float* W, int64_t N, int64_t K,
                                          uint32_t* packed, float* D,
                                          void* ws, size_t ws_bytes, bl_stream_t stream);
 
+/* Bytes of scratch that bitlinear_forward_blocks needs: the forward
+ * workspace plus one int32 per token and block (the row sums of the codes per
+ * block, for the tensor-core route). */
+BL_API size_t bitlinear_blocks_workspace_size(int64_t M, int64_t N, int64_t K);
+
 /* y [M, N] from per-block scaled weights (packed and D from
- * bitlinear_pack_weights_blocks): ActQuant of x into ws (as bitlinear_forward
- * does), then a CUDA-core kernel that contracts each 256-column block with
- * dp4a and adds the block terms in ascending order. Any M (tiles of up to 16
- * tokens per CTA; there is no tensor-core path for this variant). Same
- * workspace as bitlinear_forward (bitlinear_workspace_size(M, N, K)); every
- * device pointer 16-byte aligned, ws 256-byte aligned. Asynchronous. */
+ * bitlinear_pack_weights_blocks). One token with K % 256 == 0 and K <= 8192:
+ * one launch that quantises x in every CTA. M < 128: ActQuant into ws, then a
+ * CUDA-core kernel that contracts each 256-column block with dp4a and adds the
+ * block terms in ascending order. M >= 128: ActQuant into ws, the codes' row
+ * sums per block, then one tcgen05 tensor-core GEMM per block over its 256
+ * columns whose epilogue applies that block's D and adds the term to y (the
+ * first block stores it). ws_bytes >= bitlinear_blocks_workspace_size(M, N,
+ * K); every device pointer 16-byte aligned, ws 256-byte aligned.
+ * Asynchronous. */
 BL_API int bitlinear_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K,
                                     const uint32_t* packed, const float* D, float* y,
                                     void* ws, size_t ws_bytes, bl_stream_t stream);

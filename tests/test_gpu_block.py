@@ -146,6 +146,8 @@ FWD_CASES = [
     # one token, K % 256 == 0, at most 32 blocks per row (activation codes held in registers)
     (1, 1000, 2560), (1, 77, 6912), (1, 129, 8192), (1, 5, 768), (1, 4097, 512),
     (1, 300, 2048), (1, 1025, 3072),
+    # M >= 128: one tensor-core GEMM per block, the epilogue adding each term to y
+    (128, 300, 528), (200, 256, 2560), (300, 1000, 1152), (256, 4304, 4304), (129, 33, 6912), (385, 130, 272),
 ]
 
 
@@ -178,6 +180,10 @@ def test_forward_blocks_zero_sizes_and_validation(B):
     small = torch.empty(64, dtype=torch.uint8, device="cuda")
     with pytest.raises(BitLinearError, match="WORKSPACE"):
         B.forward_blocks(torch.zeros((1, 272), device="cuda"), packed, D, ws=small)
+    # the tensor-core route needs the per-block row sums too: the plain forward workspace is short
+    short = torch.empty(B.workspace_size(200, 8, 272), dtype=torch.uint8, device="cuda")
+    with pytest.raises(BitLinearError, match="WORKSPACE"):
+        B.forward_blocks(torch.zeros((200, 272), device="cuda"), packed, D, ws=short)
 
 
 def _rows(n, k=64):
