@@ -1103,6 +1103,51 @@ def bench_rmsnorm(B, torch, dev, stream, capture, time_graph, max_ranks, hbm_pea
                       "frac_true_roofline": round(max(nb / (hbm_peak * 1e9), ops / (i8_burst * 1e12)) / t, 4)}
     del gg, x, y, ws
     torch.cuda.empty_cache()
+    # The decode layer set (M=1) with a norm before every projection: four
+    # bitlinear_forward_rmsnorm calls per step, each one decode launch that
+    # normalises and quantises x in every CTA. Bytes per layer: the BitLinear's
+    # plus 4K of norm weight.
+    dl = WL.WORKLOADS[HEADLINE]
+    layers = list(dl.layers)
+    rot = 16
+    with torch.cuda.stream(stream):
+        base = []
+        for li, lay in enumerate(layers):
+            W = torch.from_numpy(WL.weight(lay.N, lay.K, dl.w_dist, dl.seed, layer=li)).to(dev)
+            base.append(B.pack_weights(W))
+            del W
+        packs = [[(pp.clone(), DD.clone()) for (pp, DD) in base] for _ in range(rot)]
+        gs = [torch.from_numpy(WL.weight(1, lay.K, "normal", 30 + li).reshape(-1) + np.float32(1.0)).to(dev)
+              for li, lay in enumerate(layers)]
+        xs = [[torch.from_numpy(WL.activations(1, lay.K, dl.x_dist, dl.seed + r, layer=li, meta=dl.meta)).to(dev)
+               for li, lay in enumerate(layers)] for r in range(rot)]
+        ys = [torch.empty((1, lay.N), dtype=torch.float32, device=dev) for lay in layers]
+        wss = [torch.zeros(max(256, B.workspace_size(1, lay.N, lay.K)), dtype=torch.uint8, device=dev)
+               for lay in layers]
+    torch.cuda.synchronize(dev)
+
+    def step(i):
+        r = i % rot
+        for li in range(len(layers)):
+            pp, DD = packs[r][li]
+            B.forward_rmsnorm(xs[r][li], gs[li], pp, DD, out=ys[li], ws=wss[li])
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            step(i)
+    torch.cuda.synchronize(dev)
+    n = 64
+    gd = capture(step, n)
+    with torch.cuda.stream(stream):
+        gd.replay()
+    t = max_ranks(time_graph(gd)) / n * 1e-3
+    tot = sum(lay.N * lay.K // 4 + 4 * lay.N + 4 * lay.K + 4 * lay.N + 4 * lay.K for lay in layers)
+    out["decode_layer_set"] = {"us_per_step": round(t * 1e6, 2), "GB/s": round(tot / t / 1e9, 1),
+                               "frac_hbm": round(tot / t / 1e9 / hbm_peak, 4),
+                               "note": "four bitlinear_forward_rmsnorm calls per step (M=1, one decode launch "
+                                       f"each, norm + ActQuant in every CTA), weights rotating over {rot} copies"}
+    del gd, packs, xs
+    torch.cuda.empty_cache()
     return out
 
 
