@@ -278,6 +278,30 @@ __device__ __forceinline__ float rescale(int32_t acc, float s_x, float d) {
   return __fmul_rn(__fdiv_rn(__int2float_rn(acc), s_x), d);
 }
 
+// RN(a / s) for an integer-valued a (|a| <= 2^24) and s > 0, given r = RN(1/s)
+// (one division per token instead of one per output). Markstein's correction
+// (IBM J. Res. Dev. 34(1), 1990; Muller et al., "Handbook of Floating-Point
+// Arithmetic", division with a fused multiply-add): if r is within half an
+// ulp of 1/s and q within one ulp of a/s, the residual e = a - s*q is exact in
+// one FMA and RN(q + e*r) is the correctly rounded quotient. q0 = RN(a*r) may
+// be up to ~1.5 ulp off, so a first correction brings it within one ulp and
+// the second yields RN(a/s). A quotient at the edge of the fp32 range (only
+// for max|x| beyond ~1e33) takes the IEEE division instead.
+__device__ __forceinline__ float div_rn_by_rcp(float a, float s, float r) {
+  float q = __fmul_rn(a, r);
+  float e = __fmaf_rn(-q, s, a);
+  q = __fmaf_rn(e, r, q);
+  e = __fmaf_rn(-q, s, a);
+  q = __fmaf_rn(e, r, q);
+  if (!(fabsf(q) < 0x1p127f)) q = __fdiv_rn(a, s);
+  return q;
+}
+
+// The rescale y = RN(RN(float(acc) / s_x) * d) with r = RN(1 / s_x) given.
+__device__ __forceinline__ float rescale_rcp(int32_t acc, float s_x, float r, float d) {
+  return __fmul_rn(div_rn_by_rcp(__int2float_rn(acc), s_x, r), d);
+}
+
 // Inputs are fp32, or bf16 given as 16-bit patterns. A bf16 is the upper half
 // of the fp32 with the same value, so widening it is exact. load4 reads the
 // four consecutive elements 4*i4 .. 4*i4+3 (16 bytes of fp32 or 8 of bf16).

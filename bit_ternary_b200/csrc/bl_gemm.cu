@@ -78,6 +78,7 @@ constexpr uint32_t kYChunkBytes = kEpiChunk * 32 * 4;  // one epilogue chunk: 32
 
 struct TokConst {
   float sx;    // s_x = 127 / max|x|
+  float rx;    // RN(1 / s_x), for the rescale's corrected division
   int32_t rs;  // sum_k q[m, k]
 };
 
@@ -342,6 +343,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 #pragma unroll
       for (int h = 0; h < kBN / 32; ++h) {
         S.cst[r][32 * h + lane].sx = sx[h];
+        S.cst[r][32 * h + lane].rx = __fdiv_rn(1.0f, sx[h]);
         S.cst[r][32 * h + lane].rs = rs[h];
       }
       __syncwarp();
@@ -445,7 +447,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int t = 0; t < kEpiChunk; ++t) {
           const TokConst kc = cst[c0 + t];
           const int a = (int)v[t] - kc.rs;
-          const uint32_t out = kAccOut ? (uint32_t)a : __float_as_uint(rescale(a, kc.sx, dn));
+          const uint32_t out = kAccOut ? (uint32_t)a : __float_as_uint(rescale_rcp(a, kc.sx, kc.rx, dn));
           if (kTmaStore) {
             sy[t * 32 + lane] = out;
           } else {

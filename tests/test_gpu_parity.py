@@ -263,6 +263,28 @@ def test_forward_gemm(B, M, N, K):
     run_case(B, M, N, K, wdist="laplace", xdist="outlier_channels", seed=M + N * 7 + K)
 
 
+def test_gemm_rescale_extreme_token_scales(B):
+    """The tensor-core epilogue divides by s_x through a reciprocal with two
+    FMA corrections. Tokens whose max|x| spans 1e-30 .. 3e38 (s_x from ~1e32
+    down to ~4e-37, quotients from 0 to beyond the fp32 range, where the
+    IEEE division takes over) must still match the oracle bit for bit,
+    infinities included."""
+    M, N, K = 160, 96, 512
+    W = WL.weight(N, K, "normal", 77)
+    x = WL.activations(M, K, "normal", 78)
+    with np.errstate(over="ignore"):
+        scales = (10.0 ** np.linspace(-31, 38, M)).astype(np.float32)
+        x = (x * scales[:, None]).astype(np.float32)
+    x[~np.isfinite(x)] = np.float32(3e38)
+    packed, D = B.pack_weights(dev(W))
+    p_ref, D_ref = O.pack_weights(W)
+    y = B.forward(dev(x), packed, D).cpu().numpy()
+    with np.errstate(over="ignore"):
+        y_ref = O.bitlinear_forward(x, p_ref, D_ref, K)
+    assert np.array_equal(y.view(np.uint32), y_ref.view(np.uint32))
+    assert np.isinf(y_ref).any() and np.isfinite(y_ref).any()
+
+
 def test_gemm_edge_zero_tokens_and_rows(B):
     """All-zero token (floor path) and rows whose weights ternarise to 0."""
     M, N, K = 40, 200, 512
