@@ -329,21 +329,28 @@ __global__ void __launch_bounds__(256) ternarize_pack_kernel(const void* __restr
   const float s = scal[1];
   const int lane = threadIdx.x & 31;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  // Loop bound is warp-uniform so every lane reaches the shuffles.
+  // Loop bound is warp-uniform so every lane reaches the shuffles. Two chunks
+  // per iteration, both loads issued before either is used.
   const int64_t nchunks = (n4 + 31) >> 5;
   const int64_t cstride = stride >> 5;
-  for (int64_t c = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; c < nchunks; c += cstride) {
-    const int64_t i = ((nchunks - 1 - c) << 5) + lane;
-    uint32_t byte = 0u;
-    if (i < n4) {
-      const float4 v = load4<kBf16>(W, i);
-      byte = code_plus_one(v.x, s) | (code_plus_one(v.y, s) << 2) | (code_plus_one(v.z, s) << 4) |
-             (code_plus_one(v.w, s) << 6);
+  for (int64_t c = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5; c < nchunks; c += 2 * cstride) {
+    int64_t i[2];
+    float4 v[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int64_t ch = c + h * cstride;
+      i[h] = ch < nchunks ? ((nchunks - 1 - ch) << 5) + lane : n4;
+      v[h] = i[h] < n4 ? load4<kBf16>(W, i[h]) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    uint32_t word = byte << (8 * (lane & 3));
-    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
-    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
-    if ((lane & 3) == 0 && i < n4) packed[i >> 2] = word;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t byte = code_plus_one(v[h].x, s) | (code_plus_one(v[h].y, s) << 2) |
+                            (code_plus_one(v[h].z, s) << 4) | (code_plus_one(v[h].w, s) << 6);
+      uint32_t word = byte << (8 * (lane & 3));
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+      if ((lane & 3) == 0 && i[h] < n4) packed[i[h] >> 2] = word;
+    }
   }
   for (int64_t n = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; n < N; n += stride) D[n] = mean_c;
 }
