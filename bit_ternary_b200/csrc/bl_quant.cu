@@ -452,6 +452,76 @@ cudaError_t launch_selftest_wait(uint32_t* err, uint64_t limit_ns, cudaStream_t 
 // Register-resident variant for rows of up to 256 * 16 * kG columns: each
 // thread loads its kG groups of 16 values once, the block reduces max|x|, and
 // the same registers are quantised and stored (one read of x, one write of q).
+// ActQuant with one warp per token, for rows of up to 32 * kWG groups of 16
+// columns (K <= 3072): every lane keeps its groups in registers (up to 24
+// 16-byte loads in flight), max|x| and the row sum are warp reductions, and no
+// block barrier is needed. The same arithmetic as act_quant_reg_kernel.
+template <bool kPerm, int kWG, bool kBf16>
+__global__ void __launch_bounds__(256) act_quant_warp_kernel(const void* __restrict__ x, int64_t M, int64_t K,
+                                                             int8_t* __restrict__ q, float* __restrict__ s_out,
+                                                             int32_t* __restrict__ rowsum_out,
+                                                             uint32_t* __restrict__ err_reset) {
+  // A decode launch that waits on these codes may start streaming its weights.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if (err_reset != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *err_reset = 0u;
+  const int lane = threadIdx.x & 31;
+  const int ngroups = (int)(K >> 4);
+  const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t m = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); m < M; m += nwarps) {
+    const int64_t xr = m * (K >> 2);
+    float4 f[kWG][4];
+#pragma unroll
+    for (int i = 0; i < kWG; ++i) {
+      const int gi = lane + 32 * i;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) f[i][j] = gi < ngroups ? load4<kBf16>(x, xr + 4 * gi + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kWG; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(f[i][j].x), fabsf(f[i][j].y)), fmaxf(fabsf(f[i][j].z), fabsf(f[i][j].w))));
+    // |x| >= 0, so the order of the bit patterns is the order of the values.
+    amax = __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(amax)));
+    const float sx = __fdiv_rn(kQmax, fmaxf(amax, kFloor));
+    int rsum = 0;
+    int8_t* qr = q + m * K;
+#pragma unroll
+    for (int i = 0; i < kWG; ++i) {
+      const int gi = lane + 32 * i;
+      if (gi >= ngroups) continue;
+      int v[16];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[4 * j + 0] = quant_code(f[i][j].x, sx);
+        v[4 * j + 1] = quant_code(f[i][j].y, sx);
+        v[4 * j + 2] = quant_code(f[i][j].z, sx);
+        v[4 * j + 3] = quant_code(f[i][j].w, sx);
+      }
+      uint32_t w4[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        uint32_t word = 0u;
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int pp = 4 * r + b;
+          word |= (uint32_t)(v[kPerm ? perm16(pp) : pp] & 0xFF) << (8 * b);
+        }
+        w4[r] = word;
+      }
+#pragma unroll
+      for (int j = 0; j < 16; ++j) rsum += v[j];
+      *reinterpret_cast<uint4*>(qr + 16 * (int64_t)gi) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+    rsum = __reduce_add_sync(0xFFFFFFFFu, rsum);
+    if (lane == 0) {
+      s_out[m] = sx;
+      if (rowsum_out != nullptr) rowsum_out[m] = rsum;
+    }
+  }
+}
+
 template <bool kPerm, int kG, bool kBf16>
 __global__ void __launch_bounds__(256) act_quant_reg_kernel(const void* __restrict__ x, int64_t K,
                                                             int8_t* __restrict__ q, float* __restrict__ s_out,
@@ -799,6 +869,30 @@ template <bool kBf16>
 static cudaError_t launch_act_quant_t(const void* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
                                       bool permuted, cudaStream_t stream, uint32_t* err_reset) {
   const int64_t ngroups = K / 16;
+  // Rows of up to 6 groups per lane: one warp per token, no block barrier.
+  if (ngroups <= 32 * 6) {
+    const int wg = (int)((ngroups + 31) / 32);
+    const int64_t want = (M + 7) / 8;
+    const unsigned grid = (unsigned)(want < 1 ? 1 : (want < 148 * 16 ? want : 148 * 16));
+#define BL_AQW(P, G) act_quant_warp_kernel<P, G, kBf16><<<grid, 256, 0, stream>>>(x, M, K, q, s_x, rowsum, err_reset)
+#define BL_AQW_G(P)                                                                                         \
+  switch (wg) {                                                                                             \
+    case 1: BL_AQW(P, 1); break;                                                                            \
+    case 2: BL_AQW(P, 2); break;                                                                            \
+    case 3: BL_AQW(P, 3); break;                                                                            \
+    case 4: BL_AQW(P, 4); break;                                                                            \
+    case 5: BL_AQW(P, 5); break;                                                                            \
+    default: BL_AQW(P, 6); break;                                                                           \
+  }
+    if (permuted) {
+      BL_AQW_G(true)
+    } else {
+      BL_AQW_G(false)
+    }
+#undef BL_AQW_G
+#undef BL_AQW
+    return cudaGetLastError();
+  }
   // Rows of up to 256 threads x 4 groups x 16 values stay in registers.
   int kg = (int)((ngroups + 255) / 256);
   if (kg <= 4) {
