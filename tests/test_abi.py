@@ -207,3 +207,54 @@ def test_python_constants_match_header_defines():
     statuses = dict((k, int(v)) for k, v in re.findall(r"(BL_(?:OK|ERR_\w+))\s*=\s*(\d+)", text))
     for code, name in _lib.STATUS_NAMES.items():
         assert statuses[name] == code, name
+
+
+# ------------------------------------------------- per-256-block scale variant
+@pytest.mark.parametrize("K,nb", [(16, 1), (256, 1), (272, 2), (2560, 10), (6912, 27), (4304, 17), (131072, 512)])
+def test_block_scales_count(L, K, nb):
+    assert L.bitlinear_block_scales(K) == nb
+
+
+@pytest.mark.parametrize("K", [0, -16, 24, 131072 + 16])
+def test_block_scales_invalid_k(L, K):
+    assert L.bitlinear_block_scales(K) == 0
+    assert L.bitlinear_blocks_workspace_size(4, 4, K) == 0
+
+
+def test_blocks_workspace_adds_row_sums_per_block(L):
+    for M, K in ((1, 2560), (200, 272), (4096, 6912)):
+        base = L.bitlinear_workspace_size(M, 8, K)
+        blk = L.bitlinear_blocks_workspace_size(M, 8, K)
+        nb = L.bitlinear_block_scales(K)
+        assert blk >= base + 4 * M * nb and blk % 256 == 0
+
+
+@pytest.mark.parametrize("K", [0, 8, 24, 131072 + 16])
+def test_block_entry_points_reject_bad_k(L, K):
+    assert L.bitlinear_forward_blocks(FAKE, 1, 1, K, FAKE, FAKE, FAKE, FAKE, 1 << 20, None) == 2
+    assert L.bitlinear_pack_weights_blocks(FAKE, 1, K, FAKE, FAKE, FAKE, 1 << 16, None) == 2
+
+
+def test_block_entry_points_validate_before_cuda(L):
+    big = 1 << 24
+    assert L.bitlinear_forward_blocks(None, 0, 5, 16, None, None, None, None, 0, None) == 0  # empty: no-op
+    assert L.bitlinear_forward_blocks(None, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, big, None) == 1
+    assert L.bitlinear_forward_blocks(FAKE, 1, 1, 16, FAKE, None, FAKE, FAKE, big, None) == 1
+    assert L.bitlinear_forward_blocks(FAKE + 4, 1, 1, 16, FAKE, FAKE, FAKE, FAKE, big, None) == 3
+    assert L.bitlinear_forward_blocks(FAKE, 1, 1, 16, FAKE, FAKE, FAKE, FAKE + 16, big, None) == 3
+    # the plain forward workspace is short for the block route (it also holds per-block row sums)
+    short = L.bitlinear_workspace_size(200, 8, 272)
+    assert L.bitlinear_forward_blocks(FAKE, 200, 8, 272, FAKE, FAKE, FAKE, FAKE, short, None) == 4
+    assert L.bitlinear_pack_weights_blocks(FAKE, 0, 16, FAKE, FAKE, FAKE, big, None) == 2
+    assert L.bitlinear_pack_weights_blocks(None, 4, 16, FAKE, FAKE, FAKE, big, None) == 1
+    assert L.bitlinear_pack_weights_blocks(FAKE, 4, 16, FAKE, FAKE, FAKE, 16, None) == 4
+
+
+def test_async_pack_and_status_validate_before_cuda(L):
+    ws = L.bitlinear_pack_workspace_size(1, 16)
+    assert L.bitlinear_pack_weights_async(FAKE, 1, 24, FAKE, FAKE, FAKE, ws, None) == 2
+    assert L.bitlinear_pack_weights_async(FAKE, 4, 16, FAKE, FAKE, FAKE, 16, None) == 4
+    assert L.bitlinear_pack_weights_async(FAKE + 4, 4, 16, FAKE, FAKE, FAKE, ws, None) == 3
+    assert L.bitlinear_pack_status(None, ws, None) == 1
+    assert L.bitlinear_pack_status(FAKE + 16, ws, None) == 3
+    assert L.bitlinear_pack_status(FAKE, 16, None) == 4
