@@ -75,6 +75,8 @@ SIGNATURES = {
     "bitlinear_blocks_workspace_size": (_SZ, [_I64, _I64, _I64]),
     "bitlinear_pack_weights_blocks": (ctypes.c_int, [_VP, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
     "bitlinear_forward_blocks": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "bitlinear_pack_weights_blocks_bf16": (ctypes.c_int, [_VP, _I64, _I64, _VP, _VP, _VP, _SZ, _VP]),
+    "bitlinear_forward_blocks_bf16": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "bitlinear_workspace_error": (ctypes.c_int, [_VP, _SZ, _VP]),
     "bitlinear_selftest_wait_timeout": (ctypes.c_int, [_VP, _SZ, ctypes.c_uint64, _VP]),
     "bitlinear_forward_noalloc": (ctypes.c_int, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _VP]),

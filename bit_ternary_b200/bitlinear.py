@@ -261,8 +261,8 @@ def blocks_workspace_size(M: int, N: int, K: int) -> int:
 
 
 def pack_weights_blocks(W: torch.Tensor, ws: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Per-256-block WeightQuant + pack: fp32 W [N, K] -> (packed int32 [N, K/16], D fp32 [N, nb])."""
-    _need_cuda(W, "W", torch.float32)
+    """Per-256-block WeightQuant + pack: fp32 or bf16 W [N, K] -> (packed int32 [N, K/16], D fp32 [N, nb])."""
+    sfx = _float_input(W, "W")
     N, K = W.shape
     nb = block_scales(K)
     packed = torch.empty((N, K // 16), dtype=torch.int32, device=W.device)
@@ -270,16 +270,17 @@ def pack_weights_blocks(W: torch.Tensor, ws: Optional[torch.Tensor] = None) -> T
     L = _lib.lib()
     if ws is None:
         ws = _alloc_ws(L.bitlinear_pack_workspace_size(N, K), W.device)
-    _lib.call("bitlinear_pack_weights_blocks", W.data_ptr(), N, K, packed.data_ptr(), D.data_ptr(),
+    _lib.call("bitlinear_pack_weights_blocks" + sfx, W.data_ptr(), N, K, packed.data_ptr(), D.data_ptr(),
               ws.data_ptr(), ws.numel(), _stream_handle(W.device))
     return packed, D
 
 
 def forward_blocks(x: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,
                    out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """y [M, N] from per-256-block scaled weights (D fp32 [N, ceil(K/256)])."""
+    """y [M, N] from per-256-block scaled weights (D fp32 [N, ceil(K/256)]); x fp32 or bf16, y fp32."""
     K = x.shape[-1]
-    M, N = _fwd_args(x, packed, K)
+    M, N = _fwd_args(x, packed, K, allow_bf16=True)
+    fn = "bitlinear_forward_blocks_bf16" if x.dtype == torch.bfloat16 else "bitlinear_forward_blocks"
     nb = block_scales(K)
     if tuple(D.shape) != (N, nb):
         raise ValueError(f"D must have shape [N, nb] = [{N}, {nb}], got {list(D.shape)}")
@@ -288,7 +289,7 @@ def forward_blocks(x: torch.Tensor, packed: torch.Tensor, D: torch.Tensor,
     _need_cuda(y, "out", torch.float32)
     if ws is None:
         ws = _alloc_ws(blocks_workspace_size(M, N, K), x.device)
-    _lib.call("bitlinear_forward_blocks", x.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(), y.data_ptr(),
+    _lib.call(fn, x.data_ptr(), M, N, K, packed.data_ptr(), D.data_ptr(), y.data_ptr(),
               ws.data_ptr(), ws.numel(), _stream_handle(x.device))
     return y
 

@@ -360,8 +360,8 @@ int64_t bitlinear_block_scales(int64_t K) {
   return bl::scale_blocks(K);
 }
 
-int bitlinear_pack_weights_blocks(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
-                                  size_t ws_bytes, bl_stream_t stream) {
+static int pack_blocks_impl(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
+                            size_t ws_bytes, bl_stream_t stream) {
   int st = check_k(K);
   if (st != BL_OK) return st;
   if (N <= 0 || N > 0x7FFFFFFF) return BL_ERR_SHAPE;
@@ -373,7 +373,7 @@ int bitlinear_pack_weights_blocks(const float* W, int64_t N, int64_t K, uint32_t
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   uint32_t* word = static_cast<uint32_t*>(ws);
   if (cudaMemsetAsync(word, 0, sizeof(uint32_t), s) != cudaSuccess) return BL_ERR_CUDA;
-  if (bl::launch_pack_blocks(W, N, K, packed, D, word, s, sms) != cudaSuccess) return BL_ERR_CUDA;
+  if (bl::launch_pack_blocks(W, bf16, N, K, packed, D, word, s, sms) != cudaSuccess) return BL_ERR_CUDA;
   uint32_t status = 0;
   if (cudaMemcpyAsync(&status, word, sizeof(status), cudaMemcpyDeviceToHost, s) != cudaSuccess) return BL_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return BL_ERR_CUDA;
@@ -386,8 +386,18 @@ size_t bitlinear_blocks_workspace_size(int64_t M, int64_t N, int64_t K) {
   return bl::ws_blocks_bytes(M, K);
 }
 
-int bitlinear_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
-                             const float* D, float* y, void* ws, size_t ws_bytes, bl_stream_t stream) {
+int bitlinear_pack_weights_blocks(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, void* ws,
+                                  size_t ws_bytes, bl_stream_t stream) {
+  return pack_blocks_impl(W, false, N, K, packed, D, ws, ws_bytes, stream);
+}
+
+int bitlinear_pack_weights_blocks_bf16(const uint16_t* W, int64_t N, int64_t K, uint32_t* packed, float* D,
+                                       void* ws, size_t ws_bytes, bl_stream_t stream) {
+  return pack_blocks_impl(W, true, N, K, packed, D, ws, ws_bytes, stream);
+}
+
+static int forward_blocks_impl(const void* x, bool bf16, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                               const float* D, float* y, void* ws, size_t ws_bytes, bl_stream_t stream) {
   int st = check_k(K);
   if (st != BL_OK) return st;
   st = check_mn(M, N);
@@ -399,7 +409,17 @@ int bitlinear_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, co
   const int sms = num_sms_current();
   if (sms <= 0) return BL_ERR_CUDA;
   return cuda_status(
-      bl::launch_forward_blocks(x, M, N, K, packed, D, y, ws, reinterpret_cast<cudaStream_t>(stream), sms));
+      bl::launch_forward_blocks(x, bf16, M, N, K, packed, D, y, ws, reinterpret_cast<cudaStream_t>(stream), sms));
+}
+
+int bitlinear_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                             const float* D, float* y, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  return forward_blocks_impl(x, false, M, N, K, packed, D, y, ws, ws_bytes, stream);
+}
+
+int bitlinear_forward_blocks_bf16(const uint16_t* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                                  const float* D, float* y, void* ws, size_t ws_bytes, bl_stream_t stream) {
+  return forward_blocks_impl(x, true, M, N, K, packed, D, y, ws, ws_bytes, stream);
 }
 
 size_t bitlinear_batch_workspace_size(const bl_linear_call* calls, int count) {

@@ -36,12 +36,15 @@ constexpr int kLimbs = 9;  // 288 bits: 256 values below 2^277 units of 2^-149
 // units. B is an fp64 value that is an integer multiple of 2^-149 (the
 // midpoint of two fp32 values times a multiple of 16). One thread; used only
 // when the fp64 interval cannot decide the rounding.
-__device__ __noinline__ int compare_abs_sum(const float* __restrict__ w, int cnt, double B) {
+template <bool kBf16>
+__device__ __noinline__ int compare_abs_sum(const void* __restrict__ wv, int cnt, double B) {
   uint32_t A[kLimbs];
 #pragma unroll
   for (int i = 0; i < kLimbs; ++i) A[i] = 0u;
   for (int j = 0; j < cnt; ++j) {
-    const uint32_t b = __float_as_uint(__ldg(w + j)) & 0x7FFFFFFFu;
+    const float wj = kBf16 ? bf16_bits_to_float(__ldg(static_cast<const uint16_t*>(wv) + j))
+                           : __ldg(static_cast<const float*>(wv) + j);
+    const uint32_t b = __float_as_uint(wj) & 0x7FFFFFFFu;
     uint32_t e = b >> 23, m = b & 0x7FFFFFu;
     if (e != 0u) m |= 0x800000u; else e = 1u;
     const int sh = (int)e - 1;  // 0 .. 253
@@ -82,7 +85,8 @@ __device__ __noinline__ int compare_abs_sum(const float* __restrict__ w, int cnt
 
 // One warp per (row, block). Lane l holds columns 4l..4l+3 and 128+4l..128+4l+3
 // of the block; four lanes make one packed word.
-__global__ void __launch_bounds__(256) bl_block_scale_pack_kernel(const float* __restrict__ W, int64_t N, int64_t K,
+template <bool kBf16>
+__global__ void __launch_bounds__(256) bl_block_scale_pack_kernel(const void* __restrict__ W, int64_t N, int64_t K,
                                                          uint32_t* __restrict__ packed, float* __restrict__ D,
                                                          uint32_t* __restrict__ status) {
   const int lane = threadIdx.x & 31;
@@ -93,14 +97,16 @@ __global__ void __launch_bounds__(256) bl_block_scale_pack_kernel(const float* _
     const int64_t n = blk / nb, b = blk - n * nb;
     const int64_t k0 = b * kScaleBlock;
     const int cnt = (int)std::min<int64_t>(kScaleBlock, K - k0);
-    const float* src = W + n * K + k0;
+    const int64_t e0 = n * K + k0;  // first element of the block
+    const void* src = kBf16 ? static_cast<const void*>(static_cast<const uint16_t*>(W) + e0)
+                            : static_cast<const void*>(static_cast<const float*>(W) + e0);
     float4 v[2];
     bool ok[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int c = 128 * h + 4 * lane;
       ok[h] = c < cnt;
-      v[h] = ok[h] ? __ldg(reinterpret_cast<const float4*>(src + c)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[h] = ok[h] ? load4<kBf16>(W, (e0 + c) >> 2) : make_float4(0.f, 0.f, 0.f, 0.f);
     }
     // Non-finite weights: record and leave this block unwritten.
     bool bad = false;
@@ -132,7 +138,7 @@ __global__ void __launch_bounds__(256) bl_block_scale_pack_kernel(const float* _
       // midpoint, to c2 above it, to the even one on it. Midpoint * cnt is
       // exact in fp64 (25 + 9 significant bits).
       int cmp = 0;
-      if (lane == 0) cmp = compare_abs_sum(src, cnt, 0.5 * ((double)c1 + (double)c2) * (double)cnt);
+      if (lane == 0) cmp = compare_abs_sum<kBf16>(src, cnt, 0.5 * ((double)c1 + (double)c2) * (double)cnt);
       cmp = __shfl_sync(0xFFFFFFFFu, cmp, 0);
       mean = cmp < 0 ? c1 : (cmp > 0 ? c2 : ((__float_as_uint(c1) & 1u) ? c2 : c1));
     }
@@ -467,7 +473,7 @@ cudaError_t launch_block_forward_aligned_t(const BlockFwdArgs& a, unsigned grid,
 // dp4a per class accumulates 4^c times the class sum; the four sums are
 // recombined exactly by arithmetic shifts (each is an exact multiple).
 struct BlockDecArgs {
-  const float* x;   // [1, K] fp32, quantised by every CTA
+  const void* x;    // [1, K] fp32 (or bf16 bit patterns), quantised by every CTA
   const uint32_t* packed;
   const float* D;   // [N, nb]
   float* y;         // [1, N]
@@ -483,7 +489,7 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
 
 // NBT != 0 fixes the number of blocks per row at compile time (the per-row
 // sum then unrolls); NBT == 0 reads it from the arguments.
-template <int NBT>
+template <int NBT, bool kBf16>
 __global__ void __launch_bounds__(256, 2) bl_block_scale_decode_kernel(BlockDecArgs a) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int nb = NBT != 0 ? NBT : a.nb, R = 32 / nb;
@@ -504,11 +510,10 @@ __global__ void __launch_bounds__(256, 2) bl_block_scale_decode_kernel(BlockDecA
   // column 4j + c) in shared memory.
   __shared__ float red[kFwdWarps];
   __shared__ __align__(16) int8_t qs[kBlockDecMaxK];
-  const float4* x4 = reinterpret_cast<const float4*>(a.x);
   const int K4 = a.K >> 2;
   float amax = 0.0f;
   for (int i = threadIdx.x; i < K4; i += blockDim.x) {
-    const float4 v = __ldg(x4 + i);
+    const float4 v = load4<kBf16>(a.x, i);
     amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
   }
 #pragma unroll
@@ -523,7 +528,7 @@ __global__ void __launch_bounds__(256, 2) bl_block_scale_decode_kernel(BlockDecA
     int v[16];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float4 f = __ldg(x4 + 4 * g + j);
+      const float4 f = load4<kBf16>(a.x, 4 * g + j);
       v[4 * j + 0] = quant_code(f.x, sx);
       v[4 * j + 1] = quant_code(f.y, sx);
       v[4 * j + 2] = quant_code(f.z, sx);
@@ -641,12 +646,15 @@ __global__ void __launch_bounds__(256) bl_block_scale_rowsum_kernel(const int8_t
 
 }  // namespace
 
-cudaError_t launch_pack_blocks(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, uint32_t* status,
-                               cudaStream_t stream, int num_sms) {
+cudaError_t launch_pack_blocks(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D,
+                               uint32_t* status, cudaStream_t stream, int num_sms) {
   const int64_t total = N * scale_blocks(K);
   const int64_t want = (total + 7) / 8;
   const unsigned grid = (unsigned)std::min<int64_t>(want, (int64_t)num_sms * 32);
-  bl_block_scale_pack_kernel<<<grid, 256, 0, stream>>>(W, N, K, packed, D, status);
+  if (bf16)
+    bl_block_scale_pack_kernel<true><<<grid, 256, 0, stream>>>(W, N, K, packed, D, status);
+  else
+    bl_block_scale_pack_kernel<false><<<grid, 256, 0, stream>>>(W, N, K, packed, D, status);
   return cudaGetLastError();
 }
 
@@ -657,7 +665,7 @@ int block_forward_tile(int64_t M, int64_t K) {
   return tm;
 }
 
-cudaError_t launch_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+cudaError_t launch_forward_blocks(const void* x, bool bf16, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                                   const float* D, float* y, void* ws, cudaStream_t stream, int num_sms) {
   uint8_t* base = static_cast<uint8_t*>(ws);
   BlockFwdArgs a;
@@ -693,22 +701,29 @@ cudaError_t launch_forward_blocks(const float* x, int64_t M, int64_t N, int64_t 
     cfg.blockDim = dim3(kFwdWarps * 32);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
-    void (*kern)(BlockDecArgs) = bl_block_scale_decode_kernel<0>;
-    switch (a.nb) {
-      case 4: kern = bl_block_scale_decode_kernel<4>; break;     // K = 1024
-      case 8: kern = bl_block_scale_decode_kernel<8>; break;     // K = 2048
-      case 10: kern = bl_block_scale_decode_kernel<10>; break;   // K = 2560
-      case 12: kern = bl_block_scale_decode_kernel<12>; break;   // K = 3072
-      case 27: kern = bl_block_scale_decode_kernel<27>; break;   // K = 6912
-      default: break;
+    void (*kern)(BlockDecArgs) = nullptr;
+#define BL_BDK(B)                                                                  \
+  switch (a.nb) {                                                                  \
+    case 4: kern = bl_block_scale_decode_kernel<4, B>; break;   /* K = 1024 */     \
+    case 8: kern = bl_block_scale_decode_kernel<8, B>; break;   /* K = 2048 */     \
+    case 10: kern = bl_block_scale_decode_kernel<10, B>; break; /* K = 2560 */     \
+    case 12: kern = bl_block_scale_decode_kernel<12, B>; break; /* K = 3072 */     \
+    case 27: kern = bl_block_scale_decode_kernel<27, B>; break; /* K = 6912 */     \
+    default: kern = bl_block_scale_decode_kernel<0, B>; break;                     \
+  }
+    if (bf16) {
+      BL_BDK(true)
+    } else {
+      BL_BDK(false)
     }
+#undef BL_BDK
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, d);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
   // Otherwise the activations are quantised once into the workspace (private
   // order), and the contraction launches as a programmatic dependent of that.
-  cudaError_t eq = launch_act_quant(x, false, M, K, reinterpret_cast<int8_t*>(base + ws_q_off(M)),
+  cudaError_t eq = launch_act_quant(x, bf16, M, K, reinterpret_cast<int8_t*>(base + ws_q_off(M)),
                                     reinterpret_cast<float*>(base + ws_sx_off(M)),
                                     reinterpret_cast<int32_t*>(base + ws_rowsum_off(M)), true, stream,
                                     reinterpret_cast<uint32_t*>(base));

@@ -115,8 +115,9 @@ inline int64_t scale_blocks(int64_t K) { return (K + kScaleBlock - 1) / kScaleBl
 constexpr size_t kBlockFwdSmemMax = 200 * 1024;
 // status: a device word that gets bit 0 OR-ed in for a block holding a
 // non-finite weight (that block's words and scale are left unwritten).
-cudaError_t launch_pack_blocks(const float* W, int64_t N, int64_t K, uint32_t* packed, float* D, uint32_t* status,
-                               cudaStream_t stream, int num_sms);
+// W is fp32, or bf16 bit patterns when bf16 (widened exactly).
+cudaError_t launch_pack_blocks(const void* W, bool bf16, int64_t N, int64_t K, uint32_t* packed, float* D,
+                               uint32_t* status, cudaStream_t stream, int num_sms);
 // Tokens per CTA tile of the block forward (its activation codes fit in
 // kBlockFwdSmemMax of shared memory); always >= 1 for K <= kMaxK.
 int block_forward_tile(int64_t M, int64_t K);
@@ -130,7 +131,8 @@ constexpr int64_t kBlockGemmMinM = 128;
 inline size_t ws_blocks_bytes(int64_t M, int64_t K) {
   return ws_forward_bytes(M, K) + align256(4 * (size_t)M * (size_t)scale_blocks(K));
 }
-cudaError_t launch_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+// x is fp32, or bf16 bit patterns when bf16 (widened exactly).
+cudaError_t launch_forward_blocks(const void* x, bool bf16, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                                   const float* D, float* y, void* ws, cudaStream_t stream, int num_sms);
 
 cudaError_t launch_selftest_wait(uint32_t* err, uint64_t limit_ns, cudaStream_t stream);

@@ -262,6 +262,13 @@ BL_API int bitlinear_pack_weights_blocks(const float* W, int64_t N, int64_t K,
                                          uint32_t* packed, float* D,
                                          void* ws, size_t ws_bytes, bl_stream_t stream);
 
+/* As bitlinear_pack_weights_blocks, from a bf16 master weight (bit patterns
+ * [N, K], uint16, 16-byte aligned), each value widened to fp32 exactly.
+ * Synchronous. */
+BL_API int bitlinear_pack_weights_blocks_bf16(const uint16_t* W, int64_t N, int64_t K,
+                                              uint32_t* packed, float* D,
+                                              void* ws, size_t ws_bytes, bl_stream_t stream);
+
 /* Bytes of scratch that bitlinear_forward_blocks needs: the forward
  * workspace plus one int32 per token and block (the row sums of the codes per
  * block, for the tensor-core route). */
@@ -280,6 +287,13 @@ BL_API size_t bitlinear_blocks_workspace_size(int64_t M, int64_t N, int64_t K);
 BL_API int bitlinear_forward_blocks(const float* x, int64_t M, int64_t N, int64_t K,
                                     const uint32_t* packed, const float* D, float* y,
                                     void* ws, size_t ws_bytes, bl_stream_t stream);
+
+/* As bitlinear_forward_blocks, from bf16 activations (bit patterns [M, K],
+ * uint16, 16-byte aligned), widened to fp32 exactly in the quantiser; y fp32.
+ * Same workspace. Asynchronous. */
+BL_API int bitlinear_forward_blocks_bf16(const uint16_t* x, int64_t M, int64_t N, int64_t K,
+                                         const uint32_t* packed, const float* D, float* y,
+                                         void* ws, size_t ws_bytes, bl_stream_t stream);
 
 /* ---------------------------------------------------------------- batch --- */
 

@@ -209,3 +209,24 @@ def test_forward_blocks_workload_shapes_sampled(B, key, li, M):
     assert np.array_equal(D.cpu().numpy()[rows].view(np.uint32), D_ref.view(np.uint32))
     y_ref = O.bitlinear_forward_blocks(x[toks], p_ref, D_ref, layer.K)
     assert_y_bitexact(y[np.ix_(toks, rows)], y_ref)
+
+
+# -------------------------------------------------------------- bf16 inputs
+def _bf16(a):
+    """fp32 array -> (bf16 bit patterns uint16, the same values as fp32), by truncation."""
+    bits = (np.ascontiguousarray(a, np.float32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+    return bits, O.bf16_to_f32(bits)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 300, 2560), (1, 77, 528), (5, 64, 6912), (130, 257, 1152), (1, 129, 8192)])
+def test_blocks_bf16_inputs_bitexact(B, M, N, K):
+    """bf16 master weights and bf16 activations, widened exactly: the same as
+    the fp32 path on the widened values (pack, and each forward route)."""
+    Wb, Wf = _bf16(WL.weight(N, K, "laplace", M + N + K))
+    xb, xf = _bf16(WL.activations(M, K, "student_t", M + K, meta={"df": 3.0}))
+    packed, D = B.pack_weights_blocks(torch.from_numpy(Wb.view(np.int16)).cuda().view(torch.bfloat16))
+    p_ref, D_ref = O.pack_weights_blocks(Wf)
+    assert np.array_equal(u32(packed), p_ref)
+    assert np.array_equal(D.cpu().numpy().view(np.uint32), D_ref.view(np.uint32))
+    y = B.forward_blocks(torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16), packed, D).cpu().numpy()
+    assert_y_bitexact(y, O.bitlinear_forward_blocks(xf, p_ref, D_ref, K))
