@@ -869,8 +869,10 @@ template <bool kBf16>
 static cudaError_t launch_act_quant_t(const void* x, int64_t M, int64_t K, int8_t* q, float* s_x, int32_t* rowsum,
                                       bool permuted, cudaStream_t stream, uint32_t* err_reset) {
   const int64_t ngroups = K / 16;
-  // Rows of up to 6 groups per lane: one warp per token, no block barrier.
-  if (ngroups <= 32 * 6) {
+  // Many tokens with rows of up to 6 groups per lane: one warp per token, no
+  // block barrier. A few tokens (decode) keep one CTA per token, which
+  // finishes each token sooner (its 16-column groups spread over more warps).
+  if (ngroups <= 32 * 6 && M >= 1024) {
     const int wg = (int)((ngroups + 31) / 32);
     const int64_t want = (M + 7) / 8;
     const unsigned grid = (unsigned)(want < 1 ? 1 : (want < 148 * 16 ? want : 148 * 16));
